@@ -1,0 +1,357 @@
+"""Float64 numpy statement of the AdaSpark layer (test infrastructure only).
+
+Sources (page titles and sections; the pages print no code for this method):
+
+* "AdaSpark: Adaptive Sparsity for Efficient Long-Video Understanding"
+  (papernotes.org note), sections 整体框架 (overall framework) and 关键设计 1-4
+  (key designs: 3D cube partition, AdaS-Attn with the P_i / S_i formula,
+  AdaS-FFN with the mean-compensation formula, the shared Top-p knob).
+* The same paper's abstract and Figure 2 caption (thelatestinai.com list view):
+  relevance is scored over *preceding* cubes; text tokens pass densely through
+  the FFN.
+
+Readings taken where the pages leave a step open (each is listed, with its
+basis, in the design notes of this repository):
+
+* tokens are in cube-major order, cubes enumerated time-major (t_b, h_b, w_b),
+  tokens inside a cube in (t, h, w) order; edge cubes are truncated;
+* the index i of P_i is the query's own cube; P_i runs over cubes 0..i-1, the
+  own cube is always attended causally, the first cube selects nothing;
+* selection is per (query token, query head); query head h reads KV head
+  floor(h / (hq / hkv));
+* Top-p: order by (probability descending, index ascending), take the smallest
+  prefix whose cumulative mass reaches p, at least one element; p >= 1 keeps all;
+* the selected cubes and the own-cube causal prefix share one softmax; P_i is
+  not used as a weight;
+* text tokens are the suffix and attend densely and causally;
+* FFN importance is the linear share of the L2 norm inside the cube,
+  w_u = ||x_u|| / sum_v ||x_v||; a cube whose norms sum to 0 keeps every token;
+* the FFN is SwiGLU without bias, W_down(silu(W_gate x) * W_up x); an active
+  or text token gets y = x + FFN(x), a skipped one y = x + mean of FFN over the
+  cube's active tokens (unrounded).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def _f64(a):
+    """Exact float64 copy of a numpy array or torch tensor (bf16 widens exactly)."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Key design 1: 3D spatio-temporal cube partition.
+# ---------------------------------------------------------------------------
+def cube_partition(T, H, W, cube_h, cube_w, cube_t, n_text):
+    """Split a T x H x W video-token grid into h x w x t cubes.
+
+    Follows the partition of key design 1 (cubes are h x w x t windows of the
+    video tokens fed to the LLM).  Returns ``perm`` (perm[k] = raster index
+    t*H*W + h*W + w of the k-th token in cube-major order), ``cube_ids`` (cube of
+    each cube-major position, then -1 for each of the n_text text tokens),
+    ``cube_offsets`` [C+1] and C.  Cubes are enumerated time-major over the cube
+    grid; tokens within a cube in (t, h, w) order; edge cubes are truncated.
+    """
+    if min(T, H, W, cube_h, cube_w, cube_t) <= 0 or n_text < 0:
+        raise ValueError("sizes must be positive")
+    n_tb = -(-T // cube_t)
+    n_hb = -(-H // cube_h)
+    n_wb = -(-W // cube_w)
+    perm, ids, offsets = [], [], [0]
+    c = 0
+    for tb in range(n_tb):
+        for hb in range(n_hb):
+            for wb in range(n_wb):
+                for t in range(tb * cube_t, min(T, (tb + 1) * cube_t)):
+                    for h in range(hb * cube_h, min(H, (hb + 1) * cube_h)):
+                        for w in range(wb * cube_w, min(W, (wb + 1) * cube_w)):
+                            perm.append(t * H * W + h * W + w)
+                            ids.append(c)
+                offsets.append(len(perm))
+                c += 1
+    ids.extend([-1] * n_text)
+    return (np.asarray(perm, np.int32), np.asarray(ids, np.int32),
+            np.asarray(offsets, np.int32), c)
+
+
+# ---------------------------------------------------------------------------
+# Key design 2: AdaS-Attn.
+# ---------------------------------------------------------------------------
+def cube_mean_keys(K, cube_offsets):
+    """k_bar[j, kv, :] = mean of K over the tokens of cube j (key design 2,
+    "similarity to the cube's mean key").  K: [N, hkv, d]; returns float64
+    [C, hkv, d], accumulated token by token."""
+    K = _f64(K)
+    off = np.asarray(cube_offsets)
+    C = len(off) - 1
+    out = np.zeros((C,) + K.shape[1:], dtype=np.float64)
+    for j in range(C):
+        acc = np.zeros(K.shape[1:], dtype=np.float64)
+        for t in range(off[j], off[j + 1]):
+            acc += K[t]
+        out[j] = acc / (off[j + 1] - off[j])
+    return out
+
+
+def cube_scores(q, kbar_rows, d):
+    """s_j = q . k_bar_j / sqrt(d_k) for the preceding cubes (key design 2,
+    the argument of the softmax in the P_i formula).  q: [..., d],
+    kbar_rows: [c, d]."""
+    return (_f64(q) @ _f64(kbar_rows).T) / math.sqrt(d)
+
+
+def softmax(s, axis=-1):
+    """Softmax in float64 (the P_i formula of key design 2)."""
+    s = np.asarray(s, dtype=np.float64)
+    if s.shape[axis] == 0:
+        return s.copy()
+    m = np.max(s, axis=axis, keepdims=True)
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+def _check_p(p):
+    if not (p > 0.0 and p <= 1.0):  # also rejects NaN
+        raise ValueError("p must lie in (0, 1]")
+
+
+def top_p(P, p):
+    """Top-p (nucleus) set of a probability vector (S_i of key design 2; the same
+    rule drives AdaS-FFN per key designs 3 and 4).
+
+    Order the entries by probability descending, index ascending; keep the
+    smallest prefix whose cumulative mass reaches p (at least one entry; every
+    entry when the sum never reaches p in floating point).  p >= 1 keeps all.
+    Returns a boolean mask over the entries.
+    """
+    _check_p(p)
+    P = np.asarray(P, dtype=np.float64)
+    m = P.shape[-1]
+    keep = np.zeros(P.shape, dtype=bool)
+    if m == 0:
+        return keep
+    if p >= 1.0:
+        keep[...] = True
+        return keep
+    flat = P.reshape(-1, m)
+    kflat = keep.reshape(-1, m)
+    order = np.argsort(-flat, axis=1, kind="stable")
+    cum = np.cumsum(np.take_along_axis(flat, order, axis=1), axis=1)
+    reached = cum >= p
+    kstar = np.where(reached.any(axis=1), reached.argmax(axis=1) + 1, m)
+    for r in range(flat.shape[0]):
+        kflat[r, order[r, :kstar[r]]] = True
+    return keep
+
+
+def top_p_margin(P, p):
+    """Distance of a Top-p cut from flipping: the smallest of C_k* - p,
+    p - C_(k*-1) (k* > 1) and P_(k*) - P_(k*+1) (k* < m), in the sorted order
+    used by ``top_p``.  +inf when nothing can flip (m <= 1 or p >= 1)."""
+    _check_p(p)
+    P = np.asarray(P, dtype=np.float64)
+    m = P.shape[-1]
+    flat = P.reshape(-1, m)
+    out = np.full(flat.shape[0], np.inf)
+    if m <= 1 or p >= 1.0:
+        return out.reshape(P.shape[:-1])
+    order = np.argsort(-flat, axis=1, kind="stable")
+    srt = np.take_along_axis(flat, order, axis=1)
+    cum = np.cumsum(srt, axis=1)
+    reached = cum >= p
+    kstar = np.where(reached.any(axis=1), reached.argmax(axis=1) + 1, m)
+    for r in range(flat.shape[0]):
+        k = kstar[r]
+        cand = [cum[r, k - 1] - p]
+        if k > 1:
+            cand.append(p - cum[r, k - 2])
+        if k < m:
+            cand.append(srt[r, k - 1] - srt[r, k])
+        out[r] = min(cand)
+    return out.reshape(P.shape[:-1])
+
+
+def select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=None, with_margin=False):
+    """AdaS-Attn cube selection (key design 2, formula P_i and S_i).
+
+    For visual token t in cube i and query head h: P = softmax over the
+    preceding cubes j < i of q . k_bar_j / sqrt(d), k_bar of KV head
+    floor(h / (hq/hkv)); S = Top-p(P, p).  Returns a boolean array
+    sel[len(tokens), hq, C] (sel[r, h, j] is True when cube j is selected; the
+    own cube is not marked here, it is always attended causally) and, when
+    asked, the cut margins [len(tokens), hq] (+inf where nothing can flip).
+    ``tokens`` defaults to every visual token.
+    """
+    _check_p(p)
+    off = np.asarray(cube_offsets)
+    C = len(off) - 1
+    d = Q.shape[-1]
+    g = hq // hkv
+    kbar = cube_mean_keys(K, off)
+    if tokens is None:
+        tokens = np.arange(n_vis)
+    tokens = np.asarray(tokens)
+    cube_of = np.searchsorted(off, tokens, side="right") - 1
+    sel = np.zeros((len(tokens), hq, C), dtype=bool)
+    margin = np.full((len(tokens), hq), np.inf)
+    Qf = _f64(Q[tokens]) if not isinstance(Q, np.ndarray) else _f64(Q)[tokens]
+    for i in np.unique(cube_of):
+        rows = np.nonzero(cube_of == i)[0]
+        if i == 0:
+            continue  # no preceding cube: empty set
+        for h in range(hq):
+            kv = h // g
+            s = cube_scores(Qf[rows, h, :], kbar[:i, kv, :], d)   # [rows, i]
+            P = softmax(s, axis=1)
+            sel[rows, h, :i] = top_p(P, p)
+            if with_margin:
+                margin[rows, h] = top_p_margin(P, p)
+    if with_margin:
+        return sel, margin
+    return sel
+
+
+def attention_given_sets(Q, K, V, cube_offsets, n_vis, sel, tokens=None):
+    """GQA attention restricted to the selected cubes plus the own cube
+    (key design 2: each query attends only to the chosen cubes and always keeps
+    full attention to its own cube; causal inside the own cube).  Text tokens
+    (index >= n_vis) attend densely and causally to every earlier token.
+
+    One softmax over all admitted keys, scale 1/sqrt(d), written as a masked
+    dense softmax per (cube, head).  ``sel`` is [len(tokens), hq, C] for the
+    tokens in ``tokens`` (rows of text tokens are ignored).  Returns float64
+    out [len(tokens), hq, d].
+    """
+    off = np.asarray(cube_offsets)
+    N, hq, d = Q.shape
+    hkv = K.shape[1]
+    g = hq // hkv
+    if tokens is None:
+        tokens = np.arange(N)
+    tokens = np.asarray(tokens)
+    Kf, Vf = _f64(K), _f64(V)
+    Qf = _f64(Q)[tokens] if isinstance(Q, np.ndarray) else _f64(Q[tokens])
+    out = np.zeros((len(tokens), hq, d), dtype=np.float64)
+    key_cube = np.concatenate([np.searchsorted(off, np.arange(n_vis), side="right") - 1,
+                               np.full(N - n_vis, -1)])
+    pos = np.arange(N)
+    scale = 1.0 / math.sqrt(d)
+    group = np.where(tokens < n_vis, key_cube[np.minimum(tokens, N - 1)], -1)
+    for i in np.unique(group):
+        rows = np.nonzero(group == i)[0]
+        t = tokens[rows]
+        if i < 0:                       # text rows: dense causal over all earlier tokens
+            end = int(t.max()) + 1
+            base = pos[None, :end] <= t[:, None]
+        else:                           # visual rows of cube i
+            end = int(off[i + 1])
+            base = (key_cube[None, :end] == i) & (pos[None, :end] <= t[:, None])
+        for h in range(hq):
+            kv = h // g
+            if i < 0:
+                mask = base
+            else:
+                kc = key_cube[:end]
+                chosen = sel[rows][:, h, :][:, np.maximum(kc, 0)] & (kc < i)[None, :]
+                mask = base | chosen
+            s = (Qf[rows, h, :] @ Kf[:end, kv, :].T) * scale
+            s = np.where(mask, s, -np.inf)
+            m = np.max(s, axis=1, keepdims=True)
+            e = np.where(mask, np.exp(s - m), 0.0)
+            out[rows, h] = (e / e.sum(axis=1, keepdims=True)) @ Vf[:end, kv, :]
+    return out
+
+
+def cube_attn(Q, K, V, cube_offsets, n_vis, p, tokens=None):
+    """The whole AdaS-Attn call: selection then restricted attention."""
+    hq, hkv = Q.shape[1], K.shape[1]
+    sel = select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=tokens)
+    return attention_given_sets(Q, K, V, cube_offsets, n_vis, sel, tokens=tokens), sel
+
+
+# ---------------------------------------------------------------------------
+# Key design 3: AdaS-FFN with mean compensation.
+# ---------------------------------------------------------------------------
+def ffn_select(x, cube_offsets, n_vis, p, cubes=None, with_margin=False):
+    """AdaS-FFN token selection (key design 3): inside each cube rank tokens by
+    L2 norm, importance w_u = ||x_u|| / sum_v ||x_v||, keep Top-p(w, p).  Text
+    tokens are always active.  Returns a boolean ``active`` [N] (entries of
+    cubes not in ``cubes`` are left False) and, when asked, per-cube margins."""
+    _check_p(p)
+    X = _f64(x)
+    N = X.shape[0]
+    off = np.asarray(cube_offsets)
+    C = len(off) - 1
+    active = np.zeros(N, dtype=bool)
+    active[n_vis:] = True
+    margins = np.full(C, np.inf)
+    if cubes is None:
+        cubes = range(C)
+    for c in cubes:
+        a, b = off[c], off[c + 1]
+        norms = np.sqrt(np.sum(X[a:b] * X[a:b], axis=1))
+        total = norms.sum()
+        if total == 0.0:
+            active[a:b] = True
+            continue
+        w = norms / total
+        active[a:b] = top_p(w, p)
+        if with_margin:
+            margins[c] = top_p_margin(w, p)
+    if with_margin:
+        return active, margins
+    return active
+
+
+def swiglu_ffn(x, W_gate, W_up, W_down):
+    """FFN(x) = W_down (silu(W_gate x) * W_up x), no bias, float64."""
+    X = _f64(x)
+    gate = X @ _f64(W_gate).T
+    up = X @ _f64(W_up).T
+    h = gate / (1.0 + np.exp(-gate)) * up
+    return h @ _f64(W_down).T
+
+
+def ffn_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active, cubes=None,
+                   text=True):
+    """Outputs of AdaS-FFN for a given active set (key design 3): active and text
+    tokens y = x + FFN(x); skipped tokens y_k = x_k + m_bar_i with
+    m_bar_i = mean of FFN(x_j) over the cube's active tokens.  Returns float64
+    y [N, D] (rows of cubes outside ``cubes`` are NaN; text rows NaN when
+    ``text`` is False)."""
+    X = _f64(x)
+    N, D = X.shape
+    off = np.asarray(cube_offsets)
+    C = len(off) - 1
+    y = np.full((N, D), np.nan)
+    if cubes is None:
+        cubes = range(C)
+    for c in cubes:
+        a, b = off[c], off[c + 1]
+        idx = np.arange(a, b)
+        act = idx[active[a:b]]
+        skip = idx[~active[a:b]]
+        f = swiglu_ffn(X[act], W_gate, W_up, W_down)
+        y[act] = X[act] + f
+        if len(skip):
+            mbar = f.sum(axis=0) / len(act)
+            y[skip] = X[skip] + mbar
+    if text and N > n_vis:
+        y[n_vis:] = X[n_vis:] + swiglu_ffn(X[n_vis:], W_gate, W_up, W_down)
+    return y
+
+
+def token_ffn(x, W_gate, W_up, W_down, cube_offsets, n_vis, p, cubes=None, text=True):
+    """The whole AdaS-FFN call: selection then the given-set outputs."""
+    active = ffn_select(x, cube_offsets, n_vis, p, cubes=cubes)
+    return ffn_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active,
+                          cubes=cubes, text=text), active

@@ -1,0 +1,341 @@
+"""Pins for the float64 oracle: each test checks it against something other than
+itself -- brute force on tiny inputs, closed forms, invariants, or an
+independent library routine (torch in float64) -- so that a dropped term, a
+wrong sign or index, or a transposed operand in the oracle fails here.
+All CPU-only."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as Fn
+
+import oracle
+from oracle import adaspark_ref as ref
+
+
+# ---------------------------------------------------------------- partition
+@pytest.mark.parametrize("grid,cube,n_text", [
+    ((4, 4, 4), (2, 2, 2), 0),
+    ((5, 7, 3), (2, 3, 2), 3),      # truncated edge cubes on every axis
+    ((8, 8, 8), (4, 4, 2), 32),
+    ((3, 1, 1), (1, 1, 1), 1),      # one token per cube
+    ((2, 3, 5), (4, 4, 4), 0),      # one cube larger than the grid
+])
+def test_partition_matches_sorted_order(grid, cube, n_text):
+    T, H, W = grid
+    ch, cw, ct = cube
+    perm, ids, off, C = oracle.cube_partition(T, H, W, ch, cw, ct, n_text)
+    # Independent statement: sort raster positions by (cube t, cube h, cube w, t, h, w).
+    keys = []
+    for t in range(T):
+        for h in range(H):
+            for w in range(W):
+                keys.append(((t // ct, h // ch, w // cw), (t, h, w), t * H * W + h * W + w))
+    keys.sort()
+    cube_keys = sorted({k[0] for k in keys})
+    rank = {k: i for i, k in enumerate(cube_keys)}
+    assert C == len(cube_keys)
+    assert list(perm) == [k[2] for k in keys]
+    assert sorted(perm.tolist()) == list(range(T * H * W))       # bijection
+    assert list(ids[:T * H * W]) == [rank[k[0]] for k in keys]
+    assert list(ids[T * H * W:]) == [-1] * n_text
+    counts = np.bincount(ids[:T * H * W], minlength=C)
+    assert list(np.diff(off)) == list(counts)
+    assert off[0] == 0 and off[-1] == T * H * W
+
+
+# ---------------------------------------------------------------- top-p rule
+def _brute_top_p(P, p):
+    """Minimal cardinality, then maximal mass, then lexicographically smallest."""
+    m = len(P)
+    best = None
+    for k in range(1, m + 1):
+        cands = []
+        for S in itertools.combinations(range(m), k):
+            mass = sum(P[j] for j in S)
+            if mass >= p:
+                cands.append((-mass, S))
+        if cands:
+            cands.sort()
+            best = cands[0][1]
+            break
+    assert best is not None
+    return set(best)
+
+
+def test_top_p_brute_force():
+    rng = np.random.default_rng(5)
+    for trial in range(300):
+        m = int(rng.integers(1, 11))
+        # integer weights / 1024: every partial sum is exact in binary, so the
+        # brute force and the prefix rule see identical masses; small ranges
+        # force many ties.
+        w = rng.integers(1, 6 if trial % 2 else 200, size=m).astype(np.float64)
+        w = np.floor(w / w.sum() * 1024)
+        w[0] += 1024 - w.sum()
+        if w.min() <= 0:
+            continue
+        P = w / 1024.0
+        # p on the grid (exact equality must count as reached) or between points
+        p = float(rng.integers(1, 1024)) / 1024.0
+        if trial % 3 == 0:
+            p -= 1.0 / 4096.0
+        got = set(np.nonzero(oracle.top_p(P, p))[0].tolist())
+        assert got == _brute_top_p(P, p), (P, p)
+
+
+@pytest.mark.parametrize("m,p", [(7, 0.7), (10, 0.55), (13, 0.31), (64, 0.7), (100, 0.905)])
+def test_top_p_uniform_closed_form(m, p):
+    P = np.full(m, 1.0 / m)
+    keep = oracle.top_p(P, p)
+    k = math.ceil(p * m)
+    assert keep.sum() == k
+    assert keep[:k].all()      # ties go to the lower indices
+
+
+def test_top_p_degenerate():
+    P = np.array([0.1, 0.4, 0.4, 0.1])
+    assert np.nonzero(oracle.top_p(P, 1e-9))[0].tolist() == [1]   # argmax, first of the tie
+    assert oracle.top_p(P, 1.0).all()
+    assert oracle.top_p(np.zeros(0), 0.5).shape == (0,)
+    # cumulative mass exactly equal to p counts as reached (binary-exact values)
+    assert np.nonzero(oracle.top_p(np.array([0.25, 0.5, 0.25]), 0.75))[0].tolist() == [0, 1]
+    assert oracle.top_p(np.full(4, 0.25), 0.5).tolist() == [True, True, False, False]
+    for bad in (0.0, -0.1, 1.5, float("nan")):
+        with pytest.raises(ValueError):
+            oracle.top_p(P, bad)
+
+
+def test_top_p_margin_values():
+    P = np.array([0.5, 0.3, 0.2])
+    # p = 0.75: k* = 2, C_2 = 0.8, C_1 = 0.5, P_(2) - P_(3) = 0.1
+    assert oracle.top_p_margin(P, 0.75) == pytest.approx(min(0.05, 0.25, 0.1))
+    assert oracle.top_p_margin(np.array([0.25] * 4), 0.6) == 0.0   # exact tie at the cut
+
+
+# ---------------------------------------------------------------- cube means
+def test_cube_mean_keys_invariants():
+    rng = np.random.default_rng(1)
+    off = np.array([0, 3, 4, 9, 16])
+    K = rng.standard_normal((16, 2, 8))
+    kbar = oracle.cube_mean_keys(K, off)
+    for j in range(4):
+        resid = (K[off[j]:off[j + 1]] - kbar[j]).sum(axis=0)
+        assert np.abs(resid).max() < 1e-12
+    assert np.array_equal(kbar[1], K[3])                  # single-token cube
+    Kc = np.repeat(rng.standard_normal((4, 1, 2, 8)), np.diff(off), axis=0).reshape(16, 2, 8)
+    kc = oracle.cube_mean_keys(Kc, off)
+    for j in range(4):
+        assert np.allclose(kc[j], Kc[off[j]], atol=1e-15)   # constant cube -> that constant
+
+
+# ---------------------------------------------------------------- AdaS-Attn selection
+def _qkv(rng, N, hq, hkv, d, scale=1.0):
+    Q = rng.standard_normal((N, hq, d)) * scale
+    K = rng.standard_normal((N, hkv, d)) * scale
+    V = rng.standard_normal((N, hkv, d))
+    return Q, K, V
+
+
+@pytest.mark.parametrize("p", [0.3, 0.55, 0.7, 0.9])
+def test_select_uniform_means_closed_form(p):
+    """All cube means equal -> P uniform over the c preceding cubes -> the
+    ceil(p*c) lowest-index cubes.  Counting the own cube in P would give
+    ceil(p*(c+1)) instead."""
+    rng = np.random.default_rng(2)
+    C, n, hq, hkv, d = 12, 4, 2, 1, 16
+    off = np.arange(C + 1) * n
+    N = C * n
+    Q = rng.standard_normal((N, hq, d))
+    K = np.tile(rng.standard_normal((1, hkv, d)), (N, 1, 1))
+    sel = oracle.select_cubes(Q, K, off, N, hq, hkv, p)
+    for t in range(N):
+        c = t // n
+        if c > 0 and abs(p * c - round(p * c)) < 1e-9:
+            continue   # p*c on an integer: the cut sits exactly on a rounding tie
+        for h in range(hq):
+            k = math.ceil(p * c) if c > 0 else 0
+            assert sel[t, h].sum() == k
+            assert sel[t, h, :k].all()
+            assert not sel[t, h, c:].any()
+    # discriminates own-cube inclusion for at least one cube
+    assert any(math.ceil(p * c) != math.ceil(p * (c + 1)) for c in range(1, C))
+
+
+def test_select_two_cube_sigmoid_scale_and_sign():
+    """Rows of cube 2 see cubes 0 and 1.  q . (kbar_1 - kbar_0) / sqrt(d) = ln 3,
+    so P = (1/4, 3/4) exactly in closed form: p = 0.74 keeps cube 1 alone,
+    p = 0.76 keeps both.  Dropping 1/sqrt(d) (P_1 ~ 0.99985) or flipping the
+    sign (cube 0 preferred) changes the answer."""
+    d, n = 64, 2
+    off = np.array([0, n, 2 * n, 3 * n])
+    N = 3 * n
+    Q = np.zeros((N, 1, d))
+    K = np.zeros((N, 1, d))
+    V = np.zeros((N, 1, d))
+    Q[:, 0, 0] = 1.0
+    K[0:n, 0, 0] = 0.0
+    K[n:2 * n, 0, 0] = math.sqrt(d) * math.log(3.0)
+    sel = oracle.select_cubes(Q, K, off, N, 1, 1, 0.74)
+    assert sel[2 * n:, 0, :].tolist() == [[False, True, False]] * n
+    sel = oracle.select_cubes(Q, K, off, N, 1, 1, 0.76)
+    assert sel[2 * n:, 0, :].tolist() == [[True, True, False]] * n
+    # cube 1's rows see only cube 0: always selected; cube 0's rows: nothing
+    assert sel[n:2 * n, 0, 0].all() and not sel[:n].any()
+
+
+def test_select_gqa_head_mapping():
+    """hq = 4, hkv = 2: heads 0,1 read KV head 0 and heads 2,3 read KV head 1
+    (floor(h / g)); the two KV heads prefer opposite cubes."""
+    d, n = 8, 2
+    off = np.array([0, n, 2 * n, 3 * n])
+    N = 3 * n
+    Q = np.zeros((N, 4, d))
+    Q[:, :, 0] = 1.0
+    K = np.zeros((N, 2, d))
+    K[0:n, 0, 0] = 20.0      # KV head 0 prefers cube 0
+    K[n:2 * n, 1, 0] = 20.0  # KV head 1 prefers cube 1
+    sel = oracle.select_cubes(Q, K, off, N, 4, 2, 0.5)
+    rows = sel[2 * n:]
+    for h, want in ((0, [True, False, False]), (1, [True, False, False]),
+                    (2, [False, True, False]), (3, [False, True, False])):
+        assert rows[:, h, :].tolist() == [want] * n
+
+
+# ---------------------------------------------------------------- AdaS-Attn attention
+def _sdpa_masked(Q, K, V, mask):
+    """torch SDPA in float64 with an explicit boolean mask [hq, N, N]."""
+    hq, hkv = Q.shape[1], K.shape[1]
+    g = hq // hkv
+    q = torch.from_numpy(Q).permute(1, 0, 2)[None]
+    k = torch.from_numpy(K).repeat_interleave(g, dim=1).permute(1, 0, 2)[None]
+    v = torch.from_numpy(V).repeat_interleave(g, dim=1).permute(1, 0, 2)[None]
+    o = Fn.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(mask)[None])
+    return o[0].permute(1, 0, 2).numpy()
+
+
+def test_attention_dense_equals_causal_sdpa():
+    rng = np.random.default_rng(3)
+    off = np.array([0, 5, 9, 16, 20, 27])
+    n_vis, n_text, hq, hkv, d = 27, 6, 6, 2, 16
+    N = n_vis + n_text
+    Q, K, V = _qkv(rng, N, hq, hkv, d)
+    sel = oracle.select_cubes(Q, K, off, n_vis, hq, hkv, 1.0)
+    out = oracle.attention_given_sets(Q, K, V, off, n_vis, sel)
+    causal = np.tril(np.ones((N, N), dtype=bool))
+    want = _sdpa_masked(Q, K, V, np.broadcast_to(causal, (hq, N, N)).copy())
+    assert np.abs(out - want).max() < 1e-12
+
+
+def test_attention_given_random_sets_equals_masked_sdpa():
+    rng = np.random.default_rng(4)
+    off = np.array([0, 4, 8, 12, 16, 20, 24])
+    n_vis, n_text, hq, hkv, d = 24, 5, 4, 2, 8
+    N = n_vis + n_text
+    C = len(off) - 1
+    Q, K, V = _qkv(rng, N, hq, hkv, d)
+    sel = rng.random((N, hq, C)) < 0.4
+    out = oracle.attention_given_sets(Q, K, V, off, n_vis, sel)
+    cube = np.searchsorted(off, np.arange(n_vis), side="right") - 1
+    mask = np.zeros((hq, N, N), dtype=bool)
+    for t in range(N):
+        for h in range(hq):
+            for u in range(t + 1):
+                if t >= n_vis:
+                    mask[h, t, u] = True
+                elif cube[u] == cube[t]:
+                    mask[h, t, u] = True
+                elif cube[u] < cube[t] and sel[t, h, cube[u]]:
+                    mask[h, t, u] = True
+    want = _sdpa_masked(Q, K, V, mask)
+    assert np.abs(out - want).max() < 1e-12
+    # the very first token sees only itself
+    g = hq // hkv
+    for h in range(hq):
+        assert np.array_equal(out[0, h], V[0, h // g])
+
+
+def test_attention_smallest_p_is_argmax_cube_plus_own():
+    rng = np.random.default_rng(6)
+    off = np.arange(7) * 4
+    n_vis, hq, hkv, d = 24, 2, 1, 8
+    Q, K, V = _qkv(rng, n_vis, hq, hkv, d, scale=2.0)
+    sel = oracle.select_cubes(Q, K, off, n_vis, hq, hkv, 1e-9)
+    kbar = np.stack([K[off[j]:off[j + 1]].mean(axis=0) for j in range(6)])
+    for t in range(4, n_vis):
+        c = t // 4
+        for h in range(hq):
+            s = Q[t, h] @ kbar[:c, 0].T
+            assert np.nonzero(sel[t, h])[0].tolist() == [int(np.argmax(s))]
+
+
+# ---------------------------------------------------------------- AdaS-FFN
+def _ffn_torch(x, Wg, Wu, Wd):
+    x, Wg, Wu, Wd = (torch.from_numpy(np.asarray(a, dtype=np.float64)) for a in (x, Wg, Wu, Wd))
+    return Fn.linear(Fn.silu(Fn.linear(x, Wg)) * Fn.linear(x, Wu), Wd).numpy()
+
+
+def test_swiglu_matches_torch():
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((9, 16))
+    Wg, Wu, Wd = (rng.standard_normal(s) * 0.3 for s in ((24, 16), (24, 16), (16, 24)))
+    assert np.abs(oracle.swiglu_ffn(x, Wg, Wu, Wd) - _ffn_torch(x, Wg, Wu, Wd)).max() < 1e-12
+
+
+def test_ffn_select_closed_forms():
+    rng = np.random.default_rng(8)
+    D = 12
+    v = rng.standard_normal(D)
+    # cube 0: equal norms (sign flips keep the norm) -> uniform -> ceil(p n) lowest
+    # cube 1: x_u = a_u v with distinct a_u -> w_u = a_u / sum(a): brute force
+    # cube 2: all zeros -> everything active; cube 3: single token
+    a = np.array([3.0, 1.0, 4.0, 1.5, 5.0, 9.0, 2.0])
+    x = np.concatenate([
+        v[None] * np.array([1, -1, 1, -1, 1, -1, 1, 1])[:, None],
+        a[:, None] * v[None],
+        np.zeros((3, D)),
+        v[None] * 2.0,
+        rng.standard_normal((4, D)),          # text
+    ])
+    off = np.array([0, 8, 15, 18, 19])
+    n_vis = 19
+    for p in (0.3, 0.6, 0.8):
+        act = oracle.ffn_select(x, off, n_vis, p)
+        k = math.ceil(p * 8)
+        assert act[:8].tolist() == [True] * k + [False] * (8 - k)
+        w = a / a.sum()
+        want = _brute_top_p(w.tolist(), p)
+        assert set(np.nonzero(act[8:15])[0].tolist()) == want
+        assert act[15:18].all() and act[18] and act[19:].all()
+    act = oracle.ffn_select(x, off, n_vis, 1e-9)
+    assert np.nonzero(act[8:15])[0].tolist() == [5]     # the largest norm alone
+
+
+def test_token_ffn_dense_and_compensation():
+    rng = np.random.default_rng(9)
+    D, F = 16, 24
+    off = np.array([0, 6, 7, 15, 22])       # cube 1 holds a single token
+    n_vis, n_text = 22, 3
+    N = n_vis + n_text
+    x = rng.standard_normal((N, D)) * (1.0 + rng.random((N, 1)))
+    Wg, Wu, Wd = (rng.standard_normal(s) * 0.3 for s in ((F, D), (F, D), (D, F)))
+    full = x + _ffn_torch(x, Wg, Wu, Wd)
+    y1, act1 = oracle.token_ffn(x, Wg, Wu, Wd, off, n_vis, 1.0)
+    assert act1.all()
+    assert np.abs(y1 - full).max() < 1e-12
+    y, act = oracle.token_ffn(x, Wg, Wu, Wd, off, n_vis, 0.5)
+    f = _ffn_torch(x, Wg, Wu, Wd)
+    assert act[6] and np.abs(y[6] - full[6]).max() < 1e-12         # single-token cube
+    assert np.abs(y[n_vis:] - full[n_vis:]).max() < 1e-12           # text unaffected by p
+    for c in range(4):
+        idx = np.arange(off[c], off[c + 1])
+        A, S = idx[act[idx]], idx[~act[idx]]
+        assert len(A) >= 1
+        assert np.abs(y[A] - full[A]).max() < 1e-12
+        if len(S):
+            mbar = f[A].mean(axis=0)
+            assert np.abs((y[S] - x[S]) - mbar[None]).max() < 1e-12   # y_k - x_k = m_bar
+            assert np.abs(np.diff(y[S] - x[S], axis=0)).max() < 1e-12  # shared by the cube
+    assert (~act[:n_vis]).any()
