@@ -1,0 +1,251 @@
+// extern "C" entry points of AdaS-Attn and AdaS-FFN: host-side validation,
+// workspace carving, and the launch sequence on the caller's stream.
+#include <cmath>
+
+#include "attn_kernels.h"
+#include "ffn_kernels.h"
+
+using namespace adaspark;
+
+namespace {
+
+constexpr int kModeDense = 1;
+
+int check_device() {
+  static int cached = -2;
+  if (cached == -2) cached = device_is_sm100();
+  if (cached < 0) return ADASPARK_ECUDA;
+  return cached ? ADASPARK_OK : ADASPARK_EUNSUPPORTED;
+}
+
+bool attn_sizes_ok(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d, int dtype) {
+  if (n_tokens < 1 || n_vis < 0 || n_vis > n_tokens) return false;
+  if (n_cubes < 0 || n_cubes > kMaxCubes) return false;
+  if (n_vis > 0 && n_cubes < 1) return false;
+  if (n_vis == 0 && n_cubes != 0) return false;
+  if ((long long)n_cubes > n_vis) return false;
+  if (hq < 1 || hkv < 1 || hq % hkv != 0 || hkv * d > 1024) return false;
+  if (dtype == ADASPARK_BF16) return d == 128;
+  if (dtype == ADASPARK_FP32) return d == 64 || d == 128;
+  return false;
+}
+
+bool ffn_sizes_ok(int n_tokens, int n_vis, int n_cubes, int D, int F, int dtype) {
+  if (n_tokens < 1 || n_vis < 0 || n_vis > n_tokens) return false;
+  if (n_cubes < 0 || n_cubes > kMaxCubes) return false;
+  if (n_vis > 0 && n_cubes < 1) return false;
+  if (n_vis == 0 && n_cubes != 0) return false;
+  if ((long long)n_cubes > n_vis) return false;
+  if (D < 1 || F < 1) return false;
+  if (dtype == ADASPARK_BF16) return D % 64 == 0 && F % 64 == 0;
+  if (dtype == ADASPARK_FP32) return D % 4 == 0 && F % 4 == 0;
+  return false;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? ADASPARK_OK : ADASPARK_ECUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d,
+                                    int dtype) {
+  if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return 0;
+  const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
+  return make_attn_layout(G).total;
+}
+
+int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
+                       const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                       int n_vis, int n_tokens, int hq, int hkv, int d, float p, void* out,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !cube_ids || !cube_offsets || !out || !workspace) return ADASPARK_EINVAL;
+  if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype) || !p_valid(p))
+    return ADASPARK_EINVAL;
+  const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
+  const AttnLayout L = make_attn_layout(G);
+  if (workspace_bytes < L.total || !aligned(workspace, kAlign)) return ADASPARK_EINVAL;
+  const size_t es = dtype == ADASPARK_BF16 ? 2 : 4;
+  if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) || es == 0)
+    return ADASPARK_EINVAL;
+  int rc = check_device();
+  if (rc != ADASPARK_OK) return rc;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
+  const int dense = p >= 1.0f;
+  if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
+  if (dense && cudaMemsetAsync(&hdr->pad[0], kModeDense, 1, s) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  rc = cuda_rc(launch_validate(cube_ids, cube_offsets, nullptr, n_cubes, n_vis, n_tokens, hdr, s));
+  if (rc) return rc;
+
+  SelectArgs sa;
+  sa.Q = Q;
+  sa.cube_ids = cube_ids;
+  sa.cube_offsets = cube_offsets;
+  sa.kbar = reinterpret_cast<float*>(ws + L.kbar);
+  sa.kbar_split = reinterpret_cast<__nv_bfloat16*>(ws + L.kbar_split);
+  sa.tile_mask = reinterpret_cast<uint32_t*>(ws + L.tile_mask);
+  sa.tile_list = reinterpret_cast<uint16_t*>(ws + L.tile_list);
+  sa.tile_count = reinterpret_cast<int32_t*>(ws + L.tile_count);
+  sa.pool_z = reinterpret_cast<float*>(ws + L.pool);
+  sa.pool_j = reinterpret_cast<int32_t*>(ws + L.pool + (size_t)G.pool_rows * G.n_cubes * 4);
+  sa.hdr = hdr;
+  sa.G = G;
+  sa.p = p;
+  sa.zscale = (float)(1.4426950408889634 / std::sqrt((double)d));
+
+  if (!dense && n_vis > 0 && G.n_vtiles > 0) {
+    rc = cuda_rc(launch_cube_mean(K, dtype, cube_offsets, const_cast<float*>(sa.kbar),
+                                  const_cast<__nv_bfloat16*>(sa.kbar_split), G, hdr, s));
+    if (rc) return rc;
+    rc = cuda_rc(launch_select_simt(sa, dtype, s));
+    if (rc) return rc;
+  }
+
+  AttnArgs aa;
+  aa.Q = Q;
+  aa.K = K;
+  aa.V = V;
+  aa.out = out;
+  aa.cube_ids = cube_ids;
+  aa.cube_offsets = cube_offsets;
+  aa.tile_count = sa.tile_count;
+  aa.tile_list = sa.tile_list;
+  aa.tile_mask = sa.tile_mask;
+  aa.hdr = hdr;
+  aa.G = G;
+  aa.dense = dense;
+  aa.scale_log2 = sa.zscale;
+  return cuda_rc(launch_attn_simt(aa, dtype, s));
+}
+
+int adaspark_attn_export_sets(const void* workspace, const int32_t* cube_ids, int n_cubes,
+                              int n_vis, int n_tokens, int hq, int hkv, int d, int dtype,
+                              uint32_t* sel_bits, void* stream) {
+  if (!workspace || !sel_bits || !cube_ids) return ADASPARK_EINVAL;
+  if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return ADASPARK_EINVAL;
+  const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
+  const AttnLayout L = make_attn_layout(G);
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t mode = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ADASPARK_ECUDA;
+  const WsHeader* hdr = reinterpret_cast<const WsHeader*>(ws + L.header);
+  if (cudaMemcpy(&mode, &hdr->pad[0], 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  return cuda_rc(launch_export_sets(reinterpret_cast<const int32_t*>(ws + L.tile_count),
+                                    reinterpret_cast<const uint16_t*>(ws + L.tile_list),
+                                    reinterpret_cast<const uint32_t*>(ws + L.tile_mask),
+                                    cube_ids, G, (mode & 0xff) == kModeDense, sel_bits, s));
+}
+
+int adaspark_attn_read_stats(const void* workspace, adaspark_attn_stats* stats, void* stream) {
+  if (!workspace || !stats) return ADASPARK_EINVAL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  const WsHeader* hdr = static_cast<const WsHeader*>(workspace);
+  static_assert(sizeof(adaspark_attn_stats) == sizeof(hdr->stats), "stats size");
+  return cuda_rc(cudaMemcpy(stats, hdr->stats, sizeof(adaspark_attn_stats), cudaMemcpyDeviceToHost));
+}
+
+size_t adaspark_token_ffn_workspace(int n_tokens, int n_vis, int n_cubes, int D, int F,
+                                    int dtype) {
+  if (!ffn_sizes_ok(n_tokens, n_vis, n_cubes, D, F, dtype)) return 0;
+  return make_ffn_layout(n_tokens, n_vis, n_cubes, D, F, dtype == ADASPARK_BF16 ? 2 : 4).total;
+}
+
+int adaspark_token_ffn(const void* x, const void* W_gate, const void* W_up, const void* W_down,
+                       int dtype, const int32_t* cube_ids, const int32_t* cube_offsets,
+                       const uint8_t* text_mask, int n_cubes, int n_vis, int n_tokens, int D,
+                       int F, float p, float* y, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!x || !W_gate || !W_up || !W_down || !cube_ids || !cube_offsets || !text_mask || !y ||
+      !workspace)
+    return ADASPARK_EINVAL;
+  if (!ffn_sizes_ok(n_tokens, n_vis, n_cubes, D, F, dtype) || !p_valid(p)) return ADASPARK_EINVAL;
+  const int es = dtype == ADASPARK_BF16 ? 2 : 4;
+  const FfnLayout L = make_ffn_layout(n_tokens, n_vis, n_cubes, D, F, es);
+  if (workspace_bytes < L.total || !aligned(workspace, kAlign)) return ADASPARK_EINVAL;
+  if (!aligned(x, 16) || !aligned(W_gate, 16) || !aligned(W_up, 16) || !aligned(W_down, 16) ||
+      !aligned(y, 16))
+    return ADASPARK_EINVAL;
+  int rc = check_device();
+  if (rc != ADASPARK_OK) return rc;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  FfnArgs a;
+  a.x = x;
+  a.W_gate = W_gate;
+  a.W_up = W_up;
+  a.W_down = W_down;
+  a.cube_ids = cube_ids;
+  a.cube_offsets = cube_offsets;
+  a.y = y;
+  a.norms = reinterpret_cast<float*>(ws + L.norms);
+  a.active = ws + L.active;
+  a.cube_count = reinterpret_cast<int32_t*>(ws + L.cube_count);
+  a.cube_start = reinterpret_cast<int32_t*>(ws + L.cube_start);
+  a.idx = reinterpret_cast<int32_t*>(ws + L.idx);
+  a.row_cube = reinterpret_cast<int32_t*>(ws + L.row_cube);
+  a.xa = ws + L.xa;
+  a.h = ws + L.h;
+  a.sums = reinterpret_cast<float*>(ws + L.sums);
+  a.hdr = reinterpret_cast<WsHeader*>(ws + L.header);
+  a.n_tokens = n_tokens;
+  a.n_vis = n_vis;
+  a.n_cubes = n_cubes;
+  a.D = D;
+  a.F = F;
+  a.p = p;
+  a.dense = p >= 1.0f;
+
+  if (cudaMemsetAsync(a.hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
+  if (!a.dense && n_cubes > 0 &&
+      cudaMemsetAsync(a.sums, 0, (size_t)n_cubes * D * sizeof(float), s) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  if ((rc = cuda_rc(launch_validate(cube_ids, cube_offsets, text_mask, n_cubes, n_vis, n_tokens,
+                                    a.hdr, s))))
+    return rc;
+  if ((rc = cuda_rc(launch_ffn_select(a, dtype, s)))) return rc;
+  if ((rc = cuda_rc(launch_ffn_compact(a, dtype, s)))) return rc;
+  if ((rc = cuda_rc(launch_ffn_gemm1_simt(a, dtype, s)))) return rc;
+  if ((rc = cuda_rc(launch_ffn_gemm2_simt(a, dtype, s)))) return rc;
+  return cuda_rc(launch_ffn_compensate(a, dtype, s));
+}
+
+int adaspark_ffn_export_active(const void* workspace, int n_tokens, int n_vis, int n_cubes, int D,
+                               int F, int dtype, uint8_t* active, void* stream) {
+  if (!workspace || !active) return ADASPARK_EINVAL;
+  if (!ffn_sizes_ok(n_tokens, n_vis, n_cubes, D, F, dtype)) return ADASPARK_EINVAL;
+  const FfnLayout L =
+      make_ffn_layout(n_tokens, n_vis, n_cubes, D, F, dtype == ADASPARK_BF16 ? 2 : 4);
+  return cuda_rc(cudaMemcpyAsync(active, static_cast<const uint8_t*>(workspace) + L.active,
+                                 (size_t)n_tokens, cudaMemcpyDeviceToDevice,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+int adaspark_ffn_read_stats(const void* workspace, adaspark_ffn_stats* stats, void* stream) {
+  if (!workspace || !stats) return ADASPARK_EINVAL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  const WsHeader* hdr = static_cast<const WsHeader*>(workspace);
+  static_assert(sizeof(adaspark_ffn_stats) == sizeof(hdr->stats), "stats size");
+  return cuda_rc(cudaMemcpy(stats, hdr->stats, sizeof(adaspark_ffn_stats), cudaMemcpyDeviceToHost));
+}
+
+int adaspark_read_device_status(const void* workspace, uint32_t* detail, void* stream) {
+  if (!workspace) return ADASPARK_EINVAL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  uint32_t st[2] = {0, 0};
+  if (cudaMemcpy(st, workspace, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  if (detail) *detail = st[0];
+  return st[0] ? ADASPARK_EDEVICE : ADASPARK_OK;
+}
+
+}  // extern "C"

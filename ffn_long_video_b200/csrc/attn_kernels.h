@@ -1,0 +1,56 @@
+// Kernel argument blocks and host launchers of AdaS-Attn.
+#pragma once
+
+#include "common.cuh"
+#include "host_util.h"
+#include "layout.cuh"
+
+namespace adaspark {
+
+struct SelectArgs {
+  const void* Q;
+  const int32_t* cube_ids;
+  const int32_t* cube_offsets;
+  const float* kbar;                  // [hkv][C][d]
+  const __nv_bfloat16* kbar_split;    // [3][hkv][C][d]
+  uint32_t* tile_mask;                // [n_vtiles][C][4]
+  uint16_t* tile_list;                // [n_vtiles][C]
+  int32_t* tile_count;                // [n_vtiles]
+  float* pool_z;
+  int32_t* pool_j;
+  WsHeader* hdr;
+  AttnGeom G;
+  float p;
+  float zscale;                       // log2(e) / sqrt(d)
+};
+
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  void* out;
+  const int32_t* cube_ids;
+  const int32_t* cube_offsets;
+  const int32_t* tile_count;
+  const uint16_t* tile_list;
+  const uint32_t* tile_mask;
+  WsHeader* hdr;
+  AttnGeom G;
+  int dense;                          // p == 1: every preceding cube, no lists
+  float scale_log2;                   // log2(e) / sqrt(d)
+};
+
+cudaError_t launch_validate(const int32_t* cube_ids, const int32_t* off, const uint8_t* text_mask,
+                            int n_cubes, int n_vis, int n_tokens, WsHeader* hdr, cudaStream_t s);
+cudaError_t launch_cube_mean(const void* K, int dtype, const int32_t* off, float* kbar,
+                             __nv_bfloat16* split, const AttnGeom& G, WsHeader* hdr,
+                             cudaStream_t s);
+cudaError_t launch_select_simt(const SelectArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_select_tc(const SelectArgs& a, cudaStream_t s);
+cudaError_t launch_export_sets(const int32_t* tile_count, const uint16_t* tile_list,
+                               const uint32_t* tile_mask, const int32_t* cube_ids,
+                               const AttnGeom& G, int dense, uint32_t* bits, cudaStream_t s);
+cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
+
+}  // namespace adaspark

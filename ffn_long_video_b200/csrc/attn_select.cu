@@ -1,0 +1,289 @@
+// AdaS-Attn, selection side (key design 2 of the AdaSpark note):
+//  - layout validation of cube_ids / cube_offsets,
+//  - cube mean keys kbar_j (fp32, plus a three-part bf16 split for the tensor-core
+//    scorer),
+//  - the SIMT scorer + Top-p selection (fp32 path), emitting per-tile cube lists
+//    and 128-bit row masks,
+//  - export of the selected sets as a dense bitmap.
+#include "attn_kernels.h"
+#include "select.cuh"
+
+namespace adaspark {
+
+// ---------------------------------------------------------------------------
+// Layout validation (visual prefix in cubes, text suffix = -1).
+// ---------------------------------------------------------------------------
+__global__ void validate_layout_kernel(const int32_t* __restrict__ cube_ids,
+                                       const int32_t* __restrict__ off,
+                                       const uint8_t* __restrict__ text_mask, int n_cubes,
+                                       int n_vis, int n_tokens, WsHeader* hdr) {
+  const int stride = gridDim.x * blockDim.x;
+  for (int c = blockIdx.x * blockDim.x + threadIdx.x; c <= n_cubes; c += stride) {
+    const int a = off[c];
+    if (c == 0 && a != 0) set_status(hdr, ADASPARK_DEV_BAD_LAYOUT, 0x101u);
+    if (c == n_cubes && a != n_vis) set_status(hdr, ADASPARK_DEV_BAD_LAYOUT, 0x102u);
+    if (c < n_cubes) {
+      const int n = off[c + 1] - a;
+      if (n < 1 || n > kMaxCubeTokens) set_status(hdr, ADASPARK_DEV_BAD_LAYOUT, 0x103u);
+    }
+  }
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n_tokens; t += stride) {
+    const int c = cube_ids[t];
+    if (t < n_vis) {
+      if (c < 0 || c >= n_cubes || t < off[c] || t >= off[c + 1])
+        set_status(hdr, ADASPARK_DEV_BAD_LAYOUT, 0x104u);
+    } else if (c != -1) {
+      set_status(hdr, ADASPARK_DEV_BAD_LAYOUT, 0x105u);
+    }
+    if (text_mask && (text_mask[t] != 0) != (c == -1))
+      set_status(hdr, ADASPARK_DEV_BAD_LAYOUT, 0x106u);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// kbar[kv][j][:] = mean of K over cube j (fp64 accumulation, fp32 result) and
+// its split kbar = hi + mid + lo into bf16 parts (products with bf16 queries are
+// exact, so three tensor-core passes reproduce the fp32 dot product).
+// One block per cube, one thread per (kv, dim) element.
+// ---------------------------------------------------------------------------
+template <typename T>
+__global__ void cube_mean_kernel(const T* __restrict__ K, const int32_t* __restrict__ off,
+                                 float* __restrict__ kbar, __nv_bfloat16* __restrict__ split,
+                                 int n_cubes, int hkv, int d, WsHeader* hdr) {
+  if (status_bad(hdr)) return;
+  const int j = blockIdx.x;
+  const int e = threadIdx.x;  // kv * d + dim
+  const int row = hkv * d;
+  if (e >= row) return;
+  const int a = off[j], b = off[j + 1];
+  double acc = 0.0;
+  for (int t = a; t < b; ++t) acc += (double)to_f32(K[(size_t)t * row + e]);
+  const float mean = (float)(acc / (double)(b - a));
+  const int kv = e / d, dim = e - kv * d;
+  const size_t o = ((size_t)kv * n_cubes + j) * d + dim;
+  kbar[o] = mean;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
+  const float r1 = mean - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(mid);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+  const size_t plane = (size_t)hkv * n_cubes * d;
+  split[o] = hi;
+  split[plane + o] = mid;
+  split[2 * plane + o] = lo;
+}
+
+// ---------------------------------------------------------------------------
+// Shared tile epilogue: compact the cube columns with any row bit into the
+// tile's ascending list. 128 threads.
+// ---------------------------------------------------------------------------
+__device__ void compact_tile_list(const uint32_t* tmask, uint16_t* list, int32_t* count, int c_hi,
+                                  int* s_wcnt) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  int total = 0;
+  for (int base = 0; base <= c_hi; base += 128) {
+    const int j = base + tid;
+    bool nz = false;
+    if (j <= c_hi) {
+      const uint4 w = __ldcg(reinterpret_cast<const uint4*>(tmask + (size_t)j * 4));
+      nz = (w.x | w.y | w.z | w.w) != 0u;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, nz);
+    if (lane == 0) s_wcnt[warp] = __popc(bal);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int before = total;
+    for (int w = 0; w < warp; ++w) before += s_wcnt[w];
+    const int chunk_total = s_wcnt[0] + s_wcnt[1] + s_wcnt[2] + s_wcnt[3];
+    if (nz) list[before + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)j;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    total += chunk_total;
+  }
+  if (tid == 0) *count = total;
+}
+
+// ---------------------------------------------------------------------------
+// SIMT scorer + selection: one block per visual tile, one thread per row.
+// ---------------------------------------------------------------------------
+template <typename T, int D>
+__global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  sel::Smem* ss = reinterpret_cast<sel::Smem*>(smem_raw);
+  float* kch = reinterpret_cast<float*>(smem_raw + sizeof(sel::Smem));  // [64][D]
+  __shared__ int s_lo, s_hi, s_wcnt[4];
+  if (status_bad(a.hdr)) return;
+  const AttnGeom& G = a.G;
+  const int vt = blockIdx.x;
+  const int kv = vt / G.vtiles_per_kv;
+  const int tl = vt - kv * G.vtiles_per_kv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long r = (long long)tl * kTileRows + tid;
+  const bool valid = r < (long long)G.n_vis * G.g;
+  const int t = valid ? (int)(r / G.g) : 0;
+  const int h = kv * G.g + (valid ? (int)(r % G.g) : 0);
+  const int own = valid ? a.cube_ids[t] : -1;
+
+  if (tid == 0) {
+    s_lo = INT_MAX;
+    s_hi = -1;
+  }
+  __syncthreads();
+  if (valid) {
+    atomicMin(&s_lo, own);
+    atomicMax(&s_hi, own);
+  }
+  __syncthreads();
+  const int c_hi = s_hi;
+  if (c_hi < 0) return;
+
+  float q[D];
+  const T* qp = reinterpret_cast<const T*>(a.Q) + ((size_t)t * G.hq + h) * D;
+#pragma unroll
+  for (int e = 0; e < D; ++e) q[e] = valid ? to_f32(qp[e]) : 0.f;
+
+  sel::RowSel s;
+  s.init(ss, tid);
+  const int ncand = own > 0 ? own : 0;
+  const sel::Pool pool{a.pool_z, a.pool_j, G.pool_rows, G.n_cubes};
+  const float* kb = a.kbar + (size_t)kv * G.n_cubes * D;
+
+  for (int pass = 0; pass < 2; ++pass) {
+    uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
+    int nsel = 0;
+    for (int j0 = 0; j0 < c_hi; j0 += 64) {
+      const int nj = min(64, c_hi - j0);
+      __syncthreads();
+      for (int e = tid; e < nj * D; e += 128) kch[e] = kb[(size_t)j0 * D + e];
+      __syncthreads();
+      for (int jj = 0; jj < nj; ++jj) {
+        const int j = j0 + jj;
+        bool selb = false;
+        if (j < ncand) {
+          const float* kr = kch + jj * D;
+          float acc = 0.f;
+#pragma unroll
+          for (int e = 0; e < D; ++e) acc = fmaf(q[e], kr[e], acc);
+          const float z = acc * a.zscale;
+          if (pass == 0)
+            s.pass1(z);
+          else
+            selb = s.pass2(z, j, a.hdr, pool);
+        }
+        if (pass == 1) {
+          const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
+          if (lane == 0) tmask[(size_t)j * 4 + warp] = w;
+          nsel += selb;
+        }
+      }
+    }
+    if (pass == 0) {
+      s.finish1(a.p);
+    } else {
+      const unsigned w = __ballot_sync(0xffffffffu, own == c_hi);
+      if (lane == 0) tmask[(size_t)c_hi * 4 + warp] = w;
+      __syncwarp();
+      const int m = s.resolve();
+      for (int i = 0; i < m; ++i) atomicOr(&tmask[(size_t)s.ljv(i) * 4 + warp], 1u << lane);
+      nsel += m;
+      // statistics
+      const float rows_f = (valid && own > 0) ? 1.f : 0.f;
+      unsigned long long v_rows = __reduce_add_sync(0xffffffffu, (unsigned)rows_f);
+      unsigned long long v_cand = __reduce_add_sync(0xffffffffu, (unsigned)ncand);
+      unsigned long long v_sel = __reduce_add_sync(0xffffffffu, (unsigned)nsel);
+      unsigned long long v_ovf = __reduce_add_sync(0xffffffffu, s.gz ? 1u : 0u);
+      if (lane == 0) {
+        atomicAdd((unsigned long long*)&a.hdr->stats[0], v_rows);
+        atomicAdd((unsigned long long*)&a.hdr->stats[1], v_cand);
+        atomicAdd((unsigned long long*)&a.hdr->stats[2], v_sel);
+        atomicAdd((unsigned long long*)&a.hdr->stats[3], v_ovf);
+      }
+      __syncthreads();
+      compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes, a.tile_count + vt, c_hi,
+                        s_wcnt);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Export: tile lists + masks -> dense bitmap [n_vis][hq][W] (own cube not marked).
+// ---------------------------------------------------------------------------
+__global__ void export_sets_kernel(const int32_t* __restrict__ tile_count,
+                                   const uint16_t* __restrict__ tile_list,
+                                   const uint32_t* __restrict__ tile_mask,
+                                   const int32_t* __restrict__ cube_ids, AttnGeom G, int dense,
+                                   uint32_t* __restrict__ bits) {
+  const int vt = blockIdx.x;
+  const int kv = vt / G.vtiles_per_kv;
+  const int tl = vt - kv * G.vtiles_per_kv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long r = (long long)tl * kTileRows + tid;
+  if (r >= (long long)G.n_vis * G.g) return;
+  const int t = (int)(r / G.g), h = kv * G.g + (int)(r % G.g);
+  const int own = cube_ids[t];
+  const int W = (G.n_cubes + 31) / 32;
+  uint32_t* row = bits + ((size_t)t * G.hq + h) * W;
+  for (int w = 0; w < W; ++w) row[w] = 0u;
+  if (dense) {
+    for (int j = 0; j < own; ++j) row[j >> 5] |= 1u << (j & 31);
+    return;
+  }
+  const int n = tile_count[vt];
+  const uint16_t* list = tile_list + (size_t)vt * G.n_cubes;
+  const uint32_t* tm = tile_mask + (size_t)vt * G.n_cubes * 4;
+  for (int k = 0; k < n; ++k) {
+    const int j = list[k];
+    if (j >= own) break;
+    if ((tm[(size_t)j * 4 + warp] >> lane) & 1u) row[j >> 5] |= 1u << (j & 31);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers.
+// ---------------------------------------------------------------------------
+cudaError_t launch_validate(const int32_t* cube_ids, const int32_t* off, const uint8_t* text_mask,
+                            int n_cubes, int n_vis, int n_tokens, WsHeader* hdr,
+                            cudaStream_t s) {
+  int n = n_tokens > n_cubes + 1 ? n_tokens : n_cubes + 1;
+  int blocks = (n + 255) / 256;
+  if (blocks > 1184) blocks = 1184;
+  return launch("validate_layout", validate_layout_kernel, dim3(blocks), dim3(256), 0, s, cube_ids,
+                off, text_mask, n_cubes, n_vis, n_tokens, hdr);
+}
+
+cudaError_t launch_cube_mean(const void* K, int dtype, const int32_t* off, float* kbar,
+                             __nv_bfloat16* split, const AttnGeom& G, WsHeader* hdr,
+                             cudaStream_t s) {
+  const int threads = G.hkv * G.d;
+  if (dtype == ADASPARK_BF16)
+    return launch("cube_mean_keys", cube_mean_kernel<__nv_bfloat16>, dim3(G.n_cubes),
+                  dim3(threads), 0, s, (const __nv_bfloat16*)K, off, kbar, split, G.n_cubes,
+                  G.hkv, G.d, hdr);
+  return launch("cube_mean_keys", cube_mean_kernel<float>, dim3(G.n_cubes), dim3(threads), 0, s,
+                (const float*)K, off, kbar, split, G.n_cubes, G.hkv, G.d, hdr);
+}
+
+template <typename T, int D>
+static cudaError_t launch_select_simt_t(const SelectArgs& a, cudaStream_t s) {
+  const size_t smem = sizeof(sel::Smem) + 64 * D * sizeof(float);
+  auto k = select_simt_kernel<T, D>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch("select_simt", k, dim3(a.G.n_vtiles), dim3(128), smem, s, a);
+}
+
+cudaError_t launch_select_simt(const SelectArgs& a, int dtype, cudaStream_t s) {
+  if (dtype == ADASPARK_FP32) {
+    if (a.G.d == 64) return launch_select_simt_t<float, 64>(a, s);
+    return launch_select_simt_t<float, 128>(a, s);
+  }
+  return launch_select_simt_t<__nv_bfloat16, 128>(a, s);
+}
+
+cudaError_t launch_export_sets(const int32_t* tile_count, const uint16_t* tile_list,
+                               const uint32_t* tile_mask, const int32_t* cube_ids,
+                               const AttnGeom& G, int dense, uint32_t* bits, cudaStream_t s) {
+  if (G.n_vtiles == 0) return cudaSuccess;
+  return launch("export_sets", export_sets_kernel, dim3(G.n_vtiles), dim3(128), 0, s, tile_count,
+                tile_list, tile_mask, cube_ids, G, dense, bits);
+}
+
+}  // namespace adaspark

@@ -1,0 +1,41 @@
+// Kernel argument blocks and host launchers of AdaS-FFN.
+#pragma once
+
+#include "common.cuh"
+#include "host_util.h"
+#include "layout.cuh"
+
+namespace adaspark {
+
+struct FfnArgs {
+  const void* x;        // [N][D]
+  const void* W_gate;   // [F][D]
+  const void* W_up;     // [F][D]
+  const void* W_down;   // [D][F]
+  const int32_t* cube_ids;
+  const int32_t* cube_offsets;
+  float* y;             // [N][D] fp32
+  float* norms;         // [n_vis]
+  uint8_t* active;      // [N]
+  int32_t* cube_count;  // [C]
+  int32_t* cube_start;  // [C+1]
+  int32_t* idx;         // [N]
+  int32_t* row_cube;    // [N]
+  void* xa;             // [N][D]
+  void* h;              // [N][F]
+  float* sums;          // [C][D]
+  WsHeader* hdr;
+  int n_tokens, n_vis, n_cubes, D, F;
+  float p;
+  int dense;
+};
+
+cudaError_t launch_ffn_select(const FfnArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_ffn_compact(const FfnArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_ffn_gemm1_simt(const FfnArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_ffn_gemm2_simt(const FfnArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_ffn_gemm1_tc(const FfnArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_gemm2_tc(const FfnArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_compensate(const FfnArgs& a, int dtype, cudaStream_t s);
+
+}  // namespace adaspark

@@ -1,0 +1,232 @@
+/*
+ * adaspark.h -- C ABI of the AdaSpark layer hot path for NVIDIA B200 (sm_100a).
+ *
+ * The method (from "AdaSpark: Adaptive Sparsity for Efficient Long-Video
+ * Understanding", papernotes.org note, sections 整体框架 and 关键设计 1-4, and the
+ * paper's abstract / Figure 2 caption):
+ *   - video tokens are split into 3D h x w x t cubes (key design 1);
+ *   - AdaS-Attn: each query token scores the preceding cubes against their mean
+ *     keys, P_i = softmax(q . kbar_j / sqrt(d_k)), keeps the Top-p set S_i and
+ *     attends only to those cubes plus its own cube (key design 2);
+ *   - AdaS-FFN: inside each cube the Top-p tokens by L2 norm go through the FFN;
+ *     each skipped token is updated as y_k = x_k + mean_j FFN(x_j) over the
+ *     cube's active tokens; text tokens always take the dense FFN (key design 3);
+ *   - one threshold p drives both selections (key design 4).
+ *
+ * Conventions shared by every call:
+ *   - Ownership: the caller allocates and frees every buffer, host and device.
+ *     The library never allocates device memory; workspace sizes come from the
+ *     *_workspace queries.
+ *   - Execution: calls taking a `stream` (a cudaStream_t, NULL = legacy default
+ *     stream) are asynchronous on it. Their return code covers host-side
+ *     validation and launch errors only. Problems found on the device (a token
+ *     layout that breaks the preconditions, a bounded wait that expired, an
+ *     exhausted overflow pool) set a status word in the workspace; the kernels
+ *     then return early and adaspark_read_device_status() reports
+ *     ADASPARK_EDEVICE.
+ *   - Token layout: tokens are in cube-major order. The visual prefix holds
+ *     cubes 0..C-1 contiguously (cube_ids nondecreasing 0..C-1, cube_offsets
+ *     [C+1] with cube_offsets[0] = 0 and cube_offsets[C] = n_vis); the text
+ *     suffix n_vis..n_tokens-1 has cube_id -1. Causality follows this order.
+ *   - Calls are reentrant when they use distinct workspaces. No C++ exception
+ *     crosses this interface.
+ *   - Requires an sm_100 device; otherwise ADASPARK_EUNSUPPORTED.
+ */
+#ifndef ADASPARK_H
+#define ADASPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+typedef enum {
+  ADASPARK_OK = 0,
+  ADASPARK_EINVAL = -1,        /* bad argument (host-side validation)          */
+  ADASPARK_ECUDA = -2,         /* a CUDA runtime/driver call failed            */
+  ADASPARK_EUNSUPPORTED = -3,  /* device is not sm_100, or a shape not handled */
+  ADASPARK_EDEVICE = -4        /* a kernel flagged a problem (see status word) */
+} adaspark_status;
+
+/* Element types of the activations and weights. */
+typedef enum { ADASPARK_BF16 = 0, ADASPARK_FP32 = 1 } adaspark_dtype;
+
+/* Bits of the device status word (adaspark_read_device_status detail). */
+#define ADASPARK_DEV_BAD_LAYOUT   0x1u  /* cube_ids / cube_offsets / text_mask inconsistent */
+#define ADASPARK_DEV_TIMEOUT      0x2u  /* a bounded wait inside a kernel expired          */
+#define ADASPARK_DEV_POOL_FULL    0x4u  /* selection overflow pool exhausted               */
+
+/* Human-readable name of a return code. Never NULL. */
+const char *adaspark_status_string(int status);
+
+/* ------------------------------------------------------------------------ */
+/* Key design 1: 3D spatio-temporal cube partition (host only).             */
+/* ------------------------------------------------------------------------ */
+
+/* Number of cubes of a T x H x W grid split into cube_h x cube_w x cube_t
+ * windows (edge cubes truncated): ceil(T/cube_t)*ceil(H/cube_h)*ceil(W/cube_w).
+ * Returns ADASPARK_EINVAL for a non-positive size or a NULL n_cubes. */
+int adaspark_cube_count(int T, int H, int W, int cube_h, int cube_w, int cube_t,
+                        int32_t *n_cubes);
+
+/* Cube-major order of a video-token grid (key design 1).
+ *   perm         [T*H*W]          out: perm[k] = raster index t*H*W + h*W + w of
+ *                                      the k-th token in cube-major order
+ *   cube_ids     [T*H*W + n_text] out: cube of each cube-major position; -1 for the
+ *                                      n_text text tokens, which follow the video
+ *   cube_offsets [n_cubes + 1]    out: first position of each cube, then T*H*W
+ *   n_cubes                       out: number of cubes (size cube_offsets with
+ *                                      adaspark_cube_count)
+ * Cubes are enumerated time-major over the cube grid (t_b, h_b, w_b); tokens
+ * inside a cube in (t, h, w) order; edge cubes are truncated. All arrays are
+ * caller-allocated HOST memory. Runs on the host, once per video, outside the
+ * per-layer path. Returns ADASPARK_EINVAL on a non-positive size, negative
+ * n_text or NULL pointer. */
+int adaspark_cube_partition(int T, int H, int W, int cube_h, int cube_w, int cube_t,
+                            int n_text, int32_t *perm, int32_t *cube_ids,
+                            int32_t *cube_offsets, int32_t *n_cubes);
+
+/* ------------------------------------------------------------------------ */
+/* Key design 2: AdaS-Attn.                                                 */
+/* ------------------------------------------------------------------------ */
+
+/* Counters written by adaspark_cube_attn (read with adaspark_attn_read_stats). */
+typedef struct {
+  uint64_t visual_rows;      /* (visual token, query head) rows that ran selection */
+  uint64_t candidate_pairs;  /* sum over those rows of the preceding-cube count    */
+  uint64_t selected_pairs;   /* sum over those rows of |S_i|                        */
+  uint64_t overflow_rows;    /* rows whose cut was resolved in the overflow pool    */
+  uint64_t tiles;            /* 128-row attention tiles executed (visual + text)    */
+  uint64_t key_blocks;       /* executed (tile, key block) pairs                    */
+  uint64_t key_block_keys;   /* keys covered by those blocks (for executed FLOPs)   */
+  uint64_t reserved[9];
+} adaspark_attn_stats;
+
+/* Device workspace bytes needed by adaspark_cube_attn for these sizes
+ * (0 when the sizes are invalid). */
+size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv,
+                                    int d, int dtype);
+
+/* AdaS-Attn for one layer (key design 2 of the papernotes note; the abstract's
+ * "relevance scores computed over preceding Cubes").
+ *
+ * For a visual token t of cube i and query head h (KV head floor(h/(hq/hkv))):
+ *   kbar_j = mean of K over cube j;  P = softmax_j<i(q . kbar_j / sqrt(d));
+ *   S = Top-p(P, p): order by probability descending then cube index ascending,
+ *       keep the smallest prefix whose cumulative mass reaches p (>= 1 cube;
+ *       p = 1 keeps every preceding cube; the first cube has none);
+ *   out[t,h] = softmax attention over the keys of the cubes in S and the keys of
+ *       cube i at positions <= t, one softmax, scale 1/sqrt(d).
+ * A text token attends densely and causally to every earlier token.
+ *
+ *   Q [n_tokens, hq, d], K/V [n_tokens, hkv, d]: device, row-major, element type
+ *       `dtype` (BF16 for d = 128, FP32 for d = 64 or 128);
+ *   cube_ids [n_tokens], cube_offsets [n_cubes + 1]: device int32 (layout above);
+ *   n_vis = cube_offsets[n_cubes] (checked on the device);
+ *   p in (0, 1]; hq % hkv == 0; every cube holds 1..256 tokens;
+ *   out [n_tokens, hq, d]: device, element type `dtype`;
+ *   workspace: device, >= adaspark_cube_attn_workspace(...) bytes, 256-byte aligned.
+ * Errors: ADASPARK_EINVAL for NULL pointers, bad sizes, p outside (0, 1] or NaN,
+ * hq % hkv != 0, unsupported d, a short or misaligned workspace; ADASPARK_ECUDA
+ * for a failed launch. */
+int adaspark_cube_attn(const void *Q, const void *K, const void *V, int dtype,
+                       const int32_t *cube_ids, const int32_t *cube_offsets, int n_cubes,
+                       int n_vis, int n_tokens, int hq, int hkv, int d, float p,
+                       void *out, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Expand the selection sets of the last adaspark_cube_attn call on `workspace`
+ * into a dense bitmap: sel_bits [n_vis, hq, ceil(n_cubes/32)] uint32 in DEVICE
+ * memory, bit j of row (t, h) set when cube j is in S for that row (the own cube
+ * is not marked). Same sizes and cube_ids (device) as the call. Synchronizes
+ * `stream` once to read the call's mode, then runs asynchronously. For parity
+ * checks and analysis. */
+int adaspark_attn_export_sets(const void *workspace, const int32_t *cube_ids, int n_cubes,
+                              int n_vis, int n_tokens, int hq, int hkv, int d, int dtype,
+                              uint32_t *sel_bits, void *stream);
+
+/* Copy the counters of the last adaspark_cube_attn call to host memory.
+ * Synchronizes `stream`. */
+int adaspark_attn_read_stats(const void *workspace, adaspark_attn_stats *stats, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Key design 3: AdaS-FFN with mean compensation.                           */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+  uint64_t active_visual;   /* visual tokens that went through the FFN      */
+  uint64_t skipped_visual;  /* visual tokens updated by mean compensation   */
+  uint64_t text_tokens;     /* text tokens (always dense)                   */
+  uint64_t reserved[13];
+} adaspark_ffn_stats;
+
+/* Device workspace bytes needed by adaspark_token_ffn (0 when invalid). */
+size_t adaspark_token_ffn_workspace(int n_tokens, int n_vis, int n_cubes, int D, int F,
+                                    int dtype);
+
+/* AdaS-FFN for one layer (key design 3 of the papernotes note; Figure 2 caption).
+ *
+ * Inside each cube c, importance w_u = ||x_u||_2 / sum_{v in c} ||x_v||_2; the
+ * active set M_c = Top-p(w, p) (same rule as AdaS-Attn; a cube whose norms sum
+ * to 0 keeps every token). With FFN(x) = W_down (silu(W_gate x) * (W_up x)):
+ *   active visual or text token: y = x + FFN(x);
+ *   skipped visual token k of cube c: y_k = x_k + (1/|M_c|) sum_{j in M_c} FFN(x_j).
+ *
+ *   x [n_tokens, D]: device, type `dtype`; W_gate, W_up [F, D]; W_down [D, F]:
+ *       device, type `dtype`, row-major (nn.Linear [out, in] layout);
+ *   cube_ids [n_tokens], cube_offsets [n_cubes + 1]: device int32;
+ *   text_mask [n_tokens]: device uint8, must equal (cube_ids == -1);
+ *   p in (0, 1]; D % 64 == 0 and F % 128 == 0 for BF16 (D, F multiples of 4 for FP32);
+ *   y [n_tokens, D]: device float32 (the residual stream is kept in fp32);
+ *   workspace: device, >= adaspark_token_ffn_workspace(...) bytes, 256-byte aligned.
+ * Errors as for adaspark_cube_attn. */
+int adaspark_token_ffn(const void *x, const void *W_gate, const void *W_up, const void *W_down,
+                       int dtype, const int32_t *cube_ids, const int32_t *cube_offsets,
+                       const uint8_t *text_mask, int n_cubes, int n_vis, int n_tokens, int D,
+                       int F, float p, float *y, void *workspace, size_t workspace_bytes,
+                       void *stream);
+
+/* Copy the active flags of the last adaspark_token_ffn call on `workspace` into
+ * active [n_tokens] uint8 DEVICE memory (1 = through the FFN). Asynchronous. */
+int adaspark_ffn_export_active(const void *workspace, int n_tokens, int n_vis, int n_cubes,
+                               int D, int F, int dtype, uint8_t *active, void *stream);
+
+/* Copy the counters of the last adaspark_token_ffn call to host memory.
+ * Synchronizes `stream`. */
+int adaspark_ffn_read_stats(const void *workspace, adaspark_ffn_stats *stats, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* Status, timing and launch accounting.                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Synchronize `stream` and read the status word of a workspace of either call.
+ * Returns ADASPARK_OK, or ADASPARK_EDEVICE with *detail (if not NULL) set to the
+ * ADASPARK_DEV_* bits. The word is cleared by the next call on the workspace. */
+int adaspark_read_device_status(const void *workspace, uint32_t *detail, void *stream);
+
+/* Per-kernel timing with CUDA events recorded on the launching stream around
+ * each launch of this library. Off by default; process-wide; not thread-safe. */
+typedef struct {
+  char name[48];     /* kernel name                      */
+  uint64_t launches; /* timed launches since the last read */
+  double total_ms;   /* summed event-to-event time        */
+} adaspark_kernel_time;
+
+int adaspark_timer_enable(int on);
+/* Synchronize the recorded events, fill up to `max` entries and reset. */
+int adaspark_timer_read(adaspark_kernel_time *out, int max, int *n_out);
+
+/* Number of kernels this library has launched since it was loaded. */
+uint64_t adaspark_launch_count(void);
+
+/* ADASPARK_OK when `device` is an sm_100 GPU, else ADASPARK_EUNSUPPORTED
+ * (ADASPARK_ECUDA if the query fails). */
+int adaspark_device_check(int device);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ADASPARK_H */

@@ -1,0 +1,144 @@
+"""Helpers of the GPU parity tests: build a seeded layer on the device, run the
+library through its C ABI, run the oracle on the same values, compare.
+
+Comparison protocol:
+* selection sets (cube sets of AdaS-Attn, active tokens of AdaS-FFN) must equal
+  the oracle's bit for bit, except where the oracle's cut margin is below 1e-5;
+  those cases are counted and reported, not required to match;
+* outputs are compared with the oracle run on the library's own sets
+  (``attention_given_sets`` / ``ffn_given_sets``), so arithmetic error and
+  selection error are judged separately; bf16: max-abs 2e-2 and rel-L2 5e-3;
+  fp32: max-abs 1e-4 and rel-L2 1e-5.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import ffn_long_video_b200 as fb
+import oracle
+import workloads
+
+MARGIN = 1e-5
+TOL = {"bf16": (2e-2, 5e-3), "fp32": (1e-4, 1e-5)}
+
+
+def layout_tensors(cfg, device="cuda"):
+    sizes = cfg.sizes
+    ids = np.concatenate([np.repeat(np.arange(cfg.n_cubes, dtype=np.int32), sizes),
+                          np.full(cfg.n_text, -1, np.int32)])
+    off = cfg.offsets
+    t_ids = torch.from_numpy(ids).to(device)
+    t_off = torch.from_numpy(off).to(device)
+    t_text = torch.from_numpy((ids == -1).astype(np.uint8)).to(device)
+    return t_ids, t_off, t_text, off
+
+
+def make_case(cfg, layer=0):
+    dev = "cuda"
+    lay = workloads.make_layer(cfg, layer=layer, project_on=dev)
+    lay = {k: v.to(dev) for k, v in lay.items()}
+    ids, off, text, off_np = layout_tensors(cfg, dev)
+    return {"cfg": cfg, "t": lay, "ids": ids, "off": off, "text": text, "off_np": off_np}
+
+
+def errors(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    diff = got - want
+    max_abs = float(np.abs(diff).max()) if diff.size else 0.0
+    rel = float(np.linalg.norm(diff) / max(np.linalg.norm(want), 1e-300))
+    return max_abs, rel
+
+
+def run_attn(case, p=None):
+    cfg, t = case["cfg"], case["t"]
+    p = cfg.p if p is None else p
+    out, ws = fb.cube_attn(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis, p)
+    torch.cuda.synchronize()
+    code, detail = fb.read_device_status(ws)
+    assert code == fb.OK, (code, detail)
+    sel = fb.attn_export_sets(ws, case["ids"], cfg.n_cubes, cfg.n_vis, cfg.n_tokens, cfg.hq,
+                              cfg.hkv, cfg.d, fb.BF16 if cfg.dtype == "bf16" else fb.FP32)
+    return out, sel, ws
+
+
+def check_attn(case, p=None, tokens=None, report=None):
+    """Selection parity + output parity of AdaS-Attn on ``tokens`` (default all)."""
+    cfg, t = case["cfg"], case["t"]
+    p = cfg.p if p is None else p
+    out, gsel, ws = run_attn(case, p)
+    Qc, Kc, Vc = (t[k].cpu() for k in ("Q", "K", "V"))
+    off = case["off_np"]
+    if tokens is None:
+        tokens = np.arange(cfg.n_tokens)
+    tokens = np.asarray(tokens)
+    vis = tokens[tokens < cfg.n_vis]
+    osel, margin = oracle.select_cubes(Qc, Kc, off, cfg.n_vis, cfg.hq, cfg.hkv, p, tokens=vis,
+                                       with_margin=True)
+    g = gsel[vis]
+    diff_rows = (osel != g).any(axis=2)
+    near = margin < MARGIN
+    bad = diff_rows & ~near
+    n_near_mismatch = int((diff_rows & near).sum())
+    assert not bad.any(), f"{int(bad.sum())} selection mismatches outside the margin " \
+                          f"(first at {np.argwhere(bad)[:3].tolist()})"
+    # outputs against the oracle on the library's own sets
+    sel_full = np.zeros((len(tokens), cfg.hq, cfg.n_cubes), dtype=bool)
+    is_vis = tokens < cfg.n_vis
+    sel_full[is_vis] = gsel[tokens[is_vis]]
+    want = oracle.attention_given_sets(Qc, Kc, Vc, off, cfg.n_vis, sel_full, tokens=tokens)
+    got = out.float().cpu().numpy()[tokens]
+    max_abs, rel = errors(got, want)
+    tol_abs, tol_rel = TOL[cfg.dtype]
+    if report is not None:
+        report.update(max_abs=max_abs, rel_l2=rel, near_margin_rows=int(near.sum()),
+                      near_margin_mismatch=n_near_mismatch, rows=int(g.shape[0] * g.shape[1]))
+    assert max_abs <= tol_abs and rel <= tol_rel, (max_abs, rel)
+    return out, gsel, ws
+
+
+def run_ffn(case, p=None):
+    cfg, t = case["cfg"], case["t"]
+    p = cfg.p if p is None else p
+    y, ws = fb.token_ffn(t["x"], t["W_gate"], t["W_up"], t["W_down"], case["ids"], case["off"],
+                         case["text"], cfg.n_vis, p)
+    torch.cuda.synchronize()
+    code, detail = fb.read_device_status(ws)
+    assert code == fb.OK, (code, detail)
+    act = fb.ffn_export_active(ws, cfg.n_tokens, cfg.n_vis, cfg.n_cubes, cfg.D, cfg.F,
+                               fb.BF16 if cfg.dtype == "bf16" else fb.FP32)
+    return y, act, ws
+
+
+def check_ffn(case, p=None, cubes=None, text=True, report=None):
+    cfg, t = case["cfg"], case["t"]
+    p = cfg.p if p is None else p
+    y, gact, ws = run_ffn(case, p)
+    x = t["x"].cpu()
+    off = case["off_np"]
+    if cubes is None:
+        cubes = np.arange(cfg.n_cubes)
+    oact, margins = oracle.ffn_select(x, off, cfg.n_vis, p, cubes=cubes, with_margin=True)
+    bad_cubes, near_mismatch = [], 0
+    for c in cubes:
+        a, b = off[c], off[c + 1]
+        if not np.array_equal(oact[a:b], gact[a:b]):
+            if margins[c] < MARGIN:
+                near_mismatch += 1
+            else:
+                bad_cubes.append(int(c))
+    assert not bad_cubes, f"active-set mismatch outside the margin in cubes {bad_cubes[:5]}"
+    assert gact[cfg.n_vis:].all()
+    want = oracle.ffn_given_sets(x, t["W_gate"].cpu(), t["W_up"].cpu(), t["W_down"].cpu(), off,
+                                 cfg.n_vis, gact, cubes=cubes, text=text)
+    rows = np.isfinite(want[:, 0])
+    got = y.cpu().numpy()
+    max_abs, rel = errors(got[rows], want[rows])
+    tol_abs, tol_rel = TOL[cfg.dtype]
+    if report is not None:
+        report.update(max_abs=max_abs, rel_l2=rel,
+                      near_margin_cubes=int((margins[cubes] < MARGIN).sum()),
+                      near_margin_mismatch=near_mismatch)
+    assert max_abs <= tol_abs and rel <= tol_rel, (max_abs, rel)
+    return y, gact, ws

@@ -1,0 +1,83 @@
+"""The C-ABI library without a GPU: it loads, exports every function that
+include/adaspark.h declares, runs the host-only partition (checked against the
+oracle), and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import ffn_long_video_b200 as fb
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "adaspark.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(adaspark_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = fb.lib()
+    names = _declared()
+    assert len(names) >= 16
+    for n in names:
+        assert hasattr(L, n), n
+
+
+@pytest.mark.parametrize("grid,cube,n_text", [
+    ((8, 8, 8), (4, 4, 2), 32),
+    ((5, 7, 3), (2, 3, 2), 3),
+    ((64, 32, 32), (4, 4, 4), 256),
+    ((3, 1, 1), (1, 1, 1), 0),
+])
+def test_partition_matches_oracle(grid, cube, n_text):
+    T, H, W = grid
+    ch, cw, ct = cube
+    perm, ids, off = fb.cube_partition(T, H, W, ch, cw, ct, n_text)
+    operm, oids, ooff, C = oracle.cube_partition(T, H, W, ch, cw, ct, n_text)
+    assert np.array_equal(perm, operm)
+    assert np.array_equal(ids, oids)
+    assert np.array_equal(off, ooff)
+    assert fb.cube_count(T, H, W, ch, cw, ct) == C
+
+
+def test_partition_rejects_bad_sizes():
+    P = ctypes.POINTER(ctypes.c_int32)
+    buf = (ctypes.c_int32 * 16)()
+    n = ctypes.c_int32(0)
+    L = fb.lib()
+    assert L.adaspark_cube_partition(0, 2, 2, 1, 1, 1, 0, buf, buf, buf, ctypes.byref(n)) == fb.EINVAL
+    assert L.adaspark_cube_partition(2, 2, 2, 1, 1, 1, -1, buf, buf, buf, ctypes.byref(n)) == fb.EINVAL
+    assert L.adaspark_cube_partition(2, 2, 2, 1, 1, 1, 0, None, buf, buf, ctypes.byref(n)) == fb.EINVAL
+    assert L.adaspark_cube_count(2, 2, 2, 0, 1, 1, ctypes.byref(n)) == fb.EINVAL
+
+
+def test_workspace_queries():
+    assert fb.cube_attn_workspace_bytes(65792, 65536, 1024, 28, 4, 128, fb.BF16) > 0
+    assert fb.cube_attn_workspace_bytes(544, 512, 16, 4, 1, 64, fb.FP32) > 0
+    assert fb.cube_attn_workspace_bytes(544, 512, 16, 5, 2, 64, fb.FP32) == 0   # hq % hkv
+    assert fb.cube_attn_workspace_bytes(544, 512, 16, 4, 1, 64, fb.BF16) == 0   # bf16 needs d=128
+    assert fb.cube_attn_workspace_bytes(544, 600, 16, 4, 1, 64, fb.FP32) == 0   # n_vis > n_tokens
+    assert fb.token_ffn_workspace_bytes(65792, 65536, 1024, 3584, 18944, fb.BF16) > 0
+    assert fb.token_ffn_workspace_bytes(544, 512, 16, 250, 512, fb.FP32) == 0
+
+
+def test_calls_reject_bad_arguments_before_the_device():
+    L = fb.lib()
+    dummy = ctypes.c_void_p(256)
+    ws_bytes = fb.cube_attn_workspace_bytes(544, 512, 16, 4, 1, 64, fb.FP32)
+    args = [dummy, dummy, dummy, fb.FP32, dummy, dummy, 16, 512, 544, 4, 1, 64]
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        assert L.adaspark_cube_attn(*args, p, dummy, dummy, ws_bytes, None) == fb.EINVAL
+    assert L.adaspark_cube_attn(*args, 0.7, dummy, dummy, ws_bytes - 1, None) == fb.EINVAL
+    assert L.adaspark_cube_attn(*args, 0.7, None, dummy, ws_bytes, None) == fb.EINVAL
+    assert L.adaspark_cube_attn(*args, 0.7, dummy, ctypes.c_void_p(257), ws_bytes, None) == fb.EINVAL
+    fws = fb.token_ffn_workspace_bytes(544, 512, 16, 256, 512, fb.FP32)
+    fargs = [dummy] * 4 + [fb.FP32, dummy, dummy, dummy, 16, 512, 544, 256, 512]
+    assert L.adaspark_token_ffn(*fargs, 2.0, dummy, dummy, fws, None) == fb.EINVAL
+    assert L.adaspark_token_ffn(*fargs, 0.7, dummy, dummy, fws - 8, None) == fb.EINVAL
+    assert fb.status_string(fb.EDEVICE) == "device-side check failed"

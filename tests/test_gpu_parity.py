@@ -1,0 +1,72 @@
+"""Parity of the CUDA path against the float64 oracle (needs a B200).
+
+Element-wise on sizes the oracle finishes in seconds (several tiles, ragged
+tails, truncated and single-token cubes), and on sampled rows / cubes at the
+full Qwen2.5-VL-3B-shaped size."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny-fp32": workloads.CONFIGS[1],
+    # 8 query heads / 2 KV heads, 32-token cubes: 8 visual tiles per KV head,
+    # a ragged text tile (40 text tokens)
+    "small-bf16": workloads.small_config(),
+    # the 3B shape (16/2 heads, 64-token cubes) on a 2048-token grid
+    "mid-bf16": workloads.small_config(name="mid", grid=(8, 16, 16), cube=(4, 4, 4), n_text=72,
+                                       D=512, hq=16, hkv=2, F=1024, seed=99),
+    # truncated edge cubes, one of them a single token
+    "ragged-bf16": workloads.small_config(name="ragged", grid=(4, 8, 8), cube=(4, 4, 2),
+                                          n_text=17, D=256, hq=4, hkv=2, F=256, seed=7,
+                                          cube_sizes=(32, 1, 31, 64, 17, 47, 32, 32)),
+    "ragged-fp32": workloads.small_config(name="ragged32", grid=(4, 8, 8), cube=(4, 4, 2),
+                                          n_text=9, D=128, hq=4, hkv=1, d=64, F=256,
+                                          dtype="fp32", seed=8,
+                                          cube_sizes=(1, 63, 32, 32, 40, 24, 60, 1, 1, 2)),
+}
+
+
+@pytest.fixture(scope="module", params=list(SMALL))
+def small_case(request):
+    torch.manual_seed(0)
+    return parity.make_case(SMALL[request.param])
+
+
+@pytest.mark.parametrize("p", [0.7, 0.3, 1.0])
+def test_attn_small(small_case, p):
+    rep = {}
+    parity.check_attn(small_case, p=p, report=rep)
+    print(small_case["cfg"].name, p, rep)
+
+
+@pytest.mark.parametrize("p", [0.7, 0.45, 1.0])
+def test_ffn_small(small_case, p):
+    rep = {}
+    parity.check_ffn(small_case, p=p, report=rep)
+    print(small_case["cfg"].name, p, rep)
+
+
+def test_attn_smallest_p_picks_argmax(small_case):
+    """p -> 0+: every visual row of cube i > 0 selects exactly one cube."""
+    cfg = small_case["cfg"]
+    _, sel, _ = parity.run_attn(small_case, p=1e-7)
+    off = small_case["off_np"]
+    cube = np.searchsorted(off, np.arange(cfg.n_vis), side="right") - 1
+    counts = sel.sum(axis=2)
+    assert (counts[cube > 0] == 1).all()
+    assert (counts[cube == 0] == 0).all()
+
+
+def test_repeat_runs_identical_sets(small_case):
+    """The selection sets are deterministic run to run."""
+    _, s1, _ = parity.run_attn(small_case)
+    _, s2, _ = parity.run_attn(small_case)
+    assert np.array_equal(s1, s2)
+    _, a1, _ = parity.run_ffn(small_case)
+    _, a2, _ = parity.run_ffn(small_case)
+    assert np.array_equal(a1, a2)
