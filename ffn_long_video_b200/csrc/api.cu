@@ -37,7 +37,7 @@ bool ffn_sizes_ok(int n_tokens, int n_vis, int n_cubes, int D, int F, int dtype)
   if (n_vis == 0 && n_cubes != 0) return false;
   if ((long long)n_cubes > n_vis) return false;
   if (D < 1 || F < 1) return false;
-  if (dtype == ADASPARK_BF16) return D % 64 == 0 && F % 64 == 0;
+  if (dtype == ADASPARK_BF16) return D % 64 == 0 && F % 128 == 0;
   if (dtype == ADASPARK_FP32) return D % 4 == 0 && F % 4 == 0;
   return false;
 }
@@ -212,8 +212,13 @@ int adaspark_token_ffn(const void* x, const void* W_gate, const void* W_up, cons
     return rc;
   if ((rc = cuda_rc(launch_ffn_select(a, dtype, s)))) return rc;
   if ((rc = cuda_rc(launch_ffn_compact(a, dtype, s)))) return rc;
-  if ((rc = cuda_rc(launch_ffn_gemm1_simt(a, dtype, s)))) return rc;
-  if ((rc = cuda_rc(launch_ffn_gemm2_simt(a, dtype, s)))) return rc;
+  if (dtype == ADASPARK_BF16) {
+    if ((rc = cuda_rc(launch_ffn_gemm1_tc(a, s)))) return rc;
+    if ((rc = cuda_rc(launch_ffn_gemm2_tc(a, s)))) return rc;
+  } else {
+    if ((rc = cuda_rc(launch_ffn_gemm1_simt(a, dtype, s)))) return rc;
+    if ((rc = cuda_rc(launch_ffn_gemm2_simt(a, dtype, s)))) return rc;
+  }
   return cuda_rc(launch_ffn_compensate(a, dtype, s));
 }
 
