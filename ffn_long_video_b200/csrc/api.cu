@@ -101,7 +101,7 @@ int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
     rc = cuda_rc(launch_cube_mean(K, dtype, cube_offsets, const_cast<float*>(sa.kbar),
                                   const_cast<__nv_bfloat16*>(sa.kbar_split), G, hdr, s));
     if (rc) return rc;
-    rc = cuda_rc(launch_select_simt(sa, dtype, s));
+    rc = cuda_rc(dtype == ADASPARK_BF16 ? launch_select_tc(sa, s) : launch_select_simt(sa, dtype, s));
     if (rc) return rc;
   }
 
@@ -119,6 +119,7 @@ int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
   aa.G = G;
   aa.dense = dense;
   aa.scale_log2 = sa.zscale;
+  if (dtype == ADASPARK_BF16) return cuda_rc(launch_attn_tc(aa, s));
   return cuda_rc(launch_attn_simt(aa, dtype, s));
 }
 
@@ -194,6 +195,7 @@ int adaspark_token_ffn(const void* x, const void* W_gate, const void* W_up, cons
   a.xa = ws + L.xa;
   a.h = ws + L.h;
   a.sums = reinterpret_cast<float*>(ws + L.sums);
+  a.wd16 = ws + L.wd16;
   a.hdr = reinterpret_cast<WsHeader*>(ws + L.header);
   a.n_tokens = n_tokens;
   a.n_vis = n_vis;
@@ -213,6 +215,7 @@ int adaspark_token_ffn(const void* x, const void* W_gate, const void* W_up, cons
   if ((rc = cuda_rc(launch_ffn_select(a, dtype, s)))) return rc;
   if ((rc = cuda_rc(launch_ffn_compact(a, dtype, s)))) return rc;
   if (dtype == ADASPARK_BF16) {
+    if ((rc = cuda_rc(launch_wdown_to_fp16(a, s)))) return rc;
     if ((rc = cuda_rc(launch_ffn_gemm1_tc(a, s)))) return rc;
     if ((rc = cuda_rc(launch_ffn_gemm2_tc(a, s)))) return rc;
   } else {
@@ -243,13 +246,14 @@ int adaspark_ffn_read_stats(const void* workspace, adaspark_ffn_stats* stats, vo
 }
 
 int adaspark_read_device_status(const void* workspace, uint32_t* detail, void* stream) {
+  // detail: ADASPARK_DEV_* bits in 0..7, the code of the first failing check in 8..23
   if (!workspace) return ADASPARK_EINVAL;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return ADASPARK_ECUDA;
   uint32_t st[2] = {0, 0};
   if (cudaMemcpy(st, workspace, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess)
     return ADASPARK_ECUDA;
-  if (detail) *detail = st[0];
+  if (detail) *detail = (st[0] & 0xffu) | ((st[1] & 0xffffu) << 8);
   return st[0] ? ADASPARK_EDEVICE : ADASPARK_OK;
 }
 

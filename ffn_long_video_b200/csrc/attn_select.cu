@@ -74,34 +74,6 @@ __global__ void cube_mean_kernel(const T* __restrict__ K, const int32_t* __restr
 }
 
 // ---------------------------------------------------------------------------
-// Shared tile epilogue: compact the cube columns with any row bit into the
-// tile's ascending list. 128 threads.
-// ---------------------------------------------------------------------------
-__device__ void compact_tile_list(const uint32_t* tmask, uint16_t* list, int32_t* count, int c_hi,
-                                  int* s_wcnt) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int total = 0;
-  for (int base = 0; base <= c_hi; base += 128) {
-    const int j = base + tid;
-    bool nz = false;
-    if (j <= c_hi) {
-      const uint4 w = __ldcg(reinterpret_cast<const uint4*>(tmask + (size_t)j * 4));
-      nz = (w.x | w.y | w.z | w.w) != 0u;
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, nz);
-    if (lane == 0) s_wcnt[warp] = __popc(bal);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    int before = total;
-    for (int w = 0; w < warp; ++w) before += s_wcnt[w];
-    const int chunk_total = s_wcnt[0] + s_wcnt[1] + s_wcnt[2] + s_wcnt[3];
-    if (nz) list[before + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)j;
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    total += chunk_total;
-  }
-  if (tid == 0) *count = total;
-}
-
-// ---------------------------------------------------------------------------
 // SIMT scorer + selection: one block per visual tile, one thread per row.
 // ---------------------------------------------------------------------------
 template <typename T, int D>
@@ -114,12 +86,10 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
   const AttnGeom& G = a.G;
   const int vt = blockIdx.x;
   const int kv = vt / G.vtiles_per_kv;
-  const int tl = vt - kv * G.vtiles_per_kv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long r = (long long)tl * kTileRows + tid;
-  const bool valid = r < (long long)G.n_vis * G.g;
-  const int t = valid ? (int)(r / G.g) : 0;
-  const int h = kv * G.g + (valid ? (int)(r % G.g) : 0);
+  const TileRow R = tile_row(G, false, vt, tid);
+  const bool valid = R.valid;
+  const int t = R.t, h = R.h;
   const int own = valid ? a.cube_ids[t] : -1;
 
   if (tid == 0) {
@@ -198,7 +168,7 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
       }
       __syncthreads();
       compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes, a.tile_count + vt, c_hi,
-                        s_wcnt);
+                        s_wcnt, tid);
     }
   }
 }
@@ -212,12 +182,10 @@ __global__ void export_sets_kernel(const int32_t* __restrict__ tile_count,
                                    const int32_t* __restrict__ cube_ids, AttnGeom G, int dense,
                                    uint32_t* __restrict__ bits) {
   const int vt = blockIdx.x;
-  const int kv = vt / G.vtiles_per_kv;
-  const int tl = vt - kv * G.vtiles_per_kv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long r = (long long)tl * kTileRows + tid;
-  if (r >= (long long)G.n_vis * G.g) return;
-  const int t = (int)(r / G.g), h = kv * G.g + (int)(r % G.g);
+  const TileRow R = tile_row(G, false, vt, tid);
+  if (!R.valid) return;
+  const int t = R.t, h = R.h;
   const int own = cube_ids[t];
   const int W = (G.n_cubes + 31) / 32;
   uint32_t* row = bits + ((size_t)t * G.hq + h) * W;

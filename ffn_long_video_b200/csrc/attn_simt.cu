@@ -20,14 +20,10 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(AttnArgs a) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool text = blockIdx.x >= (unsigned)G.n_vtiles;
   const int bt = text ? blockIdx.x - G.n_vtiles : blockIdx.x;
-  const int per_kv = text ? G.ttiles_per_kv : G.vtiles_per_kv;
-  const int kv = bt / per_kv;
-  const int tl = bt - kv * per_kv;
-  const long long r = (long long)tl * kTileRows + tid;
-  const long long nrows = (long long)(text ? G.n_tokens - G.n_vis : G.n_vis) * G.g;
-  const bool valid = r < nrows;
-  const int t = (text ? G.n_vis : 0) + (valid ? (int)(r / G.g) : 0);
-  const int h = kv * G.g + (valid ? (int)(r % G.g) : 0);
+  const int kv = bt / (text ? G.ttiles_per_kv : G.vtiles_per_kv);
+  const TileRow R = tile_row(G, text, bt, tid);
+  const bool valid = R.valid;
+  const int t = R.t, h = R.h;
   const int own = (!text && valid) ? a.cube_ids[t] : -1;
 
   if (tid == 0) s_hi = -1;

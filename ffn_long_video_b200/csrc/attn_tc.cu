@@ -1,0 +1,490 @@
+// AdaS-Attn block-sparse attention on the 5th-generation tensor cores (bf16).
+//
+// Key design 2 of the AdaSpark note: a visual query attends to the keys of its
+// selected cubes and, causally, of its own cube; one softmax over all admitted
+// keys. A text query attends densely and causally.
+//
+// One CTA per 128-row tile (128 tokens of one query head). The tile walks a
+// sequence of 64-key blocks: the cubes of its selection list (cubes where any
+// row has its bit set) cut into 64-key pieces, or every cube then the text keys
+// for a text tile. Rows that did not select a cube are masked inside the block.
+//   warp 6     block-descriptor filler: reads the list, cube offsets and row
+//              masks from global memory 32 entries at a time and feeds a
+//              64-slot shared-memory ring, far ahead of the consumers
+//   warp 0     TMA producer: K and V blocks (3D maps over [token][kv][d], no
+//              multicast), 3-stage ring
+//   warp 1     TMEM allocator + tcgen05.mma issuer:
+//                S_i = Q K_i^T   (M=128, N=64, K=128; two TMEM buffers)
+//                O  += P_i V_i   (M=128, N=128, K=64; V read N-major)
+//   warps 2-5  one thread per row: Q gather, masking, online softmax with lazy
+//              rescaling of O in TMEM, P (bf16) to shared memory, final 1/l.
+#include "attn_kernels.h"
+
+namespace adaspark {
+namespace fa {
+
+constexpr int STAGES = 3;
+constexpr int THREADS = 224;
+constexpr int RING = 64;
+constexpr int Q_BYTES = 128 * 256;        // 128 rows x 128 dims bf16 (two 64-dim halves)
+constexpr int KV_BYTES = 4 * 8192;        // K (2 halves) + V (2 halves), 64 keys each
+constexpr int P_BYTES = 128 * 128;        // 128 rows x 64 keys bf16
+struct Desc {
+  int k0, nk, j, pad;
+  uint32_t mask[4];
+};
+constexpr size_t SMEM_BYTES =
+    1024 + Q_BYTES + STAGES * KV_BYTES + 2 * P_BYTES + RING * sizeof(Desc) + 2048;
+constexpr float kRescale = 8.0f;          // log2 headroom before O is rescaled
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+struct TileInfo {
+  bool text;
+  int bt;        // tile index within its kind
+  int kv;
+  int t_hi;      // last valid token of the tile
+};
+
+__device__ __forceinline__ TileInfo decode_tile(const AttnGeom& G) {
+  TileInfo T;
+  const int b = blockIdx.x;
+  T.text = b < G.n_ttiles;  // text tiles first (the heaviest)
+  if (T.text) {
+    T.bt = b;
+  } else {
+    // visual tiles, latest tokens first: rank r -> token tile, then head
+    const int r = b - G.n_ttiles;
+    const int per_head = G.vtiles_per_head;
+    const int tt = per_head - 1 - r / G.hq;
+    const int hq_idx = r % G.hq;                 // query head
+    const int kv = hq_idx / G.g, hh = hq_idx - kv * G.g;
+    T.bt = kv * G.vtiles_per_kv + hh * per_head + tt;
+  }
+  T.kv = T.bt / (T.text ? G.ttiles_per_kv : G.vtiles_per_kv);
+  const int per_head = T.text ? G.ttiles_per_head : G.vtiles_per_head;
+  const int count = T.text ? G.n_tokens - G.n_vis : G.n_vis;
+  const int tl = T.bt - T.kv * (T.text ? G.ttiles_per_kv : G.vtiles_per_kv);
+  const int tt = tl % per_head;
+  T.t_hi = (T.text ? G.n_vis : 0) + min(tt * kTileRows + kTileRows, count) - 1;
+  return T;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                   AttnArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = sQ + Q_BYTES;
+  uint8_t* sP = sKV + STAGES * KV_BYTES;
+  Desc* ring = reinterpret_cast<Desc*>(sP + 2 * P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + RING);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = kv_full + STAGES;
+  uint64_t* s_full = kv_empty + STAGES;     // [2]
+  uint64_t* s_empty = s_full + 2;           // [2]
+  uint64_t* p_full = s_empty + 2;           // [2]
+  uint64_t* pv_done = p_full + 2;           // [2]
+  uint64_t* q_full = pv_done + 2;
+  uint64_t* drain = q_full + 1;
+  uint64_t* r_full = drain + 1;             // [RING]
+  uint64_t* r_empty = r_full + RING;        // [RING]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(r_empty + RING);
+  __shared__ volatile int s_abort;
+  __shared__ int s_own_hi, s_bad;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const AttnGeom& G = a.G;
+  WsHeader* hdr = a.hdr;
+  const TileInfo T = decode_tile(G);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 128);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+    }
+    for (int r = 0; r < RING; ++r) {
+      mbar_init(&r_full[r], 1);
+      mbar_init(&r_empty[r], 128);
+    }
+    mbar_init(q_full, 128);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    s_abort = 0;
+    s_bad = status_bad(hdr) ? 1 : 0;
+    s_own_hi = (!T.text && !s_bad) ? a.cube_ids[T.t_hi] : -1;
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const bool bad = s_bad != 0;
+
+  if (warp == 6) {
+    // ------------------------------------------------------------ descriptor filler
+    int n_entries = 0, n_chunks = 0;
+    bool use_list = false;
+    if (!bad) {
+      if (T.text) {
+        n_entries = G.n_cubes;
+        n_chunks = (T.t_hi - G.n_vis) / 64 + 1;
+      } else if (a.dense) {
+        n_entries = s_own_hi + 1;
+      } else {
+        n_entries = a.tile_count[T.bt];
+        use_list = true;
+      }
+    }
+    const int n_total = n_entries + n_chunks;
+    const uint16_t* list = a.tile_list + (size_t)T.bt * G.n_cubes;
+    const uint4* tmask = reinterpret_cast<const uint4*>(a.tile_mask) + (size_t)T.bt * G.n_cubes;
+    int base = 0;
+    bool ok = true;
+    for (int e0 = 0; e0 < n_total && ok; e0 += 32) {
+      const int e = e0 + lane;
+      int j = -1, ks = 0, ke = 0;
+      uint4 m = make_uint4(~0u, ~0u, ~0u, ~0u);
+      if (e < n_entries) {
+        j = use_list ? (int)list[e] : e;
+        ks = a.cube_offsets[j];
+        ke = a.cube_offsets[j + 1];
+        if (use_list) m = tmask[j];
+      } else if (e < n_total) {
+        ks = G.n_vis + (e - n_entries) * 64;
+        ke = min(ks + 64, T.t_hi + 1);
+      }
+      const int nb = (ke - ks + 63) / 64;
+      int incl = nb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      int idx = base + incl - nb;
+      for (int b = 0; b < nb; ++b, ++idx) {
+        const int slot = idx % RING;
+        if (!mbar_wait(&r_empty[slot], ((idx / RING) & 1) ^ 1, &s_abort, hdr, 0x7a00u)) {
+          ok = false;
+          break;
+        }
+        Desc& d = ring[slot];
+        d.k0 = ks + 64 * b;
+        d.nk = min(64, ke - d.k0);
+        d.j = j;
+        d.mask[0] = m.x;
+        d.mask[1] = m.y;
+        d.mask[2] = m.z;
+        d.mask[3] = m.w;
+        mbar_arrive(&r_full[slot]);
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      base += total;
+    }
+    if (ok && lane == 0) {  // terminal descriptor
+      const int slot = base % RING;
+      if (mbar_wait(&r_empty[slot], ((base / RING) & 1) ^ 1, &s_abort, hdr, 0x7b00u)) {
+        ring[slot].nk = 0;
+        mbar_arrive(&r_full[slot]);
+      }
+    }
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int i = 0;
+      bool ok = true;
+      while (ok) {
+        const int slot = i % RING;
+        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7000u)) break;
+        const int k0 = ring[slot].k0, nk = ring[slot].nk;
+        if (nk == 0) break;
+        const int s = i % STAGES;
+        if (!mbar_wait(&kv_empty[s], ((i / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7100u)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = sKV + s * KV_BYTES;
+        mbar_expect_tx(&kv_full[s], KV_BYTES);
+        tma_load_3d(&mapK, &kv_full[s], st, 0, T.kv, k0);
+        tma_load_3d(&mapK, &kv_full[s], st + 8192, 64, T.kv, k0);
+        tma_load_3d(&mapV, &kv_full[s], st + 16384, 0, T.kv, k0);
+        tma_load_3d(&mapV, &kv_full[s], st + 24576, 64, T.kv, k0);
+        ++i;
+      }
+      if (!ok) {
+        for (int k = 0; k < STAGES; ++k) {
+          const int jj = i - 1 - k;
+          if (jj < 0) break;
+          long long t0 = clock64();
+          while (!mbar_try_wait(&kv_full[jj % STAGES], (jj / STAGES) & 1) &&
+                 clock64() - t0 < kWaitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64);
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, 128, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      bool ok = mbar_wait(q_full, 0, &s_abort, hdr, 0x7200u);
+      tc_fence_after();
+      int i = 0;
+      auto issue_pv = [&](int blk) -> bool {
+        const int pb = blk & 1;
+        if (!mbar_wait(&p_full[pb], (blk >> 1) & 1, &s_abort, hdr, 0x7300u)) return false;
+        tc_fence_after();
+        const int s = blk % STAGES;
+        const uint32_t v_addr = smem_u32(sKV + s * KV_BYTES + 16384);
+        const uint32_t p_addr = smem_u32(sP + pb * P_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = make_sdesc_sw128(p_addr + kk * 32, 16, 1024);
+          const uint64_t bd = make_sdesc_sw128(v_addr + kk * 2048, 8192, 1024);
+          umma_bf16(tmem_base, ad, bd, idesc_o, (blk > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_done[pb]);
+        umma_commit(&kv_empty[s]);
+        return true;
+      };
+      while (ok) {
+        const int slot = i % RING;
+        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7d00u)) {
+          ok = false;
+          break;
+        }
+        if (ring[slot].nk == 0) break;
+        const int s = i % STAGES;
+        const int sb = i & 1;
+        if (!mbar_wait(&kv_full[s], (i / STAGES) & 1, &s_abort, hdr, 0x7400u) ||
+            !mbar_wait(&s_empty[sb], ((i >> 1) & 1) ^ 1, &s_abort, hdr, 0x7500u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sKV + s * KV_BYTES);
+        const uint32_t d_s = tmem_base + 128 + sb * 64;
+#pragma unroll
+        for (int dc = 0; dc < 2; ++dc)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024);
+            const uint64_t bd = make_sdesc_sw128(k_addr + dc * 8192 + kk * 32, 16, 1024);
+            umma_bf16(d_s, ad, bd, idesc_s, (dc | kk) != 0 ? 1u : 0u);
+          }
+        umma_commit(&s_full[sb]);
+        if (i > 0 && !issue_pv(i - 1)) {
+          ok = false;
+          break;
+        }
+        ++i;
+      }
+      if (ok && i > 0) issue_pv(i - 1);
+      umma_commit(drain);
+      long long t0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax rows
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const TileRow R = tile_row(G, T.text, T.bt, row);
+    const bool valid = R.valid;
+    const int t = R.t, h = R.h;
+    const int own = (!T.text && valid) ? a.cube_ids[t] : -1;
+    const float scale = a.scale_log2;
+    {
+      const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
+      const uint4* src = reinterpret_cast<const uint4*>(Qg + ((size_t)t * G.hq + h) * 128);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sQ + (c >> 3) * 16384 + sw128_offset(row, c & 7)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_full);
+    }
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    float m_used = -INFINITY, l = 0.f;
+    int i = 0;
+    bool ok = true;
+    while (true) {
+      const int slot = i % RING;
+      if (!mbar_wait_warp(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7e00u)) {
+        ok = false;
+        break;
+      }
+      const Desc dsc = ring[slot];
+      if (dsc.nk == 0) break;
+      const int sb = i & 1;
+      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0x7600u)) {
+        ok = false;
+        break;
+      }
+      // S_i has landed, so the producer and the MMA issuer have both consumed
+      // descriptor i: only now may the filler reuse its slot.
+      mbar_arrive(&r_empty[slot]);
+      tc_fence_after();
+      uint32_t sr[64];
+      {
+        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        tmem_ld32(tmem_base + lane_base + 128 + sb * 64, s0);
+        tmem_ld32(tmem_base + lane_base + 128 + sb * 64 + 32, s1);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(&s_empty[sb]);
+
+      // admitted keys [0, lim) of this row in the block
+      bool row_on;
+      if (!valid) row_on = false;
+      else if (T.text) row_on = true;
+      else if (a.dense) row_on = dsc.j <= own;
+      else row_on = ((dsc.mask[wq] >> lane) & 1u) != 0u;
+      int lim = row_on ? dsc.nk : 0;
+      if (row_on && (T.text || dsc.j == own)) lim = min(lim, t - dsc.k0 + 1);
+      float mraw = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 64; ++u)
+        if (u < lim) mraw = fmaxf(mraw, __uint_as_float(sr[u]));
+      const float m_new = fmaxf(m_used, mraw * scale);
+      const bool want = m_new > m_used + kRescale;
+      if (__any_sync(0xffffffffu, want)) {
+        const float factor = (m_used == -INFINITY || m_new == -INFINITY) ? 1.f
+                                                                         : ex2(m_used - m_new);
+        if (i > 0) {
+          if (!mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr,
+                              0x7700u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(tmem_base + lane_base + c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * factor);
+            tmem_st32(tmem_base + lane_base + c, o);
+          }
+          tmem_st_wait();
+        }
+        l *= factor;
+        if (m_new != -INFINITY) m_used = m_new;
+      }
+      const int pb = i & 1;
+      if (i >= 2) {
+        if (!mbar_wait_warp(&pv_done[pb], ((i - 2) >> 1) & 1, &s_abort, hdr, 0x7800u)) {
+          ok = false;
+          break;
+        }
+      }
+      // P = 2^(s * scale - m_used) on admitted keys, bf16, 128-byte swizzled row
+      float ls0 = 0.f, ls1 = 0.f;
+      uint8_t* prow = sP + pb * P_BYTES;
+      const float neg_m = -m_used;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int u = c * 8 + q * 2;
+          const float p0 = (u < lim) ? ex2(fmaf(__uint_as_float(sr[u]), scale, neg_m)) : 0.f;
+          const float p1 =
+              (u + 1 < lim) ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, neg_m)) : 0.f;
+          ls0 += p0;
+          ls1 += p1;
+          pk[q] = pack_bf16x2(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(prow + sw128_offset(row, c)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l += ls0 + ls1;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&p_full[pb]);
+      ++i;
+    }
+    // final: O / l once the last PV has landed
+    if (ok && i > 0 &&
+        mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr, 0x7900u)) {
+      tc_fence_after();
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* dst =
+          reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem_base + lane_base + c, o);
+        tmem_ld_wait();
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            pk[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv,
+                                __uint_as_float(o[2 * x + 1]) * inv);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            d4[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        }
+      }
+    }
+    if (warp == 2 && lane == 0 && !bad) {
+      atomicAdd((unsigned long long*)&hdr->stats[4], 1ull);
+      atomicAdd((unsigned long long*)&hdr->stats[5], (unsigned long long)i);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 256);
+  }
+}
+
+}  // namespace fa
+
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
+  const AttnGeom& G = a.G;
+  const int blocks = G.n_vtiles + G.n_ttiles;
+  if (blocks == 0) return cudaSuccess;
+  CUtensorMap mK, mV;
+  const uint64_t dims[3] = {(uint64_t)G.d, (uint64_t)G.hkv, (uint64_t)G.n_tokens};
+  const uint64_t strides[2] = {(uint64_t)G.d * 2, (uint64_t)G.hkv * G.d * 2};
+  const uint32_t box[3] = {64, 1, 64};
+  if (!encode_tmap_bf16(&mK, a.K, 3, dims, strides, box) ||
+      !encode_tmap_bf16(&mV, a.V, 3, dims, strides, box))
+    return cudaErrorInvalidValue;
+  auto k = fa::attn_tc_kernel;
+  cudaError_t e =
+      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fa::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  return launch("attn_tc", k, dim3(blocks), dim3(fa::THREADS), fa::SMEM_BYTES, s, mK, mV, a);
+}
+
+}  // namespace adaspark

@@ -32,7 +32,10 @@ __host__ __device__ inline size_t align_up(size_t v, size_t a = kAlign) {
 
 __device__ __forceinline__ void set_status(WsHeader* h, uint32_t bit, uint32_t detail = 0) {
   atomicOr(&h->status, bit);
-  if (detail) atomicCAS(&h->detail, 0u, detail);
+  if (detail && atomicCAS(&h->detail, 0u, detail) == 0u) {
+    h->pad[1] = blockIdx.x;   // first failing CTA and thread, for diagnosis
+    h->pad[2] = threadIdx.x;
+  }
 }
 __device__ __forceinline__ bool status_bad(const WsHeader* h) {
   return *((volatile const uint32_t*)&h->status) != 0u;
@@ -123,6 +126,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Warp-uniform form: every lane waits, and the warp proceeds only if all lanes
+// saw the phase complete (so warp-collective tcgen05 ops after it never diverge).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag, WsHeader* hdr,
+                                               uint32_t where) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, hdr, where);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library).
 // ---------------------------------------------------------------------------
@@ -189,12 +201,13 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// Instruction descriptor, kind::f16: bf16 A/B, fp32 D, A and B K-major unless
-// b_mn_major (B stored with N contiguous), M x N tile.
-__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_major = false) {
+// Instruction descriptor, kind::f16: bf16 (or fp16) A and B of the same type,
+// fp32 D, A and B K-major unless b_mn_major (B stored with N contiguous), M x N.
+__host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_major = false,
+                                                       bool fp16 = false) {
   return (1u << 4)                          // D format: f32
-         | (1u << 7)                        // A format: bf16
-         | (1u << 10)                       // B format: bf16
+         | ((fp16 ? 0u : 1u) << 7)          // A format: bf16 (1) / f16 (0)
+         | ((fp16 ? 0u : 1u) << 10)         // B format: same as A
          | ((b_mn_major ? 1u : 0u) << 16)   // B major
          | ((uint32_t)(N >> 3) << 17)       // N / 8
          | ((uint32_t)(M >> 4) << 24);      // M / 16

@@ -1,7 +1,9 @@
 // AdaS-FFN GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
 //   mode 0 (gate/up):  H[m, n] = silu(X_a W_gate^T)[m, n] * (X_a W_up^T)[m, n]
-//   mode 1 (down):     FFN_a = H W_down^T; y[idx[m]] = x[idx[m]] + FFN_a[m];
+//                      (bf16 x bf16, fp32 accumulate; H stored as fp16, saturating)
+//   mode 1 (down):     FFN_a = H W_down^T (fp16 x fp16 with W_down converted
+//                      from bf16, fp32 accumulate); y[idx[m]] = x[idx[m]] + FFN_a[m];
 //                      sums[cube(m)] += FFN_a[m] for active visual rows
 // (key design 3 of the AdaSpark note: the FFN runs only on the active tokens; the
 // per-cube sums feed the mean compensation of the skipped ones).
@@ -15,6 +17,13 @@
 // the epilogue of tile i overlaps the MMAs of tile i+1. In mode 0 the 256 B
 // rows are 128 W_gate rows followed by the same 128 W_up rows, so one MMA chain
 // yields gate (columns 0-127) and up (128-255) for the same outputs.
+// H is kept in fp16 rather than bf16: its 3 extra mantissa bits keep the
+// rounding error of the 18944-long down-projection sums well inside the
+// output tolerance (bf16 H gave max-abs errors near 0.04 at that width).
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
 #include "ffn_kernels.h"
 
 namespace adaspark {
@@ -46,6 +55,12 @@ __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt
 }
 
 __device__ __forceinline__ float silu(float g) { return g / (1.f + __expf(-g)); }
+
+__device__ __forceinline__ uint32_t pack_f16x2_sat(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 
 // Reduce 32 per-row values (one row per lane) to 32 per-column sums; lane l
 // ends with the sum of column l (rows that should not count pass zeros).
@@ -79,6 +94,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   __shared__ volatile int s_abort;
+  __shared__ int s_M;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   WsHeader* hdr = P.f.hdr;
@@ -94,6 +110,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(drain, 1);
     fence_mbar_init();
     s_abort = 0;
+    s_M = status_bad(hdr) ? 0 : (int)*P.m_active;
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&mapA);
@@ -109,7 +126,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int M = status_bad(hdr) ? 0 : (int)*P.m_active;
+  const int M = s_M;
   const int num_m = (M + BM - 1) / BM;
   const int total = num_m * P.n_tiles;
   const int KB = P.k_blocks;
@@ -153,7 +170,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_bf16(BM, BN);
+      constexpr uint32_t idesc = make_idesc_bf16(BM, BN, false, MODE == 1);
       int it = 0, tc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
@@ -198,13 +215,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       tile_coords(t, num_m, P.n_tiles, mt, nt);
       const int b = tc & 1;
       const uint32_t aph = (tc >> 1) & 1;
-      if (!mbar_wait(&acc_full[b], aph, &s_abort, hdr, 0x6400u)) break;
+      if (!mbar_wait_warp(&acc_full[b], aph, &s_abort, hdr, 0x6400u)) break;
       tc_fence_after();
       const int m = mt * BM + row;
       const bool live = m < M;
       const uint32_t tb = tmem_base + ((uint32_t)(wq * 32) << 16) + b * BN;
       if (MODE == 0) {
-        __nv_bfloat16* H = reinterpret_cast<__nv_bfloat16*>(P.f.h);
+        __half* H = reinterpret_cast<__half*>(P.f.h);
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
           uint32_t g[32], u[32];
@@ -219,7 +236,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               const float h0 = silu(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
               const float h1 =
                   silu(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-              pk[i] = pack_bf16x2(h0, h1);
+              pk[i] = pack_f16x2_sat(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(H + (size_t)m * P.f.F + n0);
 #pragma unroll
@@ -303,11 +320,39 @@ static int num_sms() {
 }
 
 static bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
-                     uint32_t box_rows) {
+                     uint32_t box_rows, bool fp16 = false) {
   const uint64_t dims[2] = {cols, rows};
   const uint64_t strides[1] = {cols * 2};
   const uint32_t box[2] = {64, box_rows};
-  return encode_tmap_bf16(m, base, 2, dims, strides, box);
+  return encode_tmap_16(m, base, 2, dims, strides, box, fp16);
+}
+
+// W_down bf16 -> fp16 (exact for |w| >= 2^-14; smaller magnitudes keep an
+// absolute error below 2^-25). 8 elements per thread.
+__global__ void wdown_to_fp16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
+                                     size_t n8, WsHeader* hdr) {
+  if (status_bad(hdr)) return;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+    uint4 o;
+    uint32_t* op = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(b[k]);
+      const __half2 hv = __floats2half2_rn(f.x, f.y);
+      op[k] = *reinterpret_cast<const uint32_t*>(&hv);
+    }
+    reinterpret_cast<uint4*>(dst)[i] = o;
+  }
+}
+
+cudaError_t launch_wdown_to_fp16(const FfnArgs& a, cudaStream_t s) {
+  const size_t n8 = (size_t)a.D * a.F / 8;
+  const int blocks = (int)std::min<size_t>((n8 + 255) / 256, (size_t)num_sms() * 8);
+  return launch("wdown_to_fp16", wdown_to_fp16_kernel, dim3(blocks), dim3(256), 0, s,
+                (const __nv_bfloat16*)a.W_down, (__half*)a.wd16, n8, a.hdr);
 }
 
 cudaError_t launch_ffn_gemm1_tc(const FfnArgs& a, cudaStream_t s) {
@@ -331,7 +376,8 @@ cudaError_t launch_ffn_gemm1_tc(const FfnArgs& a, cudaStream_t s) {
 
 cudaError_t launch_ffn_gemm2_tc(const FfnArgs& a, cudaStream_t s) {
   CUtensorMap mA, mD;
-  if (!map_rows(&mA, a.h, a.F, a.n_tokens, 128) || !map_rows(&mD, a.W_down, a.F, a.D, 256))
+  if (!map_rows(&mA, a.h, a.F, a.n_tokens, 128, true) ||
+      !map_rows(&mD, a.wd16, a.F, a.D, 256, true))
     return cudaErrorInvalidValue;
   gemm::Params P;
   P.m_active = &a.hdr->m_active;

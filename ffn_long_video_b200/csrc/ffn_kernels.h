@@ -24,6 +24,7 @@ struct FfnArgs {
   void* xa;             // [N][D]
   void* h;              // [N][F]
   float* sums;          // [C][D]
+  void* wd16;           // [D][F] fp16 copy of W_down (bf16 path)
   WsHeader* hdr;
   int n_tokens, n_vis, n_cubes, D, F;
   float p;
@@ -37,5 +38,6 @@ cudaError_t launch_ffn_gemm2_simt(const FfnArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_ffn_gemm1_tc(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_gemm2_tc(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_compensate(const FfnArgs& a, int dtype, cudaStream_t s);
+cudaError_t launch_wdown_to_fp16(const FfnArgs& a, cudaStream_t s);
 
 }  // namespace adaspark

@@ -32,10 +32,15 @@ inline cudaError_t launch(const char* name, void (*kernel)(KArgs...), dim3 grid,
 #endif
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
-// 2D or 3D bf16 maps, 128-byte swizzle, zero fill out of bounds.
-// dims/strides are innermost first; strides in bytes for dims 1.. (dim 0 is dense).
-bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                      const uint64_t* strides_bytes, const uint32_t* box);
+// 2D or 3D maps of 16-bit elements (bf16 or fp16), 128-byte swizzle, zero fill
+// out of bounds. dims/strides are innermost first; strides in bytes for dims
+// 1.. (dim 0 is dense).
+bool encode_tmap_16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, bool fp16);
+inline bool encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                             const uint64_t* strides_bytes, const uint32_t* box) {
+  return encode_tmap_16(map, base, rank, dims, strides_bytes, box, false);
+}
 
 inline bool p_valid(float p) { return p > 0.0f && p <= 1.0f; }  // false for NaN
 

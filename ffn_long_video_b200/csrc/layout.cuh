@@ -12,14 +12,19 @@ constexpr int kTileRows = 128;      // rows of one attention / selection tile
 constexpr int kMaxCubeTokens = 256; // largest cube accepted
 constexpr int kMaxCubes = 65535;    // cube ids fit 16 bits in the selection lists
 
-// Geometry of AdaS-Attn. A "row" is one (token, query head) pair. Rows of one
-// KV head are ordered r = t * g + (h mod g) and cut into 128-row tiles; visual
-// tiles cover tokens [0, n_vis), text tiles the suffix.
+// Geometry of AdaS-Attn. A "row" is one (token, query head) pair. Rows are
+// grouped by KV head, then by query head within the group, then by token, and
+// cut into 128-token tiles that never straddle a head: tile tl of KV head kv
+// holds query head kv * g + tl / tiles_per_head and tokens
+// (tl % tiles_per_head) * 128 + [0, 128). Rows of one tile thus share the head
+// and span one or two neighbouring cubes, which keeps the union of their cube
+// sets small. Visual tiles cover tokens [0, n_vis), text tiles the suffix.
 struct AttnGeom {
   int n_tokens, n_vis, n_cubes, hq, hkv, d, g;
-  int vtiles_per_kv, ttiles_per_kv;  // tiles per KV head
+  int vtiles_per_head, ttiles_per_head;  // 128-token tiles per query head
+  int vtiles_per_kv, ttiles_per_kv;      // tiles per KV head
   int n_vtiles, n_ttiles;
-  int pool_rows;                     // overflow-pool capacity (rows)
+  int pool_rows;                         // overflow-pool capacity (rows)
 };
 
 __host__ __device__ inline AttnGeom make_attn_geom(int n_tokens, int n_vis, int n_cubes, int hq,
@@ -32,18 +37,41 @@ __host__ __device__ inline AttnGeom make_attn_geom(int n_tokens, int n_vis, int 
   G.hkv = hkv;
   G.d = d;
   G.g = hq / hkv;
-  long long vrows = (long long)n_vis * G.g;
-  long long trows = (long long)(n_tokens - n_vis) * G.g;
-  G.vtiles_per_kv = (int)((vrows + kTileRows - 1) / kTileRows);
-  G.ttiles_per_kv = (int)((trows + kTileRows - 1) / kTileRows);
+  G.vtiles_per_head = (n_vis + kTileRows - 1) / kTileRows;
+  G.ttiles_per_head = (n_tokens - n_vis + kTileRows - 1) / kTileRows;
+  G.vtiles_per_kv = G.vtiles_per_head * G.g;
+  G.ttiles_per_kv = G.ttiles_per_head * G.g;
   G.n_vtiles = G.vtiles_per_kv * hkv;
   G.n_ttiles = G.ttiles_per_kv * hkv;
-  long long rows = vrows * hkv;
-  long long pr = rows / 16;
-  if (pr < 1024) pr = 1024;
-  if (pr > 16384) pr = 16384;
+  long long rows = (long long)n_vis * hq;
+  long long pr = rows / 8;
+  if (pr < 4096) pr = 4096;
+  if (pr > 65536) pr = 65536;
+  if (pr > rows) pr = rows > 0 ? rows : 1;
   G.pool_rows = (int)pr;
   return G;
+}
+
+// Row i (0..127) of tile `bt` (index within its kind: kv * tiles_per_kv + tl).
+struct TileRow {
+  bool valid;
+  int t;   // token
+  int h;   // query head
+};
+__host__ __device__ inline TileRow tile_row(const AttnGeom& G, bool text, int bt, int i) {
+  const int per_kv = text ? G.ttiles_per_kv : G.vtiles_per_kv;
+  const int per_head = text ? G.ttiles_per_head : G.vtiles_per_head;
+  const int kv = bt / per_kv;
+  const int tl = bt - kv * per_kv;
+  const int hh = tl / per_head;
+  const int tt = (tl - hh * per_head) * kTileRows + i;
+  TileRow R;
+  const int base = text ? G.n_vis : 0;
+  const int count = text ? G.n_tokens - G.n_vis : G.n_vis;
+  R.valid = tt < count;
+  R.t = base + (R.valid ? tt : 0);
+  R.h = kv * G.g + hh;
+  return R;
 }
 
 // Workspace of adaspark_cube_attn. Offsets in bytes from the workspace base.
@@ -84,6 +112,7 @@ struct FfnLayout {
   size_t xa;          // dtype [n_tokens][D] gathered active rows
   size_t h;           // dtype [n_tokens][F] SwiGLU activations
   size_t sums;        // float [C][D] per-cube sums of FFN over active rows
+  size_t wd16;        // fp16 [D][F] copy of W_down (bf16 path)
   size_t total;
 };
 
@@ -101,6 +130,7 @@ __host__ __device__ inline FfnLayout make_ffn_layout(int n_tokens, int n_vis, in
   L.xa = o; o += align_up((size_t)n_tokens * D * esize, 1024);
   L.h = o; o += align_up((size_t)n_tokens * F * esize, 1024);
   L.sums = o; o += align_up((size_t)(n_cubes > 0 ? n_cubes : 1) * D * 4);
+  L.wd16 = o; o += align_up(esize == 2 ? (size_t)D * F * 2 : 0, 1024);
   L.total = o;
   return L;
 }

@@ -224,4 +224,33 @@ struct RowSel {
 };
 
 }  // namespace sel
+
+// ---------------------------------------------------------------------------
+// Shared tile epilogue: compact the cube columns with any row bit into the
+// tile's ascending list. 128 threads.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void compact_tile_list(const uint32_t* tmask, uint16_t* list, int32_t* count, int c_hi,
+                                  int* s_wcnt, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+  int total = 0;
+  for (int base = 0; base <= c_hi; base += 128) {
+    const int j = base + tid;
+    bool nz = false;
+    if (j <= c_hi) {
+      const uint4 w = __ldcg(reinterpret_cast<const uint4*>(tmask + (size_t)j * 4));
+      nz = (w.x | w.y | w.z | w.w) != 0u;
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, nz);
+    if (lane == 0) s_wcnt[warp] = __popc(bal);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int before = total;
+    for (int w = 0; w < warp; ++w) before += s_wcnt[w];
+    const int chunk_total = s_wcnt[0] + s_wcnt[1] + s_wcnt[2] + s_wcnt[3];
+    if (nz) list[before + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)j;
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    total += chunk_total;
+  }
+  if (tid == 0) *count = total;
+}
+
 }  // namespace adaspark

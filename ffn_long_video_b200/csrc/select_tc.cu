@@ -1,0 +1,271 @@
+// AdaS-Attn cube selection with tensor-core scores (bf16 path).
+//
+// Key design 2 of the AdaSpark note: for the 128 rows of a tile (128 tokens of
+// one query head), P_i = softmax_j<i(q . kbar_j / sqrt(d)), S_i = Top-p(P_i, p).
+// The scores of a tile against all preceding cubes form a dense 128 x c
+// contraction, computed on tcgen05 32 cubes at a time into TMEM. kbar is split
+// into three bf16 parts (hi + mid + lo, ~24 significant bits); the queries are
+// bf16, so every product is exact and the fp32-accumulated sum of the three
+// passes reproduces the fp32 dot product. Each row's Top-p cut is then found by
+// the two-pass histogram of select.cuh, one thread per row; the scores are
+// recomputed for pass 2 with the same MMA sequence, hence bit-identical.
+//   warp 0     TMA producer: kbar chunks [3 parts][2 halves][32 cubes][64 dims]
+//              from a 3D map over [part*hkv + kv][cube][dim] (no multicast)
+//   warp 1     TMEM allocator + tcgen05.mma issuer (M=128, N=32, K=16 x 24)
+//   warps 2-5  one thread per row: Q gather, histogram pass, cut, emission of the
+//              128-bit row masks, tile cube list.
+#include "attn_kernels.h"
+#include "select.cuh"
+
+namespace adaspark {
+namespace seltc {
+
+constexpr int NC = 32;                          // cubes per chunk (MMA N)
+constexpr int STAGES = 3;
+constexpr int SBUF = 4;                         // TMEM score buffers
+constexpr int THREADS = 192;
+constexpr int Q_BYTES = 128 * 256;
+constexpr int BOX_BYTES = NC * 128;             // 32 cubes x 64 dims bf16
+constexpr int CHUNK_BYTES = 6 * BOX_BYTES;      // 3 parts x 2 halves
+constexpr size_t SMEM_BYTES =
+    1024 + Q_BYTES + STAGES * CHUNK_BYTES + sizeof(sel::Smem) + 256;
+
+__global__ void __launch_bounds__(THREADS, 1)
+    select_tc_kernel(const __grid_constant__ CUtensorMap mapKb, SelectArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + Q_BYTES;
+  sel::Smem* ss = reinterpret_cast<sel::Smem*>(sK + STAGES * CHUNK_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ss) + sizeof(sel::Smem));
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + STAGES;
+  uint64_t* s_full = k_empty + STAGES;
+  uint64_t* s_empty = s_full + SBUF;
+  uint64_t* q_full = s_empty + SBUF;
+  uint64_t* drain = q_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ volatile int s_abort;
+  __shared__ int s_hi, s_bad, s_wcnt[4];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const AttnGeom& G = a.G;
+  WsHeader* hdr = a.hdr;
+  const int vt = blockIdx.x;
+  const int kv = vt / G.vtiles_per_kv;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int b = 0; b < SBUF; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], 128);
+    }
+    mbar_init(q_full, 128);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    s_abort = 0;
+    s_bad = status_bad(hdr) ? 1 : 0;
+    // rows are tokens in order: the last valid row holds the highest own cube
+    const TileRow last = tile_row(G, false, vt, 0);
+    const int t_hi = min(last.t + kTileRows, G.n_vis) - 1;
+    s_hi = s_bad ? -1 : a.cube_ids[t_hi];
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&mapKb);
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int c_hi = s_hi;                       // candidates of the tile: cubes < c_hi
+  const int nch = c_hi > 0 ? (c_hi + NC - 1) / NC : 0;
+  const int n_it = 2 * nch;                    // pass 1 then pass 2 over the same chunks
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      int it = 0;
+      for (; it < n_it && ok; ++it) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&k_empty[s], ((it / STAGES) & 1) ^ 1, &s_abort, hdr, 0x8100u)) {
+          ok = false;
+          break;
+        }
+        const int j0 = (it % nch) * NC;
+        uint8_t* st = sK + s * CHUNK_BYTES;
+        mbar_expect_tx(&k_full[s], CHUNK_BYTES);
+#pragma unroll
+        for (int part = 0; part < 3; ++part)
+#pragma unroll
+          for (int dc = 0; dc < 2; ++dc)
+            tma_load_3d(&mapKb, &k_full[s], st + (part * 2 + dc) * BOX_BYTES, dc * 64, j0,
+                        part * G.hkv + kv);
+      }
+      if (!ok) {
+        for (int k = 0; k < STAGES; ++k) {
+          const int jj = it - 1 - k;
+          if (jj < 0) break;
+          long long t0 = clock64();
+          while (!mbar_try_wait(&k_full[jj % STAGES], (jj / STAGES) & 1) &&
+                 clock64() - t0 < kWaitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_bf16(128, NC);
+      const uint32_t q_addr = smem_u32(sQ);
+      bool ok = n_it == 0 || mbar_wait(q_full, 0, &s_abort, hdr, 0x8200u);
+      tc_fence_after();
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it % STAGES, sb = it % SBUF;
+        if (!mbar_wait(&k_full[s], (it / STAGES) & 1, &s_abort, hdr, 0x8300u) ||
+            !mbar_wait(&s_empty[sb], ((it / SBUF) & 1) ^ 1, &s_abort, hdr, 0x8400u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + s * CHUNK_BYTES);
+        const uint32_t d = tmem_base + sb * NC;
+#pragma unroll
+        for (int part = 0; part < 3; ++part)
+#pragma unroll
+          for (int dc = 0; dc < 2; ++dc)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024);
+              const uint64_t bd =
+                  make_sdesc_sw128(k_addr + (part * 2 + dc) * BOX_BYTES + kk * 32, 16, 1024);
+              umma_bf16(d, ad, bd, idesc, (part | dc | kk) != 0 ? 1u : 0u);
+            }
+        umma_commit(&s_full[sb]);
+        umma_commit(&k_empty[s]);
+      }
+      umma_commit(drain);
+      long long t0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitCycles) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ selection rows
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;
+    const TileRow R = tile_row(G, false, vt, row);
+    const bool valid = R.valid;
+    const int t = R.t, h = R.h;
+    const int own = valid ? a.cube_ids[t] : -1;
+    {
+      const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
+      const uint4* src = reinterpret_cast<const uint4*>(Qg + ((size_t)t * G.hq + h) * 128);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sQ + (c >> 3) * 16384 + sw128_offset(row, c & 7)) = v;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(q_full);
+    }
+    if (c_hi >= 0) {
+      sel::RowSel s;
+      s.init(ss, row);
+      const int ncand = own > 0 ? own : 0;
+      const sel::Pool pool{a.pool_z, a.pool_j, G.pool_rows, G.n_cubes};
+      uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
+      const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+      int nsel = 0;
+      bool ok = true;
+      for (int it = 0; it < n_it; ++it) {
+        const int sb = it % SBUF;
+        const bool second = it >= nch;
+        if (!mbar_wait_warp(&s_full[sb], (it / SBUF) & 1, &s_abort, hdr, 0x8500u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t acc[32];
+        tmem_ld32(tmem_base + lane_base + sb * NC, acc);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s_empty[sb]);
+        const int j0 = (it % nch) * NC;
+        if (!second) {
+#pragma unroll 4
+          for (int c = 0; c < NC; ++c)
+            if (j0 + c < ncand) s.pass1(__uint_as_float(acc[c]) * a.zscale);
+          if (it == nch - 1) s.finish1(a.p);
+        } else {
+          uint32_t mine = 0u;  // mask word of column j0 + lane, this warp
+#pragma unroll 4
+          for (int c = 0; c < NC; ++c) {
+            const int j = j0 + c;
+            bool selb = false;
+            if (j < ncand) selb = s.pass2(__uint_as_float(acc[c]) * a.zscale, j, hdr, pool);
+            nsel += selb;
+            const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
+            if (lane == c) mine = w;
+          }
+          const int jl = j0 + lane;
+          if (jl < c_hi) tmask[(size_t)jl * 4 + wq] = mine;
+        }
+      }
+      if (ok) {
+        const unsigned w = __ballot_sync(0xffffffffu, own == c_hi);
+        if (lane == 0) tmask[(size_t)c_hi * 4 + wq] = w;
+        __syncwarp();
+        __threadfence_block();
+        const int m = s.resolve();
+        for (int i = 0; i < m; ++i) atomicOr(&tmask[(size_t)s.ljv(i) * 4 + wq], 1u << lane);
+        nsel += m;
+        const unsigned v_rows = __reduce_add_sync(0xffffffffu, (valid && own > 0) ? 1u : 0u);
+        const unsigned v_cand = __reduce_add_sync(0xffffffffu, (unsigned)ncand);
+        const unsigned v_sel = __reduce_add_sync(0xffffffffu, (unsigned)nsel);
+        const unsigned v_ovf = __reduce_add_sync(0xffffffffu, s.gz ? 1u : 0u);
+        if (lane == 0) {
+          atomicAdd((unsigned long long*)&hdr->stats[0], (unsigned long long)v_rows);
+          atomicAdd((unsigned long long*)&hdr->stats[1], (unsigned long long)v_cand);
+          atomicAdd((unsigned long long*)&hdr->stats[2], (unsigned long long)v_sel);
+          atomicAdd((unsigned long long*)&hdr->stats[3], (unsigned long long)v_ovf);
+        }
+      }
+      __threadfence_block();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!s_bad)
+        compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes, a.tile_count + vt, c_hi,
+                          s_wcnt, row);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 128);
+  }
+}
+
+}  // namespace seltc
+
+cudaError_t launch_select_tc(const SelectArgs& a, cudaStream_t s) {
+  const AttnGeom& G = a.G;
+  if (G.n_vtiles == 0) return cudaSuccess;
+  CUtensorMap m;
+  const uint64_t dims[3] = {(uint64_t)G.d, (uint64_t)G.n_cubes, (uint64_t)3 * G.hkv};
+  const uint64_t strides[2] = {(uint64_t)G.d * 2, (uint64_t)G.n_cubes * G.d * 2};
+  const uint32_t box[3] = {64, (uint32_t)seltc::NC, 1};
+  if (!encode_tmap_bf16(&m, a.kbar_split, 3, dims, strides, box)) return cudaErrorInvalidValue;
+  auto k = seltc::select_tc_kernel;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)seltc::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  return launch("select_tc", k, dim3(G.n_vtiles), dim3(seltc::THREADS), seltc::SMEM_BYTES, s, m, a);
+}
+
+}  // namespace adaspark

@@ -202,8 +202,9 @@ int adaspark_ffn_read_stats(const void *workspace, adaspark_ffn_stats *stats, vo
 /* ------------------------------------------------------------------------ */
 
 /* Synchronize `stream` and read the status word of a workspace of either call.
- * Returns ADASPARK_OK, or ADASPARK_EDEVICE with *detail (if not NULL) set to the
- * ADASPARK_DEV_* bits. The word is cleared by the next call on the workspace. */
+ * Returns ADASPARK_OK, or ADASPARK_EDEVICE with *detail (if not NULL) holding the
+ * ADASPARK_DEV_* bits in bits 0-7 and an internal code of the first failing
+ * check in bits 8-23. The word is cleared by the next call on the workspace. */
 int adaspark_read_device_status(const void *workspace, uint32_t *detail, void *stream);
 
 /* Per-kernel timing with CUDA events recorded on the launching stream around

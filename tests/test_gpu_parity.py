@@ -70,3 +70,32 @@ def test_repeat_runs_identical_sets(small_case):
     _, a1, _ = parity.run_ffn(small_case)
     _, a2, _ = parity.run_ffn(small_case)
     assert np.array_equal(a1, a2)
+
+
+# ------------------------------------------------------------------ full sizes
+def _sample_tokens(cfg, n, seed):
+    rng = np.random.default_rng(seed)
+    off = cfg.offsets
+    picks = set(rng.choice(cfg.n_vis, size=n, replace=False).tolist())
+    picks |= {0, off[1] - 1, off[1], cfg.n_vis - 1}          # first cube, second cube, last
+    picks |= set(range(cfg.n_vis, cfg.n_tokens, max(1, cfg.n_text // 8)))  # text rows
+    picks.add(cfg.n_tokens - 1)
+    return np.array(sorted(picks))
+
+
+@pytest.mark.parametrize("cfg_id", [2, 3])
+def test_full_size_sampled(cfg_id):
+    """The 3B-shaped 18K layer and the 7B-shaped 64K layer at full size, in the
+    launch configuration the bench times: selection sets and outputs of
+    sampled tokens (all heads) and sampled cubes against the oracle."""
+    cfg = workloads.CONFIGS[cfg_id]
+    case = parity.make_case(cfg)
+    rep = {}
+    parity.check_attn(case, tokens=_sample_tokens(cfg, 48, cfg_id), report=rep)
+    print(cfg.name, "attn", rep)
+    rng = np.random.default_rng(cfg_id)
+    cubes = np.unique(np.concatenate([[0, cfg.n_cubes - 1],
+                                      rng.choice(cfg.n_cubes, 10, replace=False)]))
+    rep = {}
+    parity.check_ffn(case, cubes=cubes, text=True, report=rep)
+    print(cfg.name, "ffn", rep)
