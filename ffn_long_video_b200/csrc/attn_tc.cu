@@ -12,29 +12,33 @@
 //              masks from global memory 32 entries at a time and feeds a
 //              64-slot shared-memory ring, far ahead of the consumers
 //   warp 0     TMA producer: K and V blocks (3D maps over [token][kv][d], no
-//              multicast), 3-stage ring
+//              multicast), 2-stage ring
 //   warp 1     TMEM allocator + tcgen05.mma issuer:
 //                S_i = Q K_i^T   (M=128, N=64, K=128; two TMEM buffers)
-//                O  += P_i V_i   (M=128, N=128, K=64; V read N-major)
+//                O  += P_i V_i   (M=128, N=128, K=64; P read from TMEM where it
+//                                 overwrote S_i, V read N-major from smem)
 //   warps 2-5  one thread per row: Q gather, masking, online softmax with lazy
-//              rescaling of O in TMEM, P (bf16) to shared memory, final 1/l.
+//              rescaling of O in TMEM, P (bf16) back into TMEM, final 1/l.
+// With P kept in tensor memory a CTA needs ~100 KB of shared memory and 256
+// TMEM columns, so two CTAs share an SM: while one runs its softmax the other
+// keeps the tensor core busy. MMAs issued by one thread execute in order, which
+// is what makes reusing the S buffer for P safe: S_{i+2} is issued after the
+// PV_i that reads P_i from the same columns.
 #include "attn_kernels.h"
 
 namespace adaspark {
 namespace fa {
 
-constexpr int STAGES = 3;
+constexpr int STAGES = 2;
 constexpr int THREADS = 224;
 constexpr int RING = 64;
 constexpr int Q_BYTES = 128 * 256;        // 128 rows x 128 dims bf16 (two 64-dim halves)
 constexpr int KV_BYTES = 4 * 8192;        // K (2 halves) + V (2 halves), 64 keys each
-constexpr int P_BYTES = 128 * 128;        // 128 rows x 64 keys bf16
 struct Desc {
   int k0, nk, j, pad;
   uint32_t mask[4];
 };
-constexpr size_t SMEM_BYTES =
-    1024 + Q_BYTES + STAGES * KV_BYTES + 2 * P_BYTES + RING * sizeof(Desc) + 2048;
+constexpr size_t SMEM_BYTES = 1024 + Q_BYTES + STAGES * KV_BYTES + RING * sizeof(Desc) + 2048;
 constexpr float kRescale = 8.0f;          // log2 headroom before O is rescaled
 
 __device__ __forceinline__ float ex2(float x) {
@@ -74,7 +78,7 @@ __device__ __forceinline__ TileInfo decode_tile(const AttnGeom& G) {
   return T;
 }
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -82,14 +86,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = sQ + Q_BYTES;
-  uint8_t* sP = sKV + STAGES * KV_BYTES;
-  Desc* ring = reinterpret_cast<Desc*>(sP + 2 * P_BYTES);
+  Desc* ring = reinterpret_cast<Desc*>(sKV + STAGES * KV_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + RING);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = kv_full + STAGES;
   uint64_t* s_full = kv_empty + STAGES;     // [2]
-  uint64_t* s_empty = s_full + 2;           // [2]
-  uint64_t* p_full = s_empty + 2;           // [2]
+  uint64_t* p_full = s_full + 2;            // [2]
   uint64_t* pv_done = p_full + 2;           // [2]
   uint64_t* q_full = pv_done + 2;
   uint64_t* drain = q_full + 1;
@@ -111,7 +113,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], 128);
       mbar_init(&p_full[b], 128);
       mbar_init(&pv_done[b], 1);
     }
@@ -257,12 +258,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const int s = blk % STAGES;
         const uint32_t v_addr = smem_u32(sKV + s * KV_BYTES + 16384);
-        const uint32_t p_addr = smem_u32(sP + pb * P_BYTES);
+        const uint32_t p_tmem = tmem_base + 128 + pb * 64;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = make_sdesc_sw128(p_addr + kk * 32, 16, 1024);
           const uint64_t bd = make_sdesc_sw128(v_addr + kk * 2048, 8192, 1024);
-          umma_bf16(tmem_base, ad, bd, idesc_o, (blk > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem_base, p_tmem + kk * 8, bd, idesc_o, (blk > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[pb]);
         umma_commit(&kv_empty[s]);
@@ -277,8 +277,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (ring[slot].nk == 0) break;
         const int s = i % STAGES;
         const int sb = i & 1;
-        if (!mbar_wait(&kv_full[s], (i / STAGES) & 1, &s_abort, hdr, 0x7400u) ||
-            !mbar_wait(&s_empty[sb], ((i >> 1) & 1) ^ 1, &s_abort, hdr, 0x7500u)) {
+        if (!mbar_wait(&kv_full[s], (i / STAGES) & 1, &s_abort, hdr, 0x7400u)) {
           ok = false;
           break;
         }
@@ -355,8 +354,6 @@ __global__ void __launch_bounds__(THREADS, 1)
         tmem_ld32(tmem_base + lane_base + 128 + sb * 64 + 32, s1);
       }
       tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&s_empty[sb]);
 
       // admitted keys [0, lim) of this row in the block
       bool row_on;
@@ -366,10 +363,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       else row_on = ((dsc.mask[wq] >> lane) & 1u) != 0u;
       int lim = row_on ? dsc.nk : 0;
       if (row_on && (T.text || dsc.j == own)) lim = min(lim, t - dsc.k0 + 1);
-      float mraw = -INFINITY;
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
       for (int u = 0; u < 64; ++u)
-        if (u < lim) mraw = fmaxf(mraw, __uint_as_float(sr[u]));
+        if (u < lim) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(sr[u]));
+      const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_new = fmaxf(m_used, mraw * scale);
       const bool want = m_new > m_used + kRescale;
       if (__any_sync(0xffffffffu, want)) {
@@ -391,42 +392,29 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int x = 0; x < 32; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * factor);
             tmem_st32(tmem_base + lane_base + c, o);
           }
-          tmem_st_wait();
         }
         l *= factor;
         if (m_new != -INFINITY) m_used = m_new;
       }
-      const int pb = i & 1;
-      if (i >= 2) {
-        if (!mbar_wait_warp(&pv_done[pb], ((i - 2) >> 1) & 1, &s_abort, hdr, 0x7800u)) {
-          ok = false;
-          break;
-        }
-      }
-      // P = 2^(s * scale - m_used) on admitted keys, bf16, 128-byte swizzled row
-      float ls0 = 0.f, ls1 = 0.f;
-      uint8_t* prow = sP + pb * P_BYTES;
+      // P = 2^(s * scale - m_used) on admitted keys, bf16 pairs written over S_i
+      float ls[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) ls[k] = 0.f;
       const float neg_m = -m_used;
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int u = c * 8 + q * 2;
-          const float p0 = (u < lim) ? ex2(fmaf(__uint_as_float(sr[u]), scale, neg_m)) : 0.f;
-          const float p1 =
-              (u + 1 < lim) ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, neg_m)) : 0.f;
-          ls0 += p0;
-          ls1 += p1;
-          pk[q] = pack_bf16x2(p0, p1);
-        }
-        *reinterpret_cast<uint4*>(prow + sw128_offset(row, c)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      for (int q = 0; q < 32; ++q) {
+        const int u = 2 * q;
+        const float p0 = (u < lim) ? ex2(fmaf(__uint_as_float(sr[u]), scale, neg_m)) : 0.f;
+        const float p1 = (u + 1 < lim) ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, neg_m)) : 0.f;
+        ls[q & 7] += p0 + p1;
+        pk[q] = pack_bf16x2(p0, p1);
       }
-      l += ls0 + ls1;
-      fence_proxy_async_smem();
+      tmem_st32(tmem_base + lane_base + 128 + sb * 64, pk);
+      tmem_st_wait();
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       tc_fence_before();
-      mbar_arrive(&p_full[pb]);
+      mbar_arrive(&p_full[sb]);
       ++i;
     }
     // final: O / l once the last PV has landed

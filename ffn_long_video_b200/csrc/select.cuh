@@ -29,6 +29,13 @@ constexpr int kNone = INT_MIN;        // row without candidates
 constexpr int kTail = INT_MIN + 1;    // the cut lies below the window
 constexpr int kRows = 128;
 
+// 2^x on the special-function unit (relative error below 2^-22).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct Smem {
   float hist[kB][kRows];
   float lz[kL][kRows];
@@ -69,7 +76,7 @@ struct RowSel {
     for (int k = 0; k < kB; ++k) sm->hist[k][tid] = 0.f;
   }
 
-  __device__ __forceinline__ void shift(int b) {
+  __device__ __noinline__ void shift(int b) {
     if (bmax == kNone) {
       bmax = b;
       return;
@@ -93,9 +100,9 @@ struct RowSel {
     const int b = __float2int_rd(z * (float)kR);
     if (b > bmax) shift(b);
     if (b > bmax - kB)
-      sm->hist[b & (kB - 1)][tid] += exp2f(z - (float)b * kInvR);
+      sm->hist[b & (kB - 1)][tid] += fast_exp2(z - (float)b * kInvR);
     else
-      tail += exp2f(z - (float)bmax * kInvR);
+      tail += fast_exp2(z - (float)bmax * kInvR);
   }
 
   __device__ void finish1(float p) {
@@ -123,7 +130,7 @@ struct RowSel {
     need = target - cum;
   }
 
-  __device__ void push(float z, int j, WsHeader* hdr, const Pool& pool) {
+  __device__ __noinline__ void push(float z, int j, WsHeader* hdr, const Pool& pool) {
     if (!gz) {
       if (n < kL) {
         sm->lz[n][tid] = z;

@@ -191,28 +191,35 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         tc_fence_after();
-        uint32_t acc[32];
-        tmem_ld32(tmem_base + lane_base + sb * NC, acc);
-        tmem_ld_wait();
+        const int j0 = (it % nch) * NC;
+        const uint32_t tcol = tmem_base + lane_base + sb * NC;
+        uint32_t mine = 0u;  // pass 2: mask word of column j0 + lane, this warp
+#pragma unroll 1
+        for (int q = 0; q < NC / 8; ++q) {
+          uint32_t acc[8];
+          tmem_ld8(tcol + q * 8, acc);
+          tmem_ld_wait();
+          if (!second) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              if (j0 + q * 8 + c < ncand) s.pass1(__uint_as_float(acc[c]) * a.zscale);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int j = j0 + q * 8 + c;
+              bool selb = false;
+              if (j < ncand) selb = s.pass2(__uint_as_float(acc[c]) * a.zscale, j, hdr, pool);
+              nsel += selb;
+              const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
+              if (lane == q * 8 + c) mine = w;
+            }
+          }
+        }
         tc_fence_before();
         mbar_arrive(&s_empty[sb]);
-        const int j0 = (it % nch) * NC;
         if (!second) {
-#pragma unroll 4
-          for (int c = 0; c < NC; ++c)
-            if (j0 + c < ncand) s.pass1(__uint_as_float(acc[c]) * a.zscale);
           if (it == nch - 1) s.finish1(a.p);
         } else {
-          uint32_t mine = 0u;  // mask word of column j0 + lane, this warp
-#pragma unroll 4
-          for (int c = 0; c < NC; ++c) {
-            const int j = j0 + c;
-            bool selb = false;
-            if (j < ncand) selb = s.pass2(__uint_as_float(acc[c]) * a.zscale, j, hdr, pool);
-            nsel += selb;
-            const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
-            if (lane == c) mine = w;
-          }
           const int jl = j0 + lane;
           if (jl < c_hi) tmask[(size_t)jl * 4 + wq] = mine;
         }
