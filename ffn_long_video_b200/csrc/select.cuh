@@ -23,7 +23,7 @@ namespace sel {
 
 constexpr int kR = 8;                 // bins per log2 unit
 constexpr float kInvR = 1.0f / kR;
-constexpr int kB = 128;               // bins in the window (16 log2 units)
+constexpr int kB = 64;                // bins in the window (8 log2 units)
 constexpr int kL = 24;                // cut-bin list entries kept in shared memory
 constexpr int kNone = INT_MIN;        // row without candidates
 constexpr int kTail = INT_MIN + 1;    // the cut lies below the window

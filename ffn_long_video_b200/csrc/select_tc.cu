@@ -11,9 +11,12 @@
 // recomputed for pass 2 with the same MMA sequence, hence bit-identical.
 //   warp 0     TMA producer: kbar chunks [3 parts][2 halves][32 cubes][64 dims]
 //              from a 3D map over [part*hkv + kv][cube][dim] (no multicast)
-//   warp 1     TMEM allocator + tcgen05.mma issuer (M=128, N=32, K=16 x 24)
-//   warps 2-5  one thread per row: Q gather, histogram pass, cut, emission of the
-//              128-bit row masks, tile cube list.
+//   warp 1     TMEM allocator + tcgen05.mma issuer (M=128, N=32, K=16 x 24),
+//              A = the query tile held in TMEM
+//   warps 2-5  one thread per row: Q gather into TMEM, histogram pass, cut,
+//              emission of the 128-bit row masks, tile cube list.
+// The query tile lives in tensor memory (64 columns) rather than shared memory,
+// so a CTA needs under 100 KB of shared memory and two CTAs share an SM.
 #include "attn_kernels.h"
 #include "select.cuh"
 
@@ -21,22 +24,21 @@ namespace adaspark {
 namespace seltc {
 
 constexpr int NC = 32;                          // cubes per chunk (MMA N)
-constexpr int STAGES = 3;
+constexpr int STAGES = 2;
 constexpr int SBUF = 4;                         // TMEM score buffers
 constexpr int THREADS = 192;
-constexpr int Q_BYTES = 128 * 256;
 constexpr int BOX_BYTES = NC * 128;             // 32 cubes x 64 dims bf16
 constexpr int CHUNK_BYTES = 6 * BOX_BYTES;      // 3 parts x 2 halves
-constexpr size_t SMEM_BYTES =
-    1024 + Q_BYTES + STAGES * CHUNK_BYTES + sizeof(sel::Smem) + 256;
+constexpr size_t SMEM_BYTES = 1024 + STAGES * CHUNK_BYTES + sizeof(sel::Smem) + 256;
+constexpr int TMEM_COLS = 256;                  // S buffers 0..127, Q tile 128..191
+constexpr int Q_COL = 128;
 
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, 2)
     select_tc_kernel(const __grid_constant__ CUtensorMap mapKb, SelectArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + Q_BYTES;
+  uint8_t* sK = smem;
   sel::Smem* ss = reinterpret_cast<sel::Smem*>(sK + STAGES * CHUNK_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(ss) + sizeof(sel::Smem));
   uint64_t* k_full = bars;
@@ -76,7 +78,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&mapKb);
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 128);
+    tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc_bf16(128, NC);
-      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t q_tmem = tmem_base + Q_COL;
       bool ok = n_it == 0 || mbar_wait(q_full, 0, &s_abort, hdr, 0x8200u);
       tc_fence_after();
       for (int it = 0; it < n_it && ok; ++it) {
@@ -142,10 +144,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int dc = 0; dc < 2; ++dc)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024);
               const uint64_t bd =
                   make_sdesc_sw128(k_addr + (part * 2 + dc) * BOX_BYTES + kk * 32, 16, 1024);
-              umma_bf16(d, ad, bd, idesc, (part | dc | kk) != 0 ? 1u : 0u);
+              umma_bf16_ts(d, q_tmem + dc * 32 + kk * 8, bd, idesc, (part | dc | kk) != 0 ? 1u : 0u);
             }
         umma_commit(&s_full[sb]);
         umma_commit(&k_empty[s]);
@@ -164,14 +165,25 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int t = R.t, h = R.h;
     const int own = valid ? a.cube_ids[t] : -1;
     {
+      // query row -> 64 TMEM columns of this row's lane (two bf16 per column)
       const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
       const uint4* src = reinterpret_cast<const uint4*>(Qg + ((size_t)t * G.hq + h) * 128);
+      const uint32_t qlane = tmem_base + ((uint32_t)(wq * 32) << 16) + Q_COL;
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(sQ + (c >> 3) * 16384 + sw128_offset(row, c & 7)) = v;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = valid ? src[half * 8 + c] : make_uint4(0, 0, 0, 0);
+          r[4 * c] = v.x;
+          r[4 * c + 1] = v.y;
+          r[4 * c + 2] = v.z;
+          r[4 * c + 3] = v.w;
+        }
+        tmem_st32(qlane + half * 32, r);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       mbar_arrive(q_full);
     }
     if (c_hi >= 0) {
@@ -254,7 +266,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 128);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
