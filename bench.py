@@ -130,9 +130,13 @@ def kernel_work(name, cfg, attn_stats, ffn_stats):
     if name.startswith("attn_tc"):
         # QK^T + PV per executed (128-row tile, 64-key block)
         return 4.0 * 128 * 64 * cfg.d * attn_stats["key_blocks"], "flop", "tensor"
+    if name.startswith("select_tc"):
+        # executed score MMAs: 3 bf16 parts of kbar x 2 passes x 2*d per (row, cube) pair
+        return 12.0 * cfg.d * attn_stats["candidate_pairs"], "flop", "tensor"
     if name.startswith("select"):
-        # score dot products (2*d flop) per (row, preceding cube) pair
-        return 2.0 * cfg.d * attn_stats["candidate_pairs"], "flop", "tensor"
+        return 2.0 * cfg.d * attn_stats["candidate_pairs"], "flop", "alu"
+    if name == "wdown_to_fp16":
+        return float(cfg.D) * cfg.F * 4, "byte", "hbm"
     if name == "ffn_select":
         return float(cfg.n_vis) * cfg.D * 2, "byte", "hbm"
     if name == "ffn_compact":
