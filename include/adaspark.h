@@ -151,6 +151,35 @@ int adaspark_attn_export_sets(const void *workspace, const int32_t *cube_ids, in
  * Synchronizes `stream`. */
 int adaspark_attn_read_stats(const void *workspace, adaspark_attn_stats *stats, void *stream);
 
+/* Allocation-free AdaS-Attn. (The AdaSpark pages have no counterpart: this is
+ * a calling convenience of this library.)
+ *
+ * For callers that cannot allocate device memory where they run the layer --
+ * e.g. a plugin that its host framework gives only input and output buffers, a
+ * serving loop that must not allocate (allocation may synchronize the device
+ * or fragment a fixed budget), or a process whose device memory belongs to
+ * another allocator. Same computation, arguments and errors as
+ * adaspark_cube_attn, without the workspace: the kernels use a fixed array of
+ * ADASPARK_NOALLOC_SCRATCH_BYTES that the library keeps in device memory on
+ * every GPU where its device code is loaded, until the process exits.
+ *   - Returns ADASPARK_EINVAL when the sizes are invalid or when
+ *     adaspark_cube_attn_workspace() for them exceeds
+ *     ADASPARK_NOALLOC_SCRATCH_BYTES (check that first).
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any stream
+ *     capture.
+ *   - Calls no cudaMalloc / cudaFree and no allocating routine.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents: calls whose kernels may overlap on the GPU (different streams
+ *     without ordering between them) race and give wrong results; serialize
+ *     them. adaspark_attn_export_sets / adaspark_attn_read_stats cannot read
+ *     this array (use adaspark_cube_attn for those). */
+#define ADASPARK_NOALLOC_SCRATCH_BYTES (32u << 20)
+int adaspark_cube_attn_noalloc(const void *Q, const void *K, const void *V, int dtype,
+                               const int32_t *cube_ids, const int32_t *cube_offsets,
+                               int n_cubes, int n_vis, int n_tokens, int hq, int hkv, int d,
+                               float p, void *out, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Key design 3: AdaS-FFN with mean compensation.                           */
 /* ------------------------------------------------------------------------ */
