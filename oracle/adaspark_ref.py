@@ -287,8 +287,7 @@ def ffn_select(x, cube_offsets, n_vis, p, cubes=None, with_margin=False):
     tokens are always active.  Returns a boolean ``active`` [N] (entries of
     cubes not in ``cubes`` are left False) and, when asked, per-cube margins."""
     _check_p(p)
-    X = _f64(x)
-    N = X.shape[0]
+    N = x.shape[0]
     off = np.asarray(cube_offsets)
     C = len(off) - 1
     active = np.zeros(N, dtype=bool)
@@ -298,7 +297,8 @@ def ffn_select(x, cube_offsets, n_vis, p, cubes=None, with_margin=False):
         cubes = range(C)
     for c in cubes:
         a, b = off[c], off[c + 1]
-        norms = np.sqrt(np.sum(X[a:b] * X[a:b], axis=1))
+        Xc = _f64(x[a:b])
+        norms = np.sqrt(np.sum(Xc * Xc, axis=1))
         total = norms.sum()
         if total == 0.0:
             active[a:b] = True
@@ -328,25 +328,25 @@ def ffn_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active, cubes=N
     m_bar_i = mean of FFN(x_j) over the cube's active tokens.  Returns float64
     y [N, D] (rows of cubes outside ``cubes`` are NaN; text rows NaN when
     ``text`` is False)."""
-    X = _f64(x)
-    N, D = X.shape
+    N, D = x.shape
     off = np.asarray(cube_offsets)
     C = len(off) - 1
     y = np.full((N, D), np.nan)
+    Wg, Wu, Wd = _f64(W_gate), _f64(W_up), _f64(W_down)
     if cubes is None:
         cubes = range(C)
     for c in cubes:
         a, b = off[c], off[c + 1]
-        idx = np.arange(a, b)
-        act = idx[active[a:b]]
-        skip = idx[~active[a:b]]
-        f = swiglu_ffn(X[act], W_gate, W_up, W_down)
-        y[act] = X[act] + f
-        if len(skip):
-            mbar = f.sum(axis=0) / len(act)
-            y[skip] = X[skip] + mbar
+        Xc = _f64(x[a:b])
+        act = active[a:b]
+        f = swiglu_ffn(Xc[act], Wg, Wu, Wd)
+        y[a:b][act] = Xc[act] + f
+        if (~act).any():
+            mbar = f.sum(axis=0) / int(act.sum())
+            y[a:b][~act] = Xc[~act] + mbar
     if text and N > n_vis:
-        y[n_vis:] = X[n_vis:] + swiglu_ffn(X[n_vis:], W_gate, W_up, W_down)
+        Xt = _f64(x[n_vis:])
+        y[n_vis:] = Xt + swiglu_ffn(Xt, Wg, Wu, Wd)
     return y
 
 

@@ -99,3 +99,56 @@ def test_full_size_sampled(cfg_id):
     rep = {}
     parity.check_ffn(case, cubes=cubes, text=True, report=rep)
     print(cfg.name, "ffn", rep)
+
+
+@pytest.mark.parametrize("shape", [(4, 4, 4), (8, 8, 2)])
+def test_128k_sweep_sampled(shape):
+    """The 7B-shaped 128K layer: p in {0.5, 0.7, 0.9, 1.0} on both cube shapes
+    (64-token and 128-token cubes), sampled tokens and cubes."""
+    idxs = [i for i, (p, c) in enumerate(workloads.SWEEP_4) if c == shape]
+    cfg0 = workloads.sweep_config(idxs[0])
+    case = parity.make_case(cfg0)
+    for i in idxs:
+        cfg = workloads.sweep_config(i)
+        case["cfg"] = cfg
+        rep = {}
+        parity.check_attn(case, p=cfg.p, tokens=_sample_tokens(cfg, 24, i), report=rep)
+        print(cfg.name, "attn", rep)
+        rng = np.random.default_rng(i)
+        cubes = np.unique(np.concatenate([[0, cfg.n_cubes - 1],
+                                          rng.choice(cfg.n_cubes, 6, replace=False)]))
+        rep = {}
+        parity.check_ffn(case, p=cfg.p, cubes=cubes, text=(cfg.p == 0.7), report=rep)
+        print(cfg.name, "ffn", rep)
+
+
+def test_262k_four_layer_stack_sampled():
+    """Four independently seeded 7B-shaped layers at 262K visual tokens, half of
+    the cubes near-duplicates of earlier ones. The harness wires the stack
+    (Q/K/V = x W, h = x + out W_o, next x = y); each layer's AdaS-Attn and
+    AdaS-FFN are checked against the oracle on that layer's own inputs."""
+    cfg = workloads.CONFIGS[5]
+    ids, off, text, off_np = parity.layout_tensors(cfg)
+    x = None
+    for layer in range(cfg.n_layers):
+        w = {k: v.cuda() for k, v in workloads.make_stack(cfg, layer).items()}
+        if layer == 0:
+            x = w.pop("x")
+        qkv = workloads.project_qkv(cfg, x, w["W_q"], w["W_k"], w["W_v"], project_on="cuda")
+        t = {k: v.cuda() for k, v in qkv.items()}
+        case = {"cfg": cfg, "t": dict(t), "ids": ids, "off": off, "text": text, "off_np": off_np}
+        rep = {}
+        out, _, _ = parity.check_attn(case, tokens=_sample_tokens(cfg, 16, 50 + layer), report=rep)
+        print(cfg.name, "layer", layer, "attn", rep)
+        h = (x.float() + (out.reshape(cfg.n_tokens, -1).float() @ w["W_o"].float())).to(x.dtype)
+        del out
+        case["t"] = {"x": h, "W_gate": w["W_gate"], "W_up": w["W_up"], "W_down": w["W_down"]}
+        rng = np.random.default_rng(60 + layer)
+        cubes = np.unique(np.concatenate([[0, cfg.n_cubes - 1],
+                                          rng.choice(cfg.n_cubes, 4, replace=False)]))
+        rep = {}
+        y, _, _ = parity.check_ffn(case, cubes=cubes, text=(layer == 0), report=rep)
+        print(cfg.name, "layer", layer, "ffn", rep)
+        x = y.to(x.dtype)
+        del y, h, t, qkv, w
+        torch.cuda.empty_cache()

@@ -120,13 +120,15 @@ CONFIGS = {
             structure="near_dup", n_layers=4),
 }
 
-# The sweep of the 128K workload: p values x cube shapes.
+# The sweep of the 128K workload: p values x cube shapes. The inputs depend on
+# the cube shape only (seed + 100 * shape index), so the p sweep reuses them.
 SWEEP_4 = [(p, cube) for cube in ((4, 4, 4), (8, 8, 2)) for p in (0.5, 0.7, 0.9, 1.0)]
 
 
 def sweep_config(idx: int) -> LayerConfig:
     p, cube = SWEEP_4[idx]
-    return dataclasses.replace(CONFIGS[4], p=p, cube=cube, seed=BASE_SEED + 4 + 100 * idx,
+    shape = 0 if cube == (4, 4, 4) else 1
+    return dataclasses.replace(CONFIGS[4], p=p, cube=cube, seed=BASE_SEED + 4 + 100 * shape,
                                name=f"qwen2.5-vl-7b-128k-p{p}-{cube[0]}x{cube[1]}x{cube[2]}")
 
 
@@ -219,6 +221,20 @@ def make_layer(cfg: LayerConfig, layer: int = 0, device=None, project_on=None) -
     out.update(project_qkv(cfg, out["x"], out["W_q"], out["W_k"], out["W_v"], project_on))
     if device is not None:
         out = {k: v.to(device) for k, v in out.items()}
+    return out
+
+
+def make_stack(cfg: LayerConfig, layer: int) -> dict:
+    """Stacked workload (several independent layers): the first layer draws the
+    hidden state then its weights from its own stream; later layers draw only
+    their weights (W_q, W_k, W_v, W_gate, W_up, W_down, W_o) from theirs.
+    Returns rounded torch CPU tensors ("x" only for layer 0)."""
+    rng = layer_rng(cfg, layer)
+    out = {}
+    if layer == 0:
+        out["x"] = _round(make_hidden(cfg, rng), cfg.dtype)
+    for k, v in make_weights(cfg, rng, with_o=True).items():
+        out[k] = _round(v, cfg.dtype)
     return out
 
 
