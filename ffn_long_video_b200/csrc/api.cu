@@ -90,8 +90,6 @@ int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
   sa.tile_mask = reinterpret_cast<uint32_t*>(ws + L.tile_mask);
   sa.tile_list = reinterpret_cast<uint16_t*>(ws + L.tile_list);
   sa.tile_count = reinterpret_cast<int32_t*>(ws + L.tile_count);
-  sa.pool_z = reinterpret_cast<float*>(ws + L.pool);
-  sa.pool_j = reinterpret_cast<int32_t*>(ws + L.pool + (size_t)G.pool_rows * G.n_cubes * 4);
   sa.hdr = hdr;
   sa.G = G;
   sa.p = p;

@@ -16,8 +16,6 @@ struct SelectArgs {
   uint32_t* tile_mask;                // [n_vtiles][C][4]
   uint16_t* tile_list;                // [n_vtiles][C]
   int32_t* tile_count;                // [n_vtiles]
-  float* pool_z;
-  int32_t* pool_j;
   WsHeader* hdr;
   AttnGeom G;
   float p;

@@ -113,12 +113,13 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
   sel::RowSel s;
   s.init(ss, tid);
   const int ncand = own > 0 ? own : 0;
-  const sel::Pool pool{a.pool_z, a.pool_j, G.pool_rows, G.n_cubes};
   const float* kb = a.kbar + (size_t)kv * G.n_cubes * D;
+  uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
+  __shared__ int s_more;
+  int nsel = 0, extra = 0;
 
-  for (int pass = 0; pass < 2; ++pass) {
-    uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
-    int nsel = 0;
+  // pass 0: histogram; pass 1: emission; pass >= 2: rows whose cut is still open
+  for (int pass = 0;; ++pass) {
     for (int j0 = 0; j0 < c_hi; j0 += 64) {
       const int nj = min(64, c_hi - j0);
       __syncthreads();
@@ -127,16 +128,15 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
       for (int jj = 0; jj < nj; ++jj) {
         const int j = j0 + jj;
         bool selb = false;
-        if (j < ncand) {
+        if (j < ncand && (pass < 2 || s.open)) {
           const float* kr = kch + jj * D;
           float acc = 0.f;
 #pragma unroll
           for (int e = 0; e < D; ++e) acc = fmaf(q[e], kr[e], acc);
           const float z = acc * a.zscale;
-          if (pass == 0)
-            s.pass1(z);
-          else
-            selb = s.pass2(z, j, a.hdr, pool);
+          if (pass == 0) s.pass1(z);
+          else if (pass == 1) selb = s.pass2(z, j);
+          else s.pass_more(z, j);
         }
         if (pass == 1) {
           const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
@@ -147,30 +147,40 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
     }
     if (pass == 0) {
       s.finish1(a.p);
-    } else {
+      continue;
+    }
+    if (pass == 1) {
       const unsigned w = __ballot_sync(0xffffffffu, own == c_hi);
       if (lane == 0) tmask[(size_t)c_hi * 4 + warp] = w;
       __syncwarp();
-      const int m = s.resolve();
-      for (int i = 0; i < m; ++i) atomicOr(&tmask[(size_t)s.ljv(i) * 4 + warp], 1u << lane);
-      nsel += m;
-      // statistics
-      const float rows_f = (valid && own > 0) ? 1.f : 0.f;
-      unsigned long long v_rows = __reduce_add_sync(0xffffffffu, (unsigned)rows_f);
-      unsigned long long v_cand = __reduce_add_sync(0xffffffffu, (unsigned)ncand);
-      unsigned long long v_sel = __reduce_add_sync(0xffffffffu, (unsigned)nsel);
-      unsigned long long v_ovf = __reduce_add_sync(0xffffffffu, s.gz ? 1u : 0u);
-      if (lane == 0) {
-        atomicAdd((unsigned long long*)&a.hdr->stats[0], v_rows);
-        atomicAdd((unsigned long long*)&a.hdr->stats[1], v_cand);
-        atomicAdd((unsigned long long*)&a.hdr->stats[2], v_sel);
-        atomicAdd((unsigned long long*)&a.hdr->stats[3], v_ovf);
-      }
-      __syncthreads();
-      compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes, a.tile_count + vt, c_hi,
-                        s_wcnt, tid);
     }
+    const bool was_open = s.open;
+    const int m = s.settle();
+    for (int i = 0; i < m; ++i) atomicOr(&tmask[(size_t)s.list_j(i) * 4 + warp], 1u << lane);
+    nsel += m;
+    s.reset_list();
+    if (pass >= 1 && was_open && s.open) extra = 1;
+    if (tid == 0) s_more = 0;
+    __syncthreads();
+    if (s.open) s_more = 1;
+    __syncthreads();
+    if (!s_more) break;
   }
+  // statistics
+  const unsigned v_rows = __reduce_add_sync(0xffffffffu, (valid && own > 0) ? 1u : 0u);
+  const unsigned v_cand = __reduce_add_sync(0xffffffffu, (unsigned)ncand);
+  const unsigned v_sel = __reduce_add_sync(0xffffffffu, (unsigned)nsel);
+  const unsigned v_ext = __reduce_add_sync(0xffffffffu, (unsigned)extra);
+  if (lane == 0) {
+    atomicAdd((unsigned long long*)&a.hdr->stats[0], (unsigned long long)v_rows);
+    atomicAdd((unsigned long long*)&a.hdr->stats[1], (unsigned long long)v_cand);
+    atomicAdd((unsigned long long*)&a.hdr->stats[2], (unsigned long long)v_sel);
+    atomicAdd((unsigned long long*)&a.hdr->stats[3], (unsigned long long)v_ext);
+  }
+  __threadfence_block();
+  __syncthreads();
+  compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes, a.tile_count + vt, c_hi, s_wcnt,
+                    tid);
 }
 
 // ---------------------------------------------------------------------------

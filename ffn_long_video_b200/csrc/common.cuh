@@ -17,7 +17,7 @@ namespace adaspark {
 struct WsHeader {
   uint32_t status;        // ADASPARK_DEV_* bits, cleared at the start of a call
   uint32_t detail;        // first failing check (debug aid)
-  uint32_t pool_next;     // overflow-pool slot counter (selection)
+  uint32_t spare0;
   uint32_t m_active;      // FFN: number of active rows (visual + text)
   uint32_t sched[4];      // persistent-kernel tile counters
   uint64_t stats[16];     // adaspark_attn_stats / adaspark_ffn_stats

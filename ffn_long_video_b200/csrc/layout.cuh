@@ -24,7 +24,6 @@ struct AttnGeom {
   int vtiles_per_head, ttiles_per_head;  // 128-token tiles per query head
   int vtiles_per_kv, ttiles_per_kv;      // tiles per KV head
   int n_vtiles, n_ttiles;
-  int pool_rows;                         // overflow-pool capacity (rows)
 };
 
 __host__ __device__ inline AttnGeom make_attn_geom(int n_tokens, int n_vis, int n_cubes, int hq,
@@ -43,12 +42,6 @@ __host__ __device__ inline AttnGeom make_attn_geom(int n_tokens, int n_vis, int 
   G.ttiles_per_kv = G.ttiles_per_head * G.g;
   G.n_vtiles = G.vtiles_per_kv * hkv;
   G.n_ttiles = G.ttiles_per_kv * hkv;
-  long long rows = (long long)n_vis * hq;
-  long long pr = rows / 8;
-  if (pr < 4096) pr = 4096;
-  if (pr > 65536) pr = 65536;
-  if (pr > rows) pr = rows > 0 ? rows : 1;
-  G.pool_rows = (int)pr;
   return G;
 }
 
@@ -82,7 +75,6 @@ struct AttnLayout {
   size_t tile_count;  // int32 [n_vtiles]
   size_t tile_list;   // uint16 [n_vtiles][C]  cube ids with any row bit, ascending
   size_t tile_mask;   // uint32 [n_vtiles][C][4]  128 row bits per (tile, cube)
-  size_t pool;        // overflow pool: [pool_rows][C] x (float z, int32 j)
   size_t total;
 };
 
@@ -95,7 +87,6 @@ __host__ __device__ inline AttnLayout make_attn_layout(const AttnGeom& G) {
   L.tile_count = o; o += align_up((size_t)G.n_vtiles * 4);
   L.tile_list = o; o += align_up((size_t)G.n_vtiles * G.n_cubes * 2);
   L.tile_mask = o; o += align_up((size_t)G.n_vtiles * G.n_cubes * 16);
-  L.pool = o; o += align_up((size_t)G.pool_rows * G.n_cubes * 8);
   L.total = o;
   return L;
 }

@@ -55,7 +55,7 @@ extern "C" int adaspark_cube_attn_noalloc(const void* Q, const void* K, const vo
   const int rc = scratch_on_current_device(&scratch);
   if (rc != ADASPARK_OK) return rc;
   // adaspark_cube_attn clears the parts of the workspace that must start at
-  // zero (status word, pool counter, counters) at the start of every call.
+  // zero (status word and counters) at the start of every call.
   return adaspark_cube_attn(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq,
                             hkv, d, p, out, scratch, (size_t)ADASPARK_NOALLOC_SCRATCH_BYTES,
                             stream);

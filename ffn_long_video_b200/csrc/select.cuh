@@ -1,17 +1,24 @@
 // Sort-free Top-p cut of one row of cube scores (AdaS-Attn key design 2:
-// S_i = {j | p_j in Top-p(P_i, p)}), one thread per row, in two streaming passes
-// over the scores (which the caller recomputes bit-identically in pass 2).
+// S_i = {j | p_j in Top-p(P_i, p)}), one thread per row, in streaming passes
+// over the scores (which the caller recomputes bit-identically every pass).
 //
 // Scores enter in log2 units, z_j = (q . kbar_j) * log2(e) / sqrt(d), so that
-// P_j is proportional to 2^z_j. Pass 1 keeps a mass histogram of 2^z over bins
-// of width 1/kR log2-units, in a window of kB bins below the running maximum
-// (older bins fold into a tail scalar when the maximum moves up). After pass 1
-// the bin holding the cut is known: walking down from the top, it is the first
-// bin at which the cumulative mass reaches p * Z. Pass 2 marks every element of
-// a higher bin as selected and collects the elements of the cut bin; sorting
-// that short list by (z descending, index ascending) gives the exact cut.
+// P_j is proportional to 2^z_j. The order is (z descending, index ascending).
+//  pass 1  mass histogram of 2^z over bins of width 1/kR log2-units, in a window
+//          of kB bins below the running maximum (older bins fold into a tail
+//          scalar when the maximum moves up). Walking down from the top, the
+//          cut bin is the first at which the cumulative mass reaches p * Z.
+//  pass 2  every element of a higher bin is selected outright; the elements of
+//          the cut bin are offered to a per-row top-kL list kept sorted in the
+//          (z desc, index asc) order. Walking that list until the cumulative
+//          mass reaches p * Z ends the cut.
+//  more    if the cut lies beyond the kL best elements of the cut bin, those
+//          kL are selected, the required mass is reduced by theirs, and another
+//          pass collects the next kL below the last key; repeated until the cut
+//          is found (bounded by the size of the cut bin).
 // This reproduces "smallest prefix of the (P desc, index asc) order whose
-// cumulative mass reaches p" up to fp32 rounding of the masses.
+// cumulative mass reaches p" up to fp32 rounding of the masses, for any score
+// distribution (ties included), without memory beyond the per-row list.
 #pragma once
 
 #include <limits.h>
@@ -24,7 +31,7 @@ namespace sel {
 constexpr int kR = 8;                 // bins per log2 unit
 constexpr float kInvR = 1.0f / kR;
 constexpr int kB = 64;                // bins in the window (8 log2 units)
-constexpr int kL = 24;                // cut-bin list entries kept in shared memory
+constexpr int kL = 24;                // list entries per row (shared memory)
 constexpr int kNone = INT_MIN;        // row without candidates
 constexpr int kTail = INT_MIN + 1;    // the cut lies below the window
 constexpr int kRows = 128;
@@ -36,17 +43,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// (z1, j1) comes before (z2, j2) in the (z desc, index asc) order.
+__device__ __forceinline__ bool before(float z1, int j1, float z2, int j2) {
+  return z1 > z2 || (z1 == z2 && j1 < j2);
+}
+
 struct Smem {
   float hist[kB][kRows];
   float lz[kL][kRows];
   uint16_t lj[kL][kRows];
-};
-
-struct Pool {
-  float* z;        // [rows][C]
-  int32_t* j;      // [rows][C]
-  int rows;
-  int C;
 };
 
 struct RowSel {
@@ -56,10 +61,11 @@ struct RowSel {
   float tail;
   int bstar;
   float need;
-  int n;
-  float* gz;
-  int32_t* gj;
-  bool lost;
+  int n;          // list entries
+  bool open;      // cut not found yet
+  bool bounded;   // only keys after (bz, bj) are offered (extra passes)
+  float bz;
+  int bj;
 
   __device__ void init(Smem* s, int t) {
     sm = s;
@@ -69,9 +75,10 @@ struct RowSel {
     bstar = kNone;
     need = 0.f;
     n = 0;
-    gz = nullptr;
-    gj = nullptr;
-    lost = false;
+    open = false;
+    bounded = false;
+    bz = 0.f;
+    bj = 0;
 #pragma unroll 8
     for (int k = 0; k < kB; ++k) sm->hist[k][tid] = 0.f;
   }
@@ -108,6 +115,7 @@ struct RowSel {
   __device__ void finish1(float p) {
     if (bmax == kNone) {
       bstar = kNone;
+      open = false;
       return;
     }
     float Z = tail;
@@ -128,106 +136,76 @@ struct RowSel {
       cum += m;
     }
     need = target - cum;
+    open = true;
   }
 
-  __device__ __noinline__ void push(float z, int j, WsHeader* hdr, const Pool& pool) {
-    if (!gz) {
-      if (n < kL) {
-        sm->lz[n][tid] = z;
-        sm->lj[n][tid] = (uint16_t)j;
-        ++n;
-        return;
-      }
-      const unsigned slot = atomicAdd(&hdr->pool_next, 1u);
-      if (slot >= (unsigned)pool.rows) {
-        if (!lost) set_status(hdr, ADASPARK_DEV_POOL_FULL, 0x5000u);
-        lost = true;
-        return;
-      }
-      gz = pool.z + (size_t)slot * pool.C;
-      gj = pool.j + (size_t)slot * pool.C;
-      for (int i = 0; i < n; ++i) {
-        gz[i] = sm->lz[i][tid];
-        gj[i] = sm->lj[i][tid];
-      }
-    }
-    if (n < pool.C) {
-      gz[n] = z;
-      gj[n] = j;
-      ++n;
-    }
-  }
-
-  // Returns true when z lies above the cut bin (selected outright); pushes the
-  // elements of the cut bin to the list.
-  __device__ __forceinline__ bool pass2(float z, int j, WsHeader* hdr, const Pool& pool) {
-    const int b = __float2int_rd(z * (float)kR);
-    bool above, cand;
-    if (bstar == kTail) {
-      above = b > bmax - kB;
-      cand = !above;
+  // Insert into the sorted top-kL list (keys after the bound only).
+  __device__ __noinline__ void offer(float z, int j) {
+    if (bounded && !before(bz, bj, z, j)) return;
+    int pos;
+    if (n == kL) {
+      if (!before(z, j, sm->lz[kL - 1][tid], (int)sm->lj[kL - 1][tid])) return;
+      pos = kL - 1;
     } else {
-      above = b > bstar;
-      cand = (b == bstar);
+      pos = n++;
     }
-    if (cand) push(z, j, hdr, pool);
+    while (pos > 0 && before(z, j, sm->lz[pos - 1][tid], (int)sm->lj[pos - 1][tid])) {
+      sm->lz[pos][tid] = sm->lz[pos - 1][tid];
+      sm->lj[pos][tid] = sm->lj[pos - 1][tid];
+      --pos;
+    }
+    sm->lz[pos][tid] = z;
+    sm->lj[pos][tid] = (uint16_t)j;
+  }
+
+  __device__ __forceinline__ bool in_cut_bin(int b) const {
+    return bstar == kTail ? b <= bmax - kB : b == bstar;
+  }
+
+  // Emission pass: true when z lies above the cut bin (selected outright);
+  // elements of the cut bin go to the list.
+  __device__ __forceinline__ bool pass2(float z, int j) {
+    const int b = __float2int_rd(z * (float)kR);
+    const bool above = bstar == kTail ? b > bmax - kB : b > bstar;
+    if (open && in_cut_bin(b)) offer(z, j);
     return above;
   }
 
-  __device__ __forceinline__ float lzv(int i) const { return gz ? gz[i] : sm->lz[i][tid]; }
-  __device__ __forceinline__ int ljv(int i) const { return gz ? gj[i] : (int)sm->lj[i][tid]; }
-  __device__ __forceinline__ void lset(int i, float z, int j) {
-    if (gz) {
-      gz[i] = z;
-      gj[i] = j;
-    } else {
-      sm->lz[i][tid] = z;
-      sm->lj[i][tid] = (uint16_t)j;
-    }
+  // Extra pass for a row whose cut is still open.
+  __device__ __forceinline__ void pass_more(float z, int j) {
+    if (!open) return;
+    const int b = __float2int_rd(z * (float)kR);
+    if (in_cut_bin(b)) offer(z, j);
   }
 
-  // Sort the cut-bin list by (z desc, j asc) and return how many of its leading
-  // entries complete the Top-p set.
-  __device__ int resolve() {
-    if (bstar == kNone || n == 0) return 0;
-    if (!gz) {
-      for (int i = 1; i < n; ++i) {  // insertion sort (stable; entries arrive in j order)
-        const float z = sm->lz[i][tid];
-        const uint16_t j = sm->lj[i][tid];
-        int k = i - 1;
-        while (k >= 0 && sm->lz[k][tid] < z) {
-          sm->lz[k + 1][tid] = sm->lz[k][tid];
-          sm->lj[k + 1][tid] = sm->lj[k][tid];
-          --k;
-        }
-        sm->lz[k + 1][tid] = z;
-        sm->lj[k + 1][tid] = j;
-      }
-    } else {
-      // shell sort on the full key (not stable, so the index breaks ties)
-      for (int gap = n / 2; gap > 0; gap /= 2) {
-        for (int i = gap; i < n; ++i) {
-          const float z = gz[i];
-          const int j = gj[i];
-          int k = i;
-          while (k >= gap && (gz[k - gap] < z || (gz[k - gap] == z && gj[k - gap] > j))) {
-            gz[k] = gz[k - gap];
-            gj[k] = gj[k - gap];
-            k -= gap;
-          }
-          gz[k] = z;
-          gj[k] = j;
-        }
-      }
-    }
+  // After a pass over the cut bin: how many leading list entries are selected.
+  // Closes the cut when reached (or when the bin is exhausted); otherwise all
+  // kL entries are taken and the next pass starts after the last of them.
+  __device__ int settle() {
+    if (!open) return 0;
     const float ref = (float)bmax * kInvR;
     float cum = 0.f;
     for (int i = 0; i < n; ++i) {
-      cum += exp2f(lzv(i) - ref);
-      if (cum >= need) return i + 1;
+      cum += fast_exp2(sm->lz[i][tid] - ref);
+      if (cum >= need) {
+        open = false;
+        return i + 1;
+      }
     }
-    return n;
+    const int m = n;
+    if (n < kL) {  // the whole cut bin was offered: rounding left need unmet
+      open = false;
+      return m;
+    }
+    need -= cum;
+    bounded = true;
+    bz = sm->lz[kL - 1][tid];
+    bj = (int)sm->lj[kL - 1][tid];
+    return m;
   }
+
+  __device__ __forceinline__ int list_j(int i) const { return (int)sm->lj[i][tid]; }
+  __device__ __forceinline__ void reset_list() { n = 0; }
 };
 
 }  // namespace sel
@@ -236,8 +214,8 @@ struct RowSel {
 // Shared tile epilogue: compact the cube columns with any row bit into the
 // tile's ascending list. 128 threads.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void compact_tile_list(const uint32_t* tmask, uint16_t* list, int32_t* count, int c_hi,
-                                  int* s_wcnt, int tid) {
+__device__ __forceinline__ void compact_tile_list(const uint32_t* tmask, uint16_t* list,
+                                                  int32_t* count, int c_hi, int* s_wcnt, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
   int total = 0;
   for (int base = 0; base <= c_hi; base += 128) {

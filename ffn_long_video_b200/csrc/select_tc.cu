@@ -7,8 +7,11 @@
 // into three bf16 parts (hi + mid + lo, ~24 significant bits); the queries are
 // bf16, so every product is exact and the fp32-accumulated sum of the three
 // passes reproduces the fp32 dot product. Each row's Top-p cut is then found by
-// the two-pass histogram of select.cuh, one thread per row; the scores are
-// recomputed for pass 2 with the same MMA sequence, hence bit-identical.
+// the streaming histogram cut of select.cuh, one thread per row; the scores are
+// recomputed for every pass with the same MMA sequence, hence bit-identical.
+// Passes: histogram, emission, then (only while some row's cut is still open)
+// extra passes; after each pass from the emission on, the row threads vote and
+// the producer and MMA warps read the vote through a per-round barrier.
 //   warp 0     TMA producer: kbar chunks [3 parts][2 halves][32 cubes][64 dims]
 //              from a 3D map over [part*hkv + kv][cube][dim] (no multicast)
 //   warp 1     TMEM allocator + tcgen05.mma issuer (M=128, N=32, K=16 x 24),
@@ -47,9 +50,11 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* s_empty = s_full + SBUF;
   uint64_t* q_full = s_empty + SBUF;
   uint64_t* drain = q_full + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* decide = drain + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(decide + 1);
   __shared__ volatile int s_abort;
   __shared__ int s_hi, s_bad, s_wcnt[4];
+  __shared__ volatile int s_more[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const AttnGeom& G = a.G;
@@ -68,8 +73,11 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     mbar_init(q_full, 128);
     mbar_init(drain, 1);
+    mbar_init(decide, 128);
     fence_mbar_init();
     s_abort = 0;
+    s_more[0] = 0;
+    s_more[1] = 0;
     s_bad = status_bad(hdr) ? 1 : 0;
     // rows are tokens in order: the last valid row holds the highest own cube
     const TileRow last = tile_row(G, false, vt, 0);
@@ -87,28 +95,32 @@ __global__ void __launch_bounds__(THREADS, 2)
   const uint32_t tmem_base = *tmem_holder;
   const int c_hi = s_hi;                       // candidates of the tile: cubes < c_hi
   const int nch = c_hi > 0 ? (c_hi + NC - 1) / NC : 0;
-  const int n_it = 2 * nch;                    // pass 1 then pass 2 over the same chunks
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    if (lane == 0 && nch > 0) {
       bool ok = true;
       int it = 0;
-      for (; it < n_it && ok; ++it) {
-        const int s = it % STAGES;
-        if (!mbar_wait(&k_empty[s], ((it / STAGES) & 1) ^ 1, &s_abort, hdr, 0x8100u)) {
-          ok = false;
-          break;
+      for (int pass = 0; ok; ++pass) {
+        if (pass >= 2) {  // decision of round pass - 2
+          const int r = pass - 2;
+          if (!mbar_wait(decide, r & 1, &s_abort, hdr, 0x8600u) || !s_more[r & 1]) break;
         }
-        const int j0 = (it % nch) * NC;
-        uint8_t* st = sK + s * CHUNK_BYTES;
-        mbar_expect_tx(&k_full[s], CHUNK_BYTES);
+        for (int c = 0; c < nch; ++c, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&k_empty[s], ((it / STAGES) & 1) ^ 1, &s_abort, hdr, 0x8100u)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = sK + s * CHUNK_BYTES;
+          mbar_expect_tx(&k_full[s], CHUNK_BYTES);
 #pragma unroll
-        for (int part = 0; part < 3; ++part)
+          for (int part = 0; part < 3; ++part)
 #pragma unroll
-          for (int dc = 0; dc < 2; ++dc)
-            tma_load_3d(&mapKb, &k_full[s], st + (part * 2 + dc) * BOX_BYTES, dc * 64, j0,
-                        part * G.hkv + kv);
+            for (int dc = 0; dc < 2; ++dc)
+              tma_load_3d(&mapKb, &k_full[s], st + (part * 2 + dc) * BOX_BYTES, dc * 64, c * NC,
+                          part * G.hkv + kv);
+        }
       }
       if (!ok) {
         for (int k = 0; k < STAGES; ++k) {
@@ -126,30 +138,38 @@ __global__ void __launch_bounds__(THREADS, 2)
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc_bf16(128, NC);
       const uint32_t q_tmem = tmem_base + Q_COL;
-      bool ok = n_it == 0 || mbar_wait(q_full, 0, &s_abort, hdr, 0x8200u);
+      bool ok = nch == 0 || mbar_wait(q_full, 0, &s_abort, hdr, 0x8200u);
       tc_fence_after();
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int s = it % STAGES, sb = it % SBUF;
-        if (!mbar_wait(&k_full[s], (it / STAGES) & 1, &s_abort, hdr, 0x8300u) ||
-            !mbar_wait(&s_empty[sb], ((it / SBUF) & 1) ^ 1, &s_abort, hdr, 0x8400u)) {
-          ok = false;
-          break;
+      int it = 0;
+      for (int pass = 0; ok && nch > 0; ++pass) {
+        if (pass >= 2) {
+          const int r = pass - 2;
+          if (!mbar_wait(decide, r & 1, &s_abort, hdr, 0x8700u) || !s_more[r & 1]) break;
         }
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + s * CHUNK_BYTES);
-        const uint32_t d = tmem_base + sb * NC;
+        for (int c = 0; c < nch; ++c, ++it) {
+          const int s = it % STAGES, sb = it % SBUF;
+          if (!mbar_wait(&k_full[s], (it / STAGES) & 1, &s_abort, hdr, 0x8300u) ||
+              !mbar_wait(&s_empty[sb], ((it / SBUF) & 1) ^ 1, &s_abort, hdr, 0x8400u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sK + s * CHUNK_BYTES);
+          const uint32_t d = tmem_base + sb * NC;
 #pragma unroll
-        for (int part = 0; part < 3; ++part)
+          for (int part = 0; part < 3; ++part)
 #pragma unroll
-          for (int dc = 0; dc < 2; ++dc)
+            for (int dc = 0; dc < 2; ++dc)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bd =
-                  make_sdesc_sw128(k_addr + (part * 2 + dc) * BOX_BYTES + kk * 32, 16, 1024);
-              umma_bf16_ts(d, q_tmem + dc * 32 + kk * 8, bd, idesc, (part | dc | kk) != 0 ? 1u : 0u);
-            }
-        umma_commit(&s_full[sb]);
-        umma_commit(&k_empty[s]);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd =
+                    make_sdesc_sw128(k_addr + (part * 2 + dc) * BOX_BYTES + kk * 32, 16, 1024);
+                umma_bf16_ts(d, q_tmem + dc * 32 + kk * 8, bd, idesc,
+                             (part | dc | kk) != 0 ? 1u : 0u);
+              }
+          umma_commit(&s_full[sb]);
+          umma_commit(&k_empty[s]);
+        }
       }
       umma_commit(drain);
       long long t0 = clock64();
@@ -190,69 +210,98 @@ __global__ void __launch_bounds__(THREADS, 2)
       sel::RowSel s;
       s.init(ss, row);
       const int ncand = own > 0 ? own : 0;
-      const sel::Pool pool{a.pool_z, a.pool_j, G.pool_rows, G.n_cubes};
       uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-      int nsel = 0;
+      int nsel = 0, extra = 0;
       bool ok = true;
-      for (int it = 0; it < n_it; ++it) {
-        const int sb = it % SBUF;
-        const bool second = it >= nch;
-        if (!mbar_wait_warp(&s_full[sb], (it / SBUF) & 1, &s_abort, hdr, 0x8500u)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int j0 = (it % nch) * NC;
-        const uint32_t tcol = tmem_base + lane_base + sb * NC;
-        uint32_t mine = 0u;  // pass 2: mask word of column j0 + lane, this warp
+      int it = 0;
+      for (int pass = 0; nch > 0; ++pass) {
+        for (int ch = 0; ch < nch && ok; ++ch, ++it) {
+          const int sb = it % SBUF;
+          if (!mbar_wait_warp(&s_full[sb], (it / SBUF) & 1, &s_abort, hdr, 0x8500u)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int j0 = ch * NC;
+          const uint32_t tcol = tmem_base + lane_base + sb * NC;
+          uint32_t mine = 0u;  // emission pass: mask word of column j0 + lane, this warp
 #pragma unroll 1
-        for (int q = 0; q < NC / 8; ++q) {
-          uint32_t acc[8];
-          tmem_ld8(tcol + q * 8, acc);
-          tmem_ld_wait();
-          if (!second) {
+          for (int q = 0; q < NC / 8; ++q) {
+            uint32_t acc[8];
+            tmem_ld8(tcol + q * 8, acc);
+            tmem_ld_wait();
+            if (pass == 0) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              if (j0 + q * 8 + c < ncand) s.pass1(__uint_as_float(acc[c]) * a.zscale);
-          } else {
+              for (int c = 0; c < 8; ++c)
+                if (j0 + q * 8 + c < ncand) s.pass1(__uint_as_float(acc[c]) * a.zscale);
+            } else if (pass == 1) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int j = j0 + q * 8 + c;
-              bool selb = false;
-              if (j < ncand) selb = s.pass2(__uint_as_float(acc[c]) * a.zscale, j, hdr, pool);
-              nsel += selb;
-              const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
-              if (lane == q * 8 + c) mine = w;
+              for (int c = 0; c < 8; ++c) {
+                const int j = j0 + q * 8 + c;
+                bool selb = false;
+                if (j < ncand) selb = s.pass2(__uint_as_float(acc[c]) * a.zscale, j);
+                nsel += selb;
+                const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
+                if (lane == q * 8 + c) mine = w;
+              }
+            } else if (s.open) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const int j = j0 + q * 8 + c;
+                if (j < ncand) s.pass_more(__uint_as_float(acc[c]) * a.zscale, j);
+              }
             }
           }
+          tc_fence_before();
+          mbar_arrive(&s_empty[sb]);
+          if (pass == 1) {
+            const int jl = j0 + lane;
+            if (jl < c_hi) tmask[(size_t)jl * 4 + wq] = mine;
+          }
         }
-        tc_fence_before();
-        mbar_arrive(&s_empty[sb]);
-        if (!second) {
-          if (it == nch - 1) s.finish1(a.p);
-        } else {
-          const int jl = j0 + lane;
-          if (jl < c_hi) tmask[(size_t)jl * 4 + wq] = mine;
+        // Every row warp reaches the vote barrier below, even after a failed
+        // wait (the abort flag then ends the loop), so the named barrier
+        // cannot strand the other warps.
+        if (pass == 0) {
+          if (ok) s.finish1(a.p);
+          continue;
         }
+        if (pass == 1) {
+          const unsigned w = __ballot_sync(0xffffffffu, own == c_hi);
+          if (lane == 0) tmask[(size_t)c_hi * 4 + wq] = w;
+          __syncwarp();
+          __threadfence_block();
+        }
+        const bool was_open = s.open;
+        const int m = s.settle();
+        for (int i = 0; i < m; ++i) atomicOr(&tmask[(size_t)s.list_j(i) * 4 + wq], 1u << lane);
+        nsel += m;
+        s.reset_list();
+        if (was_open && s.open) extra = 1;
+        // vote for another pass (round r = pass - 1)
+        const int r = pass - 1;
+        if (row == 0) s_more[(r + 1) & 1] = 0;
+        if (s.open) s_more[r & 1] = 1;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const bool more = s_more[r & 1] != 0 && !s_abort;
+        mbar_arrive(decide);
+        if (!more) break;
       }
-      if (ok) {
+      if (ok && nch == 0) {
         const unsigned w = __ballot_sync(0xffffffffu, own == c_hi);
         if (lane == 0) tmask[(size_t)c_hi * 4 + wq] = w;
-        __syncwarp();
-        __threadfence_block();
-        const int m = s.resolve();
-        for (int i = 0; i < m; ++i) atomicOr(&tmask[(size_t)s.ljv(i) * 4 + wq], 1u << lane);
-        nsel += m;
+      }
+      if (ok) {
         const unsigned v_rows = __reduce_add_sync(0xffffffffu, (valid && own > 0) ? 1u : 0u);
         const unsigned v_cand = __reduce_add_sync(0xffffffffu, (unsigned)ncand);
         const unsigned v_sel = __reduce_add_sync(0xffffffffu, (unsigned)nsel);
-        const unsigned v_ovf = __reduce_add_sync(0xffffffffu, s.gz ? 1u : 0u);
+        const unsigned v_ext = __reduce_add_sync(0xffffffffu, (unsigned)extra);
         if (lane == 0) {
           atomicAdd((unsigned long long*)&hdr->stats[0], (unsigned long long)v_rows);
           atomicAdd((unsigned long long*)&hdr->stats[1], (unsigned long long)v_cand);
           atomicAdd((unsigned long long*)&hdr->stats[2], (unsigned long long)v_sel);
-          atomicAdd((unsigned long long*)&hdr->stats[3], (unsigned long long)v_ovf);
+          atomicAdd((unsigned long long*)&hdr->stats[3], (unsigned long long)v_ext);
         }
       }
       __threadfence_block();

@@ -20,8 +20,8 @@
  *   - Execution: calls taking a `stream` (a cudaStream_t, NULL = legacy default
  *     stream) are asynchronous on it. Their return code covers host-side
  *     validation and launch errors only. Problems found on the device (a token
- *     layout that breaks the preconditions, a bounded wait that expired, an
- *     exhausted overflow pool) set a status word in the workspace; the kernels
+ *     layout that breaks the preconditions, a bounded wait that expired) set a
+ *     status word in the workspace; the kernels
  *     then return early and adaspark_read_device_status() reports
  *     ADASPARK_EDEVICE.
  *   - Token layout: tokens are in cube-major order. The visual prefix holds
@@ -57,7 +57,6 @@ typedef enum { ADASPARK_BF16 = 0, ADASPARK_FP32 = 1 } adaspark_dtype;
 /* Bits of the device status word (adaspark_read_device_status detail). */
 #define ADASPARK_DEV_BAD_LAYOUT   0x1u  /* cube_ids / cube_offsets / text_mask inconsistent */
 #define ADASPARK_DEV_TIMEOUT      0x2u  /* a bounded wait inside a kernel expired          */
-#define ADASPARK_DEV_POOL_FULL    0x4u  /* selection overflow pool exhausted               */
 
 /* Human-readable name of a return code. Never NULL. */
 const char *adaspark_status_string(int status);
@@ -98,7 +97,7 @@ typedef struct {
   uint64_t visual_rows;      /* (visual token, query head) rows that ran selection */
   uint64_t candidate_pairs;  /* sum over those rows of the preceding-cube count    */
   uint64_t selected_pairs;   /* sum over those rows of |S_i|                        */
-  uint64_t overflow_rows;    /* rows whose cut was resolved in the overflow pool    */
+  uint64_t overflow_rows;    /* rows whose Top-p cut needed extra score passes      */
   uint64_t tiles;            /* 128-row attention tiles executed (visual + text)    */
   uint64_t key_blocks;       /* executed (tile, key block) pairs                    */
   uint64_t key_block_keys;   /* keys covered by those blocks (for executed FLOPs)   */

@@ -152,3 +152,59 @@ def test_262k_four_layer_stack_sampled():
         x = y.to(x.dtype)
         del y, h, t, qkv, w
         torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ cut-bin stress
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("fp32", 64)])
+def test_attn_uniform_means_closed_form(dtype, d):
+    """Every key identical -> every cube mean identical -> P uniform over the c
+    preceding cubes: exact ties, the cut bin holds all of them, and the Top-p
+    set must be the ceil(p*c) lowest-index cubes (several extra passes)."""
+    import math
+    import ffn_long_video_b200 as fb
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    C, n, hq, hkv, n_text = 90, 8, 2, 1, 5
+    n_vis = C * n
+    N = n_vis + n_text
+    g = torch.Generator().manual_seed(11)
+    Q = torch.randn(N, hq, d, generator=g).to(tdt).cuda()
+    K = torch.randn(1, hkv, d, generator=g).expand(N, hkv, d).contiguous().to(tdt).cuda()
+    V = torch.randn(N, hkv, d, generator=g).to(tdt).cuda()
+    ids = torch.cat([torch.arange(C, dtype=torch.int32).repeat_interleave(n),
+                     torch.full((n_text,), -1, dtype=torch.int32)]).cuda()
+    off = (torch.arange(C + 1, dtype=torch.int32) * n).cuda()
+    for p in (0.7, 0.33):
+        out, ws = fb.cube_attn(Q, K, V, ids, off, n_vis, p)
+        torch.cuda.synchronize()
+        assert fb.read_device_status(ws)[0] == fb.OK
+        sel = fb.attn_export_sets(ws, ids, C, n_vis, N, hq, hkv, d,
+                                  fb.BF16 if dtype == "bf16" else fb.FP32)
+        for t in range(n_vis):
+            c = t // n
+            if c > 0 and abs(p * c - round(p * c)) < 1e-6:
+                continue
+            k = math.ceil(p * c) if c > 0 else 0
+            want = np.zeros(C, bool)
+            want[:k] = True
+            for h in range(hq):
+                assert np.array_equal(sel[t, h], want), (p, t, h, np.nonzero(sel[t, h])[0][:8])
+        st = fb.attn_read_stats(ws)
+        assert st["overflow_rows"] > 0          # the extra-pass path ran
+
+
+def test_attn_flat_random_scores():
+    """Unstructured Q/K (near-uniform cube relevance): wide cut bins on many
+    rows; sets and outputs still match the oracle."""
+    cfg = workloads.small_config(name="flat", grid=(8, 16, 16), cube=(4, 4, 2), n_text=30,
+                                 D=256, hq=4, hkv=2, F=256, seed=5)
+    g = torch.Generator().manual_seed(3)
+    N = cfg.n_tokens
+    t = {"Q": torch.randn(N, cfg.hq, cfg.d, generator=g).to(torch.bfloat16).cuda(),
+         "K": torch.randn(N, cfg.hkv, cfg.d, generator=g).to(torch.bfloat16).cuda(),
+         "V": torch.randn(N, cfg.hkv, cfg.d, generator=g).to(torch.bfloat16).cuda()}
+    ids, off, text, off_np = parity.layout_tensors(cfg)
+    case = {"cfg": cfg, "t": t, "ids": ids, "off": off, "text": text, "off_np": off_np}
+    for p in (0.7, 0.95):
+        rep = {}
+        parity.check_attn(case, p=p, report=rep)
+        print("flat", p, rep)
