@@ -8,7 +8,11 @@ Comparison protocol:
 * outputs are compared with the oracle run on the library's own sets
   (``attention_given_sets`` / ``ffn_given_sets``), so arithmetic error and
   selection error are judged separately; bf16: max-abs 2e-2 and rel-L2 5e-3;
-  fp32: max-abs 1e-4 and rel-L2 1e-5.
+  fp32: max-abs 1e-4 and rel-L2 1e-5.  An output stored in bf16 (the
+  attention output) cannot be closer to the exact value than its own rounding,
+  so its bound is |err| <= 2e-2 + 1 ulp_bf16(|ref|) per element (the reading
+  for bf16 outputs when |ref| reaches 8 and beyond, where half an ulp alone
+  exceeds 2e-2).
 """
 from __future__ import annotations
 
@@ -51,6 +55,19 @@ def errors(got, want):
     return max_abs, rel
 
 
+def ulp_bf16(x):
+    """Spacing of bf16 numbers at |x| (8 significant bits)."""
+    a = np.maximum(np.abs(np.asarray(x, dtype=np.float64)), 2.0 ** -126)
+    return np.exp2(np.floor(np.log2(a)) - 7)
+
+
+def excess_over_bf16(got, want):
+    """max of |got - want| - ulp_bf16(want): the error beyond one output ulp."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    return float((np.abs(got - want) - ulp_bf16(want)).max()) if got.size else 0.0
+
+
 def run_attn(case, p=None):
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
@@ -91,10 +108,13 @@ def check_attn(case, p=None, tokens=None, report=None):
     got = out.float().cpu().numpy()[tokens]
     max_abs, rel = errors(got, want)
     tol_abs, tol_rel = TOL[cfg.dtype]
+    # bf16 output: allow one ulp of the output format on top of the bound
+    worst = excess_over_bf16(got, want) if cfg.dtype == "bf16" else max_abs
     if report is not None:
-        report.update(max_abs=max_abs, rel_l2=rel, near_margin_rows=int(near.sum()),
-                      near_margin_mismatch=n_near_mismatch, rows=int(g.shape[0] * g.shape[1]))
-    assert max_abs <= tol_abs and rel <= tol_rel, (max_abs, rel)
+        report.update(max_abs=max_abs, excess_over_ulp=worst, rel_l2=rel,
+                      near_margin_rows=int(near.sum()), near_margin_mismatch=n_near_mismatch,
+                      rows=int(g.shape[0] * g.shape[1]))
+    assert worst <= tol_abs and rel <= tol_rel, (max_abs, worst, rel)
     return out, gsel, ws
 
 

@@ -125,8 +125,11 @@ def test_128k_sweep_sampled(shape):
 def test_262k_four_layer_stack_sampled():
     """Four independently seeded 7B-shaped layers at 262K visual tokens, half of
     the cubes near-duplicates of earlier ones. The harness wires the stack
-    (Q/K/V = x W, h = x + out W_o, next x = y); each layer's AdaS-Attn and
-    AdaS-FFN are checked against the oracle on that layer's own inputs."""
+    (Q/K/V = x W, h = x + out W_o, next x = y scaled to unit RMS per token, in
+    place of the RMSNorm a decoder applies between layers, so that the random
+    weights do not blow the residual stream up layer after layer); each layer's
+    AdaS-Attn and AdaS-FFN are checked against the oracle on that layer's own
+    inputs."""
     cfg = workloads.CONFIGS[5]
     ids, off, text, off_np = parity.layout_tensors(cfg)
     x = None
@@ -149,7 +152,7 @@ def test_262k_four_layer_stack_sampled():
         rep = {}
         y, _, _ = parity.check_ffn(case, cubes=cubes, text=(layer == 0), report=rep)
         print(cfg.name, "layer", layer, "ffn", rep)
-        x = y.to(x.dtype)
+        x = (y * torch.rsqrt(y.pow(2).mean(dim=1, keepdim=True) + 1e-6)).to(x.dtype)
         del y, h, t, qkv, w
         torch.cuda.empty_cache()
 
