@@ -47,6 +47,29 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Two fp32 lanes at once on the FMA pipe: (a0, a1) * s + (c, c).
+__device__ __forceinline__ void fma2_bcast(float a0, float a1, float s, float c, float& o0,
+                                           float& o1) {
+  asm("{\n\t.reg .b64 pa, ps, pc, pr;\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "mov.b64 ps, {%4, %4};\n\t"
+      "mov.b64 pc, {%5, %5};\n\t"
+      "fma.rn.f32x2 pr, pa, ps, pc;\n\t"
+      "mov.b64 {%0, %1}, pr;\n\t}"
+      : "=f"(o0), "=f"(o1)
+      : "f"(a0), "f"(a1), "f"(s), "f"(c));
+}
+// (s0, s1) += (a0, a1)
+__device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ps, pa;\n\t"
+      "mov.b64 ps, {%0, %1};\n\t"
+      "mov.b64 pa, {%2, %3};\n\t"
+      "add.rn.f32x2 ps, ps, pa;\n\t"
+      "mov.b64 {%0, %1}, ps;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
+}
+
 struct TileInfo {
   bool text;
   int bt;        // tile index within its kind
@@ -363,14 +386,31 @@ __global__ void __launch_bounds__(THREADS, 2)
       else row_on = ((dsc.mask[wq] >> lane) & 1u) != 0u;
       int lim = row_on ? dsc.nk : 0;
       if (row_on && (T.text || dsc.j == own)) lim = min(lim, t - dsc.k0 + 1);
-      float mx[8];
+      if (lim <= 0) row_on = false;
+      // Blocks where every row of the warp takes all 64 keys or none need no
+      // per-key mask: a row that takes none gets an offset of -inf, so its
+      // probabilities come out as exact zeros.
+      const bool partial = __any_sync(0xffffffffu, row_on && lim < 64);
+      float mraw = -INFINITY;
+      if (!partial) {
+        float mx[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+        for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
 #pragma unroll
-      for (int u = 0; u < 64; ++u)
-        if (u < lim) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(sr[u]));
-      const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+        for (int u = 8; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(sr[u]));
+        const float m8 = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        mraw = row_on ? m8 : -INFINITY;
+      } else {
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < 64; ++u)
+          if (u < lim) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(sr[u]));
+        mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                     fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      }
       const float m_new = fmaxf(m_used, mraw * scale);
       const bool want = m_new > m_used + kRescale;
       if (__any_sync(0xffffffffu, want)) {
@@ -397,18 +437,31 @@ __global__ void __launch_bounds__(THREADS, 2)
         if (m_new != -INFINITY) m_used = m_new;
       }
       // P = 2^(s * scale - m_used) on admitted keys, bf16 pairs written over S_i
+      const float neg_m = row_on ? -m_used : -INFINITY;
       float ls[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) ls[k] = 0.f;
-      const float neg_m = -m_used;
       uint32_t pk[32];
+      if (!partial) {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int u = 2 * q;
-        const float p0 = (u < lim) ? ex2(fmaf(__uint_as_float(sr[u]), scale, neg_m)) : 0.f;
-        const float p1 = (u + 1 < lim) ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, neg_m)) : 0.f;
-        ls[q & 7] += p0 + p1;
-        pk[q] = pack_bf16x2(p0, p1);
+        for (int q = 0; q < 32; ++q) {
+          float x0, x1;
+          fma2_bcast(__uint_as_float(sr[2 * q]), __uint_as_float(sr[2 * q + 1]), scale, neg_m,
+                     x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          add2(ls[2 * (q & 3)], ls[2 * (q & 3) + 1], p0, p1);
+          pk[q] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int u = 2 * q;
+          const float p0 = (u < lim) ? ex2(fmaf(__uint_as_float(sr[u]), scale, neg_m)) : 0.f;
+          const float p1 =
+              (u + 1 < lim) ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, neg_m)) : 0.f;
+          ls[q & 7] += p0 + p1;
+          pk[q] = pack_bf16x2(p0, p1);
+        }
       }
       tmem_st32(tmem_base + lane_base + 128 + sb * 64, pk);
       tmem_st_wait();
