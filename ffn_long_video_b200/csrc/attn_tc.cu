@@ -12,7 +12,9 @@
 //              masks from global memory 32 entries at a time and feeds a
 //              64-slot shared-memory ring, far ahead of the consumers
 //   warp 0     TMA producer: K and V blocks (3D maps over [token][kv][d], no
-//              multicast), 2-stage ring
+//              multicast) in two separate 2-stage rings; a K slot is released
+//              as soon as its S MMA completes, so K loads run a block ahead of
+//              the V loads (which wait for the PV MMA)
 //   warp 1     TMEM allocator + tcgen05.mma issuer:
 //                S_i = Q K_i^T   (M=128, N=64, K=128; two TMEM buffers)
 //                O  += P_i V_i   (M=128, N=128, K=64; P read from TMEM where it
@@ -34,6 +36,7 @@ constexpr int THREADS = 224;
 constexpr int RING = 64;
 constexpr int Q_BYTES = 128 * 256;        // 128 rows x 128 dims bf16 (two 64-dim halves)
 constexpr int KV_BYTES = 4 * 8192;        // K (2 halves) + V (2 halves), 64 keys each
+constexpr int K_BYTES = 2 * 8192;         // one K (or V) block: two 64-dim halves
 struct Desc {
   int k0, nk, j, pad;
   uint32_t mask[4];
@@ -111,9 +114,11 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint8_t* sKV = sQ + Q_BYTES;
   Desc* ring = reinterpret_cast<Desc*>(sKV + STAGES * KV_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + RING);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = kv_full + STAGES;
-  uint64_t* s_full = kv_empty + STAGES;     // [2]
+  uint64_t* k_full = bars;                  // [STAGES]
+  uint64_t* k_empty = k_full + STAGES;
+  uint64_t* v_full = k_empty + STAGES;
+  uint64_t* v_empty = v_full + STAGES;
+  uint64_t* s_full = v_empty + STAGES;      // [2]
   uint64_t* p_full = s_full + 2;            // [2]
   uint64_t* pv_done = p_full + 2;           // [2]
   uint64_t* q_full = pv_done + 2;
@@ -131,8 +136,10 @@ __global__ void __launch_bounds__(THREADS, 2)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -234,33 +241,54 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Block i: K_i into K stage i % 2 (free once S_{i-2} is done), then V_{i-1}
+    // into V stage (i-1) % 2 (free once PV_{i-3} is done).
     if (lane == 0) {
-      int i = 0;
+      uint8_t* sK = sKV;                       // [STAGES][K_BYTES]
+      uint8_t* sV = sKV + STAGES * K_BYTES;    // [STAGES][K_BYTES]
+      int i = 0, prev_k0 = 0, nv = 0;
       bool ok = true;
+      auto load_v = [&](int blk, int k0) -> bool {
+        const int s = blk % STAGES;
+        if (!mbar_wait(&v_empty[s], ((blk / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7110u)) return false;
+        mbar_expect_tx(&v_full[s], K_BYTES);
+        tma_load_3d(&mapV, &v_full[s], sV + s * K_BYTES, 0, T.kv, k0);
+        tma_load_3d(&mapV, &v_full[s], sV + s * K_BYTES + 8192, 64, T.kv, k0);
+        nv = blk + 1;
+        return true;
+      };
       while (ok) {
         const int slot = i % RING;
-        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7000u)) break;
-        const int k0 = ring[slot].k0, nk = ring[slot].nk;
-        if (nk == 0) break;
-        const int s = i % STAGES;
-        if (!mbar_wait(&kv_empty[s], ((i / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7100u)) {
+        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7000u)) {
           ok = false;
           break;
         }
-        uint8_t* st = sKV + s * KV_BYTES;
-        mbar_expect_tx(&kv_full[s], KV_BYTES);
-        tma_load_3d(&mapK, &kv_full[s], st, 0, T.kv, k0);
-        tma_load_3d(&mapK, &kv_full[s], st + 8192, 64, T.kv, k0);
-        tma_load_3d(&mapV, &kv_full[s], st + 16384, 0, T.kv, k0);
-        tma_load_3d(&mapV, &kv_full[s], st + 24576, 64, T.kv, k0);
+        const int k0 = ring[slot].k0, nk = ring[slot].nk;
+        if (nk == 0) break;
+        const int s = i % STAGES;
+        if (!mbar_wait(&k_empty[s], ((i / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7100u)) {
+          ok = false;
+          break;
+        }
+        mbar_expect_tx(&k_full[s], K_BYTES);
+        tma_load_3d(&mapK, &k_full[s], sK + s * K_BYTES, 0, T.kv, k0);
+        tma_load_3d(&mapK, &k_full[s], sK + s * K_BYTES + 8192, 64, T.kv, k0);
+        if (i > 0 && !load_v(i - 1, prev_k0)) {
+          ok = false;
+          break;
+        }
+        prev_k0 = k0;
         ++i;
       }
-      if (!ok) {
+      if (ok && i > 0) ok = load_v(i - 1, prev_k0);
+      if (!ok) {  // let copies already issued land before the CTA exits
         for (int k = 0; k < STAGES; ++k) {
-          const int jj = i - 1 - k;
-          if (jj < 0) break;
           long long t0 = clock64();
-          while (!mbar_try_wait(&kv_full[jj % STAGES], (jj / STAGES) & 1) &&
+          const int jk = i - 1 - k, jv = nv - 1 - k;
+          while (jk >= 0 && !mbar_try_wait(&k_full[jk % STAGES], (jk / STAGES) & 1) &&
+                 clock64() - t0 < kWaitCycles) {
+          }
+          while (jv >= 0 && !mbar_try_wait(&v_full[jv % STAGES], (jv / STAGES) & 1) &&
                  clock64() - t0 < kWaitCycles) {
           }
         }
@@ -278,9 +306,10 @@ __global__ void __launch_bounds__(THREADS, 2)
       auto issue_pv = [&](int blk) -> bool {
         const int pb = blk & 1;
         if (!mbar_wait(&p_full[pb], (blk >> 1) & 1, &s_abort, hdr, 0x7300u)) return false;
-        tc_fence_after();
         const int s = blk % STAGES;
-        const uint32_t v_addr = smem_u32(sKV + s * KV_BYTES + 16384);
+        if (!mbar_wait(&v_full[s], (blk / STAGES) & 1, &s_abort, hdr, 0x7310u)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sKV + STAGES * K_BYTES + s * K_BYTES);
         const uint32_t p_tmem = tmem_base + 128 + pb * 64;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -288,7 +317,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           umma_bf16_ts(tmem_base, p_tmem + kk * 8, bd, idesc_o, (blk > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[pb]);
-        umma_commit(&kv_empty[s]);
+        umma_commit(&v_empty[s]);
         return true;
       };
       while (ok) {
@@ -300,12 +329,12 @@ __global__ void __launch_bounds__(THREADS, 2)
         if (ring[slot].nk == 0) break;
         const int s = i % STAGES;
         const int sb = i & 1;
-        if (!mbar_wait(&kv_full[s], (i / STAGES) & 1, &s_abort, hdr, 0x7400u)) {
+        if (!mbar_wait(&k_full[s], (i / STAGES) & 1, &s_abort, hdr, 0x7400u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sKV + s * KV_BYTES);
+        const uint32_t k_addr = smem_u32(sKV + s * K_BYTES);
         const uint32_t d_s = tmem_base + 128 + sb * 64;
 #pragma unroll
         for (int dc = 0; dc < 2; ++dc)
@@ -316,6 +345,7 @@ __global__ void __launch_bounds__(THREADS, 2)
             umma_bf16(d_s, ad, bd, idesc_s, (dc | kk) != 0 ? 1u : 0u);
           }
         umma_commit(&s_full[sb]);
+        umma_commit(&k_empty[s]);
         if (i > 0 && !issue_pv(i - 1)) {
           ok = false;
           break;
