@@ -110,6 +110,8 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
 #pragma unroll
   for (int e = 0; e < D; ++e) q[e] = valid ? to_f32(qp[e]) : 0.f;
 
+  sel::init_table(ss, tid);
+  __syncthreads();
   sel::RowSel s;
   s.init(ss, tid);
   const int ncand = own > 0 ? own : 0;

@@ -9,9 +9,9 @@
 //          scalar when the maximum moves up). Walking down from the top, the
 //          cut bin is the first at which the cumulative mass reaches p * Z.
 //  pass 2  every element of a higher bin is selected outright; the elements of
-//          the cut bin are offered to a per-row top-kL list kept sorted in the
-//          (z desc, index asc) order. Walking that list until the cumulative
-//          mass reaches p * Z ends the cut.
+//          the cut bin are offered to a per-row list that keeps the kL best in
+//          the (z desc, index asc) order. Walking that list in order until the
+//          cumulative mass reaches p * Z ends the cut.
 //  more    if the cut lies beyond the kL best elements of the cut bin, those
 //          kL are selected, the required mass is reduced by theirs, and another
 //          pass collects the next kL below the last key; repeated until the cut
@@ -52,7 +52,13 @@ struct Smem {
   float hist[kB][kRows];
   float lz[kL][kRows];
   uint16_t lj[kL][kRows];
+  float wbin[kB];          // 2^(-i/kR), i = 0..kB-1 (filled by init_table)
 };
+
+// Fill the bin-weight table once per CTA (threads [0, kB) of the caller).
+__device__ __forceinline__ void init_table(Smem* s, int tid) {
+  if (tid < kB) s->wbin[tid] = exp2f(-(float)tid * kInvR);
+}
 
 struct RowSel {
   Smem* sm;
@@ -63,6 +69,7 @@ struct RowSel {
   float need;
   int n;          // list entries
   bool open;      // cut not found yet
+  bool sorted;    // list entries [0, n) are in order
   bool bounded;   // only keys after (bz, bj) are offered (extra passes)
   float bz;
   int bj;
@@ -76,6 +83,7 @@ struct RowSel {
     need = 0.f;
     n = 0;
     open = false;
+    sorted = true;
     bounded = false;
     bz = 0.f;
     bj = 0;
@@ -112,6 +120,28 @@ struct RowSel {
       tail += fast_exp2(z - (float)bmax * kInvR);
   }
 
+  // Eight scores at once (the hot loop of pass 1): one running-maximum check
+  // for the group, then the bin updates. `valid` bit c enables z[c].
+  __device__ __forceinline__ void pass1x8(const float (&z)[8], unsigned valid) {
+    int b[8];
+    int bm = kNone;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      b[c] = __float2int_rd(z[c] * (float)kR);
+      if ((valid >> c) & 1u) bm = max(bm, b[c]);
+    }
+    if (bm > bmax) shift(bm);
+    const int lo = bmax - kB;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (!((valid >> c) & 1u)) continue;
+      if (b[c] > lo)
+        sm->hist[b[c] & (kB - 1)][tid] += fast_exp2(z[c] - (float)b[c] * kInvR);
+      else
+        tail += fast_exp2(z[c] - (float)bmax * kInvR);
+    }
+  }
+
   __device__ void finish1(float p) {
     if (bmax == kNone) {
       bstar = kNone;
@@ -119,18 +149,14 @@ struct RowSel {
       return;
     }
     float Z = tail;
-    for (int i = kB - 1; i >= 0; --i) {
-      const int k = bmax - i;
-      Z += sm->hist[k & (kB - 1)][tid] * exp2f(-(float)i * kInvR);
-    }
+    for (int i = kB - 1; i >= 0; --i) Z += sm->hist[(bmax - i) & (kB - 1)][tid] * sm->wbin[i];
     const float target = p * Z;
     float cum = 0.f;
     bstar = kTail;
     for (int i = 0; i < kB; ++i) {
-      const int k = bmax - i;
-      const float m = sm->hist[k & (kB - 1)][tid] * exp2f(-(float)i * kInvR);
+      const float m = sm->hist[(bmax - i) & (kB - 1)][tid] * sm->wbin[i];
       if (cum + m >= target) {
-        bstar = k;
+        bstar = bmax - i;
         break;
       }
       cum += m;
@@ -139,16 +165,38 @@ struct RowSel {
     open = true;
   }
 
-  // Insert into the sorted top-kL list (keys after the bound only).
+  // Sort list entries [0, n) into the (z desc, index asc) order.
+  __device__ __noinline__ void sort_list() {
+    for (int i = 1; i < n; ++i) {
+      const float z = sm->lz[i][tid];
+      const uint16_t j = sm->lj[i][tid];
+      int k = i;
+      while (k > 0 && before(z, j, sm->lz[k - 1][tid], (int)sm->lj[k - 1][tid])) {
+        sm->lz[k][tid] = sm->lz[k - 1][tid];
+        sm->lj[k][tid] = sm->lj[k - 1][tid];
+        --k;
+      }
+      sm->lz[k][tid] = z;
+      sm->lj[k][tid] = j;
+    }
+    sorted = true;
+  }
+
+  // Keep the kL best offered keys (after the bound, if any). Entries are
+  // appended unsorted until the list is full; it is sorted once then, and
+  // later offers replace the last entry by sorted insertion.
   __device__ __noinline__ void offer(float z, int j) {
     if (bounded && !before(bz, bj, z, j)) return;
-    int pos;
-    if (n == kL) {
-      if (!before(z, j, sm->lz[kL - 1][tid], (int)sm->lj[kL - 1][tid])) return;
-      pos = kL - 1;
-    } else {
-      pos = n++;
+    if (n < kL) {
+      sm->lz[n][tid] = z;
+      sm->lj[n][tid] = (uint16_t)j;
+      ++n;
+      sorted = false;
+      return;
     }
+    if (!sorted) sort_list();
+    if (!before(z, j, sm->lz[kL - 1][tid], (int)sm->lj[kL - 1][tid])) return;
+    int pos = kL - 1;
     while (pos > 0 && before(z, j, sm->lz[pos - 1][tid], (int)sm->lj[pos - 1][tid])) {
       sm->lz[pos][tid] = sm->lz[pos - 1][tid];
       sm->lj[pos][tid] = sm->lj[pos - 1][tid];
@@ -183,6 +231,7 @@ struct RowSel {
   // kL entries are taken and the next pass starts after the last of them.
   __device__ int settle() {
     if (!open) return 0;
+    if (!sorted) sort_list();
     const float ref = (float)bmax * kInvR;
     float cum = 0.f;
     for (int i = 0; i < n; ++i) {
@@ -205,7 +254,10 @@ struct RowSel {
   }
 
   __device__ __forceinline__ int list_j(int i) const { return (int)sm->lj[i][tid]; }
-  __device__ __forceinline__ void reset_list() { n = 0; }
+  __device__ __forceinline__ void reset_list() {
+    n = 0;
+    sorted = true;
+  }
 };
 
 }  // namespace sel

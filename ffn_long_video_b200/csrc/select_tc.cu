@@ -206,6 +206,8 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       mbar_arrive(q_full);
     }
+    sel::init_table(ss, row);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     if (c_hi >= 0) {
       sel::RowSel s;
       s.init(ss, row);
@@ -232,9 +234,14 @@ __global__ void __launch_bounds__(THREADS, 2)
             tmem_ld8(tcol + q * 8, acc);
             tmem_ld_wait();
             if (pass == 0) {
+              float z[8];
+              unsigned valid_bits = 0u;
 #pragma unroll
-              for (int c = 0; c < 8; ++c)
-                if (j0 + q * 8 + c < ncand) s.pass1(__uint_as_float(acc[c]) * a.zscale);
+              for (int c = 0; c < 8; ++c) {
+                z[c] = __uint_as_float(acc[c]) * a.zscale;
+                if (j0 + q * 8 + c < ncand) valid_bits |= 1u << c;
+              }
+              if (valid_bits) s.pass1x8(z, valid_bits);
             } else if (pass == 1) {
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
