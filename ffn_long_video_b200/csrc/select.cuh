@@ -60,62 +60,118 @@ __device__ __forceinline__ void init_table(Smem* s, int tid) {
   if (tid < kB) s->wbin[tid] = exp2f(-(float)tid * kInvR);
 }
 
+// Out-of-line cold paths take and return plain values, so that the per-row
+// state below stays in registers (a member function called out of line would
+// force the whole state object into local memory).
+
+// The running maximum moved up from bin bmax to bin b: fold the bins leaving
+// the window into the tail and rescale it; returns the new tail.
+static __device__ __noinline__ float shift_window(float* hist_col, int bmax, int b, float tail) {
+  int nleave = b - bmax;
+  if (nleave > kB) nleave = kB;
+  tail *= exp2f((float)(bmax - b) * kInvR);
+  const int k0 = bmax - kB + 1;
+  for (int i = 0; i < nleave; ++i) {
+    const int k = k0 + i;
+    float& hv = hist_col[(k & (kB - 1)) * kRows];
+    if (hv != 0.f) {
+      tail += hv * exp2f((float)(k - b) * kInvR);
+      hv = 0.f;
+    }
+  }
+  return tail;
+}
+
+// Insertion sort of list entries [0, n) into the (z desc, index asc) order.
+static __device__ __noinline__ void sort_entries(float* lz_col, uint16_t* lj_col, int n) {
+  for (int i = 1; i < n; ++i) {
+    const float z = lz_col[i * kRows];
+    const uint16_t j = lj_col[i * kRows];
+    int k = i;
+    while (k > 0 && before(z, j, lz_col[(k - 1) * kRows], (int)lj_col[(k - 1) * kRows])) {
+      lz_col[k * kRows] = lz_col[(k - 1) * kRows];
+      lj_col[k * kRows] = lj_col[(k - 1) * kRows];
+      --k;
+    }
+    lz_col[k * kRows] = z;
+    lj_col[k * kRows] = j;
+  }
+}
+
+// Offer (z, j) to a list holding the kL best keys seen so far; state packs the
+// entry count (bits 0..7) and an "in order" flag (bit 8). Entries are appended
+// unsorted until the list is full; it is sorted once then, and later offers
+// replace the last entry by sorted insertion. Returns the new state.
+static __device__ __noinline__ int offer_entry(float* lz_col, uint16_t* lj_col, int state, float z,
+                                        int j) {
+  int n = state & 0xff;
+  bool sorted = (state >> 8) & 1;
+  if (n < kL) {
+    lz_col[n * kRows] = z;
+    lj_col[n * kRows] = (uint16_t)j;
+    return (n + 1);  // not in order any more
+  }
+  if (!sorted) sort_entries(lz_col, lj_col, n);
+  if (before(z, j, lz_col[(kL - 1) * kRows], (int)lj_col[(kL - 1) * kRows])) {
+    int pos = kL - 1;
+    while (pos > 0 && before(z, j, lz_col[(pos - 1) * kRows], (int)lj_col[(pos - 1) * kRows])) {
+      lz_col[pos * kRows] = lz_col[(pos - 1) * kRows];
+      lj_col[pos * kRows] = lj_col[(pos - 1) * kRows];
+      --pos;
+    }
+    lz_col[pos * kRows] = z;
+    lj_col[pos * kRows] = (uint16_t)j;
+  }
+  return kL | (1 << 8);
+}
+
 struct RowSel {
-  Smem* sm;
-  int tid;
+  float* hist_col;   // &hist[0][row]
+  float* lz_col;     // &lz[0][row]
+  uint16_t* lj_col;  // &lj[0][row]
+  const float* wbin;
   int bmax;
   float tail;
   int bstar;
   float need;
-  int n;          // list entries
+  int lstate;     // list entries | (in order << 8)
   bool open;      // cut not found yet
-  bool sorted;    // list entries [0, n) are in order
   bool bounded;   // only keys after (bz, bj) are offered (extra passes)
   float bz;
   int bj;
 
-  __device__ void init(Smem* s, int t) {
-    sm = s;
-    tid = t;
+  __device__ __forceinline__ void init(Smem* s, int t) {
+    hist_col = &s->hist[0][t];
+    lz_col = &s->lz[0][t];
+    lj_col = &s->lj[0][t];
+    wbin = s->wbin;
     bmax = kNone;
     tail = 0.f;
     bstar = kNone;
     need = 0.f;
-    n = 0;
+    lstate = 1 << 8;
     open = false;
-    sorted = true;
     bounded = false;
     bz = 0.f;
     bj = 0;
 #pragma unroll 8
-    for (int k = 0; k < kB; ++k) sm->hist[k][tid] = 0.f;
+    for (int k = 0; k < kB; ++k) hist_col[k * kRows] = 0.f;
   }
 
-  __device__ __noinline__ void shift(int b) {
+  __device__ __forceinline__ void raise_max(int b) {
     if (bmax == kNone) {
       bmax = b;
       return;
     }
-    int nleave = b - bmax;
-    if (nleave > kB) nleave = kB;
-    tail *= exp2f((float)(bmax - b) * kInvR);
-    const int k0 = bmax - kB + 1;
-    for (int i = 0; i < nleave; ++i) {
-      const int k = k0 + i;
-      float& hv = sm->hist[k & (kB - 1)][tid];
-      if (hv != 0.f) {
-        tail += hv * exp2f((float)(k - b) * kInvR);
-        hv = 0.f;
-      }
-    }
+    tail = shift_window(hist_col, bmax, b, tail);
     bmax = b;
   }
 
   __device__ __forceinline__ void pass1(float z) {
     const int b = __float2int_rd(z * (float)kR);
-    if (b > bmax) shift(b);
+    if (b > bmax) raise_max(b);
     if (b > bmax - kB)
-      sm->hist[b & (kB - 1)][tid] += fast_exp2(z - (float)b * kInvR);
+      hist_col[(b & (kB - 1)) * kRows] += fast_exp2(z - (float)b * kInvR);
     else
       tail += fast_exp2(z - (float)bmax * kInvR);
   }
@@ -130,31 +186,31 @@ struct RowSel {
       b[c] = __float2int_rd(z[c] * (float)kR);
       if ((valid >> c) & 1u) bm = max(bm, b[c]);
     }
-    if (bm > bmax) shift(bm);
+    if (bm > bmax) raise_max(bm);
     const int lo = bmax - kB;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       if (!((valid >> c) & 1u)) continue;
       if (b[c] > lo)
-        sm->hist[b[c] & (kB - 1)][tid] += fast_exp2(z[c] - (float)b[c] * kInvR);
+        hist_col[(b[c] & (kB - 1)) * kRows] += fast_exp2(z[c] - (float)b[c] * kInvR);
       else
         tail += fast_exp2(z[c] - (float)bmax * kInvR);
     }
   }
 
-  __device__ void finish1(float p) {
+  __device__ __forceinline__ void finish1(float p) {
     if (bmax == kNone) {
       bstar = kNone;
       open = false;
       return;
     }
     float Z = tail;
-    for (int i = kB - 1; i >= 0; --i) Z += sm->hist[(bmax - i) & (kB - 1)][tid] * sm->wbin[i];
+    for (int i = kB - 1; i >= 0; --i) Z += hist_col[((bmax - i) & (kB - 1)) * kRows] * wbin[i];
     const float target = p * Z;
     float cum = 0.f;
     bstar = kTail;
     for (int i = 0; i < kB; ++i) {
-      const float m = sm->hist[(bmax - i) & (kB - 1)][tid] * sm->wbin[i];
+      const float m = hist_col[((bmax - i) & (kB - 1)) * kRows] * wbin[i];
       if (cum + m >= target) {
         bstar = bmax - i;
         break;
@@ -165,45 +221,9 @@ struct RowSel {
     open = true;
   }
 
-  // Sort list entries [0, n) into the (z desc, index asc) order.
-  __device__ __noinline__ void sort_list() {
-    for (int i = 1; i < n; ++i) {
-      const float z = sm->lz[i][tid];
-      const uint16_t j = sm->lj[i][tid];
-      int k = i;
-      while (k > 0 && before(z, j, sm->lz[k - 1][tid], (int)sm->lj[k - 1][tid])) {
-        sm->lz[k][tid] = sm->lz[k - 1][tid];
-        sm->lj[k][tid] = sm->lj[k - 1][tid];
-        --k;
-      }
-      sm->lz[k][tid] = z;
-      sm->lj[k][tid] = j;
-    }
-    sorted = true;
-  }
-
-  // Keep the kL best offered keys (after the bound, if any). Entries are
-  // appended unsorted until the list is full; it is sorted once then, and
-  // later offers replace the last entry by sorted insertion.
-  __device__ __noinline__ void offer(float z, int j) {
+  __device__ __forceinline__ void offer(float z, int j) {
     if (bounded && !before(bz, bj, z, j)) return;
-    if (n < kL) {
-      sm->lz[n][tid] = z;
-      sm->lj[n][tid] = (uint16_t)j;
-      ++n;
-      sorted = false;
-      return;
-    }
-    if (!sorted) sort_list();
-    if (!before(z, j, sm->lz[kL - 1][tid], (int)sm->lj[kL - 1][tid])) return;
-    int pos = kL - 1;
-    while (pos > 0 && before(z, j, sm->lz[pos - 1][tid], (int)sm->lj[pos - 1][tid])) {
-      sm->lz[pos][tid] = sm->lz[pos - 1][tid];
-      sm->lj[pos][tid] = sm->lj[pos - 1][tid];
-      --pos;
-    }
-    sm->lz[pos][tid] = z;
-    sm->lj[pos][tid] = (uint16_t)j;
+    lstate = offer_entry(lz_col, lj_col, lstate, z, j);
   }
 
   __device__ __forceinline__ bool in_cut_bin(int b) const {
@@ -229,35 +249,33 @@ struct RowSel {
   // After a pass over the cut bin: how many leading list entries are selected.
   // Closes the cut when reached (or when the bin is exhausted); otherwise all
   // kL entries are taken and the next pass starts after the last of them.
-  __device__ int settle() {
+  __device__ __forceinline__ int settle() {
     if (!open) return 0;
-    if (!sorted) sort_list();
+    const int n = lstate & 0xff;
+    if (!((lstate >> 8) & 1)) sort_entries(lz_col, lj_col, n);
+    lstate = n | (1 << 8);
     const float ref = (float)bmax * kInvR;
     float cum = 0.f;
     for (int i = 0; i < n; ++i) {
-      cum += fast_exp2(sm->lz[i][tid] - ref);
+      cum += fast_exp2(lz_col[i * kRows] - ref);
       if (cum >= need) {
         open = false;
         return i + 1;
       }
     }
-    const int m = n;
     if (n < kL) {  // the whole cut bin was offered: rounding left need unmet
       open = false;
-      return m;
+      return n;
     }
     need -= cum;
     bounded = true;
-    bz = sm->lz[kL - 1][tid];
-    bj = (int)sm->lj[kL - 1][tid];
-    return m;
+    bz = lz_col[(kL - 1) * kRows];
+    bj = (int)lj_col[(kL - 1) * kRows];
+    return n;
   }
 
-  __device__ __forceinline__ int list_j(int i) const { return (int)sm->lj[i][tid]; }
-  __device__ __forceinline__ void reset_list() {
-    n = 0;
-    sorted = true;
-  }
+  __device__ __forceinline__ int list_j(int i) const { return (int)lj_col[i * kRows]; }
+  __device__ __forceinline__ void reset_list() { lstate = 1 << 8; }
 };
 
 }  // namespace sel
