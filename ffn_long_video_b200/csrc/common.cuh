@@ -104,6 +104,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread is parked in hardware until the
+// phase completes or the hint (ns) runs out, instead of spinning on issue slots.
+constexpr uint32_t kSuspendHintNs = 16384;
+__device__ __forceinline__ bool mbar_try_wait_parked(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // A wait that gives up after ~2^31 SM cycles (about a second): on expiry it
 // records ADASPARK_DEV_TIMEOUT, raises the CTA-wide abort flag and returns
 // false so the caller can leave its loop. It also returns false at once when
@@ -112,12 +127,10 @@ constexpr long long kWaitCycles = 2000000000LL;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           WsHeader* hdr, uint32_t where) {
   if (mbar_try_wait(bar, parity)) return true;
-  long long start = clock64();
-  int spins = 0;
+  const long long start = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_parked(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (++spins > 16) __nanosleep(64);
     if (clock64() - start > kWaitCycles) {
       *abort_flag = 1;
       set_status(hdr, ADASPARK_DEV_TIMEOUT, where);
