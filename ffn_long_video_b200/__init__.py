@@ -21,7 +21,7 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libadaspar
 
 OK, EINVAL, ECUDA, EUNSUPPORTED, EDEVICE = 0, -1, -2, -3, -4
 BF16, FP32 = 0, 1
-DEV_BAD_LAYOUT, DEV_TIMEOUT = 0x1, 0x2
+DEV_BAD_LAYOUT, DEV_TIMEOUT, DEV_RANGE = 0x1, 0x2, 0x4
 
 
 class AdasparkError(RuntimeError):

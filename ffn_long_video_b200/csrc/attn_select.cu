@@ -110,10 +110,8 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
 #pragma unroll
   for (int e = 0; e < D; ++e) q[e] = valid ? to_f32(qp[e]) : 0.f;
 
-  sel::init_table(ss, tid);
-  __syncthreads();
   sel::RowSel s;
-  s.init(ss, tid);
+  s.init(ss, tid, a.zscale);
   const int ncand = own > 0 ? own : 0;
   const float* kb = a.kbar + (size_t)kv * G.n_cubes * D;
   uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
@@ -135,10 +133,9 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
           float acc = 0.f;
 #pragma unroll
           for (int e = 0; e < D; ++e) acc = fmaf(q[e], kr[e], acc);
-          const float z = acc * a.zscale;
-          if (pass == 0) s.pass1(z);
-          else if (pass == 1) selb = s.pass2(z, j);
-          else s.pass_more(z, j);
+          if (pass == 0) s.pass1(acc);
+          else if (pass == 1) selb = s.pass2(acc, j, true);
+          else s.pass_more(acc, j);
         }
         if (pass == 1) {
           const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
@@ -149,6 +146,7 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
     }
     if (pass == 0) {
       s.finish1(a.p);
+      if (s.range_err) set_status(a.hdr, ADASPARK_DEV_RANGE, 0x8900u);
       continue;
     }
     if (pass == 1) {

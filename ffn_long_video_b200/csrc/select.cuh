@@ -2,19 +2,22 @@
 // S_i = {j | p_j in Top-p(P_i, p)}), one thread per row, in streaming passes
 // over the scores (which the caller recomputes bit-identically every pass).
 //
-// Scores enter in log2 units, z_j = (q . kbar_j) * log2(e) / sqrt(d), so that
-// P_j is proportional to 2^z_j. The order is (z descending, index ascending).
-//  pass 1  mass histogram of 2^z over bins of width 1/kR log2-units, in a window
-//          of kB bins below the running maximum (older bins fold into a tail
-//          scalar when the maximum moves up). Walking down from the top, the
-//          cut bin is the first at which the cumulative mass reaches p * Z.
-//  pass 2  every element of a higher bin is selected outright; the elements of
-//          the cut bin are offered to a per-row list that keeps the kL best in
-//          the (z desc, index asc) order. Walking that list in order until the
-//          cumulative mass reaches p * Z ends the cut.
-//  more    if the cut lies beyond the kL best elements of the cut bin, those
-//          kL are selected, the required mass is reduced by theirs, and another
-//          pass collects the next kL below the last key; repeated until the cut
+// Scores enter raw (s_j = q . kbar_j); z_j = s_j * log2(e) / sqrt(d) is the
+// score in log2 units, so P_j is proportional to 2^z_j. The order is (s desc,
+// index asc).
+//  pass 1  mass histogram of 2^z over bins of 1/8 octave (keys of mass_key),
+//          in a window of kB bins below the running maximum; the lowest bin
+//          also takes every score below the window (bins leaving the window
+//          fold into it when the maximum moves up). Walking down from the top,
+//          the cut bin is the first at which the cumulative mass reaches p * Z.
+//  pass 2  every score of a higher bin is selected outright; the scores of the
+//          cut bin are appended to a per-row list of kL entries. Sorted into
+//          the (s desc, index asc) order and walked until the cumulative mass
+//          reaches p * Z, the list ends the cut. A cut bin larger than the
+//          list is collected again in the next pass, keeping its kL best.
+//  more    if the cut lies beyond the kL best scores of the cut bin, those kL
+//          are selected, the required mass is reduced by theirs, and another
+//          pass collects the next kL below the last one; repeated until the cut
 //          is found (bounded by the size of the cut bin).
 // This reproduces "smallest prefix of the (P desc, index asc) order whose
 // cumulative mass reaches p" up to fp32 rounding of the masses, for any score
@@ -28,13 +31,20 @@
 namespace adaspark {
 namespace sel {
 
-constexpr int kR = 8;                 // bins per log2 unit
-constexpr float kInvR = 1.0f / kR;
-constexpr int kB = 64;                // bins in the window (8 log2 units)
-constexpr int kL = 24;                // list entries per row (shared memory)
-constexpr int kNone = INT_MIN;        // row without candidates
-constexpr int kTail = INT_MIN + 1;    // the cut lies below the window
+constexpr int kB = 64;                // bins in the window (8 log2 units, 8 bins each)
+constexpr int kL = 32;                // list entries per row (one more slot as scratch)
 constexpr int kRows = 128;
+constexpr int kNoKey = INT_MIN;       // row without candidates
+constexpr float kRefStep = 64.f;      // new reference once the maximum passes ref + 64
+constexpr float kZLimit = 1048576.f;  // supported |z|: below 2^20 log2 units
+
+// Masses are kept relative to a per-row reference ref (an integer, in log2
+// units): u = 2^(z - ref). For a positive float, bits >> 20 is 8 x exponent +
+// the top three mantissa bits, an integer that grows with u and steps 8 times
+// per doubling; it is the bin key (bins 1/8 of an octave wide in the mantissa,
+// at most a factor 1.125 between the ends of a bin). u = 0 (far below the
+// reference) has key 0.
+__device__ __forceinline__ int mass_key(float u) { return __float_as_int(u) >> 20; }
 
 // 2^x on the special-function unit (relative error below 2^-22).
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -43,46 +53,49 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// (z1, j1) comes before (z2, j2) in the (z desc, index asc) order.
-__device__ __forceinline__ bool before(float z1, int j1, float z2, int j2) {
-  return z1 > z2 || (z1 == z2 && j1 < j2);
+// (s1, j1) comes before (s2, j2) in the (score desc, index asc) order.
+__device__ __forceinline__ bool before(float s1, int j1, float s2, int j2) {
+  return s1 > s2 || (s1 == s2 && j1 < j2);
 }
 
 struct Smem {
   float hist[kB][kRows];
-  float lz[kL][kRows];
-  uint16_t lj[kL][kRows];
-  float wbin[kB];          // 2^(-i/kR), i = 0..kB-1 (filled by init_table)
+  float lz[kL + 1][kRows];     // raw scores q . kbar_j of the list entries
+  uint16_t lj[kL + 1][kRows];  // their cube indices
 };
-
-// Fill the bin-weight table once per CTA (threads [0, kB) of the caller).
-__device__ __forceinline__ void init_table(Smem* s, int tid) {
-  if (tid < kB) s->wbin[tid] = exp2f(-(float)tid * kInvR);
-}
 
 // Out-of-line cold paths take and return plain values, so that the per-row
 // state below stays in registers (a member function called out of line would
 // force the whole state object into local memory).
 
-// The running maximum moved up from bin bmax to bin b: fold the bins leaving
-// the window into the tail and rescale it; returns the new tail.
-static __device__ __noinline__ float shift_window(float* hist_col, int bmax, int b, float tail) {
-  int nleave = b - bmax;
-  if (nleave > kB) nleave = kB;
-  tail *= exp2f((float)(bmax - b) * kInvR);
-  const int k0 = bmax - kB + 1;
-  for (int i = 0; i < nleave; ++i) {
-    const int k = k0 + i;
+// The window's lowest bin moves up from key klo to key nlo: bins leaving the
+// window add their mass to the new lowest bin, which holds every score below
+// the window.
+static __device__ __noinline__ void fold_window(float* hist_col, int klo, int nlo) {
+  const int k1 = min(nlo - 1, klo + kB - 1);
+  float acc = 0.f;
+  for (int k = klo; k <= k1; ++k) {
     float& hv = hist_col[(k & (kB - 1)) * kRows];
-    if (hv != 0.f) {
-      tail += hv * exp2f((float)(k - b) * kInvR);
-      hv = 0.f;
-    }
+    acc += hv;
+    hv = 0.f;
   }
-  return tail;
+  hist_col[(nlo & (kB - 1)) * kRows] += acc;
 }
 
-// Insertion sort of list entries [0, n) into the (z desc, index asc) order.
+// The reference moves up by `shift` log2 units: every mass scales by 2^-shift
+// (exact, barring underflow) and every key moves down by 8 * shift.
+static __device__ __noinline__ void rebase_window(float* hist_col, int kmax, int shift) {
+  float v[kB];
+  for (int i = 0; i < kB; ++i) {
+    float& hv = hist_col[((kmax - i) & (kB - 1)) * kRows];
+    v[i] = hv;
+    hv = 0.f;
+  }
+  for (int i = 0; i < kB; ++i)
+    hist_col[((kmax - i - 8 * shift) & (kB - 1)) * kRows] = ldexpf(v[i], -shift);
+}
+
+// Insertion sort of list entries [0, n) into the (score desc, index asc) order.
 static __device__ __noinline__ void sort_entries(float* lz_col, uint16_t* lj_col, int n) {
   for (int i = 1; i < n; ++i) {
     const float z = lz_col[i * kRows];
@@ -98,20 +111,12 @@ static __device__ __noinline__ void sort_entries(float* lz_col, uint16_t* lj_col
   }
 }
 
-// Offer (z, j) to a list holding the kL best keys seen so far; state packs the
-// entry count (bits 0..7) and an "in order" flag (bit 8). Entries are appended
-// unsorted until the list is full; it is sorted once then, and later offers
-// replace the last entry by sorted insertion. Returns the new state.
-static __device__ __noinline__ int offer_entry(float* lz_col, uint16_t* lj_col, int state, float z,
-                                        int j) {
-  int n = state & 0xff;
-  bool sorted = (state >> 8) & 1;
-  if (n < kL) {
-    lz_col[n * kRows] = z;
-    lj_col[n * kRows] = (uint16_t)j;
-    return (n + 1);  // not in order any more
-  }
-  if (!sorted) sort_entries(lz_col, lj_col, n);
+// Offer (z, j) to a full list (kL entries) of the best keys seen so far; sorts
+// the list first when it is not in order. The entry replaces the last one by
+// sorted insertion when it comes before it.
+static __device__ __noinline__ void offer_full(float* lz_col, uint16_t* lj_col, bool sorted,
+                                               float z, int j) {
+  if (!sorted) sort_entries(lz_col, lj_col, kL);
   if (before(z, j, lz_col[(kL - 1) * kRows], (int)lj_col[(kL - 1) * kRows])) {
     int pos = kL - 1;
     while (pos > 0 && before(z, j, lz_col[(pos - 1) * kRows], (int)lj_col[(pos - 1) * kRows])) {
@@ -122,142 +127,178 @@ static __device__ __noinline__ int offer_entry(float* lz_col, uint16_t* lj_col, 
     lz_col[pos * kRows] = z;
     lj_col[pos * kRows] = (uint16_t)j;
   }
-  return kL | (1 << 8);
 }
 
 struct RowSel {
   float* hist_col;   // &hist[0][row]
   float* lz_col;     // &lz[0][row]
   uint16_t* lj_col;  // &lj[0][row]
-  const float* wbin;
-  int bmax;
-  float tail;
-  int bstar;
-  float need;
-  int lstate;     // list entries | (in order << 8)
-  bool open;      // cut not found yet
-  bool bounded;   // only keys after (bz, bj) are offered (extra passes)
+  float zs;          // log2(e) / sqrt(d): z = score * zs in log2 units
+  float ref;         // reference of the masses (integer, log2 units)
+  int kmax;          // key of the running maximum (kNoKey before the first score)
+  int klo;           // key of the lowest window bin (kmax - kB + 1)
+  int kcut;          // after finish1: keys above kcut are selected outright ...
+  int kcut_lo;       // ... keys in [kcut_lo, kcut] form the cut bin
+  float need;        // mass still to take from the cut bin (units of 2^ref)
+  int ln;            // list entries
+  bool lsorted;      // list in (score desc, index asc) order
+  bool ovf;          // the emission pass met more cut-bin scores than the list holds
+  bool open;         // cut not found yet
+  bool bounded;      // only keys after (bz, bj) are offered (extra passes)
+  bool range_err;    // a score outside +-kZLimit log2 units
   float bz;
   int bj;
 
-  __device__ __forceinline__ void init(Smem* s, int t) {
+  __device__ __forceinline__ void init(Smem* s, int t, float zscale) {
     hist_col = &s->hist[0][t];
     lz_col = &s->lz[0][t];
     lj_col = &s->lj[0][t];
-    wbin = s->wbin;
-    bmax = kNone;
-    tail = 0.f;
-    bstar = kNone;
+    zs = zscale;
+    ref = 0.f;
+    kmax = kNoKey;
+    klo = 0;
+    kcut = INT_MAX;     // nothing above, nothing in the cut bin until finish1
+    kcut_lo = INT_MAX;
     need = 0.f;
-    lstate = 1 << 8;
+    ln = 0;
+    lsorted = true;
+    ovf = false;
     open = false;
     bounded = false;
+    range_err = false;
     bz = 0.f;
     bj = 0;
 #pragma unroll 8
     for (int k = 0; k < kB; ++k) hist_col[k * kRows] = 0.f;
   }
 
-  __device__ __forceinline__ void raise_max(int b) {
-    if (bmax == kNone) {
-      bmax = b;
+  __device__ __forceinline__ float mass(float score) const {
+    return fast_exp2(fmaf(score, zs, -ref));
+  }
+
+  // Make the window reach the raw score sm (a maximum of scores to come).
+  __device__ __forceinline__ void raise(float sm) {
+    const float zm = sm * zs;
+    if (!(fabsf(zm) < kZLimit)) {
+      range_err = true;
       return;
     }
-    tail = shift_window(hist_col, bmax, b, tail);
-    bmax = b;
+    if (kmax == kNoKey) {
+      ref = ceilf(zm);
+      kmax = mass_key(mass(sm));
+      klo = kmax - (kB - 1);
+      return;
+    }
+    if (zm > ref + kRefStep) {  // keep masses far from overflow
+      const int shift = (int)(ceilf(zm) - ref);
+      rebase_window(hist_col, kmax, shift);
+      ref += (float)shift;
+      kmax -= 8 * shift;
+      klo -= 8 * shift;
+    }
+    const int k = mass_key(mass(sm));
+    if (k > kmax) {
+      fold_window(hist_col, klo, k - (kB - 1));
+      kmax = k;
+      klo = k - (kB - 1);
+    }
   }
 
-  __device__ __forceinline__ void pass1(float z) {
-    const int b = __float2int_rd(z * (float)kR);
-    if (b > bmax) raise_max(b);
-    if (b > bmax - kB)
-      hist_col[(b & (kB - 1)) * kRows] += fast_exp2(z - (float)b * kInvR);
-    else
-      tail += fast_exp2(z - (float)bmax * kInvR);
+  // Histogram update with mass u (0 for a column that is not a candidate)
+  // whose key does not exceed kmax; keys below the window land in its lowest
+  // bin.
+  __device__ __forceinline__ void add_mass(float u) {
+    const int k = max(mass_key(u), klo);
+    hist_col[(k & (kB - 1)) * kRows] += u;
   }
 
-  // Eight scores at once (the hot loop of pass 1): one running-maximum check
-  // for the group, then the bin updates. `valid` bit c enables z[c].
-  __device__ __forceinline__ void pass1x8(const float (&z)[8], unsigned valid) {
-    int b[8];
-    int bm = kNone;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      b[c] = __float2int_rd(z[c] * (float)kR);
-      if ((valid >> c) & 1u) bm = max(bm, b[c]);
-    }
-    if (bm > bmax) raise_max(bm);
-    const int lo = bmax - kB;
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      if (!((valid >> c) & 1u)) continue;
-      if (b[c] > lo)
-        hist_col[(b[c] & (kB - 1)) * kRows] += fast_exp2(z[c] - (float)b[c] * kInvR);
-      else
-        tail += fast_exp2(z[c] - (float)bmax * kInvR);
-    }
+  // One score of the histogram pass (raises the window when needed).
+  __device__ __forceinline__ void pass1(float score) {
+    raise(score);
+    if (!range_err) add_mass(mass(score));
   }
 
   __device__ __forceinline__ void finish1(float p) {
-    if (bmax == kNone) {
-      bstar = kNone;
+    if (kmax == kNoKey || range_err) {
       open = false;
       return;
     }
-    float Z = tail;
-    for (int i = kB - 1; i >= 0; --i) Z += hist_col[((bmax - i) & (kB - 1)) * kRows] * wbin[i];
+    float Z = 0.f;  // smallest bins first
+    for (int i = kB - 1; i >= 0; --i) Z += hist_col[((kmax - i) & (kB - 1)) * kRows];
     const float target = p * Z;
     float cum = 0.f;
-    bstar = kTail;
-    for (int i = 0; i < kB; ++i) {
-      const float m = hist_col[((bmax - i) & (kB - 1)) * kRows] * wbin[i];
+    int kc = klo;
+    for (int i = 0; i < kB - 1; ++i) {
+      const float m = hist_col[((kmax - i) & (kB - 1)) * kRows];
       if (cum + m >= target) {
-        bstar = bmax - i;
+        kc = kmax - i;
         break;
       }
       cum += m;
     }
     need = target - cum;
     open = true;
+    lsorted = false;   // the emission pass appends the cut bin in column order
+    kcut = kc;
+    kcut_lo = kc == klo ? INT_MIN : kc;   // the lowest bin holds everything below it
+  }
+
+  // Emission pass, one score, without branches: true when the score lies
+  // above the cut bin (selected outright); a cut-bin score is appended to the
+  // list. The list has one spare slot, so the append writes unconditionally;
+  // a cut-bin score that finds the list full sets ovf, and the row then
+  // collects its cut bin again, in order, in an extra pass.
+  __device__ __forceinline__ bool pass2(float score, int j, bool valid) {
+    const int k = mass_key(mass(score));
+    const bool above = valid && k > kcut;
+    const bool inb = valid && k >= kcut_lo && k <= kcut;
+    lz_col[ln * kRows] = score;
+    lj_col[ln * kRows] = (uint16_t)j;
+    const bool room = ln < kL;
+    ovf = ovf || (inb && !room);
+    ln += (inb && room) ? 1 : 0;
+    return above;
   }
 
   __device__ __forceinline__ void offer(float z, int j) {
     if (bounded && !before(bz, bj, z, j)) return;
-    lstate = offer_entry(lz_col, lj_col, lstate, z, j);
-  }
-
-  __device__ __forceinline__ bool in_cut_bin(int b) const {
-    return bstar == kTail ? b <= bmax - kB : b == bstar;
-  }
-
-  // Emission pass: true when z lies above the cut bin (selected outright);
-  // elements of the cut bin go to the list.
-  __device__ __forceinline__ bool pass2(float z, int j) {
-    const int b = __float2int_rd(z * (float)kR);
-    const bool above = bstar == kTail ? b > bmax - kB : b > bstar;
-    if (open && in_cut_bin(b)) offer(z, j);
-    return above;
+    if (ln < kL) {
+      lz_col[ln * kRows] = z;
+      lj_col[ln * kRows] = (uint16_t)j;
+      ++ln;
+      lsorted = false;
+    } else {
+      offer_full(lz_col, lj_col, lsorted, z, j);
+      lsorted = true;
+    }
   }
 
   // Extra pass for a row whose cut is still open.
-  __device__ __forceinline__ void pass_more(float z, int j) {
+  __device__ __forceinline__ void pass_more(float score, int j) {
     if (!open) return;
-    const int b = __float2int_rd(z * (float)kR);
-    if (in_cut_bin(b)) offer(z, j);
+    const int k = mass_key(mass(score));
+    if (k >= kcut_lo && k <= kcut) offer(score, j);
   }
 
   // After a pass over the cut bin: how many leading list entries are selected.
   // Closes the cut when reached (or when the bin is exhausted); otherwise all
-  // kL entries are taken and the next pass starts after the last of them.
+  // kL entries are taken and the next pass starts after the last of them. A
+  // list that overflowed during the emission pass is dropped unused: the next
+  // pass collects the best kL of the cut bin in order.
   __device__ __forceinline__ int settle() {
     if (!open) return 0;
-    const int n = lstate & 0xff;
-    if (!((lstate >> 8) & 1)) sort_entries(lz_col, lj_col, n);
-    lstate = n | (1 << 8);
-    const float ref = (float)bmax * kInvR;
+    if (ovf) {
+      ovf = false;
+      ln = 0;
+      lsorted = true;
+      return 0;
+    }
+    const int n = ln;
+    if (!lsorted) sort_entries(lz_col, lj_col, n);
+    lsorted = true;
     float cum = 0.f;
     for (int i = 0; i < n; ++i) {
-      cum += fast_exp2(lz_col[i * kRows] - ref);
+      cum += mass(lz_col[i * kRows]);
       if (cum >= need) {
         open = false;
         return i + 1;
@@ -275,8 +316,28 @@ struct RowSel {
   }
 
   __device__ __forceinline__ int list_j(int i) const { return (int)lj_col[i * kRows]; }
-  __device__ __forceinline__ void reset_list() { lstate = 1 << 8; }
+  __device__ __forceinline__ void reset_list() {
+    ln = 0;
+    lsorted = true;
+  }
 };
+
+// 32 x 32 bit transpose across a warp: on entry lane r holds row r (bit c =
+// column c), on return lane c holds column c (bit r = row r). Each stage swaps
+// the off-diagonal blocks of one size with the partner lane.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) {
+    const uint32_t mhi = s == 16 ? 0xFFFF0000u
+                       : s == 8  ? 0xFF00FF00u
+                       : s == 4  ? 0xF0F0F0F0u
+                       : s == 2  ? 0xCCCCCCCCu
+                                 : 0xAAAAAAAAu;
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, s);
+    x = (lane & s) ? ((x & mhi) | ((y >> s) & ~mhi)) : ((x & ~mhi) | ((y << s) & mhi));
+  }
+  return x;
+}
 
 }  // namespace sel
 

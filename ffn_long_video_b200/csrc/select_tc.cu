@@ -206,11 +206,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_before();
       mbar_arrive(q_full);
     }
-    sel::init_table(ss, row);
-    asm volatile("bar.sync 1, 128;" ::: "memory");
     if (c_hi >= 0) {
       sel::RowSel s;
-      s.init(ss, row);
+      s.init(ss, row, a.zscale);
       const int ncand = own > 0 ? own : 0;
       uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
@@ -227,51 +225,76 @@ __global__ void __launch_bounds__(THREADS, 2)
           tc_fence_after();
           const int j0 = ch * NC;
           const uint32_t tcol = tmem_base + lane_base + sb * NC;
-          uint32_t mine = 0u;  // emission pass: mask word of column j0 + lane, this warp
+          // candidates of this row in the chunk: columns [0, nv)
+          const int nv = min(max(ncand - j0, 0), NC);
+          if (pass == 0) {
+            // histogram: the whole chunk in registers, the buffer released at once
+            uint32_t acc[NC];
+            tmem_ld32(tcol, acc);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&s_empty[sb]);
+            if (nv > 0) {
+              // the chunk maximum first: the window moves at most once per chunk
+              float m = -INFINITY;
+#pragma unroll
+              for (int c = 0; c < NC; ++c)
+                if (c < nv) m = fmaxf(m, __uint_as_float(acc[c]));
+              s.raise(m);
+              if (!s.range_err) {
+#pragma unroll
+                for (int c = 0; c < NC; ++c)
+                  s.add_mass(c < nv ? s.mass(__uint_as_float(acc[c])) : 0.f);
+              }
+            }
+            continue;
+          }
+          // emission (pass 1) and extra passes, 8 columns at a time
+          uint32_t bits = 0u;  // bit c: column j0 + c selected outright by this row
 #pragma unroll 1
           for (int q = 0; q < NC / 8; ++q) {
             uint32_t acc[8];
             tmem_ld8(tcol + q * 8, acc);
             tmem_ld_wait();
-            if (pass == 0) {
-              float z[8];
-              unsigned valid_bits = 0u;
+            if (pass == 1) {
+              uint32_t gb = 0u;
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                z[c] = __uint_as_float(acc[c]) * a.zscale;
-                if (j0 + q * 8 + c < ncand) valid_bits |= 1u << c;
-              }
-              if (valid_bits) s.pass1x8(z, valid_bits);
-            } else if (pass == 1) {
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const int j = j0 + q * 8 + c;
-                bool selb = false;
-                if (j < ncand) selb = s.pass2(__uint_as_float(acc[c]) * a.zscale, j);
-                nsel += selb;
-                const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
-                if (lane == q * 8 + c) mine = w;
-              }
+              for (int c = 0; c < 8; ++c)
+                if (s.pass2(__uint_as_float(acc[c]), j0 + q * 8 + c, q * 8 + c < nv)) gb |= 1u << c;
+              bits |= gb << (q * 8);
             } else if (s.open) {
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const int j = j0 + q * 8 + c;
-                if (j < ncand) s.pass_more(__uint_as_float(acc[c]) * a.zscale, j);
-              }
+              for (int c = 0; c < 8; ++c)
+                if (q * 8 + c < nv) s.pass_more(__uint_as_float(acc[c]), j0 + q * 8 + c);
             }
           }
           tc_fence_before();
           mbar_arrive(&s_empty[sb]);
           if (pass == 1) {
+            nsel += __popc(bits);
+            // lane L now takes the mask word of column j0 + L (bit r = row r)
+            uint32_t word = sel::warp_transpose32(bits, lane);
+            // the own cube of each row, for the rows whose own cube is in the chunk
+            const int rel = own - j0;
+            unsigned pending = __ballot_sync(0xffffffffu, rel >= 0 && rel < NC);
+            while (pending) {
+              const int o = __shfl_sync(0xffffffffu, rel, __ffs(pending) - 1);
+              const unsigned same = __ballot_sync(0xffffffffu, rel == o);
+              if (lane == o) word |= same;
+              pending &= ~same;
+            }
             const int jl = j0 + lane;
-            if (jl < c_hi) tmask[(size_t)jl * 4 + wq] = mine;
+            if (jl < c_hi) tmask[(size_t)jl * 4 + wq] = word;
           }
         }
         // Every row warp reaches the vote barrier below, even after a failed
         // wait (the abort flag then ends the loop), so the named barrier
         // cannot strand the other warps.
         if (pass == 0) {
-          if (ok) s.finish1(a.p);
+          if (ok) {
+            s.finish1(a.p);
+            if (s.range_err) set_status(hdr, ADASPARK_DEV_RANGE, 0x8800u);
+          }
           continue;
         }
         if (pass == 1) {

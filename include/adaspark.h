@@ -57,6 +57,9 @@ typedef enum { ADASPARK_BF16 = 0, ADASPARK_FP32 = 1 } adaspark_dtype;
 /* Bits of the device status word (adaspark_read_device_status detail). */
 #define ADASPARK_DEV_BAD_LAYOUT   0x1u  /* cube_ids / cube_offsets / text_mask inconsistent */
 #define ADASPARK_DEV_TIMEOUT      0x2u  /* a bounded wait inside a kernel expired          */
+#define ADASPARK_DEV_RANGE        0x4u  /* a row's largest cube score is out of range:     */
+                                        /* |q.kbar| * log2(e) / sqrt(d) must stay below    */
+                                        /* 2^18; such a row keeps only its own cube        */
 
 /* Human-readable name of a return code. Never NULL. */
 const char *adaspark_status_string(int status);
