@@ -32,7 +32,7 @@ namespace adaspark {
 namespace sel {
 
 constexpr int kB = 64;                // bins in the window (8 log2 units, 8 bins each)
-constexpr int kL = 32;                // list entries per row (one more slot as scratch)
+constexpr int kL = 31;                // list entries per row (one more slot as scratch)
 constexpr int kRows = 128;
 constexpr int kNoKey = INT_MIN;       // row without candidates
 constexpr float kRefStep = 64.f;      // new reference once the maximum passes ref + 64
@@ -58,11 +58,15 @@ __device__ __forceinline__ bool before(float s1, int j1, float s2, int j2) {
   return s1 > s2 || (s1 == s2 && j1 < j2);
 }
 
+// Per-row storage, one column per row. The histogram is dead once the cut bin
+// is known, and the list is only used from then on, so the list (raw scores
+// q . kbar_j in rows [0, kL], cube indices in rows [kL + 1, 2 kL + 1]) takes
+// the histogram's place. Each thread touches only its own column, so the reuse
+// needs no synchronization between rows.
 struct Smem {
   float hist[kB][kRows];
-  float lz[kL + 1][kRows];     // raw scores q . kbar_j of the list entries
-  uint16_t lj[kL + 1][kRows];  // their cube indices
 };
+static_assert(2 * (kL + 1) <= kB, "the cut list must fit in the histogram's storage");
 
 // Out-of-line cold paths take and return plain values, so that the per-row
 // state below stays in registers (a member function called out of line would
@@ -96,12 +100,12 @@ static __device__ __noinline__ void rebase_window(float* hist_col, int kmax, int
 }
 
 // Insertion sort of list entries [0, n) into the (score desc, index asc) order.
-static __device__ __noinline__ void sort_entries(float* lz_col, uint16_t* lj_col, int n) {
+static __device__ __noinline__ void sort_entries(float* lz_col, int* lj_col, int n) {
   for (int i = 1; i < n; ++i) {
     const float z = lz_col[i * kRows];
-    const uint16_t j = lj_col[i * kRows];
+    const int j = lj_col[i * kRows];
     int k = i;
-    while (k > 0 && before(z, j, lz_col[(k - 1) * kRows], (int)lj_col[(k - 1) * kRows])) {
+    while (k > 0 && before(z, j, lz_col[(k - 1) * kRows], lj_col[(k - 1) * kRows])) {
       lz_col[k * kRows] = lz_col[(k - 1) * kRows];
       lj_col[k * kRows] = lj_col[(k - 1) * kRows];
       --k;
@@ -114,25 +118,25 @@ static __device__ __noinline__ void sort_entries(float* lz_col, uint16_t* lj_col
 // Offer (z, j) to a full list (kL entries) of the best keys seen so far; sorts
 // the list first when it is not in order. The entry replaces the last one by
 // sorted insertion when it comes before it.
-static __device__ __noinline__ void offer_full(float* lz_col, uint16_t* lj_col, bool sorted,
+static __device__ __noinline__ void offer_full(float* lz_col, int* lj_col, bool sorted,
                                                float z, int j) {
   if (!sorted) sort_entries(lz_col, lj_col, kL);
-  if (before(z, j, lz_col[(kL - 1) * kRows], (int)lj_col[(kL - 1) * kRows])) {
+  if (before(z, j, lz_col[(kL - 1) * kRows], lj_col[(kL - 1) * kRows])) {
     int pos = kL - 1;
-    while (pos > 0 && before(z, j, lz_col[(pos - 1) * kRows], (int)lj_col[(pos - 1) * kRows])) {
+    while (pos > 0 && before(z, j, lz_col[(pos - 1) * kRows], lj_col[(pos - 1) * kRows])) {
       lz_col[pos * kRows] = lz_col[(pos - 1) * kRows];
       lj_col[pos * kRows] = lj_col[(pos - 1) * kRows];
       --pos;
     }
     lz_col[pos * kRows] = z;
-    lj_col[pos * kRows] = (uint16_t)j;
+    lj_col[pos * kRows] = j;
   }
 }
 
 struct RowSel {
   float* hist_col;   // &hist[0][row]
-  float* lz_col;     // &lz[0][row]
-  uint16_t* lj_col;  // &lj[0][row]
+  float* lz_col;     // list scores, in the histogram's place
+  int* lj_col;       // list cube indices, likewise
   float zs;          // log2(e) / sqrt(d): z = score * zs in log2 units
   float ref;         // reference of the masses (integer, log2 units)
   int kmax;          // key of the running maximum (kNoKey before the first score)
@@ -151,8 +155,8 @@ struct RowSel {
 
   __device__ __forceinline__ void init(Smem* s, int t, float zscale) {
     hist_col = &s->hist[0][t];
-    lz_col = &s->lz[0][t];
-    lj_col = &s->lj[0][t];
+    lz_col = &s->hist[0][t];
+    lj_col = reinterpret_cast<int*>(&s->hist[kL + 1][t]);
     zs = zscale;
     ref = 0.f;
     kmax = kNoKey;
@@ -253,7 +257,7 @@ struct RowSel {
     const bool above = valid && k > kcut;
     const bool inb = valid && k >= kcut_lo && k <= kcut;
     lz_col[ln * kRows] = score;
-    lj_col[ln * kRows] = (uint16_t)j;
+    lj_col[ln * kRows] = j;
     const bool room = ln < kL;
     ovf = ovf || (inb && !room);
     ln += (inb && room) ? 1 : 0;
@@ -264,7 +268,7 @@ struct RowSel {
     if (bounded && !before(bz, bj, z, j)) return;
     if (ln < kL) {
       lz_col[ln * kRows] = z;
-      lj_col[ln * kRows] = (uint16_t)j;
+      lj_col[ln * kRows] = j;
       ++ln;
       lsorted = false;
     } else {
@@ -311,11 +315,11 @@ struct RowSel {
     need -= cum;
     bounded = true;
     bz = lz_col[(kL - 1) * kRows];
-    bj = (int)lj_col[(kL - 1) * kRows];
+    bj = lj_col[(kL - 1) * kRows];
     return n;
   }
 
-  __device__ __forceinline__ int list_j(int i) const { return (int)lj_col[i * kRows]; }
+  __device__ __forceinline__ int list_j(int i) const { return lj_col[i * kRows]; }
   __device__ __forceinline__ void reset_list() {
     ln = 0;
     lsorted = true;

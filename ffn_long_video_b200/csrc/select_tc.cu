@@ -18,8 +18,10 @@
 //              A = the query tile held in TMEM
 //   warps 2-5  one thread per row: Q gather into TMEM, histogram pass, cut,
 //              emission of the 128-bit row masks, tile cube list.
-// The query tile lives in tensor memory (64 columns) rather than shared memory,
-// so a CTA needs under 100 KB of shared memory and two CTAs share an SM.
+// The query tile lives in tensor memory (64 columns) rather than shared memory
+// and the cut lists reuse the histogram's storage, so a CTA needs about 105 KB
+// of shared memory (three K stages and the per-row histograms) and two CTAs
+// share an SM.
 #include "attn_kernels.h"
 #include "select.cuh"
 
@@ -27,7 +29,7 @@ namespace adaspark {
 namespace seltc {
 
 constexpr int NC = 32;                          // cubes per chunk (MMA N)
-constexpr int STAGES = 2;
+constexpr int STAGES = 3;
 constexpr int SBUF = 4;                         // TMEM score buffers
 constexpr int THREADS = 192;
 constexpr int BOX_BYTES = NC * 128;             // 32 cubes x 64 dims bf16
