@@ -12,6 +12,7 @@ Parity status per function (what pins it is in ``tests/test_oracle_pins.py``):
 * ``cube_partition``        pinned (brute-force sort order on small grids)
 * ``cube_mean_keys``        pinned (invariants: zero residual sum, constant cubes)
 * ``top_p``                 pinned (exhaustive subset enumeration, closed forms)
+* ``top_k``                 pinned (exhaustive k-subset enumeration, closed forms)
 * ``select_cubes``          pinned (uniform closed form, 2-cube sigmoid cut, GQA map)
 * ``attention_given_sets``  pinned (torch SDPA in float64 with a mask; first token)
 * ``ffn_select``            pinned (closed forms on scaled tokens, brute force)
@@ -27,6 +28,8 @@ from .adaspark_ref import (  # noqa: F401
     softmax,
     top_p,
     top_p_margin,
+    top_k,
+    top_k_margin,
     select_cubes,
     attention_given_sets,
     cube_attn,

@@ -180,18 +180,56 @@ def top_p_margin(P, p):
     return out.reshape(P.shape[:-1])
 
 
-def select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=None, with_margin=False):
+def top_k(P, k):
+    """Top-K set of a probability vector: the fixed-size selection that the
+    AdaSpark paper compares with Top-p (ablation table of selection strategies,
+    row "Top-K"). The k entries of largest probability in the (probability
+    descending, index ascending) order; every entry when there are at most k.
+    Returns a boolean mask over the entries."""
+    if int(k) != k or k < 1:
+        raise ValueError("k must be a positive integer")
+    P = np.asarray(P, dtype=np.float64)
+    m = P.shape[-1]
+    keep = np.zeros(P.shape, dtype=bool)
+    if m == 0:
+        return keep
+    flat = P.reshape(-1, m)
+    kflat = keep.reshape(-1, m)
+    order = np.argsort(-flat, axis=1, kind="stable")
+    kk = min(int(k), m)
+    for r in range(flat.shape[0]):
+        kflat[r, order[r, :kk]] = True
+    return keep
+
+
+def top_k_margin(P, k):
+    """Distance of a Top-K set from flipping: P_(k) - P_(k+1) in the sorted
+    order used by ``top_k`` (+inf when there are at most k entries)."""
+    P = np.asarray(P, dtype=np.float64)
+    m = P.shape[-1]
+    flat = P.reshape(-1, m)
+    out = np.full(flat.shape[0], np.inf)
+    if m > k:
+        srt = -np.sort(-flat, axis=1)
+        out = srt[:, k - 1] - srt[:, k]
+    return out.reshape(P.shape[:-1])
+
+
+def select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=None, with_margin=False,
+                 k=None):
     """AdaS-Attn cube selection (key design 2, formula P_i and S_i).
 
     For visual token t in cube i and query head h: P = softmax over the
     preceding cubes j < i of q . k_bar_j / sqrt(d), k_bar of KV head
-    floor(h / (hq/hkv)); S = Top-p(P, p).  Returns a boolean array
+    floor(h / (hq/hkv)); S = Top-p(P, p), or Top-K(P, k) when ``k`` is given
+    (then ``p`` is ignored).  Returns a boolean array
     sel[len(tokens), hq, C] (sel[r, h, j] is True when cube j is selected; the
     own cube is not marked here, it is always attended causally) and, when
     asked, the cut margins [len(tokens), hq] (+inf where nothing can flip).
     ``tokens`` defaults to every visual token.
     """
-    _check_p(p)
+    if k is None:
+        _check_p(p)
     off = np.asarray(cube_offsets)
     C = len(off) - 1
     d = Q.shape[-1]
@@ -212,9 +250,14 @@ def select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=None, with_margin
             kv = h // g
             s = cube_scores(Qf[rows, h, :], kbar[:i, kv, :], d)   # [rows, i]
             P = softmax(s, axis=1)
-            sel[rows, h, :i] = top_p(P, p)
-            if with_margin:
-                margin[rows, h] = top_p_margin(P, p)
+            if k is None:
+                sel[rows, h, :i] = top_p(P, p)
+                if with_margin:
+                    margin[rows, h] = top_p_margin(P, p)
+            else:
+                sel[rows, h, :i] = top_k(P, k)
+                if with_margin:
+                    margin[rows, h] = top_k_margin(P, k)
     if with_margin:
         return sel, margin
     return sel

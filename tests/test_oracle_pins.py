@@ -115,6 +115,70 @@ def test_top_p_margin_values():
     assert oracle.top_p_margin(np.array([0.25] * 4), 0.6) == 0.0   # exact tie at the cut
 
 
+def _brute_top_k(P, k):
+    """Among all subsets of size min(k, m): maximal mass, then lexicographically
+    lowest index tuple (the tie rule), by enumeration."""
+    m = len(P)
+    kk = min(k, m)
+    best = None
+    for S in itertools.combinations(range(m), kk):
+        key = (-sum(P[j] for j in S), S)
+        if best is None or key < best:
+            best = key
+    return set(best[1])
+
+
+def test_top_k_brute_force():
+    rng = np.random.default_rng(9)
+    for trial in range(300):
+        m = int(rng.integers(1, 11))
+        k = int(rng.integers(1, 12))
+        # binary-exact masses with many ties
+        w = rng.integers(1, 5 if trial % 2 else 300, size=m).astype(np.float64) / 1024.0
+        got = set(np.nonzero(oracle.top_k(w, k))[0].tolist())
+        assert got == _brute_top_k(w, k), (w, k)
+
+
+@pytest.mark.parametrize("m,k", [(7, 3), (10, 1), (13, 13), (5, 9), (64, 20)])
+def test_top_k_uniform_closed_form(m, k):
+    keep = oracle.top_k(np.full(m, 1.0 / m), k)
+    assert keep.sum() == min(k, m)
+    assert keep[:min(k, m)].all()        # ties go to the lower indices
+
+
+def test_top_k_degenerate_and_margin():
+    P = np.array([0.1, 0.4, 0.4, 0.1])
+    assert np.nonzero(oracle.top_k(P, 1))[0].tolist() == [1]
+    assert np.nonzero(oracle.top_k(P, 3))[0].tolist() == [0, 1, 2]
+    assert oracle.top_k(np.zeros(0), 2).shape == (0,)
+    for bad in (0, -1, 1.5):
+        with pytest.raises(ValueError):
+            oracle.top_k(P, bad)
+    assert oracle.top_k_margin(np.array([0.5, 0.3, 0.2]), 1) == pytest.approx(0.2)
+    assert oracle.top_k_margin(np.array([0.5, 0.3, 0.2]), 2) == pytest.approx(0.1)
+    assert oracle.top_k_margin(np.array([0.5, 0.3, 0.2]), 3) == np.inf
+    assert oracle.top_k_margin(P, 1) == 0.0     # exact tie at the cut (0.4 / 0.4)
+    assert oracle.top_k_margin(P, 2) == pytest.approx(0.3)   # both 0.4 taken
+
+
+def test_select_top_k_uniform_means():
+    """Identical cube means with Top-K: the min(k, c) lowest-index preceding
+    cubes (own cube excluded from the candidates)."""
+    rng = np.random.default_rng(4)
+    C, n, hq, hkv, d = 9, 3, 2, 1, 8
+    off = np.arange(C + 1) * n
+    N = C * n
+    Q = rng.standard_normal((N, hq, d))
+    K = np.tile(rng.standard_normal((1, hkv, d)), (N, 1, 1))
+    for k in (1, 3, 20):
+        sel = oracle.select_cubes(Q, K, off, N, hq, hkv, 0.5, k=k)
+        for t in range(N):
+            c = t // n
+            kk = min(k, c)
+            assert (sel[t].sum(axis=1) == kk).all()
+            assert sel[t, :, :kk].all() and not sel[t, :, c:].any()
+
+
 # ---------------------------------------------------------------- cube means
 def test_cube_mean_keys_invariants():
     rng = np.random.default_rng(1)
