@@ -38,6 +38,36 @@ sys.path.insert(0, ROOT)
 METRIC = "AdaSpark layer tokens/s at 64K visual tokens (7B shape); % bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
+# kernel (timer name) -> source file whose build the DRAM counters were taken on
+KERNEL_SOURCES = {"attn_tc": "attn_tc.cu", "select_tc": "select_tc.cu",
+                  "ffn_gemm1_tc": "ffn_gemm_tc.cu", "ffn_gemm2_tc": "ffn_gemm_tc.cu"}
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+    `kernel` on `workload`, from the ncu summary profiles/<kernel>_<workload>.md,
+    which records the counters and the SHA-256 of the kernel's source file at
+    capture time. None when there is no summary or the source has changed
+    since (the counters then describe another kernel)."""
+    import hashlib
+    src = KERNEL_SOURCES.get(kernel)
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if src is None or not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    try:
+        want = fields["source-sha256"]
+        nbytes = int(fields["traffic-bytes-per-launch"])
+    except (KeyError, ValueError):
+        return None
+    with open(os.path.join(ROOT, "ffn_long_video_b200", "csrc", src), "rb") as f:
+        have = hashlib.sha256(f.read()).hexdigest()
+    return nbytes if have == want else None
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -225,6 +255,7 @@ def run_ours(args, rank, world, device):
 
     # ---------------- roofline of the dominant kernel
     peaks, peak_src = load_peaks()
+    traffic_of = lambda name: load_traffic(name, cfg.name)
     dom = max(ktimes.items(), key=lambda kv: kv[1][1])
     dname, (dn, dms) = dom
     work, unit, bound = kernel_work(dname, cfg, attn_stats, ffn_stats)
@@ -237,13 +268,13 @@ def run_ours(args, rank, world, device):
             roof = {"kernel": dname, "bound": "tensor", "achieved": round(achieved, 1),
                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a step)",
-                    "traffic": None, "ms_per_launch": round(per_launch_ms, 4)}
+                    "traffic": traffic_of(dname), "ms_per_launch": round(per_launch_ms, 4)}
         else:
             achieved = work / (per_launch_ms / 1e3) / 1e9
             peak = peaks["hbm_gbs"]
             roof = {"kernel": dname, "bound": "hbm", "achieved": round(achieved, 1),
                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                    "peak_source": f"{peak_src} hbm_gbs", "traffic": None,
+                    "peak_source": f"{peak_src} hbm_gbs", "traffic": traffic_of(dname),
                     "ms_per_launch": round(per_launch_ms, 4)}
     kernels = {}
     for k, (n, ms) in sorted(ktimes.items(), key=lambda kv: -kv[1][1]):

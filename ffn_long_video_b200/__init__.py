@@ -5,7 +5,7 @@ kernels.  Torch tensors supply device memory and the current CUDA stream.  The
 binding fails loudly when the library is missing; there is no fallback.
 
 Entry points (same names as include/adaspark.h, without the prefix):
-``cube_count``, ``cube_partition``, ``cube_attn``, ``attn_export_sets``,
+``cube_count``, ``cube_partition``, ``cube_attn``, ``cube_attn_topk``, ``attn_export_sets``,
 ``attn_read_stats``, ``token_ffn``, ``ffn_export_active``, ``ffn_read_stats``,
 ``read_device_status``, ``timer_enable``, ``timer_read``, ``launch_count``,
 ``device_check``, ``status_string``.
@@ -68,6 +68,8 @@ def lib():
             "adaspark_cube_attn_workspace": (sz, [i32] * 7),
             "adaspark_cube_attn": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 6 + [f32, vp, vp, sz,
                                                                                    vp]),
+            "adaspark_cube_attn_topk": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 7 + [vp, vp, sz,
+                                                                                    vp]),
             "adaspark_attn_export_sets": (i32, [vp, vp] + [i32] * 7 + [vp, vp]),
             "adaspark_attn_read_stats": (i32, [vp, ctypes.POINTER(_AttnStats), vp]),
             "adaspark_token_ffn_workspace": (sz, [i32] * 6),
@@ -178,6 +180,33 @@ def cube_attn(Q, K, V, cube_ids, cube_offsets, n_vis, p, out=None, workspace=Non
                                     _ptr(out), _ptr(workspace), workspace.numel(),
                                     _stream(stream)),
            "adaspark_cube_attn")
+    return out, workspace
+
+
+def cube_attn_topk(Q, K, V, cube_ids, cube_offsets, n_vis, k, out=None, workspace=None,
+                   stream=None):
+    """AdaS-Attn with Top-K selection (the k most probable preceding cubes);
+    returns (out, workspace)."""
+    import torch
+    for t, nm in ((Q, "Q"), (K, "K"), (V, "V"), (cube_ids, "cube_ids"),
+                  (cube_offsets, "cube_offsets")):
+        _need(t, nm)
+    N, hq, d = Q.shape
+    hkv = K.shape[1]
+    C = cube_offsets.numel() - 1
+    dt = _dtype_code(Q)
+    if out is None:
+        out = torch.empty_like(Q)
+    if workspace is None:
+        nb = cube_attn_workspace_bytes(N, n_vis, C, hq, hkv, d, dt)
+        if nb == 0:
+            raise AdasparkError(EINVAL, "adaspark_cube_attn_workspace")
+        workspace = torch.empty(nb, dtype=torch.uint8, device=Q.device)
+    _check(lib().adaspark_cube_attn_topk(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(cube_ids),
+                                         _ptr(cube_offsets), C, n_vis, N, hq, hkv, d, int(k),
+                                         _ptr(out), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)),
+           "adaspark_cube_attn_topk")
     return out, workspace
 
 

@@ -55,13 +55,16 @@ size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq
   return make_attn_layout(G).total;
 }
 
-int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
-                       const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
-                       int n_vis, int n_tokens, int hq, int hkv, int d, float p, void* out,
-                       void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+// AdaS-Attn with Top-p (topk == 0) or Top-K (topk > 0, p unused) selection.
+static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype,
+                          const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                          int n_vis, int n_tokens, int hq, int hkv, int d, float p, int topk,
+                          void* out, void* workspace, size_t workspace_bytes, void* stream) {
   if (!Q || !K || !V || !cube_ids || !cube_offsets || !out || !workspace) return ADASPARK_EINVAL;
-  if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype) || !p_valid(p))
-    return ADASPARK_EINVAL;
+  if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return ADASPARK_EINVAL;
+  if (topk < 0 || (topk == 0 && !p_valid(p))) return ADASPARK_EINVAL;
   const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
   const AttnLayout L = make_attn_layout(G);
   if (workspace_bytes < L.total || !aligned(workspace, kAlign)) return ADASPARK_EINVAL;
@@ -74,7 +77,7 @@ int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.header);
-  const int dense = p >= 1.0f;
+  const int dense = topk == 0 && p >= 1.0f;
   if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
   if (dense && cudaMemsetAsync(&hdr->pad[0], kModeDense, 1, s) != cudaSuccess)
     return ADASPARK_ECUDA;
@@ -94,6 +97,7 @@ int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
   sa.G = G;
   sa.p = p;
   sa.zscale = (float)(1.4426950408889634 / std::sqrt((double)d));
+  sa.topk = topk;
 
   if (!dense && n_vis > 0 && G.n_vtiles > 0) {
     rc = cuda_rc(launch_cube_mean(K, dtype, cube_offsets, const_cast<float*>(sa.kbar),
@@ -117,8 +121,33 @@ int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
   aa.G = G;
   aa.dense = dense;
   aa.scale_log2 = sa.zscale;
+  // When the layer's K and V outgrow what L2 holds alongside the other
+  // traffic, visual tiles run one KV head after another, so that the blocks in
+  // use belong to one head; otherwise all heads of a token range run together
+  // (fewer CTAs then read the same lines at once).
+  const double kv_bytes = 2.0 * n_tokens * hkv * d * (dtype == ADASPARK_BF16 ? 2 : 4);
+  aa.kv_major = kv_bytes > 64.0 * 1024 * 1024 ? 1 : 0;
   if (dtype == ADASPARK_BF16) return cuda_rc(launch_attn_tc(aa, s));
   return cuda_rc(launch_attn_simt(aa, dtype, s));
+}
+
+extern "C" {
+
+int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
+                       const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                       int n_vis, int n_tokens, int hq, int hkv, int d, float p, void* out,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  return cube_attn_impl(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq, hkv,
+                        d, p, 0, out, workspace, workspace_bytes, stream);
+}
+
+int adaspark_cube_attn_topk(const void* Q, const void* K, const void* V, int dtype,
+                            const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                            int n_vis, int n_tokens, int hq, int hkv, int d, int k, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (k < 1) return ADASPARK_EINVAL;
+  return cube_attn_impl(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq, hkv,
+                        d, 0.5f, k, out, workspace, workspace_bytes, stream);
 }
 
 int adaspark_attn_export_sets(const void* workspace, const int32_t* cube_ids, int n_cubes,

@@ -20,6 +20,7 @@ struct SelectArgs {
   AttnGeom G;
   float p;
   float zscale;                       // log2(e) / sqrt(d)
+  int topk;                           // > 0: Top-K with this k instead of Top-p
 };
 
 struct AttnArgs {
@@ -36,6 +37,7 @@ struct AttnArgs {
   AttnGeom G;
   int dense;                          // p == 1: every preceding cube, no lists
   float scale_log2;                   // log2(e) / sqrt(d)
+  int kv_major;                       // visual tiles ordered one KV head after another
 };
 
 cudaError_t launch_validate(const int32_t* cube_ids, const int32_t* off, const uint8_t* text_mask,

@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
   for (int e = 0; e < D; ++e) q[e] = valid ? to_f32(qp[e]) : 0.f;
 
   sel::RowSel s;
-  s.init(ss, tid, a.zscale);
+  s.init(ss, tid, a.zscale, a.topk > 0);
   const int ncand = own > 0 ? own : 0;
   const float* kb = a.kbar + (size_t)kv * G.n_cubes * D;
   uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
       }
     }
     if (pass == 0) {
-      s.finish1(a.p);
+      s.finish1(a.topk > 0 ? (float)a.topk : a.p);
       if (s.range_err) set_status(a.hdr, ADASPARK_DEV_RANGE, 0x8900u);
       continue;
     }

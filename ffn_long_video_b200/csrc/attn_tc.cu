@@ -80,12 +80,23 @@ struct TileInfo {
   int t_hi;      // last valid token of the tile
 };
 
-__device__ __forceinline__ TileInfo decode_tile(const AttnGeom& G) {
+__device__ __forceinline__ TileInfo decode_tile(const AttnGeom& G, bool kv_major) {
   TileInfo T;
   const int b = blockIdx.x;
   T.text = b < G.n_ttiles;  // text tiles first (the heaviest)
   if (T.text) {
     T.bt = b;
+  } else if (kv_major) {
+    // Visual tiles, one KV head after the other (the K/V blocks in use then fit
+    // in L2), latest tokens first within a KV head (the heaviest tiles first):
+    // rank r -> KV head, token tile, then query head of the group.
+    const int r = b - G.n_ttiles;
+    const int per_head = G.vtiles_per_head;
+    const int kv = r / G.vtiles_per_kv;
+    const int rk = r - kv * G.vtiles_per_kv;
+    const int tt = per_head - 1 - rk / G.g;
+    const int hh = rk % G.g;
+    T.bt = kv * G.vtiles_per_kv + hh * per_head + tt;
   } else {
     // visual tiles, latest tokens first: rank r -> token tile, then head
     const int r = b - G.n_ttiles;
@@ -132,7 +143,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const AttnGeom& G = a.G;
   WsHeader* hdr = a.hdr;
-  const TileInfo T = decode_tile(G);
+  const TileInfo T = decode_tile(G, a.kv_major != 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {

@@ -150,10 +150,12 @@ struct RowSel {
   bool open;         // cut not found yet
   bool bounded;      // only keys after (bz, bj) are offered (extra passes)
   bool range_err;    // a score outside +-kZLimit log2 units
+  bool count_mode;   // Top-K: bins count scores instead of summing masses
   float bz;
   int bj;
 
-  __device__ __forceinline__ void init(Smem* s, int t, float zscale) {
+  // count = true selects Top-K (finish1 then takes k instead of p).
+  __device__ __forceinline__ void init(Smem* s, int t, float zscale, bool count = false) {
     hist_col = &s->hist[0][t];
     lz_col = &s->hist[0][t];
     lj_col = reinterpret_cast<int*>(&s->hist[kL + 1][t]);
@@ -170,6 +172,7 @@ struct RowSel {
     open = false;
     bounded = false;
     range_err = false;
+    count_mode = count;
     bz = 0.f;
     bj = 0;
 #pragma unroll 8
@@ -208,20 +211,22 @@ struct RowSel {
     }
   }
 
-  // Histogram update with mass u (0 for a column that is not a candidate)
-  // whose key does not exceed kmax; keys below the window land in its lowest
-  // bin.
-  __device__ __forceinline__ void add_mass(float u) {
-    const int k = max(mass_key(u), klo);
-    hist_col[(k & (kB - 1)) * kRows] += u;
+  // Histogram update for a score of mass u whose key does not exceed kmax;
+  // keys below the window land in its lowest bin. The bin gains u, or one
+  // score in count mode; a column that is not a candidate (valid = false)
+  // adds nothing.
+  __device__ __forceinline__ void add_score(float u, bool valid) {
+    const int k = max(mass_key(valid ? u : 0.f), klo);
+    hist_col[(k & (kB - 1)) * kRows] += valid ? (count_mode ? 1.f : u) : 0.f;
   }
 
   // One score of the histogram pass (raises the window when needed).
   __device__ __forceinline__ void pass1(float score) {
     raise(score);
-    if (!range_err) add_mass(mass(score));
+    if (!range_err) add_score(mass(score), true);
   }
 
+  // p: the Top-p mass fraction; in count mode the number k of scores to keep.
   __device__ __forceinline__ void finish1(float p) {
     if (kmax == kNoKey || range_err) {
       open = false;
@@ -229,7 +234,7 @@ struct RowSel {
     }
     float Z = 0.f;  // smallest bins first
     for (int i = kB - 1; i >= 0; --i) Z += hist_col[((kmax - i) & (kB - 1)) * kRows];
-    const float target = p * Z;
+    const float target = count_mode ? p : p * Z;
     float cum = 0.f;
     int kc = klo;
     for (int i = 0; i < kB - 1; ++i) {
@@ -302,7 +307,7 @@ struct RowSel {
     lsorted = true;
     float cum = 0.f;
     for (int i = 0; i < n; ++i) {
-      cum += mass(lz_col[i * kRows]);
+      cum += count_mode ? 1.f : mass(lz_col[i * kRows]);
       if (cum >= need) {
         open = false;
         return i + 1;

@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     if (c_hi >= 0) {
       sel::RowSel s;
-      s.init(ss, row, a.zscale);
+      s.init(ss, row, a.zscale, a.topk > 0);
       const int ncand = own > 0 ? own : 0;
       uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
       const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 2)
               if (!s.range_err) {
 #pragma unroll
                 for (int c = 0; c < NC; ++c)
-                  s.add_mass(c < nv ? s.mass(__uint_as_float(acc[c])) : 0.f);
+                  s.add_score(s.mass(__uint_as_float(acc[c])), c < nv);
               }
             }
             continue;
@@ -294,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         // cannot strand the other warps.
         if (pass == 0) {
           if (ok) {
-            s.finish1(a.p);
+            s.finish1(a.topk > 0 ? (float)a.topk : a.p);
             if (s.range_err) set_status(hdr, ADASPARK_DEV_RANGE, 0x8800u);
           }
           continue;

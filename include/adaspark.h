@@ -139,6 +139,19 @@ int adaspark_cube_attn(const void *Q, const void *K, const void *V, int dtype,
                        int n_vis, int n_tokens, int hq, int hkv, int d, float p,
                        void *out, void *workspace, size_t workspace_bytes, void *stream);
 
+/* AdaS-Attn with Top-K in place of Top-p: S = the k preceding cubes of largest
+ * probability P (same order: probability descending, cube index ascending;
+ * every preceding cube when there are at most k). This is the fixed-size
+ * selection that the AdaSpark paper compares with Top-p in its ablation of
+ * selection strategies (row "Top-K"); everything else, arguments, layout,
+ * workspace and outputs, is as for adaspark_cube_attn, with k (>= 1) in place
+ * of p. adaspark_attn_export_sets reads the sets of either call.
+ * Errors: as adaspark_cube_attn, and ADASPARK_EINVAL for k < 1. */
+int adaspark_cube_attn_topk(const void *Q, const void *K, const void *V, int dtype,
+                            const int32_t *cube_ids, const int32_t *cube_offsets, int n_cubes,
+                            int n_vis, int n_tokens, int hq, int hkv, int d, int k, void *out,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
 /* Expand the selection sets of the last adaspark_cube_attn call on `workspace`
  * into a dense bitmap: sel_bits [n_vis, hq, ceil(n_cubes/32)] uint32 in DEVICE
  * memory, bit j of row (t, h) set when cube j is in S for that row (the own cube

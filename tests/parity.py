@@ -68,10 +68,15 @@ def excess_over_bf16(got, want):
     return float((np.abs(got - want) - ulp_bf16(want)).max()) if got.size else 0.0
 
 
-def run_attn(case, p=None):
+def run_attn(case, p=None, k=None):
+    """Run AdaS-Attn (Top-p, or Top-K when k is given) and export its sets."""
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
-    out, ws = fb.cube_attn(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis, p)
+    if k is None:
+        out, ws = fb.cube_attn(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis, p)
+    else:
+        out, ws = fb.cube_attn_topk(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis,
+                                    k)
     torch.cuda.synchronize()
     code, detail = fb.read_device_status(ws)
     assert code == fb.OK, (code, detail)
@@ -80,11 +85,12 @@ def run_attn(case, p=None):
     return out, sel, ws
 
 
-def check_attn(case, p=None, tokens=None, report=None):
-    """Selection parity + output parity of AdaS-Attn on ``tokens`` (default all)."""
+def check_attn(case, p=None, tokens=None, report=None, k=None):
+    """Selection parity + output parity of AdaS-Attn on ``tokens`` (default all);
+    Top-K selection when ``k`` is given."""
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
-    out, gsel, ws = run_attn(case, p)
+    out, gsel, ws = run_attn(case, p, k)
     Qc, Kc, Vc = (t[k].cpu() for k in ("Q", "K", "V"))
     off = case["off_np"]
     if tokens is None:
@@ -92,7 +98,7 @@ def check_attn(case, p=None, tokens=None, report=None):
     tokens = np.asarray(tokens)
     vis = tokens[tokens < cfg.n_vis]
     osel, margin = oracle.select_cubes(Qc, Kc, off, cfg.n_vis, cfg.hq, cfg.hkv, p, tokens=vis,
-                                       with_margin=True)
+                                       with_margin=True, k=k)
     g = gsel[vis]
     diff_rows = (osel != g).any(axis=2)
     near = margin < MARGIN

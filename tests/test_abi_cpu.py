@@ -76,6 +76,9 @@ def test_calls_reject_bad_arguments_before_the_device():
     assert L.adaspark_cube_attn(*args, 0.7, dummy, dummy, ws_bytes - 1, None) == fb.EINVAL
     assert L.adaspark_cube_attn(*args, 0.7, None, dummy, ws_bytes, None) == fb.EINVAL
     assert L.adaspark_cube_attn(*args, 0.7, dummy, ctypes.c_void_p(257), ws_bytes, None) == fb.EINVAL
+    for k in (0, -3):
+        assert L.adaspark_cube_attn_topk(*args, k, dummy, dummy, ws_bytes, None) == fb.EINVAL
+    assert L.adaspark_cube_attn_topk(*args, 4, dummy, dummy, ws_bytes - 1, None) == fb.EINVAL
     fws = fb.token_ffn_workspace_bytes(544, 512, 16, 256, 512, fb.FP32)
     fargs = [dummy] * 4 + [fb.FP32, dummy, dummy, dummy, 16, 512, 544, 256, 512]
     assert L.adaspark_token_ffn(*fargs, 2.0, dummy, dummy, fws, None) == fb.EINVAL
