@@ -324,11 +324,36 @@ def cube_attn(Q, K, V, cube_offsets, n_vis, p, tokens=None):
 # ---------------------------------------------------------------------------
 # Key design 3: AdaS-FFN with mean compensation.
 # ---------------------------------------------------------------------------
-def ffn_select(x, cube_offsets, n_vis, p, cubes=None, with_margin=False):
+IMPORTANCE = ("l2", "l2sq", "softmax")
+
+
+def token_importance(norms, importance="l2"):
+    """Importance of a cube's tokens from their L2 norms (key design 3 says only
+    "importance by L2 norm", then the same Top-p rule). "l2": the linear share
+    ||x_u|| / sum ||x_v|| (the reading this build takes); the two alternatives
+    the pages do not exclude: "l2sq", the energy share ||x_u||^2 / sum ||x_v||^2,
+    and "softmax", softmax over the cube of ||x_u||. All three rank tokens in
+    the same order as their norms. Returns None when the norms sum to 0 (l2,
+    l2sq: no importance is defined; the cube keeps every token)."""
+    norms = np.asarray(norms, dtype=np.float64)
+    if importance == "l2":
+        total = norms.sum()
+        return None if total == 0.0 else norms / total
+    if importance == "l2sq":
+        sq = norms * norms
+        total = sq.sum()
+        return None if total == 0.0 else sq / total
+    if importance == "softmax":
+        return softmax(norms)
+    raise ValueError(f"importance must be one of {IMPORTANCE}")
+
+
+def ffn_select(x, cube_offsets, n_vis, p, cubes=None, with_margin=False, importance="l2"):
     """AdaS-FFN token selection (key design 3): inside each cube rank tokens by
-    L2 norm, importance w_u = ||x_u|| / sum_v ||x_v||, keep Top-p(w, p).  Text
-    tokens are always active.  Returns a boolean ``active`` [N] (entries of
-    cubes not in ``cubes`` are left False) and, when asked, per-cube margins."""
+    L2 norm, importance w_u = ||x_u|| / sum_v ||x_v|| (or a variant of
+    ``token_importance``), keep Top-p(w, p).  Text tokens are always active.
+    Returns a boolean ``active`` [N] (entries of cubes not in ``cubes`` are left
+    False) and, when asked, per-cube margins."""
     _check_p(p)
     N = x.shape[0]
     off = np.asarray(cube_offsets)
@@ -342,11 +367,10 @@ def ffn_select(x, cube_offsets, n_vis, p, cubes=None, with_margin=False):
         a, b = off[c], off[c + 1]
         Xc = _f64(x[a:b])
         norms = np.sqrt(np.sum(Xc * Xc, axis=1))
-        total = norms.sum()
-        if total == 0.0:
+        w = token_importance(norms, importance)
+        if w is None:
             active[a:b] = True
             continue
-        w = norms / total
         active[a:b] = top_p(w, p)
         if with_margin:
             margins[c] = top_p_margin(w, p)

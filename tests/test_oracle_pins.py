@@ -377,6 +377,33 @@ def test_ffn_select_closed_forms():
     assert np.nonzero(act[8:15])[0].tolist() == [5]     # the largest norm alone
 
 
+def test_token_importance_closed_forms():
+    """Tokens x_u = s_u v with |v| = 1 have norms s_u: the three normalisations
+    have closed forms, and p = 0.5 tells them apart on s = (1, 2, 3, 4)."""
+    s = np.array([1.0, 2.0, 3.0, 4.0])
+    assert np.allclose(oracle.token_importance(s, "l2"), s / 10.0)
+    assert np.allclose(oracle.token_importance(s, "l2sq"), s ** 2 / 30.0)
+    e = np.exp(s - 4.0)
+    assert np.allclose(oracle.token_importance(s, "softmax"), e / e.sum())
+    assert oracle.token_importance(np.zeros(3), "l2") is None
+    assert oracle.token_importance(np.zeros(3), "l2sq") is None
+    assert np.allclose(oracle.token_importance(np.zeros(3), "softmax"), 1.0 / 3.0)
+    with pytest.raises(ValueError):
+        oracle.token_importance(s, "l1")
+    v = np.zeros(6)
+    v[2] = 1.0
+    x = np.concatenate([s[:, None] * v[None], np.ones((2, 6))])     # one cube + 2 text
+    off = np.array([0, 4])
+    # l2: 0.4 < 0.5 -> {3, 2}; l2sq: 16/30 >= 0.5 -> {3}; softmax: 0.644 -> {3}
+    for imp, want in (("l2", [2, 3]), ("l2sq", [3]), ("softmax", [3])):
+        act = oracle.ffn_select(x, off, 4, 0.5, importance=imp)
+        assert np.nonzero(act[:4])[0].tolist() == want, imp
+        assert act[4:].all()
+    # p = 0.85: l2 0.4+0.3+0.2 = 0.9 -> 3 tokens; l2sq 0.533+0.3+0.133 -> 3; softmax 0.644+0.237 -> 2
+    for imp, n in (("l2", 3), ("l2sq", 3), ("softmax", 2)):
+        assert oracle.ffn_select(x, off, 4, 0.85, importance=imp)[:4].sum() == n, imp
+
+
 def test_token_ffn_dense_and_compensation():
     rng = np.random.default_rng(9)
     D, F = 16, 24
