@@ -22,6 +22,8 @@ _LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libadaspar
 OK, EINVAL, ECUDA, EUNSUPPORTED, EDEVICE = 0, -1, -2, -3, -4
 BF16, FP32 = 0, 1
 DEV_BAD_LAYOUT, DEV_TIMEOUT, DEV_RANGE = 0x1, 0x2, 0x4
+# AdaS-FFN token importance (ADASPARK_IMPORTANCE_*)
+IMPORTANCE_L2_SHARE, IMPORTANCE_L2SQ_SHARE, IMPORTANCE_SOFTMAX = 0, 1, 2
 
 
 class AdasparkError(RuntimeError):
@@ -75,6 +77,8 @@ def lib():
             "adaspark_token_ffn_workspace": (sz, [i32] * 6),
             "adaspark_token_ffn": (i32, [vp, vp, vp, vp, i32, vp, vp, vp] + [i32] * 5 +
                                    [f32, vp, vp, sz, vp]),
+            "adaspark_token_ffn_ex": (i32, [vp, vp, vp, vp, i32, vp, vp, vp] + [i32] * 5 +
+                                      [f32, i32, vp, vp, sz, vp]),
             "adaspark_ffn_export_active": (i32, [vp] + [i32] * 6 + [vp, vp]),
             "adaspark_ffn_read_stats": (i32, [vp, ctypes.POINTER(_FfnStats), vp]),
             "adaspark_read_device_status": (i32, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
@@ -239,8 +243,9 @@ def token_ffn_workspace_bytes(n_tokens, n_vis, n_cubes, D, F, dtype) -> int:
 
 
 def token_ffn(x, W_gate, W_up, W_down, cube_ids, cube_offsets, text_mask, n_vis, p, y=None,
-              workspace=None, stream=None):
-    """AdaS-FFN on device tensors; returns (y fp32 [N, D], workspace)."""
+              workspace=None, stream=None, importance=IMPORTANCE_L2_SHARE):
+    """AdaS-FFN on device tensors; returns (y fp32 [N, D], workspace).
+    ``importance`` other than the linear L2 share calls adaspark_token_ffn_ex."""
     import torch
     for t, nm in ((x, "x"), (W_gate, "W_gate"), (W_up, "W_up"), (W_down, "W_down"),
                   (cube_ids, "cube_ids"), (cube_offsets, "cube_offsets"),
@@ -257,11 +262,18 @@ def token_ffn(x, W_gate, W_up, W_down, cube_ids, cube_offsets, text_mask, n_vis,
         if nb == 0:
             raise AdasparkError(EINVAL, "adaspark_token_ffn_workspace")
         workspace = torch.empty(nb, dtype=torch.uint8, device=x.device)
-    _check(lib().adaspark_token_ffn(_ptr(x), _ptr(W_gate), _ptr(W_up), _ptr(W_down), dt,
-                                    _ptr(cube_ids), _ptr(cube_offsets), _ptr(text_mask), C, n_vis,
-                                    N, D, F, float(p), _ptr(y), _ptr(workspace),
-                                    workspace.numel(), _stream(stream)),
-           "adaspark_token_ffn")
+    if importance == IMPORTANCE_L2_SHARE:
+        _check(lib().adaspark_token_ffn(_ptr(x), _ptr(W_gate), _ptr(W_up), _ptr(W_down), dt,
+                                        _ptr(cube_ids), _ptr(cube_offsets), _ptr(text_mask), C,
+                                        n_vis, N, D, F, float(p), _ptr(y), _ptr(workspace),
+                                        workspace.numel(), _stream(stream)),
+               "adaspark_token_ffn")
+    else:
+        _check(lib().adaspark_token_ffn_ex(_ptr(x), _ptr(W_gate), _ptr(W_up), _ptr(W_down), dt,
+                                           _ptr(cube_ids), _ptr(cube_offsets), _ptr(text_mask), C,
+                                           n_vis, N, D, F, float(p), int(importance), _ptr(y),
+                                           _ptr(workspace), workspace.numel(), _stream(stream)),
+               "adaspark_token_ffn_ex")
     return y, workspace
 
 

@@ -190,10 +190,23 @@ int adaspark_token_ffn(const void* x, const void* W_gate, const void* W_up, cons
                        const uint8_t* text_mask, int n_cubes, int n_vis, int n_tokens, int D,
                        int F, float p, float* y, void* workspace, size_t workspace_bytes,
                        void* stream) {
+  return adaspark_token_ffn_ex(x, W_gate, W_up, W_down, dtype, cube_ids, cube_offsets, text_mask,
+                               n_cubes, n_vis, n_tokens, D, F, p, ADASPARK_IMPORTANCE_L2_SHARE, y,
+                               workspace, workspace_bytes, stream);
+}
+
+int adaspark_token_ffn_ex(const void* x, const void* W_gate, const void* W_up,
+                          const void* W_down, int dtype, const int32_t* cube_ids,
+                          const int32_t* cube_offsets, const uint8_t* text_mask, int n_cubes,
+                          int n_vis, int n_tokens, int D, int F, float p, int importance,
+                          float* y, void* workspace, size_t workspace_bytes, void* stream) {
   if (!x || !W_gate || !W_up || !W_down || !cube_ids || !cube_offsets || !text_mask || !y ||
       !workspace)
     return ADASPARK_EINVAL;
   if (!ffn_sizes_ok(n_tokens, n_vis, n_cubes, D, F, dtype) || !p_valid(p)) return ADASPARK_EINVAL;
+  if (importance != ADASPARK_IMPORTANCE_L2_SHARE && importance != ADASPARK_IMPORTANCE_L2SQ_SHARE &&
+      importance != ADASPARK_IMPORTANCE_SOFTMAX)
+    return ADASPARK_EINVAL;
   const int es = dtype == ADASPARK_BF16 ? 2 : 4;
   const FfnLayout L = make_ffn_layout(n_tokens, n_vis, n_cubes, D, F, es);
   if (workspace_bytes < L.total || !aligned(workspace, kAlign)) return ADASPARK_EINVAL;
@@ -231,6 +244,7 @@ int adaspark_token_ffn(const void* x, const void* W_gate, const void* W_up, cons
   a.F = F;
   a.p = p;
   a.dense = p >= 1.0f;
+  a.importance = importance;
 
   if (cudaMemsetAsync(a.hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
   if (!a.dense && n_cubes > 0 &&

@@ -56,9 +56,17 @@ __global__ void cube_mean_kernel(const T* __restrict__ K, const int32_t* __restr
   const int row = hkv * d;
   if (e >= row) return;
   const int a = off[j], b = off[j + 1];
-  double acc = 0.0;
-  for (int t = a; t < b; ++t) acc += (double)to_f32(K[(size_t)t * row + e]);
-  const float mean = (float)(acc / (double)(b - a));
+  // four independent partial sums keep several loads in flight (bf16 sums of
+  // a cube are exact in fp64, so the order does not change the result)
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  int t = a;
+  for (; t + 4 <= b; t += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc[u] += (double)to_f32(K[(size_t)(t + u) * row + e]);
+  }
+  for (; t < b; ++t) acc[0] += (double)to_f32(K[(size_t)t * row + e]);
+  const double sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  const float mean = (float)(sum / (double)(b - a));
   const int kv = e / d, dim = e - kv * d;
   const size_t o = ((size_t)kv * n_cubes + j) * d + dim;
   kbar[o] = mean;

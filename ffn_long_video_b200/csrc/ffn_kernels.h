@@ -29,6 +29,7 @@ struct FfnArgs {
   int n_tokens, n_vis, n_cubes, D, F;
   float p;
   int dense;
+  int importance;       // ADASPARK_IMPORTANCE_*: share of ||x||, of ||x||^2, or softmax
 };
 
 cudaError_t launch_ffn_select(const FfnArgs& a, int dtype, cudaStream_t s);

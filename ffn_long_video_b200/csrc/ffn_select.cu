@@ -27,12 +27,15 @@ template <> struct Vec8<float> {
   }
 };
 
-// One block per cube: L2 norms of its tokens, then the Top-p cut over
-// w_u = ||x_u|| / sum ||x_v|| by (norm desc, index asc), exactly as in AdaS-Attn.
+// One block per cube: L2 norms of its tokens, then the Top-p cut over the
+// importance w_u = ||x_u|| / sum ||x_v|| (or ||x_u||^2 / sum ||x_v||^2, or the
+// softmax of the norms) by (norm desc, index asc), exactly as in AdaS-Attn. All
+// three weights rank the tokens like their norms.
 template <typename T>
 __global__ void __launch_bounds__(256) ffn_select_kernel(FfnArgs a) {
   __shared__ unsigned long long keys[kMaxCubeTokens];
   __shared__ float s_norm[kMaxCubeTokens];
+  __shared__ float s_w[kMaxCubeTokens];   // unnormalised importance
   __shared__ int s_k;
   if (status_bad(a.hdr)) return;
   const int j = blockIdx.x;
@@ -54,10 +57,21 @@ __global__ void __launch_bounds__(256) ffn_select_kernel(FfnArgs a) {
     if (lane == 0) {
       const float nu = sqrtf(acc);
       s_norm[u] = nu;
+      s_w[u] = a.importance == ADASPARK_IMPORTANCE_L2SQ_SHARE ? acc : nu;
       a.norms[base + u] = nu;
     }
   }
   __syncthreads();
+  if (a.importance == ADASPARK_IMPORTANCE_SOFTMAX) {
+    // exp(||x_u|| - max ||x||): the softmax numerators
+    if (threadIdx.x < 32) {
+      float m = -INFINITY;
+      for (int u = threadIdx.x; u < n; u += 32) m = fmaxf(m, s_norm[u]);
+      m = warp_max(m);
+      for (int u = threadIdx.x; u < n; u += 32) s_w[u] = expf(s_norm[u] - m);
+    }
+    __syncthreads();
+  }
   const int tid = threadIdx.x;
   if (a.dense) {
     for (int u = tid; u < n; u += 256) a.active[base + u] = 1;
@@ -85,13 +99,13 @@ __global__ void __launch_bounds__(256) ffn_select_kernel(FfnArgs a) {
   }
   if (tid == 0) {
     float total = 0.f;
-    for (int u = 0; u < n; ++u) total += s_norm[u];
+    for (int u = 0; u < n; ++u) total += s_w[u];
     int k = n;
     if (total > 0.f) {
       const float target = a.p * total;
       float cum = 0.f;
       for (int i = 0; i < n; ++i) {
-        cum += __uint_as_float((unsigned)(keys[i] >> 32));
+        cum += s_w[(int)(0xFFFFFFFFu - (unsigned)(keys[i] & 0xFFFFFFFFull))];
         if (cum >= target) {
           k = i + 1;
           break;
@@ -211,17 +225,23 @@ __global__ void __launch_bounds__(256) ffn_compensate_kernel(FfnArgs a) {
   const T* xr = reinterpret_cast<const T*>(a.x) + (size_t)t * a.D;
   const float* sr = a.sums + (size_t)c * a.D;
   float* yr = a.y + (size_t)t * a.D;
-  for (int e = lane * 4; e < a.D; e += 128) {
-    const float4 sv = *reinterpret_cast<const float4*>(sr + e);
-    float xv[4];
+  // one 16-byte load of x per lane and step (8 bf16 or 4 fp32 features), the
+  // matching sums and stores; two steps in flight
+  constexpr int kN = Vec8<T>::kN;
+#pragma unroll 2
+  for (int e = lane * kN; e < a.D; e += 32 * kN) {
+    float xv[8];
+    Vec8<T>::load(xr + e, xv);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) xv[i] = to_f32(xr[e + i]);
-    float4 out;
-    out.x = xv[0] + sv.x * inv;
-    out.y = xv[1] + sv.y * inv;
-    out.z = xv[2] + sv.z * inv;
-    out.w = xv[3] + sv.w * inv;
-    *reinterpret_cast<float4*>(yr + e) = out;
+    for (int h = 0; h < kN; h += 4) {
+      const float4 sv = *reinterpret_cast<const float4*>(sr + e + h);
+      float4 o;
+      o.x = xv[h] + sv.x * inv;
+      o.y = xv[h + 1] + sv.y * inv;
+      o.z = xv[h + 2] + sv.z * inv;
+      o.w = xv[h + 3] + sv.w * inv;
+      *reinterpret_cast<float4*>(yr + e + h) = o;
+    }
   }
 }
 

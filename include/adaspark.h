@@ -232,6 +232,25 @@ int adaspark_token_ffn(const void *x, const void *W_gate, const void *W_up, cons
                        int F, float p, float *y, void *workspace, size_t workspace_bytes,
                        void *stream);
 
+/* Importance of a token inside its cube for AdaS-FFN (key design 3 says only
+ * "importance by L2 norm", then the Top-p rule). The linear share is the
+ * reading adaspark_token_ffn takes; the other two are alternatives the text
+ * does not exclude. All three rank a cube's tokens like their L2 norms. */
+#define ADASPARK_IMPORTANCE_L2_SHARE   0  /* ||x_u|| / sum_v ||x_v||          */
+#define ADASPARK_IMPORTANCE_L2SQ_SHARE 1  /* ||x_u||^2 / sum_v ||x_v||^2      */
+#define ADASPARK_IMPORTANCE_SOFTMAX    2  /* softmax over the cube of ||x_u|| */
+
+/* adaspark_token_ffn with the token importance chosen by `importance` (one of
+ * ADASPARK_IMPORTANCE_*); everything else as for adaspark_token_ffn, whose
+ * workspace query applies. A cube whose importance sums to 0 keeps every
+ * token. Errors: as adaspark_token_ffn, and ADASPARK_EINVAL for an unknown
+ * importance code. */
+int adaspark_token_ffn_ex(const void *x, const void *W_gate, const void *W_up,
+                          const void *W_down, int dtype, const int32_t *cube_ids,
+                          const int32_t *cube_offsets, const uint8_t *text_mask, int n_cubes,
+                          int n_vis, int n_tokens, int D, int F, float p, int importance,
+                          float *y, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Copy the active flags of the last adaspark_token_ffn call on `workspace` into
  * active [n_tokens] uint8 DEVICE memory (1 = through the FFN). Asynchronous. */
 int adaspark_ffn_export_active(const void *workspace, int n_tokens, int n_vis, int n_cubes,

@@ -124,11 +124,15 @@ def check_attn(case, p=None, tokens=None, report=None, k=None):
     return out, gsel, ws
 
 
-def run_ffn(case, p=None):
+IMPORTANCE_CODES = {"l2": fb.IMPORTANCE_L2_SHARE, "l2sq": fb.IMPORTANCE_L2SQ_SHARE,
+                    "softmax": fb.IMPORTANCE_SOFTMAX}
+
+
+def run_ffn(case, p=None, importance="l2"):
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
     y, ws = fb.token_ffn(t["x"], t["W_gate"], t["W_up"], t["W_down"], case["ids"], case["off"],
-                         case["text"], cfg.n_vis, p)
+                         case["text"], cfg.n_vis, p, importance=IMPORTANCE_CODES[importance])
     torch.cuda.synchronize()
     code, detail = fb.read_device_status(ws)
     assert code == fb.OK, (code, detail)
@@ -137,15 +141,16 @@ def run_ffn(case, p=None):
     return y, act, ws
 
 
-def check_ffn(case, p=None, cubes=None, text=True, report=None):
+def check_ffn(case, p=None, cubes=None, text=True, report=None, importance="l2"):
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
-    y, gact, ws = run_ffn(case, p)
+    y, gact, ws = run_ffn(case, p, importance)
     x = t["x"].cpu()
     off = case["off_np"]
     if cubes is None:
         cubes = np.arange(cfg.n_cubes)
-    oact, margins = oracle.ffn_select(x, off, cfg.n_vis, p, cubes=cubes, with_margin=True)
+    oact, margins = oracle.ffn_select(x, off, cfg.n_vis, p, cubes=cubes, with_margin=True,
+                                      importance=importance)
     bad_cubes, near_mismatch = [], 0
     for c in cubes:
         a, b = off[c], off[c + 1]

@@ -83,4 +83,6 @@ def test_calls_reject_bad_arguments_before_the_device():
     fargs = [dummy] * 4 + [fb.FP32, dummy, dummy, dummy, 16, 512, 544, 256, 512]
     assert L.adaspark_token_ffn(*fargs, 2.0, dummy, dummy, fws, None) == fb.EINVAL
     assert L.adaspark_token_ffn(*fargs, 0.7, dummy, dummy, fws - 8, None) == fb.EINVAL
+    for code in (-1, 3):
+        assert L.adaspark_token_ffn_ex(*fargs, 0.7, code, dummy, dummy, fws, None) == fb.EINVAL
     assert fb.status_string(fb.EDEVICE) == "device-side check failed"

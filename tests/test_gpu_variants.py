@@ -1,7 +1,9 @@
-"""Top-K cube selection (the fixed-size strategy of the paper's ablation of
-selection strategies) against the float64 oracle (needs a B200): sets bit for
-bit except at near-ties (P_(k) - P_(k+1) below the 1e-5 margin), outputs on
-the library's own sets within the stated tolerance."""
+"""Selection variants against the float64 oracle (needs a B200): Top-K cube
+selection (the fixed-size strategy of the paper's ablation of selection
+strategies; sets bit for bit except at near-ties, P_(k) - P_(k+1) below the
+1e-5 margin) and the AdaS-FFN importance alternatives (energy share, softmax of
+norms). Outputs are compared on the library's own sets within the stated
+tolerance."""
 import numpy as np
 import pytest
 import torch
@@ -44,3 +46,15 @@ def test_topk_full_size_sampled():
     rep = {}
     parity.check_attn(c, k=16, tokens=_sample_tokens(cfg, 32, 5), report=rep)
     print(cfg.name, "top-16", rep)
+
+
+# ------------------------------------------------- AdaS-FFN importance variants
+@pytest.mark.parametrize("importance", ["l2sq", "softmax"])
+@pytest.mark.parametrize("p", [0.5, 0.8])
+def test_ffn_importance_variants(case, importance, p):
+    """The energy share and the softmax of norms (alternatives to the linear
+    L2-norm share) against the oracle: active sets bit for bit outside the
+    margin, outputs on the library's own sets."""
+    rep = {}
+    parity.check_ffn(case, p=p, importance=importance, report=rep)
+    print(case["cfg"].name, importance, p, rep)
