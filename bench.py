@@ -179,6 +179,26 @@ def kernel_work(name, cfg, attn_stats, ffn_stats):
     return None, None, None
 
 
+def max_over_ranks(v, world, device="cpu"):
+    """The largest of the ranks' values (all ranks get it): multi-GPU times are
+    the slowest replica's, taken on the device by each rank."""
+    if world <= 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(ms_total_local, steps, tokens_per_replica, world, device="cpu"):
+    """Whole-job tokens/s of `world` independent replicas: every replica
+    processes its own layer per step, the job's step time is the slowest
+    replica's (max over ranks). Returns (ms_per_step, tokens/s)."""
+    ms_step = max_over_ranks(ms_total_local, world, device) / steps
+    return ms_step, world * tokens_per_replica / (ms_step / 1e3)
+
+
 def run_ours(args, rank, world, device):
     import torch
     import ffn_long_video_b200 as fb
@@ -211,12 +231,7 @@ def run_ours(args, rank, world, device):
             dist.barrier()
 
     def reduce_max(v):
-        if world > 1:
-            import torch.distributed as dist
-            t = torch.tensor([v], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            return float(t.item())
-        return v
+        return max_over_ranks(v, world, device)
 
     for _ in range(args.warmup):
         step()
@@ -246,9 +261,7 @@ def run_ours(args, rank, world, device):
     barrier()
     ktimes = fb.timer_read()
     fb.timer_enable(False)
-    ms_total = reduce_max(ms_total)
-    ms_step = ms_total / args.steps
-    value = world * N / (ms_step / 1e3)
+    ms_step, value = replica_throughput(ms_total, args.steps, N, world, device)
 
     attn_stats = fb.attn_read_stats(aws)
     ffn_stats = fb.ffn_read_stats(fws)
