@@ -11,9 +11,10 @@ inputs resident in HBM.  Prints one JSON line (rank 0).
 * value: tokens/s over all ranks (each rank runs its own replica of the layer;
   the path has no exchange step), timed with CUDA events between barriers,
   max over ranks.
-* e2e: the same metric through the C ABI with the step's inputs (Q, K, V, x)
-  copied from pinned host memory and the outputs (out, y) copied back inside
-  the timed region.
+* e2e: the same metric through the C ABI with every step's inputs (Q, K, V, x)
+  copied from pinned host memory and its outputs (out, y) copied back inside
+  the timed region; the copies of neighbouring steps overlap the computation
+  (copy-in, compute and copy-out streams, two device buffers of each).
 * roofline: the kernel with the largest share of the step, its algorithmic
   FLOPs (or bytes) per launch over its event-timed average duration.
 * cpu_baseline / --impl reference: the float64 oracle, timed on the host cores
@@ -302,28 +303,64 @@ def run_ours(args, rank, world, device):
         kernels[k] = e
 
     # ---------------- e2e through the C ABI with host buffers
+    # Every step copies its inputs (Q, K, V, x) from pinned host memory and its
+    # outputs (out, y) back, as a serving loop would: on a copy-in stream, the
+    # compute stream and a copy-out stream, with two device buffers of each
+    # kind, so that step k's outputs leave and step k+1's inputs arrive while
+    # step k+1 computes. The timed region runs from before the first input
+    # copy to the end of the last output copy.
     pinned = {k: torch.empty(lay[k].shape, dtype=lay[k].dtype, pin_memory=True)
               for k in ("Q", "K", "V", "x")}
     for k in pinned:
         pinned[k].copy_(lay[k])
-    dev_in = {k: torch.empty_like(lay[k]) for k in pinned}
-    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    host_y = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    dev_in = [{k: torch.empty_like(lay[k]) for k in pinned} for _ in range(2)]
+    dev_out = [torch.empty_like(out) for _ in range(2)]
+    dev_y = [torch.empty_like(y) for _ in range(2)]
+    host_out = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+    host_y = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    d2h = host_out.numel() * host_out.element_size() + host_y.numel() * host_y.element_size()
-    e2e_steps = max(1, min(args.steps, 5))
+    d2h = host_out[0].numel() * host_out[0].element_size() + \
+        host_y[0].numel() * host_y[0].element_size()
+    e2e_steps = max(2, args.steps)
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    mk = lambda: torch.cuda.Event()
+    ev_in = [mk() for _ in range(e2e_steps)]
+    ev_cmp = [mk() for _ in range(e2e_steps)]
+    ev_out = [mk() for _ in range(e2e_steps)]
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        for k in pinned:
-            dev_in[k].copy_(pinned[k], non_blocking=True)
-        step(Q=dev_in["Q"], K=dev_in["K"], V=dev_in["V"], x=dev_in["x"])
-        host_out.copy_(out, non_blocking=True)
-        host_y.copy_(y, non_blocking=True)
-    e1.record(stream)
+    e0.record(s_in)
+    for k in range(e2e_steps):
+        b = k % 2
+        if k >= 2:
+            s_in.wait_event(ev_cmp[k - 2])           # inputs of buffer b consumed
+        with torch.cuda.stream(s_in):
+            for name in pinned:
+                dev_in[b][name].copy_(pinned[name], non_blocking=True)
+            ev_in[k].record(s_in)
+        s_cmp.wait_event(ev_in[k])
+        if k >= 2:
+            s_cmp.wait_event(ev_out[k - 2])          # outputs of buffer b copied out
+        with torch.cuda.stream(s_cmp):
+            d = dev_in[b]
+            fb.cube_attn(d["Q"], d["K"], d["V"], lay["cube_ids"], lay["cube_offsets"], n_vis,
+                         cfg.p, out=dev_out[b], workspace=aws, stream=s_cmp)
+            fb.token_ffn(d["x"], lay["W_gate"], lay["W_up"], lay["W_down"], lay["cube_ids"],
+                         lay["cube_offsets"], lay["text_mask"], n_vis, cfg.p, y=dev_y[b],
+                         workspace=fws, stream=s_cmp)
+            ev_cmp[k].record(s_cmp)
+        s_out.wait_event(ev_cmp[k])
+        with torch.cuda.stream(s_out):
+            host_out[b].copy_(dev_out[b], non_blocking=True)
+            host_y[b].copy_(dev_y[b], non_blocking=True)
+            ev_out[k].record(s_out)
+    e1.record(s_out)
     torch.cuda.synchronize()
+    for ws in (aws, fws):
+        code, det = fb.read_device_status(ws)
+        if code != fb.OK:
+            raise RuntimeError(f"device status {code} detail {det:#x} in the e2e steps")
     e2e_ms = reduce_max(e0.elapsed_time(e1)) / e2e_steps
     e2e = {"value": world * N / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
