@@ -17,6 +17,7 @@ Parity status per function (what pins it is in ``tests/test_oracle_pins.py``):
 * ``attention_given_sets``  pinned (torch SDPA in float64 with a mask; first token)
 * ``ffn_select``            pinned (closed forms on scaled tokens, brute force)
 * ``token_importance``      pinned (closed forms for the three normalisations)
+* ``linear``, ``rmsnorm``   pinned (explicit loops; closed forms and invariances)
 * ``swiglu_ffn``            pinned (torch.nn.functional in float64)
 * ``token_ffn``             pinned (p=1 dense, compensation identity, text rows)
 * agreement with the authors' own numbers: parity unpinned (the pages print
@@ -33,6 +34,8 @@ from .adaspark_ref import (  # noqa: F401
     top_k_margin,
     select_cubes,
     token_importance,
+    linear,
+    rmsnorm,
     attention_given_sets,
     cube_attn,
     ffn_select,

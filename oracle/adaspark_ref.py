@@ -422,3 +422,22 @@ def token_ffn(x, W_gate, W_up, W_down, cube_offsets, n_vis, p, cubes=None, text=
     active = ffn_select(x, cube_offsets, n_vis, p, cubes=cubes)
     return ffn_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active,
                           cubes=cubes, text=text), active
+
+
+# ---------------------------------------------------------------------------
+# Around the two modules: the projections and the normalization of a layer.
+# ---------------------------------------------------------------------------
+def linear(x, W):
+    """x W^T in float64 (W in [out, in] layout): the Q/K/V/O projections of the
+    layer around AdaS-Attn and AdaS-FFN (the pages place the two modules in a
+    decoder layer but say nothing about these matrices)."""
+    return _f64(x) @ _f64(W).T
+
+
+def rmsnorm(x, w=None, eps=1e-6):
+    """x / sqrt(mean(x^2) + eps) per row, times w when given, in float64."""
+    xf = _f64(x)
+    r = 1.0 / np.sqrt(np.mean(xf * xf, axis=-1, keepdims=True) + eps)
+    out = xf * r
+    return out * _f64(w) if w is not None else out
+

@@ -430,3 +430,25 @@ def test_token_ffn_dense_and_compensation():
             assert np.abs((y[S] - x[S]) - mbar[None]).max() < 1e-12   # y_k - x_k = m_bar
             assert np.abs(np.diff(y[S] - x[S], axis=0)).max() < 1e-12  # shared by the cube
     assert (~act[:n_vis]).any()
+
+
+def test_linear_matches_explicit_sums():
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((5, 7))
+    W = rng.standard_normal((3, 7))
+    want = np.array([[sum(x[i, k] * W[j, k] for k in range(7)) for j in range(3)]
+                     for i in range(5)])
+    assert np.allclose(oracle.linear(x, W), want, rtol=0, atol=1e-12)
+
+
+def test_rmsnorm_closed_forms():
+    x = np.array([[2.0, -2.0, 2.0, -2.0], [3.0, 4.0, 0.0, 0.0]])
+    out = oracle.rmsnorm(x, eps=0.0)
+    assert np.allclose(out[0], [1, -1, 1, -1])
+    assert np.allclose(out[1], np.array([3, 4, 0, 0]) / np.sqrt(25 / 4))
+    assert np.allclose(np.mean(out ** 2, axis=1), 1.0)            # unit RMS
+    assert np.allclose(oracle.rmsnorm(7.5 * x, eps=0.0), out)     # scale invariant
+    w = np.array([1.0, 2.0, 0.5, 0.0])
+    assert np.allclose(oracle.rmsnorm(x, w, eps=0.0), out * w)
+    assert np.allclose(oracle.rmsnorm(np.zeros((1, 4)), eps=1e-6), 0.0)
+
