@@ -7,6 +7,7 @@ binding fails loudly when the library is missing; there is no fallback.
 Entry points (same names as include/adaspark.h, without the prefix):
 ``cube_count``, ``cube_partition``, ``cube_attn``, ``cube_attn_topk``, ``attn_export_sets``,
 ``attn_read_stats``, ``token_ffn``, ``ffn_export_active``, ``ffn_read_stats``,
+``layer``, ``layer_buffers``, ``rmsnorm``,
 ``read_device_status``, ``timer_enable``, ``timer_read``, ``launch_count``,
 ``device_check``, ``status_string``.
 """
@@ -79,6 +80,11 @@ def lib():
                                    [f32, vp, vp, sz, vp]),
             "adaspark_token_ffn_ex": (i32, [vp, vp, vp, vp, i32, vp, vp, vp] + [i32] * 5 +
                                       [f32, i32, vp, vp, sz, vp]),
+            "adaspark_layer_workspace": (sz, [i32] * 9),
+            "adaspark_layer_buffers": (i32, [i32] * 9 + [ctypes.POINTER(ctypes.c_size_t)]),
+            "adaspark_layer": (i32, [vp] * 8 + [i32, vp, vp, vp] + [i32] * 8 +
+                               [f32, f32, vp, vp, sz, vp]),
+            "adaspark_rmsnorm": (i32, [vp, i32, vp, vp, i32, i32, f32, vp]),
             "adaspark_ffn_export_active": (i32, [vp] + [i32] * 6 + [vp, vp]),
             "adaspark_ffn_read_stats": (i32, [vp, ctypes.POINTER(_FfnStats), vp]),
             "adaspark_read_device_status": (i32, [vp, ctypes.POINTER(ctypes.c_uint32), vp]),
@@ -275,6 +281,74 @@ def token_ffn(x, W_gate, W_up, W_down, cube_ids, cube_offsets, text_mask, n_vis,
                                            _ptr(workspace), workspace.numel(), _stream(stream)),
                "adaspark_token_ffn_ex")
     return y, workspace
+
+
+def layer_workspace_bytes(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, dtype=BF16) -> int:
+    return int(lib().adaspark_layer_workspace(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, dtype))
+
+
+def layer(x, W_q, W_k, W_v, W_o, W_gate, W_up, W_down, cube_ids, cube_offsets, text_mask, n_vis,
+          hq, hkv, p_attn, p_ffn, y=None, workspace=None, stream=None):
+    """A whole AdaSpark layer (projections, AdaS-Attn, output projection with the
+    residual, AdaS-FFN); weights in [out, in] layout. Returns (y fp32, workspace)."""
+    import torch
+    for t, nm in ((x, "x"), (W_q, "W_q"), (W_k, "W_k"), (W_v, "W_v"), (W_o, "W_o"),
+                  (W_gate, "W_gate"), (W_up, "W_up"), (W_down, "W_down"),
+                  (cube_ids, "cube_ids"), (cube_offsets, "cube_offsets"),
+                  (text_mask, "text_mask")):
+        _need(t, nm)
+    N, D = x.shape
+    d = W_q.shape[0] // hq
+    F = W_gate.shape[0]
+    C = cube_offsets.numel() - 1
+    dt = _dtype_code(x)
+    if y is None:
+        y = torch.empty((N, D), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        nb = layer_workspace_bytes(N, n_vis, C, hq, hkv, d, D, F, dt)
+        if nb == 0:
+            raise AdasparkError(EINVAL, "adaspark_layer_workspace")
+        workspace = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    _check(lib().adaspark_layer(_ptr(x), _ptr(W_q), _ptr(W_k), _ptr(W_v), _ptr(W_o),
+                                _ptr(W_gate), _ptr(W_up), _ptr(W_down), dt, _ptr(cube_ids),
+                                _ptr(cube_offsets), _ptr(text_mask), C, n_vis, N, hq, hkv, d, D, F,
+                                float(p_attn), float(p_ffn), _ptr(y), _ptr(workspace),
+                                workspace.numel(), _stream(stream)),
+           "adaspark_layer")
+    return y, workspace
+
+
+def layer_buffers(workspace, n_tokens, n_vis, n_cubes, hq, hkv, d, D, F):
+    """Views of a layer workspace's intermediates: Q, K, V, a (attention output),
+    h (bf16 tensors) and the AdaS-Attn / AdaS-FFN sub-workspaces (uint8)."""
+    import torch
+    off = (ctypes.c_size_t * 7)()
+    _check(lib().adaspark_layer_buffers(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, BF16, off),
+           "adaspark_layer_buffers")
+    N = n_tokens
+
+    def view(o, count, shape):
+        return workspace[o:o + 2 * count].view(torch.bfloat16).view(*shape)
+
+    attn_b = cube_attn_workspace_bytes(N, n_vis, n_cubes, hq, hkv, d, BF16)
+    ffn_b = token_ffn_workspace_bytes(N, n_vis, n_cubes, D, F, BF16)
+    return {"Q": view(off[0], N * hq * d, (N, hq, d)), "K": view(off[1], N * hkv * d, (N, hkv, d)),
+            "V": view(off[2], N * hkv * d, (N, hkv, d)), "a": view(off[3], N * hq * d, (N, hq, d)),
+            "h": view(off[4], N * D, (N, D)),
+            "attn_ws": workspace[off[5]:off[5] + attn_b], "ffn_ws": workspace[off[6]:off[6] + ffn_b]}
+
+
+def rmsnorm(x, weight=None, eps=1e-6, out=None, stream=None):
+    """RMSNorm of the rows of x (bf16 or fp32) into a bf16 tensor."""
+    import torch
+    _need(x, "x")
+    n, D = x.shape
+    if out is None:
+        out = torch.empty((n, D), dtype=torch.bfloat16, device=x.device)
+    _check(lib().adaspark_rmsnorm(_ptr(x), _dtype_code(x), _ptr(weight) if weight is not None
+                                  else None, _ptr(out), n, D, float(eps), _stream(stream)),
+           "adaspark_rmsnorm")
+    return out
 
 
 def ffn_export_active(workspace, n_tokens, n_vis, n_cubes, D, F, dtype, stream=None):

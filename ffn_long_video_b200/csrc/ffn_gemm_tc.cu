@@ -5,6 +5,9 @@
 //   mode 1 (down):     FFN_a = H W_down^T (fp16 x fp16 with W_down converted
 //                      from bf16, fp32 accumulate); y[idx[m]] = x[idx[m]] + FFN_a[m];
 //                      sums[cube(m)] += FFN_a[m] for active visual rows
+//   mode 2 (linear):   out[m, n] = R[m, n] + (A W^T)[m, n] over every row m
+//                      (bf16 x bf16, fp32 accumulate, bf16 out; R optional): the
+//                      projections of a whole layer around AdaS-Attn
 // (key design 3 of the AdaSpark note: the FFN runs only on the active tokens; the
 // per-cube sums feed the mean compensation of the skipped ones).
 //
@@ -38,11 +41,15 @@ constexpr int GROUP_M = 16;
 constexpr size_t SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
 
 struct Params {
-  const uint32_t* m_active;  // device: active rows
+  const uint32_t* m_active;  // device: active rows (modes 0, 1)
   int n_tiles;               // tiles along N
   int k_blocks;              // K / 64
-  int n_cols;                // valid output columns (F for mode 0, D for mode 1)
-  FfnArgs f;
+  int n_cols;                // valid output columns (F for mode 0, D for mode 1, N for 2)
+  FfnArgs f;                 // modes 0, 1; f.hdr is the status word in every mode
+  // mode 2
+  int m_rows;                // rows of A and out
+  const __nv_bfloat16* R;    // residual [m_rows][n_cols] or null
+  __nv_bfloat16* out;        // [m_rows][n_cols]
 };
 
 __device__ __forceinline__ void tile_coords(int t, int num_m, int num_n, int& mt, int& nt) {
@@ -110,7 +117,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(drain, 1);
     fence_mbar_init();
     s_abort = 0;
-    s_M = status_bad(hdr) ? 0 : (int)*P.m_active;
+    s_M = status_bad(hdr) ? 0 : (MODE == 2 ? P.m_rows : (int)*P.m_active);
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&mapA);
@@ -244,6 +251,42 @@ __global__ void __launch_bounds__(THREADS, 1)
               dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
+      } else if (MODE == 2) {
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          uint32_t acc[32];
+          tmem_ld32(tb + c, acc);
+          tmem_ld_wait();
+          const int n0 = nt * BN + c;
+          if (n0 >= P.n_cols || !live) continue;
+          const size_t o = (size_t)m * P.n_cols + n0;
+          float r[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = 0.f;
+          if (P.R) {
+            const uint4* rs = reinterpret_cast<const uint4*>(P.R + o);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 rv = rs[q];
+              const __nv_bfloat162* rb = reinterpret_cast<const __nv_bfloat162*>(&rv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(rb[e]);
+                r[q * 8 + 2 * e] = f.x;
+                r[q * 8 + 2 * e + 1] = f.y;
+              }
+            }
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(r[2 * i] + __uint_as_float(acc[2 * i]),
+                                r[2 * i + 1] + __uint_as_float(acc[2 * i + 1]));
+          uint4* dst = reinterpret_cast<uint4*>(P.out + o);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
       } else {
         const __nv_bfloat16* X = reinterpret_cast<const __nv_bfloat16*>(P.f.x);
         const int orig = live ? P.f.idx[m] : 0;
@@ -372,6 +415,30 @@ cudaError_t launch_ffn_gemm1_tc(const FfnArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   return launch("ffn_gemm1_tc", k, dim3(num_sms()), dim3(gemm::THREADS), gemm::SMEM_BYTES, s, mA,
                 mG, mU, P);
+}
+
+cudaError_t launch_linear_tc(const __nv_bfloat16* A, const __nv_bfloat16* W,
+                             const __nv_bfloat16* R, __nv_bfloat16* out, int M, int N, int K,
+                             WsHeader* hdr, cudaStream_t s) {
+  CUtensorMap mA, mW;
+  if (!map_rows(&mA, A, K, M, 128) || !map_rows(&mW, W, K, N, 256)) return cudaErrorInvalidValue;
+  gemm::Params P;
+  P.m_active = nullptr;
+  P.n_tiles = (N + 255) / 256;
+  P.k_blocks = K / 64;
+  P.n_cols = N;
+  P.f = FfnArgs{};
+  P.f.hdr = hdr;
+  P.m_rows = M;
+  P.R = R;
+  P.out = out;
+  auto k = gemm::ffn_gemm_tc_kernel<2>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)gemm::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int tiles = ((M + 127) / 128) * P.n_tiles;
+  return launch("linear_tc", k, dim3(std::min(tiles, num_sms())), dim3(gemm::THREADS),
+                gemm::SMEM_BYTES, s, mA, mW, mW, P);
 }
 
 cudaError_t launch_ffn_gemm2_tc(const FfnArgs& a, cudaStream_t s) {

@@ -38,6 +38,10 @@ cudaError_t launch_ffn_gemm1_simt(const FfnArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_ffn_gemm2_simt(const FfnArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_ffn_gemm1_tc(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_ffn_gemm2_tc(const FfnArgs& a, cudaStream_t s);
+// out[M][N] = R[M][N] + A[M][K] W[N][K]^T (bf16; R may be null), tcgen05.
+cudaError_t launch_linear_tc(const __nv_bfloat16* A, const __nv_bfloat16* W,
+                             const __nv_bfloat16* R, __nv_bfloat16* out, int M, int N, int K,
+                             WsHeader* hdr, cudaStream_t s);
 cudaError_t launch_ffn_compensate(const FfnArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_wdown_to_fp16(const FfnArgs& a, cudaStream_t s);
 

@@ -264,6 +264,54 @@ int adaspark_ffn_read_stats(const void *workspace, adaspark_ffn_stats *stats, vo
 /* Status, timing and launch accounting.                                    */
 /* ------------------------------------------------------------------------ */
 
+/* ------------------------------------------------------------------------ */
+/* A whole layer around the two calls (beyond the pages' problem statement:  */
+/* the pages describe where AdaS-Attn and AdaS-FFN sit in a decoder layer,   */
+/* not its projections), and RMSNorm.                                        */
+/* ------------------------------------------------------------------------ */
+
+/* Device workspace bytes for adaspark_layer (0 when the sizes are invalid or
+ * dtype is not ADASPARK_BF16). */
+size_t adaspark_layer_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d,
+                                int D, int F, int dtype);
+
+/* One AdaSpark layer, wired as the stacked configuration uses it:
+ *   Q = x W_q^T, K = x W_k^T, V = x W_v^T   (bf16, fp32 accumulation)
+ *   a = AdaS-Attn(Q, K, V) with p_attn      (as adaspark_cube_attn)
+ *   h = x + a W_o^T                         (bf16, fp32 accumulation)
+ *   y = AdaS-FFN(h) with p_ffn              (as adaspark_token_ffn; y fp32)
+ * The projections run on the library's tensor-core GEMM.
+ *   x [n_tokens, D] bf16; W_q [hq*d, D], W_k/W_v [hkv*d, D], W_o [D, hq*d],
+ *   W_gate/W_up [F, D], W_down [D, F]: bf16, row-major (output rows first);
+ *   layout arguments and p as for the two calls; y [n_tokens, D] fp32;
+ *   workspace: device, >= adaspark_layer_workspace(...) bytes, 256-byte aligned;
+ *   it also holds Q, K, V, a and h (see adaspark_layer_buffers).
+ * Requires d = 128 and D a multiple of 64. ADASPARK_EUNSUPPORTED for FP32,
+ * ADASPARK_EINVAL for bad arguments; device-detected problems of any stage are
+ * reported by adaspark_read_device_status on the layer workspace. */
+int adaspark_layer(const void *x, const void *W_q, const void *W_k, const void *W_v,
+                   const void *W_o, const void *W_gate, const void *W_up, const void *W_down,
+                   int dtype, const int32_t *cube_ids, const int32_t *cube_offsets,
+                   const uint8_t *text_mask, int n_cubes, int n_vis, int n_tokens, int hq,
+                   int hkv, int d, int D, int F, float p_attn, float p_ffn, float *y,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Byte offsets inside an adaspark_layer workspace of the layer's intermediate
+ * tensors after a call: offsets[0..6] = Q, K, V, a (attention output), h, the
+ * AdaS-Attn workspace and the AdaS-FFN workspace (for their export and stats
+ * calls). `offsets` is host memory of 7 entries. */
+int adaspark_layer_buffers(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d, int D,
+                           int F, int dtype, size_t *offsets);
+
+/* RMSNorm: out[r] = x[r] / sqrt(mean_j x[r, j]^2 + eps) * weight (weight may be
+ * NULL: no scaling), for the normalization between stacked layers.
+ *   x [n_rows, D] device, element type x_dtype (BF16 or FP32); weight [D] bf16
+ *   device or NULL; out [n_rows, D] bf16 device. Asynchronous on `stream`.
+ * Errors: ADASPARK_EINVAL for NULL x/out, negative sizes, eps < 0 or NaN, an
+ * unknown dtype. */
+int adaspark_rmsnorm(const void *x, int x_dtype, const void *weight, void *out, int n_rows, int D,
+                     float eps, void *stream);
+
 /* Synchronize `stream` and read the status word of a workspace of either call.
  * Returns ADASPARK_OK, or ADASPARK_EDEVICE with *detail (if not NULL) holding the
  * ADASPARK_DEV_* bits in bits 0-7 and an internal code of the first failing
