@@ -20,6 +20,11 @@ Parity status per function (what pins it is in ``tests/test_oracle_pins.py``):
 * ``linear``, ``rmsnorm``   pinned (explicit loops; closed forms and invariances)
 * ``swiglu_ffn``            pinned (torch.nn.functional in float64)
 * ``token_ffn``             pinned (p=1 dense, compensation identity, text rows)
+* ``attention_backward_given_sets``, ``swiglu_ffn_backward``,
+  ``ffn_backward_given_sets``
+                            pinned (full central-difference Jacobians of the
+                            pinned forward functions; torch autograd in float64
+                            on the dense cases; sum invariants)
 * agreement with the authors' own numbers: parity unpinned (the pages print
   no worked example for any step; see the module docstring of adaspark_ref).
 """
@@ -42,4 +47,7 @@ from .adaspark_ref import (  # noqa: F401
     swiglu_ffn,
     ffn_given_sets,
     token_ffn,
+    attention_backward_given_sets,
+    swiglu_ffn_backward,
+    ffn_backward_given_sets,
 )

@@ -441,3 +441,114 @@ def rmsnorm(x, w=None, eps=1e-6):
     out = xf * r
     return out * _f64(w) if w is not None else out
 
+
+
+# ---------------------------------------------------------------------------
+# Backward pass for light fine-tuning (the note's "AdaSpark can be adapted with
+# a small amount of fine-tuning"), selection straight-through: the cube sets of
+# key design 2 and the active sets of key design 3 are held fixed, so no
+# gradient reaches the cube mean keys, the relevance softmax, or the token
+# norms; everything the sets admit is differentiated as computed.
+# ---------------------------------------------------------------------------
+def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel):
+    """Gradients of ``attention_given_sets`` (all tokens) for the upstream
+    gradient dO [N, hq, d], with the sets ``sel`` [N, hq, C] held fixed.
+
+    Per (row, head), with P the row's softmax over its admitted keys and
+    dP = dO . V^T: dS = P * (dP - sum(P * dP)); dQ = dS K / sqrt(d); the key
+    and value gradients collect dS^T Q / sqrt(d) and P^T dO over every row of
+    every query head that reads the KV head (GQA).  Returns float64 (dQ, dK, dV)
+    shaped like Q, K, V.
+    """
+    off = np.asarray(cube_offsets)
+    N, hq, d = Q.shape
+    hkv = K.shape[1]
+    g = hq // hkv
+    Qf, Kf, Vf, dOf = _f64(Q), _f64(K), _f64(V), _f64(dO)
+    dQ = np.zeros_like(Qf)
+    dK = np.zeros_like(Kf)
+    dV = np.zeros_like(Vf)
+    key_cube = np.concatenate([np.searchsorted(off, np.arange(n_vis), side="right") - 1,
+                               np.full(N - n_vis, -1)])
+    pos = np.arange(N)
+    scale = 1.0 / math.sqrt(d)
+    tokens = np.arange(N)
+    group = np.where(tokens < n_vis, key_cube, -1)
+    for i in np.unique(group):
+        t = np.nonzero(group == i)[0]
+        if i < 0:
+            end = int(t.max()) + 1
+            base = pos[None, :end] <= t[:, None]
+        else:
+            end = int(off[i + 1])
+            base = (key_cube[None, :end] == i) & (pos[None, :end] <= t[:, None])
+        for h in range(hq):
+            kv = h // g
+            if i < 0:
+                mask = base
+            else:
+                kc = key_cube[:end]
+                chosen = sel[t][:, h, :][:, np.maximum(kc, 0)] & (kc < i)[None, :]
+                mask = base | chosen
+            q, k, v, do = Qf[t, h, :], Kf[:end, kv, :], Vf[:end, kv, :], dOf[t, h, :]
+            s = np.where(mask, (q @ k.T) * scale, -np.inf)
+            m = np.max(s, axis=1, keepdims=True)
+            e = np.where(mask, np.exp(s - m), 0.0)
+            P = e / e.sum(axis=1, keepdims=True)
+            dP = do @ v.T
+            dS = P * (dP - np.sum(P * dP, axis=1, keepdims=True))
+            dQ[t, h] = (dS @ k) * scale
+            dK[:end, kv] += (dS.T @ q) * scale
+            dV[:end, kv] += P.T @ do
+    return dQ, dK, dV
+
+
+def swiglu_ffn_backward(x, W_gate, W_up, W_down, df):
+    """Gradients of f = swiglu_ffn(x) for the upstream gradient df [n, D]:
+    with g = x W_gate^T, u = x W_up^T, silu(g) = g sigma(g), h = silu(g) u,
+    dh = df W_down; du = dh silu(g); dg = dh u sigma(g) (1 + g (1 - sigma(g)));
+    dx = dg W_gate + du W_up; dW_gate = dg^T x; dW_up = du^T x; dW_down = df^T h.
+    Returns float64 (dx, dW_gate, dW_up, dW_down)."""
+    X, Wg, Wu, Wd, dF = _f64(x), _f64(W_gate), _f64(W_up), _f64(W_down), _f64(df)
+    gate = X @ Wg.T
+    up = X @ Wu.T
+    sig = 1.0 / (1.0 + np.exp(-gate))
+    silu = gate * sig
+    h = silu * up
+    dh = dF @ Wd
+    du = dh * silu
+    dg = dh * up * sig * (1.0 + gate * (1.0 - sig))
+    dx = dg @ Wg + du @ Wu
+    return dx, dg.T @ X, du.T @ X, dF.T @ h
+
+
+def ffn_backward_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active, dy):
+    """Gradients of ``ffn_given_sets`` (all cubes and the text rows) for the
+    upstream gradient dy [N, D], the active set held fixed.
+
+    A skipped token's output is x_k + m_bar of its cube, so its own gradient is
+    dy_k and its dy_k also reaches every active token of the cube through the
+    mean: the FFN of active token a receives df_a = dy_a + (sum of dy_k over
+    the cube's skipped tokens) / (number of active tokens).  Text tokens get
+    df = dy.  Then dx = dy + the FFN's input gradient for computed rows, and
+    the weight gradients sum over every computed row.  Returns float64
+    (dx [N, D], dW_gate [F, D], dW_up [F, D], dW_down [D, F])."""
+    N, D = x.shape
+    off = np.asarray(cube_offsets)
+    C = len(off) - 1
+    X, dY = _f64(x), _f64(dy)
+    active = np.asarray(active, dtype=bool).copy()
+    active[n_vis:] = True
+    df = np.zeros_like(dY)
+    for c in range(C):
+        a, b = off[c], off[c + 1]
+        act = active[a:b]
+        df[a:b][act] = dY[a:b][act]
+        if (~act).any():
+            df[a:b][act] += dY[a:b][~act].sum(axis=0) / int(act.sum())
+    df[n_vis:] = dY[n_vis:]
+    rows = np.nonzero(active)[0]
+    dxr, dWg, dWu, dWd = swiglu_ffn_backward(X[rows], W_gate, W_up, W_down, df[rows])
+    dx = dY.copy()
+    dx[rows] += dxr
+    return dx, dWg, dWu, dWd

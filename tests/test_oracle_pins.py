@@ -452,3 +452,151 @@ def test_rmsnorm_closed_forms():
     assert np.allclose(oracle.rmsnorm(x, w, eps=0.0), out * w)
     assert np.allclose(oracle.rmsnorm(np.zeros((1, 4)), eps=1e-6), 0.0)
 
+
+
+# ---------------------------------------------------------------- backward (fixed sets)
+def _central_diff(fn, arrays, eps=1e-6):
+    """Gradient of the scalar fn(*arrays) w.r.t. every element of every array by
+    central differences (float64)."""
+    grads = []
+    for a in arrays:
+        g = np.zeros_like(a)
+        it = np.nditer(a, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            old = a[i]
+            a[i] = old + eps
+            up = fn(*arrays)
+            a[i] = old - eps
+            dn = fn(*arrays)
+            a[i] = old
+            g[i] = (up - dn) / (2 * eps)
+        grads.append(g)
+    return grads
+
+
+def _tiny_attn_case(seed, sel_density=0.5):
+    rng = np.random.default_rng(seed)
+    off = np.array([0, 3, 5, 8])
+    n_vis, n_text, hq, hkv, d = 8, 2, 4, 2, 3
+    N = n_vis + n_text
+    Q, K, V = _qkv(rng, N, hq, hkv, d)
+    sel = rng.random((N, hq, 3)) < sel_density
+    dO = rng.standard_normal((N, hq, d))
+    return off, n_vis, Q, K, V, sel, dO
+
+
+@pytest.mark.parametrize("seed,density", [(21, 0.5), (22, 0.0), (23, 1.0)])
+def test_attention_backward_equals_central_differences(seed, density):
+    off, n_vis, Q, K, V, sel, dO = _tiny_attn_case(seed, density)
+
+    def loss(Q, K, V):
+        return float(np.sum(dO * oracle.attention_given_sets(Q, K, V, off, n_vis, sel)))
+
+    want = _central_diff(loss, [Q.copy(), K.copy(), V.copy()])
+    got = oracle.attention_backward_given_sets(Q, K, V, dO, off, n_vis, sel)
+    for g, w in zip(got, want):
+        assert np.abs(g - w).max() < 1e-7
+
+
+def test_attention_backward_dense_equals_autograd():
+    rng = np.random.default_rng(24)
+    off = np.array([0, 5, 9, 16, 20, 27])
+    n_vis, n_text, hq, hkv, d = 27, 6, 6, 2, 16
+    N = n_vis + n_text
+    g = hq // hkv
+    Q, K, V = _qkv(rng, N, hq, hkv, d)
+    dO = rng.standard_normal((N, hq, d))
+    sel = np.ones((N, hq, len(off) - 1), dtype=bool)
+    dQ, dK, dV = oracle.attention_backward_given_sets(Q, K, V, dO, off, n_vis, sel)
+    q, k, v = (torch.from_numpy(a.copy()).requires_grad_() for a in (Q, K, V))
+    causal = torch.ones(N, N, dtype=torch.bool).tril()
+    o = Fn.scaled_dot_product_attention(
+        q.permute(1, 0, 2)[None], k.repeat_interleave(g, dim=1).permute(1, 0, 2)[None],
+        v.repeat_interleave(g, dim=1).permute(1, 0, 2)[None], attn_mask=causal)
+    (o[0].permute(1, 0, 2) * torch.from_numpy(dO)).sum().backward()
+    for got, t in ((dQ, q), (dK, k), (dV, v)):
+        assert np.abs(got - t.grad.numpy()).max() < 1e-12
+
+
+def test_attention_backward_sum_invariants():
+    """Every row's probabilities sum to one and its dS sums to zero, so per KV
+    head sum_j dV_j = sum of dO over the rows of its query heads and
+    sum_j dK_j = 0, whatever the sets."""
+    rng = np.random.default_rng(25)
+    off = np.array([0, 4, 8, 12, 16, 20, 24])
+    n_vis, n_text, hq, hkv, d = 24, 5, 4, 2, 8
+    N = n_vis + n_text
+    g = hq // hkv
+    Q, K, V = _qkv(rng, N, hq, hkv, d)
+    sel = rng.random((N, hq, len(off) - 1)) < 0.4
+    dO = rng.standard_normal((N, hq, d))
+    dQ, dK, dV = oracle.attention_backward_given_sets(Q, K, V, dO, off, n_vis, sel)
+    for kv in range(hkv):
+        assert np.abs(dV[:, kv].sum(0) - dO[:, kv * g:(kv + 1) * g].sum((0, 1))).max() < 1e-12
+        assert np.abs(dK[:, kv].sum(0)).max() < 1e-12
+    # the first token sees only itself: its dS is zero, so no query gradient
+    assert np.abs(dQ[0]).max() < 1e-15
+
+
+def _tiny_ffn_case(seed):
+    rng = np.random.default_rng(seed)
+    D, F = 3, 4
+    off = np.array([0, 3, 4, 7])
+    n_vis, n_text = 7, 2
+    N = n_vis + n_text
+    x = rng.standard_normal((N, D))
+    Wg, Wu, Wd = (rng.standard_normal(s) * 0.7 for s in ((F, D), (F, D), (D, F)))
+    active = np.array([True, False, True, True, False, True, False, True, True])
+    dy = rng.standard_normal((N, D))
+    return off, n_vis, x, Wg, Wu, Wd, active, dy
+
+
+def test_ffn_backward_equals_central_differences():
+    off, n_vis, x, Wg, Wu, Wd, active, dy = _tiny_ffn_case(26)
+
+    def loss(x, Wg, Wu, Wd):
+        return float(np.sum(dy * oracle.ffn_given_sets(x, Wg, Wu, Wd, off, n_vis, active)))
+
+    want = _central_diff(loss, [x.copy(), Wg.copy(), Wu.copy(), Wd.copy()])
+    got = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd, off, n_vis, active, dy)
+    for g, w in zip(got, want):
+        assert np.abs(g - w).max() < 1e-7
+
+
+def test_ffn_backward_dense_equals_autograd_and_skipped_rows():
+    rng = np.random.default_rng(27)
+    D, F = 16, 24
+    off = np.array([0, 6, 7, 15, 22])
+    n_vis, n_text = 22, 3
+    N = n_vis + n_text
+    x = rng.standard_normal((N, D))
+    Wg, Wu, Wd = (rng.standard_normal(s) * 0.3 for s in ((F, D), (F, D), (D, F)))
+    dy = rng.standard_normal((N, D))
+    got = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd, off, n_vis, np.ones(N, bool), dy)
+    t = [torch.from_numpy(a.copy()).requires_grad_() for a in (x, Wg, Wu, Wd)]
+    y = t[0] + Fn.linear(Fn.silu(Fn.linear(t[0], t[1])) * Fn.linear(t[0], t[2]), t[3])
+    (y * torch.from_numpy(dy)).sum().backward()
+    for g, tt in zip(got, t):
+        assert np.abs(g - tt.grad.numpy()).max() < 1e-11
+    # sparse set: a skipped token's own gradient is dy; the cube's active tokens
+    # share sum(dy_skipped) / |active| on top of their own dy
+    active = rng.random(N) < 0.5
+    active[[0, 6, 7, 15]] = True
+    dx, _, _, _ = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd, off, n_vis, active, dy)
+    skipped = ~active
+    skipped[n_vis:] = False
+    assert np.array_equal(dx[skipped], dy[skipped])
+    # W_down = 0: the FFN's input and gate gradients vanish
+    Wd0 = np.zeros_like(Wd)
+    dx0, dWg0, _, dWd0 = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd0, off, n_vis, active, dy)
+    assert np.array_equal(dx0, dy) and not dWg0.any()
+    # dW_down collects h^T df: with the compensation term for cube 0 checked by hand
+    a0 = np.nonzero(active[:6])[0]
+    s0 = np.nonzero(~active[:6])[0]
+    df0 = dy[a0] + dy[s0].sum(0) / len(a0)
+    gate, up = x[a0] @ Wg.T, x[a0] @ Wu.T
+    h = gate / (1 + np.exp(-gate)) * up
+    _, _, _, dWd_c0 = oracle.ffn_backward_given_sets(x[:6], Wg, Wu, Wd, off[:2], 6, active[:6],
+                                                     dy[:6])
+    assert np.abs(dWd_c0 - df0.T @ h).max() < 1e-12
