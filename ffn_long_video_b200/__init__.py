@@ -6,7 +6,8 @@ binding fails loudly when the library is missing; there is no fallback.
 
 Entry points (same names as include/adaspark.h, without the prefix):
 ``cube_count``, ``cube_partition``, ``cube_attn``, ``cube_attn_topk``, ``attn_export_sets``,
-``attn_read_stats``, ``token_ffn``, ``ffn_export_active``, ``ffn_read_stats``,
+``attn_read_stats``, ``token_ffn``, ``token_ffn_backward``, ``ffn_export_active``,
+``ffn_read_stats``,
 ``layer``, ``layer_buffers``, ``rmsnorm``,
 ``read_device_status``, ``timer_enable``, ``timer_read``, ``launch_count``,
 ``device_check``, ``status_string``.
@@ -80,6 +81,9 @@ def lib():
                                    [f32, vp, vp, sz, vp]),
             "adaspark_token_ffn_ex": (i32, [vp, vp, vp, vp, i32, vp, vp, vp] + [i32] * 5 +
                                       [f32, i32, vp, vp, sz, vp]),
+            "adaspark_token_ffn_backward_workspace": (sz, [i32] * 6),
+            "adaspark_token_ffn_backward": (i32, [vp, vp, vp, i32, vp] + [i32] * 5 +
+                                            [vp] * 7 + [sz, vp]),
             "adaspark_layer_workspace": (sz, [i32] * 9),
             "adaspark_layer_buffers": (i32, [i32] * 9 + [ctypes.POINTER(ctypes.c_size_t)]),
             "adaspark_layer": (i32, [vp] * 8 + [i32, vp, vp, vp] + [i32] * 8 +
@@ -281,6 +285,42 @@ def token_ffn(x, W_gate, W_up, W_down, cube_ids, cube_offsets, text_mask, n_vis,
                                            _ptr(workspace), workspace.numel(), _stream(stream)),
                "adaspark_token_ffn_ex")
     return y, workspace
+
+
+def token_ffn_backward_workspace_bytes(n_tokens, n_vis, n_cubes, D, F, dtype=BF16) -> int:
+    return int(lib().adaspark_token_ffn_backward_workspace(n_tokens, n_vis, n_cubes, D, F, dtype))
+
+
+def token_ffn_backward(W_gate, W_up, W_down, cube_offsets, n_vis, dy, fwd_workspace, dx=None,
+                       dW_gate=None, dW_up=None, dW_down=None, workspace=None, stream=None):
+    """Backward of AdaS-FFN with the active set of the forward call that filled
+    ``fwd_workspace`` held fixed. Returns (dx, dW_gate, dW_up, dW_down, workspace),
+    all fp32 (allocated when not given)."""
+    import torch
+    for t, nm in ((W_gate, "W_gate"), (W_up, "W_up"), (W_down, "W_down"),
+                  (cube_offsets, "cube_offsets"), (dy, "dy"), (fwd_workspace, "fwd_workspace")):
+        _need(t, nm)
+    N, D = dy.shape
+    F = W_gate.shape[0]
+    C = cube_offsets.numel() - 1
+    dt = _dtype_code(W_gate)
+    dev = dy.device
+    f32 = torch.float32
+    dx = torch.empty((N, D), dtype=f32, device=dev) if dx is None else dx
+    dW_gate = torch.empty((F, D), dtype=f32, device=dev) if dW_gate is None else dW_gate
+    dW_up = torch.empty((F, D), dtype=f32, device=dev) if dW_up is None else dW_up
+    dW_down = torch.empty((D, F), dtype=f32, device=dev) if dW_down is None else dW_down
+    if workspace is None:
+        nb = token_ffn_backward_workspace_bytes(N, n_vis, C, D, F, dt)
+        if nb == 0:
+            raise AdasparkError(EUNSUPPORTED if dt == FP32 else EINVAL,
+                                "adaspark_token_ffn_backward_workspace")
+        workspace = torch.empty(nb, dtype=torch.uint8, device=dev)
+    _check(lib().adaspark_token_ffn_backward(
+        _ptr(W_gate), _ptr(W_up), _ptr(W_down), dt, _ptr(cube_offsets), C, n_vis, N, D, F,
+        _ptr(dy), _ptr(fwd_workspace), _ptr(dx), _ptr(dW_gate), _ptr(dW_up), _ptr(dW_down),
+        _ptr(workspace), workspace.numel(), _stream(stream)), "adaspark_token_ffn_backward")
+    return dx, dW_gate, dW_up, dW_down, workspace
 
 
 def layer_workspace_bytes(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, dtype=BF16) -> int:

@@ -266,6 +266,75 @@ int adaspark_token_ffn_ex(const void* x, const void* W_gate, const void* W_up,
   return cuda_rc(launch_ffn_compensate(a, dtype, s));
 }
 
+size_t adaspark_token_ffn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int D, int F,
+                                             int dtype) {
+  if (dtype != ADASPARK_BF16 || !ffn_sizes_ok(n_tokens, n_vis, n_cubes, D, F, dtype)) return 0;
+  return make_ffn_bwd_layout(n_tokens, n_cubes, D, F).total;
+}
+
+int adaspark_token_ffn_backward(const void* W_gate, const void* W_up, const void* W_down,
+                                int dtype, const int32_t* cube_offsets, int n_cubes, int n_vis,
+                                int n_tokens, int D, int F, const float* dy,
+                                const void* fwd_workspace, float* dx, float* dW_gate,
+                                float* dW_up, float* dW_down, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!W_gate || !W_up || !W_down || !cube_offsets || !dy || !fwd_workspace || !dx || !dW_gate ||
+      !dW_up || !dW_down || !workspace)
+    return ADASPARK_EINVAL;
+  if (dtype == ADASPARK_FP32) return ADASPARK_EUNSUPPORTED;
+  if (dtype != ADASPARK_BF16 || !ffn_sizes_ok(n_tokens, n_vis, n_cubes, D, F, dtype))
+    return ADASPARK_EINVAL;
+  const FfnBwdLayout L = make_ffn_bwd_layout(n_tokens, n_cubes, D, F);
+  if (workspace_bytes < L.total || !aligned(workspace, kAlign) || !aligned(fwd_workspace, kAlign))
+    return ADASPARK_EINVAL;
+  for (const void* ptr : {W_gate, W_up, W_down, static_cast<const void*>(dy),
+                          static_cast<const void*>(dx), static_cast<const void*>(dW_gate),
+                          static_cast<const void*>(dW_up), static_cast<const void*>(dW_down)})
+    if (!aligned(ptr, 16)) return ADASPARK_EINVAL;
+  int rc = check_device();
+  if (rc != ADASPARK_OK) return rc;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const FfnLayout FL = make_ffn_layout(n_tokens, n_vis, n_cubes, D, F, 2);
+  const uint8_t* fws = static_cast<const uint8_t*>(fwd_workspace);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  FfnBwdArgs a;
+  a.W_gate = static_cast<const __nv_bfloat16*>(W_gate);
+  a.W_up = static_cast<const __nv_bfloat16*>(W_up);
+  a.W_down = static_cast<const __nv_bfloat16*>(W_down);
+  a.cube_offsets = cube_offsets;
+  a.dy = dy;
+  a.dx = dx;
+  a.dWg = dW_gate;
+  a.dWu = dW_up;
+  a.dWd = dW_down;
+  a.fhdr = reinterpret_cast<const WsHeader*>(fws + FL.header);
+  a.m_active = &a.fhdr->m_active;
+  a.active = fws + FL.active;
+  a.cube_count = reinterpret_cast<const int32_t*>(fws + FL.cube_count);
+  a.idx = reinterpret_cast<const int32_t*>(fws + FL.idx);
+  a.row_cube = reinterpret_cast<const int32_t*>(fws + FL.row_cube);
+  a.xa = reinterpret_cast<const __nv_bfloat16*>(fws + FL.xa);
+  a.hdr = reinterpret_cast<WsHeader*>(ws + L.header);
+  a.gsum = reinterpret_cast<float*>(ws + L.gsum);
+  a.df = reinterpret_cast<__nv_bfloat16*>(ws + L.df);
+  a.dfT = reinterpret_cast<__nv_bfloat16*>(ws + L.dfT);
+  a.xaT = reinterpret_cast<__nv_bfloat16*>(ws + L.xaT);
+  a.wdT = reinterpret_cast<__nv_bfloat16*>(ws + L.wdT);
+  a.wguT = reinterpret_cast<__nv_bfloat16*>(ws + L.wguT);
+  a.dgu = reinterpret_cast<__nv_bfloat16*>(ws + L.dgu);
+  a.dguT = reinterpret_cast<__nv_bfloat16*>(ws + L.dguT);
+  a.hT = reinterpret_cast<__nv_bfloat16*>(ws + L.hT);
+  a.n_tokens = n_tokens;
+  a.n_vis = n_vis;
+  a.n_cubes = n_cubes;
+  a.D = D;
+  a.F = F;
+  a.mp = L.mp;
+  if (cudaMemsetAsync(a.hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
+  return cuda_rc(launch_ffn_backward_tc(a, s));
+}
+
 int adaspark_ffn_export_active(const void* workspace, int n_tokens, int n_vis, int n_cubes, int D,
                                int F, int dtype, uint8_t* active, void* stream) {
   if (!workspace || !active) return ADASPARK_EINVAL;

@@ -126,4 +126,40 @@ __host__ __device__ inline FfnLayout make_ffn_layout(int n_tokens, int n_vis, in
   return L;
 }
 
+// Workspace of adaspark_token_ffn_backward (bf16 path).
+struct FfnBwdLayout {
+  size_t header;
+  size_t gsum;   // float [C][D]
+  size_t df;     // bf16 [N][D]
+  size_t dfT;    // bf16 [D][mp]
+  size_t xaT;    // bf16 [D][mp]
+  size_t wdT;    // bf16 [F][D]
+  size_t wguT;   // bf16 [D][2F]
+  size_t dgu;    // bf16 [N][2F]
+  size_t dguT;   // bf16 [2F][mp]
+  size_t hT;     // bf16 [F][mp]
+  size_t mp;     // N rounded up to 64
+  size_t total;
+};
+
+__host__ __device__ inline FfnBwdLayout make_ffn_bwd_layout(int n_tokens, int n_cubes, int D,
+                                                            int F) {
+  FfnBwdLayout L;
+  const size_t N = (size_t)n_tokens;
+  L.mp = (N + 63) / 64 * 64;
+  size_t o = 0;
+  L.header = o; o += align_up(sizeof(WsHeader));
+  L.gsum = o; o += align_up((size_t)(n_cubes > 0 ? n_cubes : 1) * D * 4, 1024);
+  L.df = o; o += align_up(N * D * 2, 1024);
+  L.dfT = o; o += align_up((size_t)D * L.mp * 2, 1024);
+  L.xaT = o; o += align_up((size_t)D * L.mp * 2, 1024);
+  L.wdT = o; o += align_up((size_t)F * D * 2, 1024);
+  L.wguT = o; o += align_up((size_t)D * 2 * F * 2, 1024);
+  L.dgu = o; o += align_up(N * 2 * F * 2, 1024);
+  L.dguT = o; o += align_up((size_t)2 * F * L.mp * 2, 1024);
+  L.hT = o; o += align_up((size_t)F * L.mp * 2, 1024);
+  L.total = o;
+  return L;
+}
+
 }  // namespace adaspark

@@ -251,6 +251,49 @@ int adaspark_token_ffn_ex(const void *x, const void *W_gate, const void *W_up,
                           int n_vis, int n_tokens, int D, int F, float p, int importance,
                           float *y, void *workspace, size_t workspace_bytes, void *stream);
 
+/* Device workspace bytes needed by adaspark_token_ffn_backward (0 when the
+ * sizes are invalid or dtype is not ADASPARK_BF16). */
+size_t adaspark_token_ffn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int D, int F,
+                                             int dtype);
+
+/* Backward pass of AdaS-FFN for fine-tuning (the AdaSpark note adapts the model
+ * with light fine-tuning), selection straight-through: the active sets of the
+ * forward call that filled `fwd_workspace` are held fixed, the token norms get
+ * no gradient. For the forward of key design 3 and the upstream dy:
+ *   skipped visual token k of cube c:  dx_k = dy_k;
+ *   active token a of cube c:          df_a = dy_a + (sum of dy_k over the
+ *                                      cube's skipped tokens) / |M_c|;
+ *   text token:                        df = dy;
+ *   computed rows (active and text), with g = W_gate x, u = W_up x:
+ *     dh = W_down^T df, du = dh * silu(g), dg = dh * u * silu'(g),
+ *     dx = dy + W_gate^T dg + W_up^T du;
+ *   dW_gate = sum dg x^T, dW_up = sum du x^T, dW_down = sum df h^T over the
+ *   computed rows, h = silu(g) * u.
+ *
+ *   W_gate, W_up [F, D], W_down [D, F]: device bf16, the forward's weights;
+ *   cube_offsets [n_cubes + 1]: device int32, the forward's;
+ *   dy [n_tokens, D]: device float32 (the gradient of the forward's y);
+ *   fwd_workspace: the workspace of an adaspark_token_ffn / _ex call with the
+ *       same sizes, weights and x, left untouched since (the backward reads its
+ *       active set, compaction and gathered rows; it does not modify it);
+ *   dx [n_tokens, D], dW_gate / dW_up [F, D], dW_down [D, F]: device float32,
+ *       written in full (not accumulated into);
+ *   workspace: device, >= adaspark_token_ffn_backward_workspace(...) bytes,
+ *       256-byte aligned; also 256-byte alignment for fwd_workspace, 16 bytes
+ *       for every array.
+ * Contractions run in bf16 on the tensor cores with fp32 accumulation (df, dg,
+ * du and h are rounded to bf16 as operands). Only ADASPARK_BF16:
+ * ADASPARK_FP32 returns ADASPARK_EUNSUPPORTED. A forward call that reported a
+ * device error makes this call report ADASPARK_EDEVICE (read with
+ * adaspark_read_device_status on `workspace`). Other errors as for
+ * adaspark_token_ffn. */
+int adaspark_token_ffn_backward(const void *W_gate, const void *W_up, const void *W_down,
+                                int dtype, const int32_t *cube_offsets, int n_cubes, int n_vis,
+                                int n_tokens, int D, int F, const float *dy,
+                                const void *fwd_workspace, float *dx, float *dW_gate,
+                                float *dW_up, float *dW_down, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
 /* Copy the active flags of the last adaspark_token_ffn call on `workspace` into
  * active [n_tokens] uint8 DEVICE memory (1 = through the FFN). Asynchronous. */
 int adaspark_ffn_export_active(const void *workspace, int n_tokens, int n_vis, int n_cubes,

@@ -173,3 +173,57 @@ def check_ffn(case, p=None, cubes=None, text=True, report=None, importance="l2")
                       near_margin_mismatch=near_mismatch)
     assert max_abs <= tol_abs and rel <= tol_rel, (max_abs, rel)
     return y, gact, ws
+
+
+# ----------------------------------------------------------------- backward
+# Gradients have no unit scale of their own, so the bf16 bar is applied to the
+# gradient measured in units of its own RMS, with the same one-ulp allowance as
+# the bf16 outputs of the forward: per element |err| <= 2e-2 * rms(ref) +
+# ulp_bf16(|ref|), and rel-L2 <= 5e-3. The ulp term covers sums whose terms
+# share a sign (tokens of one cube are near-duplicates), where the bf16
+# rounding of an operand (dS, P, df, dg, du, h) adds up in proportion to the
+# sum itself instead of averaging out.
+GRAD_TOL = (2e-2, 5e-3)
+
+
+def check_grad(got, want, what, report=None):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(want * want))) if want.size else 0.0
+    max_abs, rel = errors(got, want)
+    excess = (np.abs(got - want) - GRAD_TOL[0] * rms - ulp_bf16(want)).max() if want.size else 0.0
+    if report is not None:
+        report[what] = {"max_abs": max_abs, "rms_ref": rms,
+                        "max_over_rms": max_abs / rms if rms > 0 else max_abs,
+                        "worst_excess": float(excess), "rel_l2": rel}
+    assert excess <= 0.0 and rel <= GRAD_TOL[1], (what, max_abs, rms, float(excess), rel)
+
+
+def run_ffn_backward(case, p=None):
+    """Forward AdaS-FFN, then its backward for the case's seeded dy; returns the
+    library's gradients, the forward's active set and dy."""
+    cfg, t = case["cfg"], case["t"]
+    _, act, fws = run_ffn(case, p)
+    dy = workloads.make_upstream(cfg)["dy"].to(t["x"].device)
+    dx, dWg, dWu, dWd, bws = fb.token_ffn_backward(t["W_gate"], t["W_up"], t["W_down"],
+                                                   case["off"], cfg.n_vis, dy, fws)
+    torch.cuda.synchronize()
+    code, detail = fb.read_device_status(bws)
+    assert code == fb.OK, (code, detail)
+    return (dx, dWg, dWu, dWd), act, dy
+
+
+def check_ffn_backward(case, p=None, report=None):
+    cfg, t = case["cfg"], case["t"]
+    grads, act, dy = run_ffn_backward(case, p)
+    want = oracle.ffn_backward_given_sets(t["x"].cpu(), t["W_gate"].cpu(), t["W_up"].cpu(),
+                                          t["W_down"].cpu(), case["off_np"], cfg.n_vis, act,
+                                          dy.cpu())
+    for g, w, nm in zip(grads, want, ("dx", "dW_gate", "dW_up", "dW_down")):
+        check_grad(g.cpu().numpy(), w, nm, report)
+    # a skipped token's gradient is its upstream gradient, bit for bit
+    skipped = ~act
+    skipped[cfg.n_vis:] = False
+    assert torch.equal(grads[0].cpu()[torch.from_numpy(skipped)],
+                       dy.cpu()[torch.from_numpy(skipped)])
+    return grads, act

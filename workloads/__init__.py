@@ -224,6 +224,18 @@ def make_layer(cfg: LayerConfig, layer: int = 0, device=None, project_on=None) -
     return out
 
 
+def make_upstream(cfg: LayerConfig, layer: int = 0) -> dict:
+    """Upstream gradients for the backward pass, from their own stream (seed +
+    500 + 1000 * layer): dO [N, hq, d] in the working dtype (the attention
+    output's type) and dy [N, D] float32 (the FFN output's type), both N(0, 1).
+    Torch CPU tensors."""
+    import torch
+    rng = np.random.Generator(np.random.PCG64(cfg.seed + 500 + 1000 * layer))
+    dO = _normal(rng, (cfg.n_tokens, cfg.hq, cfg.d))
+    dy = _normal(rng, (cfg.n_tokens, cfg.D))
+    return {"dO": _round(dO, cfg.dtype), "dy": torch.from_numpy(dy)}
+
+
 def make_stack(cfg: LayerConfig, layer: int) -> dict:
     """Stacked workload (several independent layers): the first layer draws the
     hidden state then its weights from its own stream; later layers draw only
