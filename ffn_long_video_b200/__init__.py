@@ -5,7 +5,8 @@ kernels.  Torch tensors supply device memory and the current CUDA stream.  The
 binding fails loudly when the library is missing; there is no fallback.
 
 Entry points (same names as include/adaspark.h, without the prefix):
-``cube_count``, ``cube_partition``, ``cube_attn``, ``cube_attn_topk``, ``attn_export_sets``,
+``cube_count``, ``cube_partition``, ``cube_attn``, ``cube_attn_topk``, ``cube_attn_backward``,
+``attn_export_sets``,
 ``attn_read_stats``, ``token_ffn``, ``token_ffn_backward``, ``ffn_export_active``,
 ``ffn_read_stats``,
 ``layer``, ``layer_buffers``, ``rmsnorm``,
@@ -74,6 +75,9 @@ def lib():
                                                                                    vp]),
             "adaspark_cube_attn_topk": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 7 + [vp, vp, sz,
                                                                                     vp]),
+            "adaspark_cube_attn_backward_workspace": (sz, [i32] * 7),
+            "adaspark_cube_attn_backward": (i32, [vp] * 4 + [i32, vp, vp] + [i32] * 6 +
+                                            [vp] * 5 + [sz, vp]),
             "adaspark_attn_export_sets": (i32, [vp, vp] + [i32] * 7 + [vp, vp]),
             "adaspark_attn_read_stats": (i32, [vp, ctypes.POINTER(_AttnStats), vp]),
             "adaspark_token_ffn_workspace": (sz, [i32] * 6),
@@ -285,6 +289,42 @@ def token_ffn(x, W_gate, W_up, W_down, cube_ids, cube_offsets, text_mask, n_vis,
                                            _ptr(workspace), workspace.numel(), _stream(stream)),
                "adaspark_token_ffn_ex")
     return y, workspace
+
+
+def cube_attn_backward_workspace_bytes(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype=BF16) -> int:
+    return int(lib().adaspark_cube_attn_backward_workspace(n_tokens, n_vis, n_cubes, hq, hkv, d,
+                                                            dtype))
+
+
+def cube_attn_backward(Q, K, V, dO, cube_ids, cube_offsets, n_vis, fwd_workspace, dQ=None,
+                       dK=None, dV=None, workspace=None, stream=None):
+    """Backward of AdaS-Attn with the sets of the forward call that filled
+    ``fwd_workspace`` held fixed. Returns (dQ, dK, dV, workspace), fp32
+    (allocated when not given)."""
+    import torch
+    for t, nm in ((Q, "Q"), (K, "K"), (V, "V"), (dO, "dO"),
+                  (cube_ids, "cube_ids"), (cube_offsets, "cube_offsets"),
+                  (fwd_workspace, "fwd_workspace")):
+        _need(t, nm)
+    N, hq, d = Q.shape
+    hkv = K.shape[1]
+    C = cube_offsets.numel() - 1
+    dt = _dtype_code(Q)
+    f32 = torch.float32
+    dQ = torch.empty((N, hq, d), dtype=f32, device=Q.device) if dQ is None else dQ
+    dK = torch.empty((N, hkv, d), dtype=f32, device=Q.device) if dK is None else dK
+    dV = torch.empty((N, hkv, d), dtype=f32, device=Q.device) if dV is None else dV
+    if workspace is None:
+        nb = cube_attn_backward_workspace_bytes(N, n_vis, C, hq, hkv, d, dt)
+        if nb == 0:
+            raise AdasparkError(EUNSUPPORTED if dt == FP32 else EINVAL,
+                                "adaspark_cube_attn_backward_workspace")
+        workspace = torch.empty(nb, dtype=torch.uint8, device=Q.device)
+    _check(lib().adaspark_cube_attn_backward(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(dO), dt, _ptr(cube_ids), _ptr(cube_offsets), C,
+        n_vis, N, hq, hkv, d, _ptr(fwd_workspace), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(workspace),
+        workspace.numel(), _stream(stream)), "adaspark_cube_attn_backward")
+    return dQ, dK, dV, workspace
 
 
 def token_ffn_backward_workspace_bytes(n_tokens, n_vis, n_cubes, D, F, dtype=BF16) -> int:

@@ -121,6 +121,7 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   aa.G = G;
   aa.dense = dense;
   aa.scale_log2 = sa.zscale;
+  aa.lse = reinterpret_cast<float*>(ws + L.lse);
   // When the layer's K and V outgrow what L2 holds alongside the other
   // traffic, visual tiles run one KV head after another, so that the blocks in
   // use belong to one head; otherwise all heads of a token range run together
@@ -264,6 +265,68 @@ int adaspark_token_ffn_ex(const void* x, const void* W_gate, const void* W_up,
     if ((rc = cuda_rc(launch_ffn_gemm2_simt(a, dtype, s)))) return rc;
   }
   return cuda_rc(launch_ffn_compensate(a, dtype, s));
+}
+
+size_t adaspark_cube_attn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int hq,
+                                             int hkv, int d, int dtype) {
+  if (dtype != ADASPARK_BF16 || !attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype))
+    return 0;
+  return make_attn_bwd_layout(make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d)).total;
+}
+
+int adaspark_cube_attn_backward(const void* Q, const void* K, const void* V, const void* dO,
+                                int dtype, const int32_t* cube_ids,
+                                const int32_t* cube_offsets, int n_cubes, int n_vis,
+                                int n_tokens, int hq, int hkv, int d,
+                                const void* fwd_workspace, float* dQ, float* dK, float* dV,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q || !K || !V || !dO || !cube_ids || !cube_offsets || !fwd_workspace || !dQ ||
+      !dK || !dV || !workspace)
+    return ADASPARK_EINVAL;
+  if (dtype == ADASPARK_FP32) return ADASPARK_EUNSUPPORTED;
+  if (dtype != ADASPARK_BF16 || !attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype))
+    return ADASPARK_EINVAL;
+  const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
+  const AttnBwdLayout L = make_attn_bwd_layout(G);
+  if (workspace_bytes < L.total || !aligned(workspace, kAlign) || !aligned(fwd_workspace, kAlign))
+    return ADASPARK_EINVAL;
+  for (const void* ptr : {Q, K, V, dO, static_cast<const void*>(dQ),
+                          static_cast<const void*>(dK), static_cast<const void*>(dV)})
+    if (!aligned(ptr, 16)) return ADASPARK_EINVAL;
+  int rc = check_device();
+  if (rc != ADASPARK_OK) return rc;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const AttnLayout FL = make_attn_layout(G);
+  const uint8_t* fws = static_cast<const uint8_t*>(fwd_workspace);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  AttnBwdArgs a;
+  a.Q = static_cast<const __nv_bfloat16*>(Q);
+  a.K = static_cast<const __nv_bfloat16*>(K);
+  a.V = static_cast<const __nv_bfloat16*>(V);
+  a.dO = static_cast<const __nv_bfloat16*>(dO);
+  a.dQ = dQ;
+  a.dK = dK;
+  a.dV = dV;
+  a.cube_ids = cube_ids;
+  a.cube_offsets = cube_offsets;
+  a.fhdr = reinterpret_cast<const WsHeader*>(fws + FL.header);
+  a.tile_count = reinterpret_cast<const int32_t*>(fws + FL.tile_count);
+  a.tile_list = reinterpret_cast<const uint16_t*>(fws + FL.tile_list);
+  a.tile_mask = reinterpret_cast<const uint32_t*>(fws + FL.tile_mask);
+  a.lse = reinterpret_cast<const float*>(fws + FL.lse);
+  a.hdr = reinterpret_cast<WsHeader*>(ws + L.header);
+  a.dot = reinterpret_cast<float*>(ws + L.dot);
+  a.inv_count = reinterpret_cast<int32_t*>(ws + L.inv_count);
+  a.inv_start = reinterpret_cast<int32_t*>(ws + L.inv_start);
+  a.inv_list = reinterpret_cast<int32_t*>(ws + L.inv_list);
+  a.G = G;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
+  a.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));
+  const double kv_bytes = 2.0 * n_tokens * hkv * d * 2;
+  a.kv_major = kv_bytes > 64.0 * 1024 * 1024 ? 1 : 0;
+  if (cudaMemsetAsync(a.hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
+  return cuda_rc(launch_attn_backward_tc(a, s));
 }
 
 size_t adaspark_token_ffn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int D, int F,

@@ -38,7 +38,43 @@ struct AttnArgs {
   int dense;                          // p == 1: every preceding cube, no lists
   float scale_log2;                   // log2(e) / sqrt(d)
   int kv_major;                       // visual tiles ordered one KV head after another
+  float* lse;                         // [N][hq] m + log2(l) per row (bf16 path), for the backward
 };
+
+// Backward of AdaS-Attn (sets of a forward call held fixed).
+struct AttnBwdArgs {
+  const __nv_bfloat16* Q;             // [N][hq][d]
+  const __nv_bfloat16* K;             // [N][hkv][d]
+  const __nv_bfloat16* V;             // [N][hkv][d]
+  const __nv_bfloat16* dO;            // [N][hq][d]
+  float* dQ;                          // [N][hq][d]
+  float* dK;                          // [N][hkv][d]
+  float* dV;                          // [N][hkv][d]
+  const int32_t* cube_ids;
+  const int32_t* cube_offsets;
+  // from the forward workspace
+  const WsHeader* fhdr;
+  const int32_t* tile_count;
+  const uint16_t* tile_list;
+  const uint32_t* tile_mask;
+  const float* lse;                   // [N][hq]
+  // backward workspace
+  WsHeader* hdr;
+  float* dot;                         // [N][hq] D_r = sum_j P_rj dP_rj (from attn_bwd_dq)
+  int32_t* inv_count;                 // [hkv][C] visual tiles that admit cube j
+  int32_t* inv_start;                 // [hkv * C + 1]
+  int32_t* inv_list;                  // tile indices, ascending per (kv, j)
+  AttnGeom G;
+  int kv_major;
+  float scale_log2;                   // log2(e) / sqrt(d)
+  float inv_sqrt_d;
+};
+// The forward call ran dense (p = 1: every preceding cube, no lists): the
+// first byte of its header's pad[0], set by the forward's host code.
+__device__ __forceinline__ bool fwd_was_dense(const WsHeader* fhdr) {
+  return reinterpret_cast<const volatile uint8_t*>(&fhdr->pad[0])[0] == 1u;
+}
+cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a, cudaStream_t s);
 
 cudaError_t launch_validate(const int32_t* cube_ids, const int32_t* off, const uint8_t* text_mask,
                             int n_cubes, int n_vis, int n_tokens, WsHeader* hdr, cudaStream_t s);

@@ -27,6 +27,7 @@
 // is what makes reusing the S buffer for P safe: S_{i+2} is issued after the
 // PV_i that reads P_i from the same columns.
 #include "attn_kernels.h"
+#include "attn_tile.cuh"
 
 namespace adaspark {
 namespace fa {
@@ -73,47 +74,6 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
       : "f"(a0), "f"(a1));
 }
 
-struct TileInfo {
-  bool text;
-  int bt;        // tile index within its kind
-  int kv;
-  int t_hi;      // last valid token of the tile
-};
-
-__device__ __forceinline__ TileInfo decode_tile(const AttnGeom& G, bool kv_major) {
-  TileInfo T;
-  const int b = blockIdx.x;
-  T.text = b < G.n_ttiles;  // text tiles first (the heaviest)
-  if (T.text) {
-    T.bt = b;
-  } else if (kv_major) {
-    // Visual tiles, one KV head after the other (the K/V blocks in use then fit
-    // in L2), latest tokens first within a KV head (the heaviest tiles first):
-    // rank r -> KV head, token tile, then query head of the group.
-    const int r = b - G.n_ttiles;
-    const int per_head = G.vtiles_per_head;
-    const int kv = r / G.vtiles_per_kv;
-    const int rk = r - kv * G.vtiles_per_kv;
-    const int tt = per_head - 1 - rk / G.g;
-    const int hh = rk % G.g;
-    T.bt = kv * G.vtiles_per_kv + hh * per_head + tt;
-  } else {
-    // visual tiles, latest tokens first: rank r -> token tile, then head
-    const int r = b - G.n_ttiles;
-    const int per_head = G.vtiles_per_head;
-    const int tt = per_head - 1 - r / G.hq;
-    const int hq_idx = r % G.hq;                 // query head
-    const int kv = hq_idx / G.g, hh = hq_idx - kv * G.g;
-    T.bt = kv * G.vtiles_per_kv + hh * per_head + tt;
-  }
-  T.kv = T.bt / (T.text ? G.ttiles_per_kv : G.vtiles_per_kv);
-  const int per_head = T.text ? G.ttiles_per_head : G.vtiles_per_head;
-  const int count = T.text ? G.n_tokens - G.n_vis : G.n_vis;
-  const int tl = T.bt - T.kv * (T.text ? G.ttiles_per_kv : G.vtiles_per_kv);
-  const int tt = tl % per_head;
-  T.t_hi = (T.text ? G.n_vis : 0) + min(tt * kTileRows + kTileRows, count) - 1;
-  return T;
-}
 
 __global__ void __launch_bounds__(THREADS, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
@@ -516,6 +476,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr, 0x7900u)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      // the row's softmax is 2^(s * scale - lse): kept for the backward pass
+      if (valid && a.lse) a.lse[(size_t)t * G.hq + h] = m_used + __log2f(l);
       __nv_bfloat16* dst =
           reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * 128;
 #pragma unroll 1

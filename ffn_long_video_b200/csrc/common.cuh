@@ -236,6 +236,12 @@ __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_m
          | ((uint32_t)(M >> 4) << 24);      // M / 16
 }
 
+// Same with both A and B stored MN-major (A with M contiguous, B with N
+// contiguous): the form of a product whose operands are transposed tiles.
+__host__ __device__ constexpr uint32_t make_idesc_bf16_mn(int M, int N) {
+  return make_idesc_bf16(M, N, true) | (1u << 15);  // A major: MN
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled canonical layout
 // (8-row x 128-byte swizzle atoms). K-major: rows of 128 B along K, atoms stacked
 // along M/N every `sbo` bytes (1024 for dense packing). MN-major: 64 MN elements

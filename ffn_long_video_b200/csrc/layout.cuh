@@ -75,6 +75,7 @@ struct AttnLayout {
   size_t tile_count;  // int32 [n_vtiles]
   size_t tile_list;   // uint16 [n_vtiles][C]  cube ids with any row bit, ascending
   size_t tile_mask;   // uint32 [n_vtiles][C][4]  128 row bits per (tile, cube)
+  size_t lse;         // float [N][hq]  log2-sum-exp of each row's scaled logits
   size_t total;
 };
 
@@ -87,6 +88,30 @@ __host__ __device__ inline AttnLayout make_attn_layout(const AttnGeom& G) {
   L.tile_count = o; o += align_up((size_t)G.n_vtiles * 4);
   L.tile_list = o; o += align_up((size_t)G.n_vtiles * G.n_cubes * 2);
   L.tile_mask = o; o += align_up((size_t)G.n_vtiles * G.n_cubes * 16);
+  L.lse = o; o += align_up((size_t)G.n_tokens * G.hq * 4);
+  L.total = o;
+  return L;
+}
+
+// Workspace of adaspark_cube_attn_backward.
+struct AttnBwdLayout {
+  size_t header;
+  size_t dot;        // float [N][hq]
+  size_t inv_count;  // int32 [hkv][C]
+  size_t inv_start;  // int32 [hkv * C + 1]
+  size_t inv_list;   // int32 [n_vtiles][C] (capacity; filled per (kv, j) segment)
+  size_t total;
+};
+
+__host__ __device__ inline AttnBwdLayout make_attn_bwd_layout(const AttnGeom& G) {
+  AttnBwdLayout L;
+  size_t o = 0;
+  L.header = o; o += align_up(sizeof(WsHeader));
+  L.dot = o; o += align_up((size_t)G.n_tokens * G.hq * 4);
+  L.inv_count = o; o += align_up((size_t)G.hkv * (G.n_cubes > 0 ? G.n_cubes : 1) * 4);
+  L.inv_start = o; o += align_up(((size_t)G.hkv * G.n_cubes + 1) * 4);
+  L.inv_list = o; o += align_up((size_t)(G.n_vtiles > 0 ? G.n_vtiles : 1) *
+                                (G.n_cubes > 0 ? G.n_cubes : 1) * 4);
   L.total = o;
   return L;
 }

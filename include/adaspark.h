@@ -152,6 +152,45 @@ int adaspark_cube_attn_topk(const void *Q, const void *K, const void *V, int dty
                             int n_vis, int n_tokens, int hq, int hkv, int d, int k, void *out,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Device workspace bytes needed by adaspark_cube_attn_backward (0 when the
+ * sizes are invalid or dtype is not ADASPARK_BF16). */
+size_t adaspark_cube_attn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int hq,
+                                             int hkv, int d, int dtype);
+
+/* Backward pass of AdaS-Attn for fine-tuning (the AdaSpark note adapts the
+ * model with light fine-tuning), selection straight-through: the cube sets of
+ * the forward call (adaspark_cube_attn or _topk) that filled `fwd_workspace`
+ * are held fixed; the cube mean keys and the relevance softmax receive no
+ * gradient. For row r (token, query head) with admitted keys A_r (selected
+ * cubes, own cube causally; text rows: every earlier token), logits
+ * z = q . k / sqrt(d), P = softmax over A_r, and the upstream dO:
+ *   D_r = sum_j P_rj (dO_r . v_j)  (= dO_r . O_r),  dS_rj = P_rj (dO_r . v_j - D_r);
+ *   dQ_r = sum_j dS_rj k_j / sqrt(d);
+ *   dK_j = sum dS_rj q_r / sqrt(d), dV_j = sum P_rj dO_r over the rows of every
+ *   query head of the KV group that admit key j.
+ *
+ *   Q, K, V, cube_ids, cube_offsets, sizes: exactly those of the forward call;
+ *   dO [n_tokens, hq, d]: device bf16, the gradient of the forward's output;
+ *   fwd_workspace: the forward call's workspace, untouched since (the backward
+ *       reads its sets, mode and per-row log-sum-exp; it does not modify it);
+ *   dQ [n_tokens, hq, d], dK / dV [n_tokens, hkv, d]: device float32, written
+ *       in full (not accumulated into);
+ *   workspace: device, >= adaspark_cube_attn_backward_workspace(...) bytes,
+ *       256-byte aligned (fwd_workspace too), 16-byte alignment for the arrays.
+ * The products run in bf16 on the tensor cores with fp32 accumulation (P and
+ * dS are rounded to bf16 as operands; the softmax is recomputed in fp32, and
+ * D_r is summed from the same fp32 P and dP rather than taken from the bf16
+ * output, so each row's dS sums to zero up to fp32 rounding).
+ * Deterministic: no atomics. Only ADASPARK_BF16 (ADASPARK_FP32 returns
+ * ADASPARK_EUNSUPPORTED); a forward call that reported a device error makes
+ * this call report ADASPARK_EDEVICE. Other errors as for adaspark_cube_attn. */
+int adaspark_cube_attn_backward(const void *Q, const void *K, const void *V, const void *dO,
+                                int dtype, const int32_t *cube_ids,
+                                const int32_t *cube_offsets, int n_cubes, int n_vis,
+                                int n_tokens, int hq, int hkv, int d,
+                                const void *fwd_workspace, float *dQ, float *dK, float *dV,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
 /* Expand the selection sets of the last adaspark_cube_attn call on `workspace`
  * into a dense bitmap: sel_bits [n_vis, hq, ceil(n_cubes/32)] uint32 in DEVICE
  * memory, bit j of row (t, h) set when cube j is in S for that row (the own cube

@@ -450,7 +450,7 @@ def rmsnorm(x, w=None, eps=1e-6):
 # gradient reaches the cube mean keys, the relevance softmax, or the token
 # norms; everything the sets admit is differentiated as computed.
 # ---------------------------------------------------------------------------
-def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel):
+def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel, with_magnitudes=False):
     """Gradients of ``attention_given_sets`` (all tokens) for the upstream
     gradient dO [N, hq, d], with the sets ``sel`` [N, hq, C] held fixed.
 
@@ -458,7 +458,10 @@ def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel):
     dP = dO . V^T: dS = P * (dP - sum(P * dP)); dQ = dS K / sqrt(d); the key
     and value gradients collect dS^T Q / sqrt(d) and P^T dO over every row of
     every query head that reads the KV head (GQA).  Returns float64 (dQ, dK, dV)
-    shaped like Q, K, V.
+    shaped like Q, K, V.  With ``with_magnitudes`` it also returns the same
+    three sums taken over absolute values (|dS| |K| / sqrt(d), |dS|^T |Q| /
+    sqrt(d), P^T |dO|): the scale a rounding of dS or P enters each gradient
+    element with, for comparisons that round those operands.
     """
     off = np.asarray(cube_offsets)
     N, hq, d = Q.shape
@@ -468,6 +471,7 @@ def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel):
     dQ = np.zeros_like(Qf)
     dK = np.zeros_like(Kf)
     dV = np.zeros_like(Vf)
+    mQ, mK, mV = np.zeros_like(Qf), np.zeros_like(Kf), np.zeros_like(Vf)
     key_cube = np.concatenate([np.searchsorted(off, np.arange(n_vis), side="right") - 1,
                                np.full(N - n_vis, -1)])
     pos = np.arange(N)
@@ -500,6 +504,13 @@ def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel):
             dQ[t, h] = (dS @ k) * scale
             dK[:end, kv] += (dS.T @ q) * scale
             dV[:end, kv] += P.T @ do
+            if with_magnitudes:
+                aS = np.abs(dS)
+                mQ[t, h] = (aS @ np.abs(k)) * scale
+                mK[:end, kv] += (aS.T @ np.abs(q)) * scale
+                mV[:end, kv] += P.T @ np.abs(do)
+    if with_magnitudes:
+        return dQ, dK, dV, (mQ, mK, mV)
     return dQ, dK, dV
 
 

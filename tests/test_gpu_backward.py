@@ -1,7 +1,8 @@
 """Backward pass (selection straight-through) against the float64 oracle
-(needs a B200): AdaS-FFN gradients of x and the three weights on the sets of
-the library's own forward call."""
+(needs a B200): AdaS-FFN gradients of x and the three weights, AdaS-Attn
+gradients of Q, K and V, each on the sets of the library's own forward call."""
 import pytest
+import torch
 
 import workloads
 from tests import parity
@@ -30,3 +31,19 @@ def test_ffn_backward(bcase, p):
     rep = {}
     parity.check_ffn_backward(bcase, p=p, report=rep)
     print(bcase["cfg"].name, p, rep)
+
+
+@pytest.mark.parametrize("p", [0.7, 0.4, 1.0])
+def test_attn_backward(bcase, p):
+    rep = {}
+    parity.check_attn_backward(bcase, p=p, report=rep)
+    print(bcase["cfg"].name, "attn", p, rep)
+
+
+def test_attn_backward_topk_and_determinism(bcase):
+    rep = {}
+    g1, _ = parity.check_attn_backward(bcase, k=3, report=rep)
+    print(bcase["cfg"].name, "attn top-3", rep)
+    g2, _, _, _ = parity.run_attn_backward(bcase, k=3)
+    for a, b in zip(g1, g2):      # no atomics: repeat runs agree bit for bit
+        assert torch.equal(a, b)

@@ -537,6 +537,15 @@ def test_attention_backward_sum_invariants():
         assert np.abs(dK[:, kv].sum(0)).max() < 1e-12
     # the first token sees only itself: its dS is zero, so no query gradient
     assert np.abs(dQ[0]).max() < 1e-15
+    # the magnitude sums bound the gradients, and equal them when every term is
+    # positive (dV with dO > 0)
+    *g, mags = oracle.attention_backward_given_sets(Q, K, V, dO, off, n_vis, sel,
+                                                   with_magnitudes=True)
+    for gg, mm in zip(g, mags):
+        assert (np.abs(gg) <= mm + 1e-12).all()
+    _, _, dVp, (_, _, mVp) = oracle.attention_backward_given_sets(
+        Q, K, V, np.abs(dO), off, n_vis, sel, with_magnitudes=True)
+    assert np.abs(dVp - mVp).max() < 1e-12
 
 
 def _tiny_ffn_case(seed):
