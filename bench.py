@@ -93,24 +93,39 @@ class ClockSampler:
         self.thread = None
 
     def start(self):
+        """Start sampling every 100 ms and return once the first sample has
+        arrived (nvidia-smi takes a moment to start), so that a short timed
+        region that begins afterwards is sampled."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        t_end = time.time() + 10.0
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, begin: bool):
+        """Host time of the start / end of the timed region."""
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
 
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        # one more period so that the last sample of the region has arrived
+        time.sleep(0.15)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -120,7 +135,12 @@ class ClockSampler:
             self.thread.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", float("inf"))
+        for ts, ln in self.lines:
+            # a sample describes the period before it arrives: keep those that
+            # arrived inside the region or within one period after its end
+            if ts < t0 or ts > t1 + 0.1:
+                continue
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -166,6 +186,20 @@ def kernel_work(name, cfg, attn_stats, ffn_stats):
         return 12.0 * cfg.d * attn_stats["candidate_pairs"], "flop", "tensor"
     if name.startswith("select"):
         return 2.0 * cfg.d * attn_stats["candidate_pairs"], "flop", "alu"
+    # backward (selection straight-through); pairs = executed (tile, key block) pairs
+    pairs = attn_stats["key_blocks"]
+    if name == "attn_bwd_dq_tc":
+        # two passes of S = Q K^T and dP = dO V^T, then dQ += dS K
+        return 10.0 * 128 * 64 * cfg.d * pairs, "flop", "tensor"
+    if name == "attn_bwd_dkv_tc":
+        # S, dP, dV^T += dO^T P, dK^T += Q^T dS
+        return 8.0 * 128 * 64 * cfg.d * pairs, "flop", "tensor"
+    if name == "ffn_bwd_gemm_hdg_tc":
+        return 6.0 * M * cfg.D * cfg.F, "flop", "tensor"
+    if name in ("ffn_bwd_gemm_dx_tc", "ffn_bwd_gemm_dwgu_tc"):
+        return 4.0 * M * cfg.D * cfg.F, "flop", "tensor"
+    if name == "ffn_bwd_gemm_dwd_tc":
+        return 2.0 * M * cfg.D * cfg.F, "flop", "tensor"
     if name == "wdown_to_fp16":
         return float(cfg.D) * cfg.F * 4, "byte", "hbm"
     if name == "ffn_select":
@@ -178,6 +212,44 @@ def kernel_work(name, cfg, attn_stats, ffn_stats):
     if name == "cube_mean_keys":
         return float(cfg.n_vis) * cfg.hkv * cfg.d * 2, "byte", "hbm"
     return None, None, None
+
+
+def kernel_table(ktimes, cfg, attn_stats, ffn_stats):
+    """Per kernel: ms per launch, share of the summed kernel time, and the
+    achieved TFLOP/s or GB/s where its algorithmic work is known."""
+    total = sum(v[1] for v in ktimes.values()) or 1.0
+    kernels = {}
+    for k, (n, ms) in sorted(ktimes.items(), key=lambda kv: -kv[1][1]):
+        w, u, b = kernel_work(k, cfg, attn_stats, ffn_stats)
+        e = {"ms_per_launch": round(ms / n, 4), "share": round(ms / total, 4)}
+        if w is not None:
+            if b == "tensor":
+                e["tflops"] = round(w / (ms / n / 1e3) / 1e12, 1)
+            else:
+                e["gbs"] = round(w / (ms / n / 1e3) / 1e9, 1)
+        kernels[k] = e
+    return kernels
+
+
+def roofline_of(name, n, ms, cfg, attn_stats, ffn_stats, traffic):
+    """Roofline entry of one kernel from its timer totals (n launches, ms)."""
+    work, unit, bound = kernel_work(name, cfg, attn_stats, ffn_stats)
+    if work is None:
+        return None
+    peaks, peak_src = load_peaks()
+    per_launch_ms = ms / n
+    if bound == "tensor":
+        achieved = work / (per_launch_ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a step)",
+                "traffic": traffic, "ms_per_launch": round(per_launch_ms, 4)}
+    achieved = work / (per_launch_ms / 1e3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
+            "traffic": traffic, "ms_per_launch": round(per_launch_ms, 4)}
 
 
 def max_over_ranks(v, world, device="cpu"):
@@ -251,11 +323,13 @@ def run_ours(args, rank, world, device):
     clocks.start()
     l0 = fb.launch_count()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark(True)
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
     torch.cuda.synchronize()
+    clocks.mark(False)
     launches = fb.launch_count() - l0
     ms_total = ev0.elapsed_time(ev1)
     clk = clocks.stop()
@@ -268,39 +342,9 @@ def run_ours(args, rank, world, device):
     ffn_stats = fb.ffn_read_stats(fws)
 
     # ---------------- roofline of the dominant kernel
-    peaks, peak_src = load_peaks()
-    traffic_of = lambda name: load_traffic(name, cfg.name)
-    dom = max(ktimes.items(), key=lambda kv: kv[1][1])
-    dname, (dn, dms) = dom
-    work, unit, bound = kernel_work(dname, cfg, attn_stats, ffn_stats)
-    per_launch_ms = dms / dn
-    roof = None
-    if work is not None:
-        if bound == "tensor":
-            achieved = work / (per_launch_ms / 1e3) / 1e12
-            peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-            roof = {"kernel": dname, "bound": "tensor", "achieved": round(achieved, 1),
-                    "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                    "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a step)",
-                    "traffic": traffic_of(dname), "ms_per_launch": round(per_launch_ms, 4)}
-        else:
-            achieved = work / (per_launch_ms / 1e3) / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"kernel": dname, "bound": "hbm", "achieved": round(achieved, 1),
-                    "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                    "peak_source": f"{peak_src} hbm_gbs", "traffic": traffic_of(dname),
-                    "ms_per_launch": round(per_launch_ms, 4)}
-    kernels = {}
-    for k, (n, ms) in sorted(ktimes.items(), key=lambda kv: -kv[1][1]):
-        w, u, b = kernel_work(k, cfg, attn_stats, ffn_stats)
-        e = {"ms_per_launch": round(ms / n, 4), "share": round(ms / sum(v[1] for v in
-                                                                      ktimes.values()), 4)}
-        if w is not None:
-            if b == "tensor":
-                e["tflops"] = round(w / (ms / n / 1e3) / 1e12, 1)
-            else:
-                e["gbs"] = round(w / (ms / n / 1e3) / 1e9, 1)
-        kernels[k] = e
+    dname, (dn, dms) = max(ktimes.items(), key=lambda kv: kv[1][1])
+    roof = roofline_of(dname, dn, dms, cfg, attn_stats, ffn_stats, load_traffic(dname, cfg.name))
+    kernels = kernel_table(ktimes, cfg, attn_stats, ffn_stats)
 
     # ---------------- e2e through the C ABI with host buffers
     # Every step copies its inputs (Q, K, V, x) from pinned host memory and its
@@ -378,6 +422,13 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     dense_ms = d0.elapsed_time(d1) / 2
 
+    # ---------------- backward (fine-tuning step), the forward's sets held fixed
+    backward = None
+    if not args.no_backward:
+        step()  # the sets of the timed workload (p = cfg.p) back in the workspaces
+        backward = measure_backward(args, cfg, lay, aws, fws, attn_stats, ffn_stats, world,
+                                    device, ms_step)
+
     dense = workloads.dense_flops(cfg)
     sparsity = {
         "mean_selected_cubes_per_row": attn_stats["selected_pairs"] / max(1,
@@ -393,7 +444,63 @@ def run_ours(args, rank, world, device):
         "dense_contrast": {"ms_per_step": round(dense_ms, 3),
                            "value": world * N / (dense_ms / 1e3),
                            "dense_tflop": round((dense["attn"] + dense["ffn"]) / 1e12, 2)},
-        "sparsity": sparsity, "cfg": cfg, "lay": lay,
+        "sparsity": sparsity, "backward": backward, "cfg": cfg, "lay": lay,
+    }
+
+
+def measure_backward(args, cfg, lay, aws, fws, attn_stats, ffn_stats, world, device,
+                     forward_ms):
+    """One backward step = adaspark_cube_attn_backward + adaspark_token_ffn_backward
+    on the sets the forward left in its workspaces, for seeded upstream
+    gradients (dO bf16, dy fp32) resident in HBM; device-timed like the forward."""
+    import torch
+    import ffn_long_video_b200 as fb
+    import workloads
+    N, n_vis = cfg.n_tokens, cfg.n_vis
+    up = workloads.make_upstream(cfg)
+    dO, dy = up["dO"].to(device), up["dy"].to(device)
+    bufs = {"a": {}, "f": {}}
+
+    def bwd():
+        ga = fb.cube_attn_backward(lay["Q"], lay["K"], lay["V"], dO, lay["cube_ids"],
+                                   lay["cube_offsets"], n_vis, aws, **bufs["a"])
+        gf = fb.token_ffn_backward(lay["W_gate"], lay["W_up"], lay["W_down"], lay["cube_offsets"],
+                                   n_vis, dy, fws, **bufs["f"])
+        bufs["a"] = dict(dQ=ga[0], dK=ga[1], dV=ga[2], workspace=ga[3])
+        bufs["f"] = dict(dx=gf[0], dW_gate=gf[1], dW_up=gf[2], dW_down=gf[3], workspace=gf[4])
+
+    steps = max(1, min(args.steps, 5))
+    for _ in range(max(1, args.warmup)):
+        bwd()
+    torch.cuda.synchronize()
+    for ws in (bufs["a"]["workspace"], bufs["f"]["workspace"]):
+        code, det = fb.read_device_status(ws)
+        if code != fb.OK:
+            raise RuntimeError(f"backward device status {code} detail {det:#x}")
+    fb.timer_enable(True)
+    fb.timer_read()
+    torch.cuda.synchronize()
+    l0 = fb.launch_count()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b0.record()
+    for _ in range(steps):
+        bwd()
+    b1.record()
+    torch.cuda.synchronize()
+    launches = fb.launch_count() - l0
+    ktimes = fb.timer_read()
+    fb.timer_enable(False)
+    ms = max_over_ranks(b0.elapsed_time(b1), world, device) / steps
+    dname, (dn, dms) = max(ktimes.items(), key=lambda kv: kv[1][1])
+    return {
+        "what": "attention + FFN backward of the timed layer, cube and token sets of its "
+                "forward held fixed (straight-through selection); gradients fp32",
+        "ms_per_step": round(ms, 3), "value": world * N / (ms / 1e3), "unit": "tokens/s",
+        "steps": steps, "forward_plus_backward_ms": round(forward_ms + ms, 3),
+        "gpu_launches": launches,
+        "roofline": roofline_of(dname, dn, dms, cfg, attn_stats, ffn_stats,
+                                load_traffic(dname, cfg.name)),
+        "kernels": kernel_table(ktimes, cfg, attn_stats, ffn_stats),
     }
 
 
@@ -448,6 +555,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward-pass measurement")
     args = ap.parse_args()
 
     import torch
@@ -517,7 +626,7 @@ def main():
             "roofline": res["roofline"], "cpu_baseline": cpu, "e2e": res["e2e"],
             "gpu_launches": res["launches"] * args.steps, "clocks": res["clocks"],
             "kernels": res["kernels"], "dense_contrast": res["dense_contrast"],
-            "sparsity": res["sparsity"],
+            "sparsity": res["sparsity"], "backward": res["backward"],
             "tensor_pct_of_peak": res["roofline"]["frac"] if res["roofline"] else None,
         }
         print(json.dumps(line))

@@ -60,24 +60,30 @@ __global__ void __launch_bounds__(32) check_kernel(WsHeader* hdr, const WsHeader
 }
 
 // Per (KV head, cube j): the visual tiles of the KV head with any row admitting
-// cube j, in ascending tile order. fill = 0 counts, fill = 1 writes the lists.
-__global__ void __launch_bounds__(128) inv_lists_kernel(AttnBwdArgs a, int fill) {
+// cube j, in ascending tile order. The tiles of a KV head are cut into chunks
+// of kInvChunk; thread (kv, j, chunk) counts (fill = 0) or writes (fill = 1)
+// its chunk's entries, at the offset of the exclusive prefix over
+// (kv, j, chunk) in that order, so each (kv, j) list is contiguous and sorted.
+__global__ void __launch_bounds__(128) inv_lists_kernel(AttnBwdArgs a, int fill, int n_chunks) {
   if (status_bad(a.hdr)) return;
   const AttnGeom& G = a.G;
-  const int j = blockIdx.x * blockDim.x + threadIdx.x, kv = blockIdx.y;
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  const int kv = blockIdx.y / n_chunks, chunk = blockIdx.y - kv * n_chunks;
   if (j >= G.n_cubes) return;
   const bool dense = fwd_was_dense(a.fhdr);
-  const size_t key = (size_t)kv * G.n_cubes + j;
+  const size_t key = ((size_t)kv * G.n_cubes + j) * n_chunks + chunk;
   int32_t* out = fill ? a.inv_list + a.inv_start[key] : nullptr;
   int cnt = 0;
-  for (int tl = 0; tl < G.vtiles_per_kv; ++tl) {
+  const int tl_end = min((chunk + 1) * kInvChunk, G.vtiles_per_kv);
+  for (int tl = chunk * kInvChunk; tl < tl_end; ++tl) {
     const int tt = tl % G.vtiles_per_head;
     const int t_hi = min(tt * kTileRows + kTileRows, G.n_vis) - 1;
     if (j > a.cube_ids[t_hi]) continue;  // cube j follows every row of the tile
     const int bt = kv * G.vtiles_per_kv + tl;
     bool nz = true;
     if (!dense) {
-      const uint4 w = *reinterpret_cast<const uint4*>(a.tile_mask + ((size_t)bt * G.n_cubes + j) * 4);
+      const uint4 w =
+          *reinterpret_cast<const uint4*>(a.tile_mask + ((size_t)bt * G.n_cubes + j) * 4);
       nz = (w.x | w.y | w.z | w.w) != 0u;
     }
     if (nz) {
@@ -558,7 +564,8 @@ __device__ __forceinline__ KeyBlock decode_key_block(const AttnBwdArgs& a) {
     B.k0 = a.cube_offsets[B.j] + 64 * (u & 3);
     B.ok = B.k0 < ke;
     B.nk = min(64, ke - B.k0);
-    B.n_vis_entries = B.ok ? a.inv_count[(size_t)B.kv * G.n_cubes + B.j] : 0;
+    const size_t key = ((size_t)B.kv * G.n_cubes + B.j) * a.inv_chunks;
+    B.n_vis_entries = B.ok ? a.inv_start[key + a.inv_chunks] - a.inv_start[key] : 0;
     B.tt_min = 0;
   } else {
     B.visual = false;
@@ -619,7 +626,8 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
   const KeyBlock B = decode_key_block(a);
   if (!B.ok) return;
   const int n_entries = B.n_vis_entries + B.n_text_entries;
-  const int32_t* list = a.inv_list + (B.visual ? a.inv_start[(size_t)B.kv * G.n_cubes + B.j] : 0);
+  const int32_t* list =
+      a.inv_list + (B.visual ? a.inv_start[((size_t)B.kv * G.n_cubes + B.j) * a.inv_chunks] : 0);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -877,12 +885,15 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a, cudaStream_t s) {
   if ((e = launch("attn_bwd_check", check_kernel, dim3(1), dim3(32), 0, s, a.hdr, a.fhdr)))
     return e;
   if (G.n_cubes > 0) {
-    const dim3 g((G.n_cubes + 127) / 128, G.hkv);
-    if ((e = launch("attn_bwd_inv_count", inv_lists_kernel, g, dim3(128), 0, s, a, 0))) return e;
-    if ((e = launch("attn_bwd_scan", scan_kernel, dim3(1), dim3(1024), 0, s, a.inv_count,
-                    a.inv_start, G.hkv * G.n_cubes, a.hdr)))
+    const int nc = a.inv_chunks;
+    const dim3 g((G.n_cubes + 127) / 128, G.hkv * nc);
+    if ((e = launch("attn_bwd_inv_count", inv_lists_kernel, g, dim3(128), 0, s, a, 0, nc)))
       return e;
-    if ((e = launch("attn_bwd_inv_fill", inv_lists_kernel, g, dim3(128), 0, s, a, 1))) return e;
+    if ((e = launch("attn_bwd_scan", scan_kernel, dim3(1), dim3(1024), 0, s, a.inv_count,
+                    a.inv_start, G.hkv * G.n_cubes * nc, a.hdr)))
+      return e;
+    if ((e = launch("attn_bwd_inv_fill", inv_lists_kernel, g, dim3(128), 0, s, a, 1, nc)))
+      return e;
   }
   CUtensorMap mQ, mdO, mK, mV;
   const uint64_t qdims[3] = {(uint64_t)G.d, (uint64_t)G.hq, (uint64_t)G.n_tokens};

@@ -61,9 +61,10 @@ struct AttnBwdArgs {
   // backward workspace
   WsHeader* hdr;
   float* dot;                         // [N][hq] D_r = sum_j P_rj dP_rj (from attn_bwd_dq)
-  int32_t* inv_count;                 // [hkv][C] visual tiles that admit cube j
-  int32_t* inv_start;                 // [hkv * C + 1]
+  int32_t* inv_count;                 // [hkv][C][inv_chunks] tiles admitting cube j, per chunk
+  int32_t* inv_start;                 // [hkv * C * inv_chunks + 1] exclusive prefix
   int32_t* inv_list;                  // tile indices, ascending per (kv, j)
+  int inv_chunks;                     // chunks of kInvChunk visual tiles per KV head
   AttnGeom G;
   int kv_major;
   float scale_log2;                   // log2(e) / sqrt(d)

@@ -517,17 +517,15 @@ bool map2d(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint6
 }
 
 template <int MODE>
-cudaError_t launch_bwd_gemm(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b0,
-                            const CUtensorMap& b1, const CUtensorMap& b2, const fbwd::GemmP& P,
-                            int max_tiles, cudaStream_t s) {
+cudaError_t launch_bwd_gemm(const char* name, const CUtensorMap& a0, const CUtensorMap& a1,
+                            const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& b2,
+                            const fbwd::GemmP& P, int max_tiles, cudaStream_t s) {
   auto k = fbwd::ffn_bwd_gemm_kernel<MODE>;
   const int smem = (int)fbwd::Cfg<MODE>::SMEM;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(max_tiles, bwd_num_sms()));
-  static const char* names[3] = {"ffn_bwd_gemm0_tc", "ffn_bwd_gemm1_tc", "ffn_bwd_gemm2_tc"};
-  return launch(names[MODE], k, dim3(grid), dim3(fbwd::THREADS), (size_t)smem, s, a0, a1, b0, b1,
-                b2, P);
+  return launch(name, k, dim3(grid), dim3(fbwd::THREADS), (size_t)smem, s, a0, a1, b0, b1, b2, P);
 }
 
 cudaError_t launch_transpose(const __nv_bfloat16* src, __nv_bfloat16* dst, int rows_host,
@@ -585,7 +583,9 @@ cudaError_t launch_ffn_backward_tc(const FfnBwdArgs& a, cudaStream_t s) {
   P.dguT = a.dguT;
   P.hT = a.hT;
   const int mtiles = (N + 127) / 128;
-  if ((e = launch_bwd_gemm<0>(mXa, mDf, mWg, mWu, mWdT, P, mtiles * P.n_tiles, s))) return e;
+  if ((e = launch_bwd_gemm<0>("ffn_bwd_gemm_hdg_tc", mXa, mDf, mWg, mWu, mWdT, P,
+                              mtiles * P.n_tiles, s)))
+    return e;
   // dx of the computed rows
   P.k_blocks = 2 * F / 64;
   P.n_tiles = (D + 255) / 256;
@@ -593,7 +593,8 @@ cudaError_t launch_ffn_backward_tc(const FfnBwdArgs& a, cudaStream_t s) {
   P.dy = a.dy;
   P.dx = a.dx;
   P.idx = a.idx;
-  if ((e = launch_bwd_gemm<1>(mDgu, mDgu, mWguT, mWguT, mWguT, P, mtiles * P.n_tiles, s)))
+  if ((e = launch_bwd_gemm<1>("ffn_bwd_gemm_dx_tc", mDgu, mDgu, mWguT, mWguT, mWguT, P,
+                              mtiles * P.n_tiles, s)))
     return e;
   // [dW_gate; dW_up] = [dg du]^T x_a
   P.m_host = 2 * F;
@@ -602,7 +603,7 @@ cudaError_t launch_ffn_backward_tc(const FfnBwdArgs& a, cudaStream_t s) {
   P.out0 = a.dWg;
   P.out1 = a.dWu;
   P.split = F;
-  if ((e = launch_bwd_gemm<2>(mDguT, mDguT, mXaT, mXaT, mXaT, P,
+  if ((e = launch_bwd_gemm<2>("ffn_bwd_gemm_dwgu_tc", mDguT, mDguT, mXaT, mXaT, mXaT, P,
                               ((2 * F + 127) / 128) * P.n_tiles, s)))
     return e;
   // dW_down = df^T h
@@ -612,7 +613,8 @@ cudaError_t launch_ffn_backward_tc(const FfnBwdArgs& a, cudaStream_t s) {
   P.out0 = a.dWd;
   P.out1 = a.dWd;
   P.split = D;
-  return launch_bwd_gemm<2>(mDfT, mDfT, mHT, mHT, mHT, P, ((D + 127) / 128) * P.n_tiles, s);
+  return launch_bwd_gemm<2>("ffn_bwd_gemm_dwd_tc", mDfT, mDfT, mHT, mHT, mHT, P,
+                            ((D + 127) / 128) * P.n_tiles, s);
 }
 
 }  // namespace adaspark

@@ -11,6 +11,7 @@ namespace adaspark {
 constexpr int kTileRows = 128;      // rows of one attention / selection tile
 constexpr int kMaxCubeTokens = 256; // largest cube accepted
 constexpr int kMaxCubes = 65535;    // cube ids fit 16 bits in the selection lists
+constexpr int kInvChunk = 128;      // visual tiles per chunk of the backward's inverted lists
 
 // Geometry of AdaS-Attn. A "row" is one (token, query head) pair. Rows are
 // grouped by KV head, then by query head within the group, then by token, and
@@ -97,19 +98,23 @@ __host__ __device__ inline AttnLayout make_attn_layout(const AttnGeom& G) {
 struct AttnBwdLayout {
   size_t header;
   size_t dot;        // float [N][hq]
-  size_t inv_count;  // int32 [hkv][C]
-  size_t inv_start;  // int32 [hkv * C + 1]
+  size_t inv_count;  // int32 [hkv][C][chunks]
+  size_t inv_start;  // int32 [hkv * C * chunks + 1]
   size_t inv_list;   // int32 [n_vtiles][C] (capacity; filled per (kv, j) segment)
+  int chunks;        // chunks of kInvChunk visual tiles per KV head
   size_t total;
 };
 
 __host__ __device__ inline AttnBwdLayout make_attn_bwd_layout(const AttnGeom& G) {
   AttnBwdLayout L;
+  L.chunks = (G.vtiles_per_kv + kInvChunk - 1) / kInvChunk;
+  if (L.chunks < 1) L.chunks = 1;
+  const size_t nkey = (size_t)G.hkv * (G.n_cubes > 0 ? G.n_cubes : 1) * L.chunks;
   size_t o = 0;
   L.header = o; o += align_up(sizeof(WsHeader));
   L.dot = o; o += align_up((size_t)G.n_tokens * G.hq * 4);
-  L.inv_count = o; o += align_up((size_t)G.hkv * (G.n_cubes > 0 ? G.n_cubes : 1) * 4);
-  L.inv_start = o; o += align_up(((size_t)G.hkv * G.n_cubes + 1) * 4);
+  L.inv_count = o; o += align_up(nkey * 4);
+  L.inv_start = o; o += align_up((nkey + 1) * 4);
   L.inv_list = o; o += align_up((size_t)(G.n_vtiles > 0 ? G.n_vtiles : 1) *
                                 (G.n_cubes > 0 ? G.n_cubes : 1) * 4);
   L.total = o;
