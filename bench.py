@@ -41,7 +41,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # kernel (timer name) -> source file whose build the DRAM counters were taken on
 KERNEL_SOURCES = {"attn_tc": "attn_tc.cu", "select_tc": "select_tc.cu",
-                  "ffn_gemm1_tc": "ffn_gemm_tc.cu", "ffn_gemm2_tc": "ffn_gemm_tc.cu"}
+                  "ffn_gemm1_tc": "ffn_gemm_tc.cu", "ffn_gemm2_tc": "ffn_gemm_tc.cu",
+                  "attn_bwd_dq_tc": "attn_bwd.cu", "attn_bwd_dkv_tc": "attn_bwd.cu"}
 
 
 def load_traffic(kernel, workload):
