@@ -450,7 +450,8 @@ def rmsnorm(x, w=None, eps=1e-6):
 # gradient reaches the cube mean keys, the relevance softmax, or the token
 # norms; everything the sets admit is differentiated as computed.
 # ---------------------------------------------------------------------------
-def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel, with_magnitudes=False):
+def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel, with_magnitudes=False,
+                                  cubes=None, text=True):
     """Gradients of ``attention_given_sets`` (all tokens) for the upstream
     gradient dO [N, hq, d], with the sets ``sel`` [N, hq, C] held fixed.
 
@@ -461,7 +462,11 @@ def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel, with_ma
     shaped like Q, K, V.  With ``with_magnitudes`` it also returns the same
     three sums taken over absolute values (|dS| |K| / sqrt(d), |dS|^T |Q| /
     sqrt(d), P^T |dO|): the scale a rounding of dS or P enters each gradient
-    element with, for comparisons that round those operands.
+    element with, for comparisons that round those operands.  ``cubes`` /
+    ``text`` restrict the query rows to the visual tokens of those cubes and
+    (or not) the text tokens: dQ is then exact on those rows (zero elsewhere)
+    and dK, dV hold only their contributions, exact for keys that no other row
+    admits (e.g. the last cube's keys with ``cubes=[C-1]`` and the text rows).
     """
     off = np.asarray(cube_offsets)
     N, hq, d = Q.shape
@@ -478,7 +483,12 @@ def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel, with_ma
     scale = 1.0 / math.sqrt(d)
     tokens = np.arange(N)
     group = np.where(tokens < n_vis, key_cube, -1)
+    wanted = set(range(len(off) - 1)) if cubes is None else set(int(c) for c in cubes)
+    if text:
+        wanted.add(-1)
     for i in np.unique(group):
+        if int(i) not in wanted:
+            continue
         t = np.nonzero(group == i)[0]
         if i < 0:
             end = int(t.max()) + 1
@@ -533,7 +543,8 @@ def swiglu_ffn_backward(x, W_gate, W_up, W_down, df):
     return dx, dg.T @ X, du.T @ X, dF.T @ h
 
 
-def ffn_backward_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active, dy):
+def ffn_backward_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active, dy,
+                            cubes=None, text=True):
     """Gradients of ``ffn_given_sets`` (all cubes and the text rows) for the
     upstream gradient dy [N, D], the active set held fixed.
 
@@ -543,23 +554,32 @@ def ffn_backward_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active
     the cube's skipped tokens) / (number of active tokens).  Text tokens get
     df = dy.  Then dx = dy + the FFN's input gradient for computed rows, and
     the weight gradients sum over every computed row.  Returns float64
-    (dx [N, D], dW_gate [F, D], dW_up [F, D], dW_down [D, F])."""
+    (dx [N, D], dW_gate [F, D], dW_up [F, D], dW_down [D, F]).  ``cubes`` /
+    ``text`` restrict the rows to those cubes and (or not) the text tokens: dx
+    is exact on them (NaN elsewhere) and the weight gradients hold only their
+    rows' contributions."""
     N, D = x.shape
     off = np.asarray(cube_offsets)
     C = len(off) - 1
     X, dY = _f64(x), _f64(dy)
     active = np.asarray(active, dtype=bool).copy()
     active[n_vis:] = True
+    keep = np.zeros(N, dtype=bool)
+    for c in (range(C) if cubes is None else cubes):
+        keep[off[c]:off[c + 1]] = True
+    keep[n_vis:] = text
     df = np.zeros_like(dY)
     for c in range(C):
         a, b = off[c], off[c + 1]
+        if not keep[a:b].any():
+            continue
         act = active[a:b]
         df[a:b][act] = dY[a:b][act]
         if (~act).any():
             df[a:b][act] += dY[a:b][~act].sum(axis=0) / int(act.sum())
     df[n_vis:] = dY[n_vis:]
-    rows = np.nonzero(active)[0]
+    rows = np.nonzero(active & keep)[0]
     dxr, dWg, dWu, dWd = swiglu_ffn_backward(X[rows], W_gate, W_up, W_down, df[rows])
-    dx = dY.copy()
+    dx = np.where(keep[:, None], dY, np.nan)
     dx[rows] += dxr
     return dx, dWg, dWu, dWd

@@ -548,6 +548,38 @@ def test_attention_backward_sum_invariants():
     assert np.abs(dVp - mVp).max() < 1e-12
 
 
+def test_backward_row_restrictions_agree_with_full():
+    """Restricting the rows (cubes / text) gives the full result on those rows,
+    and for the attention the full dK, dV on keys only those rows admit."""
+    rng = np.random.default_rng(28)
+    off = np.array([0, 4, 8, 12, 16, 20, 24])
+    n_vis, n_text, hq, hkv, d = 24, 5, 4, 2, 8
+    N = n_vis + n_text
+    Q, K, V = _qkv(rng, N, hq, hkv, d)
+    sel = rng.random((N, hq, len(off) - 1)) < 0.4
+    dO = rng.standard_normal((N, hq, d))
+    full = oracle.attention_backward_given_sets(Q, K, V, dO, off, n_vis, sel)
+    part = oracle.attention_backward_given_sets(Q, K, V, dO, off, n_vis, sel, cubes=[5])
+    rows = np.r_[20:24, n_vis:N]
+    assert np.abs(part[0][rows] - full[0][rows]).max() < 1e-12
+    assert not part[0][:20].any()
+    for a, b in ((part[1], full[1]), (part[2], full[2])):
+        assert np.abs(a[20:] - b[20:]).max() < 1e-12      # last cube's and text keys
+    D, F = 6, 10
+    x = rng.standard_normal((N, D))
+    Wg, Wu, Wd = (rng.standard_normal(sh) * 0.5 for sh in ((F, D), (F, D), (D, F)))
+    act = rng.random(N) < 0.6
+    for c in range(len(off) - 1):
+        act[off[c]] = True
+    dy = rng.standard_normal((N, D))
+    fdx = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd, off, n_vis, act, dy)[0]
+    pdx = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd, off, n_vis, act, dy, cubes=[1, 3],
+                                         text=False)[0]
+    rows = np.r_[4:8, 12:16]
+    assert np.abs(pdx[rows] - fdx[rows]).max() < 1e-12
+    assert np.isnan(pdx[np.r_[0:4, 8:12, 16:N]]).all()
+
+
 def _tiny_ffn_case(seed):
     rng = np.random.default_rng(seed)
     D, F = 3, 4
