@@ -765,33 +765,59 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const float scale = a.scale_log2;
     const bool dense = fwd_was_dense(a.fhdr);
-    bool ok = true;
-    for (int e = 0; e < n_entries; ++e) {
-      bool text;
-      int bt;
-      walk_entry(a, B, list, e, text, bt);
+    // Per-row data of an entry (log2-sum-exp, D, own cube, mask word) comes from
+    // global memory behind the entry's list value. The loads are software-
+    // pipelined: entry e + 2's list value and entry e + 1's row data are
+    // requested during entry e, so their latency overlaps its MMAs.
+    struct RowData {
+      float lse2, dot;
+      int t, own;
+      uint32_t w;
+      bool valid, text;
+    };
+    auto request = [&](bool text, int bt) {
+      RowData r;
       const TileRow R = tile_row(G, text, bt, row);
       const size_t rix = (size_t)R.t * G.hq + R.h;
-      const float lse2 = R.valid ? a.lse[rix] : 0.f;
-      const float dot = R.valid ? a.dot[rix] : 0.f;
-      bool row_on = R.valid;
+      r.t = R.t;
+      r.valid = R.valid;
+      r.text = text;
+      r.lse2 = R.valid ? a.lse[rix] : 0.f;
+      r.dot = R.valid ? a.dot[rix] : 0.f;
+      r.own = (!text && R.valid) ? a.cube_ids[R.t] : -1;
+      r.w = (B.visual && !text && !dense)
+                ? a.tile_mask[((size_t)bt * G.n_cubes + B.j) * 4 + wq]
+                : 0u;
+      return r;
+    };
+    bool text_n = false, text_nn = false;
+    int bt_n = 0, bt_nn = 0;
+    RowData cur{}, nxt{};
+    if (n_entries > 0) {
+      walk_entry(a, B, list, 0, text_n, bt_n);
+      cur = request(text_n, bt_n);
+    }
+    if (n_entries > 1) walk_entry(a, B, list, 1, text_n, bt_n);
+    bool ok = true;
+    for (int e = 0; e < n_entries; ++e) {
+      if (e + 1 < n_entries) nxt = request(text_n, bt_n);
+      if (e + 2 < n_entries) walk_entry(a, B, list, e + 2, text_nn, bt_nn);
+      const float lse2 = cur.lse2, dot = cur.dot;
+      bool row_on = cur.valid;
       int lim = B.nk;
       if (B.visual) {
-        if (!text && R.valid) {
-          const int own = a.cube_ids[R.t];
-          if (dense) {
-            row_on = B.j <= own;
-          } else {
-            const uint32_t w = a.tile_mask[((size_t)bt * G.n_cubes + B.j) * 4 + wq];
-            row_on = ((w >> lane) & 1u) != 0u;
-          }
-          if (B.j == own) lim = min(lim, R.t - B.k0 + 1);
+        if (!cur.text && cur.valid) {
+          row_on = dense ? B.j <= cur.own : ((cur.w >> lane) & 1u) != 0u;
+          if (B.j == cur.own) lim = min(lim, cur.t - B.k0 + 1);
         }
       } else {
-        lim = min(lim, R.t - B.k0 + 1);
+        lim = min(lim, cur.t - B.k0 + 1);
       }
       if (lim <= 0) row_on = false;
       if (!row_on) lim = 0;
+      cur = nxt;
+      text_n = text_nn;
+      bt_n = bt_nn;
       const int sb = e & 1;
       if (!mbar_wait_warp(&s_full[sb], (e >> 1) & 1, &s_abort, hdr, 0xa740u)) {
         ok = false;
