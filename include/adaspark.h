@@ -112,8 +112,8 @@ typedef struct {
 size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv,
                                     int d, int dtype);
 
-/* AdaS-Attn for one layer (key design 2 of the papernotes note; the abstract's
- * "relevance scores computed over preceding Cubes").
+/* AdaS-Attn for one layer (key design 2 of the papernotes note; the abstract
+ * scores relevance over the preceding cubes only).
  *
  * For a visual token t of cube i and query head h (KV head floor(h/(hq/hkv))):
  *   kbar_j = mean of K over cube j;  P = softmax_j<i(q . kbar_j / sqrt(d));
@@ -271,8 +271,8 @@ int adaspark_token_ffn(const void *x, const void *W_gate, const void *W_up, cons
                        int F, float p, float *y, void *workspace, size_t workspace_bytes,
                        void *stream);
 
-/* Importance of a token inside its cube for AdaS-FFN (key design 3 says only
- * "importance by L2 norm", then the Top-p rule). The linear share is the
+/* Importance of a token inside its cube for AdaS-FFN (key design 3 only says
+ * that importance comes from the L2 norm, followed by the Top-p rule). The linear share is the
  * reading adaspark_token_ffn takes; the other two are alternatives the text
  * does not exclude. All three rank a cube's tokens like their L2 norms. */
 #define ADASPARK_IMPORTANCE_L2_SHARE   0  /* ||x_u|| / sum_v ||x_v||          */

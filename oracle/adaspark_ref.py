@@ -328,10 +328,10 @@ IMPORTANCE = ("l2", "l2sq", "softmax")
 
 
 def token_importance(norms, importance="l2"):
-    """Importance of a cube's tokens from their L2 norms (key design 3 says only
-    "importance by L2 norm", then the same Top-p rule). "l2": the linear share
-    ||x_u|| / sum ||x_v|| (the reading this build takes); the two alternatives
-    the pages do not exclude: "l2sq", the energy share ||x_u||^2 / sum ||x_v||^2,
+    """Importance of a cube's tokens from their L2 norms (key design 3 only says
+    that importance comes from the L2 norm, followed by the same Top-p rule).
+    "l2": the linear share ||x_u|| / sum ||x_v|| (the default reading); the two
+    alternatives the pages do not exclude: "l2sq", the energy share ||x_u||^2 / sum ||x_v||^2,
     and "softmax", softmax over the cube of ||x_u||. All three rank tokens in
     the same order as their norms. Returns None when the norms sum to 0 (l2,
     l2sq: no importance is defined; the cube keeps every token)."""

@@ -103,7 +103,8 @@ def _cfg(i, **kw):
     return LayerConfig(seed=BASE_SEED + i, **kw)
 
 
-# The five workloads (sizes per the pages' Qwen2.5-VL shapes, grids per the spec).
+# The five workloads: Qwen2.5-VL-3B / 7B layer shapes (heads, head size, hidden and FFN
+# widths) on video-token grids of 18K to 256K tokens, plus a tiny fp32 case.
 CONFIGS = {
     1: _cfg(1, name="tiny-fp32", grid=(8, 8, 8), cube=(4, 4, 2), n_text=32, D=256,
             hq=4, hkv=1, d=64, F=512, dtype="fp32", sigma=0.3),
