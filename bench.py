@@ -351,7 +351,9 @@ def run_ours(args, rank, world, device):
     # Every step copies its inputs (Q, K, V, x) from pinned host memory and its
     # outputs (out, y) back, as a serving loop would: on a copy-in stream, the
     # compute stream and a copy-out stream, with two device buffers of each
-    # kind, so that step k's outputs leave and step k+1's inputs arrive while
+    # kind. Q, K and V go first, so that AdaS-Attn starts while x is still on
+    # its way (AdaS-FFN waits for it), and the attention output leaves while
+    # AdaS-FFN runs; step k's outputs leave and step k+1's inputs arrive while
     # step k+1 computes. The timed region runs from before the first input
     # copy to the end of the last output copy.
     pinned = {k: torch.empty(lay[k].shape, dtype=lay[k].dtype, pin_memory=True)
@@ -368,10 +370,8 @@ def run_ours(args, rank, world, device):
         host_y[0].numel() * host_y[0].element_size()
     e2e_steps = max(2, args.steps)
     s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    mk = lambda: torch.cuda.Event()
-    ev_in = [mk() for _ in range(e2e_steps)]
-    ev_cmp = [mk() for _ in range(e2e_steps)]
-    ev_out = [mk() for _ in range(e2e_steps)]
+    mk = lambda: [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_qkv, ev_x, ev_attn, ev_cmp, ev_out_a, ev_out_y = mk(), mk(), mk(), mk(), mk(), mk()
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -381,25 +381,35 @@ def run_ours(args, rank, world, device):
         if k >= 2:
             s_in.wait_event(ev_cmp[k - 2])           # inputs of buffer b consumed
         with torch.cuda.stream(s_in):
-            for name in pinned:
+            for name in ("Q", "K", "V"):
                 dev_in[b][name].copy_(pinned[name], non_blocking=True)
-            ev_in[k].record(s_in)
-        s_cmp.wait_event(ev_in[k])
+            ev_qkv[k].record(s_in)
+            dev_in[b]["x"].copy_(pinned["x"], non_blocking=True)
+            ev_x[k].record(s_in)
+        d = dev_in[b]
+        s_cmp.wait_event(ev_qkv[k])
         if k >= 2:
-            s_cmp.wait_event(ev_out[k - 2])          # outputs of buffer b copied out
+            s_cmp.wait_event(ev_out_a[k - 2])        # attention output of buffer b copied out
         with torch.cuda.stream(s_cmp):
-            d = dev_in[b]
             fb.cube_attn(d["Q"], d["K"], d["V"], lay["cube_ids"], lay["cube_offsets"], n_vis,
                          cfg.p, out=dev_out[b], workspace=aws, stream=s_cmp)
+            ev_attn[k].record(s_cmp)
+        s_cmp.wait_event(ev_x[k])
+        if k >= 2:
+            s_cmp.wait_event(ev_out_y[k - 2])        # y of buffer b copied out
+        with torch.cuda.stream(s_cmp):
             fb.token_ffn(d["x"], lay["W_gate"], lay["W_up"], lay["W_down"], lay["cube_ids"],
                          lay["cube_offsets"], lay["text_mask"], n_vis, cfg.p, y=dev_y[b],
                          workspace=fws, stream=s_cmp)
             ev_cmp[k].record(s_cmp)
-        s_out.wait_event(ev_cmp[k])
+        s_out.wait_event(ev_attn[k])
         with torch.cuda.stream(s_out):
             host_out[b].copy_(dev_out[b], non_blocking=True)
+            ev_out_a[k].record(s_out)
+        s_out.wait_event(ev_cmp[k])
+        with torch.cuda.stream(s_out):
             host_y[b].copy_(dev_y[b], non_blocking=True)
-            ev_out[k].record(s_out)
+            ev_out_y[k].record(s_out)
     e1.record(s_out)
     torch.cuda.synchronize()
     for ws in (aws, fws):
