@@ -321,6 +321,7 @@ int adaspark_cube_attn_backward(const void* Q, const void* K, const void* V, con
   a.inv_start = reinterpret_cast<int32_t*>(ws + L.inv_start);
   a.inv_list = reinterpret_cast<int32_t*>(ws + L.inv_list);
   a.inv_chunks = L.chunks;
+  a.pieces = ws + L.pieces;
   a.G = G;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d));
   a.inv_sqrt_d = (float)(1.0 / std::sqrt((double)d));

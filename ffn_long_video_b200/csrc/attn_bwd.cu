@@ -41,7 +41,6 @@ namespace abwd {
 constexpr int RING = 64;
 constexpr int Q_BYTES = 128 * 256;   // 128 rows x 128 dims bf16 (two 64-dim halves)
 constexpr int KB_BYTES = 2 * 8192;   // one 64-key block of K or V (two 64-dim halves)
-constexpr int PS_BYTES = 128 * 128;  // 128 rows x 64 keys bf16
 
 struct Desc {
   int k0, nk, j, pass;  // pass: 0 sums D_r, 1 forms dS and dQ
@@ -530,69 +529,97 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
 }
 
 // ------------------------------------------------------------------ dK / dV kernel
-// One CTA per (KV head, 64-key block). Block units per KV head: four per cube
-// (pieces of up to 64 keys; cubes hold at most 256 tokens; absent pieces exit),
-// then the 64-key pieces of the text suffix. Warps: 0 TMA producer, 1 TMEM
-// allocator + MMA issuer, 2-5 one thread per query row, then per head dimension
-// in the epilogue. TMEM (512 columns): S buffers 64 b, dP buffers 128 + 64 b,
-// dV^T 256-319, dK^T 320-383 (lane = head dimension, column = key).
+// Key pieces: the keys of each cube cut into pieces of up to 64 (cubes hold at
+// most 256 tokens), cube by cube, then the text suffix in pieces of 64. One
+// CTA per (KV head, pair of consecutive pieces) = up to 128 keys. It walks the
+// query tiles that admit either piece (the union of the two cubes' inverted
+// lists, ascending, then the text tiles) and computes, per tile,
+//   S^T = K Q^T and dP^T = V dO^T      (M = 128 keys, N = 128 rows, K = d)
+// into TMEM; one thread per key turns them into P^T and dS^T (bf16, written
+// over the scores they came from), and
+//   dV += P^T dO,  dK += dS^T Q        (M = 128 keys, N = d, K = 128 rows)
+// read P^T / dS^T from TMEM (the product form of the forward's PV), so every
+// product has N = 128 and the key block's gradients stay in TMEM until the
+// end. Warps: 0 tile walker + TMA producer, 1 TMEM allocator + MMA issuer,
+// 2-9 row threads: thread = key (TMEM lane), two warps per lane quadrant,
+// each taking 64 of the tile's 128 rows. TMEM (512 columns): S^T 0-127,
+// dP^T 128-255, dV 256-383, dK 384-511.
 namespace dkv {
-constexpr int THREADS = 192;
+constexpr int THREADS = 320;
+constexpr int ROW_THREADS = 256;
 constexpr int QST = 2;
-constexpr size_t SMEM_BYTES = 1024 + 2 * KB_BYTES + QST * 2 * Q_BYTES + 2 * PS_BYTES + 1024;
+constexpr int RINGE = 64;                 // tile-walk ring entries
+constexpr int KP_BYTES = 2 * 16384;       // 128 keys x 128 dims bf16 (two 64-dim halves)
+constexpr size_t SMEM_BYTES = 1024 + 2 * KP_BYTES + QST * 2 * Q_BYTES + 2048;
 }  // namespace dkv
 
-struct KeyBlock {
-  bool ok;        // the block exists
-  bool visual;    // keys of a visual cube (else of the text suffix)
-  int kv, j, k0, nk;
-  int n_vis_entries, tt_min, n_text_entries;
+struct Piece {
+  int cube;   // -1: text keys
+  int k0, nk;
+  int pad;
 };
 
-__device__ __forceinline__ KeyBlock decode_key_block(const AttnBwdArgs& a) {
+// Piece table (one block): pieces of every cube in order, then the text
+// pieces; the count goes to hdr->spare0.
+__global__ void __launch_bounds__(1024) piece_table_kernel(AttnBwdArgs a) {
+  __shared__ int part[1024];
+  if (status_bad(a.hdr)) return;
   const AttnGeom& G = a.G;
-  const int n_text = G.n_tokens - G.n_vis;
-  const int units = 4 * G.n_cubes + (n_text + 63) / 64;
-  KeyBlock B;
-  B.kv = blockIdx.x / units;
-  const int u = blockIdx.x - B.kv * units;
-  B.ok = true;
-  if (u < 4 * G.n_cubes) {
-    B.visual = true;
-    B.j = u >> 2;
-    const int ke = a.cube_offsets[B.j + 1];
-    B.k0 = a.cube_offsets[B.j] + 64 * (u & 3);
-    B.ok = B.k0 < ke;
-    B.nk = min(64, ke - B.k0);
-    const size_t key = ((size_t)B.kv * G.n_cubes + B.j) * a.inv_chunks;
-    B.n_vis_entries = B.ok ? a.inv_start[key + a.inv_chunks] - a.inv_start[key] : 0;
-    B.tt_min = 0;
-  } else {
-    B.visual = false;
-    B.j = -1;
-    B.k0 = G.n_vis + 64 * (u - 4 * G.n_cubes);
-    B.nk = min(64, G.n_tokens - B.k0);
-    B.n_vis_entries = 0;
-    B.tt_min = (B.k0 - G.n_vis) / kTileRows;  // text tiles before it end before k0
+  const int C = G.n_cubes, tid = threadIdx.x;
+  const int per = (C + 1023) / 1024;
+  const int b = min(tid * per, C), e = min(b + per, C);
+  int cnt = 0;
+  for (int j = b; j < e; ++j) cnt += (a.cube_offsets[j + 1] - a.cube_offsets[j] + 63) / 64;
+  part[tid] = cnt;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int v = tid >= o ? part[tid - o] : 0;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
   }
-  B.n_text_entries = G.g * (G.ttiles_per_head - B.tt_min);
-  return B;
+  int pos = part[tid] - cnt;
+  Piece* out = reinterpret_cast<Piece*>(a.pieces);
+  for (int j = b; j < e; ++j) {
+    const int k0 = a.cube_offsets[j], ke = a.cube_offsets[j + 1];
+    for (int k = k0; k < ke; k += 64) out[pos++] = Piece{j, k, min(64, ke - k), 0};
+  }
+  const int n_vis_pieces = part[1023];
+  const int n_text = G.n_tokens - G.n_vis;
+  const int n_tp = (n_text + 63) / 64;
+  for (int q = tid; q < n_tp; q += 1024) {
+    const int k0 = G.n_vis + 64 * q;
+    out[n_vis_pieces + q] = Piece{-1, k0, min(64, G.n_tokens - k0), 0};
+  }
+  if (tid == 0) a.hdr->spare0 = (uint32_t)(n_vis_pieces + n_tp);
 }
 
-// Entry e of a key block's walk: (text tile?, tile index within its kind).
-__device__ __forceinline__ void walk_entry(const AttnBwdArgs& a, const KeyBlock& B,
-                                           const int32_t* list, int e, bool& text, int& bt) {
+struct WalkEntry {
+  int bt;      // tile index within its kind; -1 terminates
+  int text;
+};
+
+// Admitted keys of row `row` of tile (text, bt) in a piece: keys [k0, k0 + lim).
+__device__ __forceinline__ int piece_limit(const AttnBwdArgs& a, const Piece& pc, bool text,
+                                           int bt, int row, const TileRow& R, int own, int c_hi,
+                                           bool dense) {
+  if (!R.valid || pc.nk <= 0) return 0;
   const AttnGeom& G = a.G;
-  if (e < B.n_vis_entries) {
-    text = false;
-    bt = list[e];
-  } else {
-    const int e2 = e - B.n_vis_entries;
-    const int nt = G.ttiles_per_head - B.tt_min;
-    const int hh = e2 / nt, tt = B.tt_min + e2 % nt;
-    text = true;
-    bt = B.kv * G.ttiles_per_kv + hh * G.ttiles_per_head + tt;
+  if (pc.cube < 0) {  // text keys: only text rows, causally
+    if (!text) return 0;
+    return max(0, min(pc.nk, R.t - pc.k0 + 1));
   }
+  if (text) return pc.nk;  // text rows see every visual key
+  if (pc.cube > c_hi) return 0;  // follows every row of the tile (mask not written)
+  bool on;
+  if (dense) {
+    on = pc.cube <= own;
+  } else {
+    const uint32_t w = a.tile_mask[((size_t)bt * G.n_cubes + pc.cube) * 4 + (row >> 5)];
+    on = ((w >> (row & 31)) & 1u) != 0u;
+  }
+  if (!on) return 0;
+  return pc.cube == own ? max(0, min(pc.nk, R.t - pc.k0 + 1)) : pc.nk;
 }
 
 __global__ void __launch_bounds__(dkv::THREADS, 1)
@@ -604,30 +631,55 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* sK = smem;                       // K block, then V block
-  uint8_t* sV = sK + KB_BYTES;
-  uint8_t* sQd = sV + KB_BYTES;             // [QST][Q tile | dO tile]
-  uint8_t* sP = sQd + QST * 2 * Q_BYTES;
-  uint8_t* sdS = sP + PS_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sdS + PS_BYTES);
+  uint8_t* sK = smem;                       // keys 0-63: piece A, 64-127: piece B
+  uint8_t* sV = sK + KP_BYTES;
+  uint8_t* sQd = sV + KP_BYTES;             // [QST][Q tile | dO tile]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sQd + QST * 2 * Q_BYTES);
   uint64_t* kv_full = bars;
   uint64_t* qd_full = kv_full + 1;          // [QST]
   uint64_t* qd_empty = qd_full + QST;       // [QST]
-  uint64_t* s_full = qd_empty + QST;        // [2]
-  uint64_t* ps_full = s_full + 2;
-  uint64_t* ps_empty = ps_full + 1;
-  uint64_t* done = ps_empty + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* s_full = qd_empty + QST;       // S^T landed
+  uint64_t* dp_full = s_full + 1;           // dP^T landed
+  uint64_t* p_ready = dp_full + 1;          // P^T stored by the row threads
+  uint64_t* ds_ready = p_ready + 1;         // dS^T stored by the row threads
+  uint64_t* meta_full = ds_ready + 1;       // [2]
+  uint64_t* done = meta_full + 2;
+  uint64_t* w_full = done + 1;              // [RINGE]
+  uint64_t* w_empty = w_full + RINGE;       // [RINGE]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(w_empty + RINGE);
+  __shared__ WalkEntry s_walk[RINGE];
+  __shared__ float s_lse[2][128], s_dot[2][128];
+  __shared__ int s_lim[2][2][128];          // [entry parity][piece][row]
   __shared__ volatile int s_abort;
 
   const AttnGeom& G = a.G;
   WsHeader* hdr = a.hdr;
   if (status_bad(hdr)) return;              // uniform: before any barrier or TMEM
-  const KeyBlock B = decode_key_block(a);
-  if (!B.ok) return;
-  const int n_entries = B.n_vis_entries + B.n_text_entries;
-  const int32_t* list =
-      a.inv_list + (B.visual ? a.inv_start[((size_t)B.kv * G.n_cubes + B.j) * a.inv_chunks] : 0);
+  const int n_pieces = (int)hdr->spare0;
+  const int units = (4 * G.n_cubes + (G.n_tokens - G.n_vis + 63) / 64 + 1) / 2;
+  const int kv = blockIdx.x / units, u = blockIdx.x - kv * units;
+  if (2 * u >= n_pieces) return;
+  const Piece* pieces = reinterpret_cast<const Piece*>(a.pieces);
+  const Piece pA = pieces[2 * u];
+  const Piece pB = 2 * u + 1 < n_pieces ? pieces[2 * u + 1] : Piece{-1, pA.k0, 0, 0};
+  const bool dense = fwd_was_dense(a.fhdr);
+  // visual lists of the two pieces' cubes (the same list once if one cube)
+  const int jA = pA.cube, jB = (pB.nk > 0 && pB.cube != pA.cube) ? pB.cube : -1;
+  const size_t nc = a.inv_chunks;
+  auto list_of = [&](int j, const int32_t*& lst, int& n) {
+    if (j < 0) {
+      lst = nullptr;
+      n = 0;
+      return;
+    }
+    const size_t key = ((size_t)kv * G.n_cubes + j) * nc;
+    lst = a.inv_list + a.inv_start[key];
+    n = a.inv_start[key + nc] - a.inv_start[key];
+  };
+  // text tiles: all of them when a visual piece is present, else those that
+  // reach the first text key
+  const bool any_visual = jA >= 0 || (pB.nk > 0 && pB.cube >= 0);
+  const int tt_min = any_visual ? 0 : (pA.k0 - G.n_vis) / kTileRows;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -636,10 +688,16 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
       mbar_init(&qd_full[s], 1);
       mbar_init(&qd_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(&s_full[b], 1);
-    mbar_init(ps_full, 128);
-    mbar_init(ps_empty, 1);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, ROW_THREADS);
+    mbar_init(ds_ready, ROW_THREADS);
+    for (int b = 0; b < 2; ++b) mbar_init(&meta_full[b], ROW_THREADS);
     mbar_init(done, 1);
+    for (int r = 0; r < RINGE; ++r) {
+      mbar_init(&w_full[r], 1);
+      mbar_init(&w_empty[r], ROW_THREADS);
+    }
     fence_mbar_init();
     s_abort = 0;
   }
@@ -657,31 +715,64 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ tile walker + producer
     if (lane == 0) {
-      mbar_expect_tx(kv_full, 2 * KB_BYTES);
-      tma_load_3d(&mapK, kv_full, sK, 0, B.kv, B.k0);
-      tma_load_3d(&mapK, kv_full, sK + 8192, 64, B.kv, B.k0);
-      tma_load_3d(&mapV, kv_full, sV, 0, B.kv, B.k0);
-      tma_load_3d(&mapV, kv_full, sV + 8192, 64, B.kv, B.k0);
-      int e = 0;
+      mbar_expect_tx(kv_full, (pB.nk > 0 ? 4u : 2u) * 8192u * 2u);
+      tma_load_3d(&mapK, kv_full, sK, 0, kv, pA.k0);
+      tma_load_3d(&mapK, kv_full, sK + 16384, 64, kv, pA.k0);
+      tma_load_3d(&mapV, kv_full, sV, 0, kv, pA.k0);
+      tma_load_3d(&mapV, kv_full, sV + 16384, 64, kv, pA.k0);
+      if (pB.nk > 0) {
+        tma_load_3d(&mapK, kv_full, sK + 8192, 0, kv, pB.k0);
+        tma_load_3d(&mapK, kv_full, sK + 16384 + 8192, 64, kv, pB.k0);
+        tma_load_3d(&mapV, kv_full, sV + 8192, 0, kv, pB.k0);
+        tma_load_3d(&mapV, kv_full, sV + 16384 + 8192, 64, kv, pB.k0);
+      }
+      const int32_t *LA, *LB;
+      int nA, nB;
+      list_of(jA, LA, nA);
+      list_of(jB, LB, nB);
+      const int nt = G.ttiles_per_head - tt_min;
+      const int n_text_entries = G.g * nt;
+      int ia = 0, ib = 0, et = 0, e = 0;
       bool ok = true;
-      for (; e < n_entries; ++e) {
-        const int st = e % QST;
-        if (!mbar_wait(&qd_empty[st], ((e / QST) & 1) ^ 1, &s_abort, hdr, 0xa700u)) {
+      while (ok) {
+        // next entry: merge of the two ascending lists, then the text tiles
+        WalkEntry we;
+        if (ia < nA || ib < nB) {
+          const int va = ia < nA ? LA[ia] : INT32_MAX, vb = ib < nB ? LB[ib] : INT32_MAX;
+          const int v = min(va, vb);
+          ia += va == v;
+          ib += vb == v;
+          we = WalkEntry{v, 0};
+        } else if (et < n_text_entries) {
+          const int hh = et / nt, tt = tt_min + et % nt;
+          we = WalkEntry{kv * G.ttiles_per_kv + hh * G.ttiles_per_head + tt, 1};
+          ++et;
+        } else {
+          we = WalkEntry{-1, 0};
+        }
+        const int slot = e % RINGE;
+        if (!mbar_wait(&w_empty[slot], ((e / RINGE) & 1) ^ 1, &s_abort, hdr, 0xa800u)) {
           ok = false;
           break;
         }
-        bool text;
-        int bt;
-        walk_entry(a, B, list, e, text, bt);
-        const TileRow R0 = tile_row(G, text, bt, 0);
+        s_walk[slot] = we;
+        mbar_arrive(&w_full[slot]);
+        if (we.bt < 0) break;
+        const int st = e % QST;
+        if (!mbar_wait(&qd_empty[st], ((e / QST) & 1) ^ 1, &s_abort, hdr, 0xa810u)) {
+          ok = false;
+          break;
+        }
+        const TileRow R0 = tile_row(G, we.text != 0, we.bt, 0);
         uint8_t* q = sQd + st * 2 * Q_BYTES;
         mbar_expect_tx(&qd_full[st], 2 * Q_BYTES);
         tma_load_3d(&mapQ, &qd_full[st], q, 0, R0.h, R0.t);
         tma_load_3d(&mapQ, &qd_full[st], q + 16384, 64, R0.h, R0.t);
         tma_load_3d(&mapdO, &qd_full[st], q + Q_BYTES, 0, R0.h, R0.t);
         tma_load_3d(&mapdO, &qd_full[st], q + Q_BYTES + 16384, 64, R0.h, R0.t);
+        ++e;
       }
       // let copies in flight land before the CTA can exit
       long long t0 = clock64();
@@ -699,60 +790,71 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64);
-      constexpr uint32_t idesc_g = make_idesc_bf16_mn(128, 64);
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128);
+      constexpr uint32_t idesc_g = make_idesc_bf16(128, 128, true);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      const uint32_t p_addr = smem_u32(sP), ds_addr = smem_u32(sdS);
-      bool ok = mbar_wait(kv_full, 0, &s_abort, hdr, 0xa710u);
+      bool ok = mbar_wait(kv_full, 0, &s_abort, hdr, 0xa820u);
       tc_fence_after();
-      auto issue_grad = [&](int f) -> bool {
-        if (!mbar_wait(ps_full, f & 1, &s_abort, hdr, 0xa720u)) return false;
-        tc_fence_after();
-        const int st = f % QST;
-        const uint32_t q_addr = smem_u32(sQd + st * 2 * Q_BYTES);
-        const uint32_t do_addr = q_addr + Q_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acc = (f > 0 || kk > 0) ? 1u : 0u;
-          // dV^T[d][key] += dO^T[d][row] P[row][key]
-          umma_bf16(tmem_base + 256, make_sdesc_sw128(do_addr + kk * 2048, 16384, 1024),
-                    make_sdesc_sw128(p_addr + kk * 2048, 8192, 1024), idesc_g, acc);
-          // dK^T[d][key] += Q^T[d][row] dS[row][key]
-          umma_bf16(tmem_base + 320, make_sdesc_sw128(q_addr + kk * 2048, 16384, 1024),
-                    make_sdesc_sw128(ds_addr + kk * 2048, 8192, 1024), idesc_g, acc);
-        }
-        umma_commit(ps_empty);
-        umma_commit(&qd_empty[st]);
-        return true;
-      };
       int e = 0;
-      for (; e < n_entries && ok; ++e) {
-        const int st = e % QST, sb = e & 1;
-        if (!mbar_wait(&qd_full[st], (e / QST) & 1, &s_abort, hdr, 0xa730u)) {
+      for (; ok; ++e) {
+        const int slot = e % RINGE;
+        if (!mbar_wait(&w_full[slot], (e / RINGE) & 1, &s_abort, hdr, 0xa830u)) {
+          ok = false;
+          break;
+        }
+        if (s_walk[slot].bt < 0) break;
+        const int st = e % QST;
+        if (!mbar_wait(&qd_full[st], (e / QST) & 1, &s_abort, hdr, 0xa840u)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQd + st * 2 * Q_BYTES);
         const uint32_t do_addr = q_addr + Q_BYTES;
+        // S^T = K Q^T, then dP^T = V dO^T (both K-major, K = d), each with its
+        // own commit so the row threads start on P while dP^T computes
 #pragma unroll
         for (int dc = 0; dc < 2; ++dc)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (dc | kk) != 0 ? 1u : 0u;
-            umma_bf16(tmem_base + sb * 64, make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024),
-                      make_sdesc_sw128(k_addr + dc * 8192 + kk * 32, 16, 1024), idesc_s, acc);
-            umma_bf16(tmem_base + 128 + sb * 64,
-                      make_sdesc_sw128(do_addr + dc * 16384 + kk * 32, 16, 1024),
-                      make_sdesc_sw128(v_addr + dc * 8192 + kk * 32, 16, 1024), idesc_s, acc);
-          }
-        umma_commit(&s_full[sb]);
-        if (e > 0 && !issue_grad(e - 1)) {
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem_base, make_sdesc_sw128(k_addr + dc * 16384 + kk * 32, 16, 1024),
+                      make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024), idesc_s,
+                      (dc | kk) != 0 ? 1u : 0u);
+        umma_commit(s_full);
+#pragma unroll
+        for (int dc = 0; dc < 2; ++dc)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem_base + 128,
+                      make_sdesc_sw128(v_addr + dc * 16384 + kk * 32, 16, 1024),
+                      make_sdesc_sw128(do_addr + dc * 16384 + kk * 32, 16, 1024), idesc_s,
+                      (dc | kk) != 0 ? 1u : 0u);
+        umma_commit(dp_full);
+        // dV += P^T dO as soon as P^T is in TMEM (rows 64 hc + r packed at
+        // column 64 hc + r / 2), while the row threads form dS
+        if (!mbar_wait(p_ready, e & 1, &s_abort, hdr, 0xa850u)) {
           ok = false;
           break;
         }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tmem_base + 256, tmem_base + (kk >> 2) * 64 + (kk & 3) * 8,
+                       make_sdesc_sw128(do_addr + kk * 2048, 16384, 1024), idesc_g,
+                       (e > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q
+        if (!mbar_wait(ds_ready, e & 1, &s_abort, hdr, 0xa855u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16_ts(tmem_base + 384, tmem_base + 128 + (kk >> 2) * 64 + (kk & 3) * 8,
+                       make_sdesc_sw128(q_addr + kk * 2048, 16384, 1024), idesc_g,
+                       (e > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&qd_empty[st]);
       }
-      if (ok && n_entries > 0) ok = issue_grad(n_entries - 1);
       umma_commit(done);
       long long t0 = clock64();
       while (!mbar_try_wait(done, 0) && clock64() - t0 < kWaitCycles) {
@@ -761,134 +863,144 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
   } else {
     // ------------------------------------------------------------ row threads
     const int wq = warp & 3;
-    const int row = wq * 32 + lane;
+    const int key = wq * 32 + lane;           // TMEM lane = key of the pair
+    const int hc = (warp - 2) >> 2;           // rows [64 hc, 64 hc + 64) of each tile
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const float scale = a.scale_log2;
-    const bool dense = fwd_was_dense(a.fhdr);
-    // Per-row data of an entry (log2-sum-exp, D, own cube, mask word) comes from
-    // global memory behind the entry's list value. The loads are software-
-    // pipelined: entry e + 2's list value and entry e + 1's row data are
-    // requested during entry e, so their latency overlaps its MMAs.
-    struct RowData {
-      float lse2, dot;
-      int t, own;
-      uint32_t w;
-      bool valid, text;
-    };
-    auto request = [&](bool text, int bt) {
-      RowData r;
-      const TileRow R = tile_row(G, text, bt, row);
-      const size_t rix = (size_t)R.t * G.hq + R.h;
-      r.t = R.t;
-      r.valid = R.valid;
-      r.text = text;
-      r.lse2 = R.valid ? a.lse[rix] : 0.f;
-      r.dot = R.valid ? a.dot[rix] : 0.f;
-      r.own = (!text && R.valid) ? a.cube_ids[R.t] : -1;
-      r.w = (B.visual && !text && !dense)
-                ? a.tile_mask[((size_t)bt * G.n_cubes + B.j) * 4 + wq]
-                : 0u;
-      return r;
-    };
-    bool text_n = false, text_nn = false;
-    int bt_n = 0, bt_nn = 0;
-    RowData cur{}, nxt{};
-    if (n_entries > 0) {
-      walk_entry(a, B, list, 0, text_n, bt_n);
-      cur = request(text_n, bt_n);
-    }
-    if (n_entries > 1) walk_entry(a, B, list, 1, text_n, bt_n);
+    const int kp = key < 64 ? 0 : 1;          // piece of this key
+    const int kl = key & 63;                  // index inside the piece
+    const int mrow = (warp - 2) * 32 + lane;  // 0..255: metadata of row mrow (first 128)
     bool ok = true;
-    for (int e = 0; e < n_entries; ++e) {
-      if (e + 1 < n_entries) nxt = request(text_n, bt_n);
-      if (e + 2 < n_entries) walk_entry(a, B, list, e + 2, text_nn, bt_nn);
-      const float lse2 = cur.lse2, dot = cur.dot;
-      bool row_on = cur.valid;
-      int lim = B.nk;
-      if (B.visual) {
-        if (!cur.text && cur.valid) {
-          row_on = dense ? B.j <= cur.own : ((cur.w >> lane) & 1u) != 0u;
-          if (B.j == cur.own) lim = min(lim, cur.t - B.k0 + 1);
-        }
-      } else {
-        lim = min(lim, cur.t - B.k0 + 1);
+    int e = 0;
+    for (;; ++e) {
+      const int slot = e % RINGE;
+      if (!mbar_wait_warp(&w_full[slot], (e / RINGE) & 1, &s_abort, hdr, 0xa860u)) {
+        ok = false;
+        break;
       }
-      if (lim <= 0) row_on = false;
-      if (!row_on) lim = 0;
-      cur = nxt;
-      text_n = text_nn;
-      bt_n = bt_nn;
-      const int sb = e & 1;
-      if (!mbar_wait_warp(&s_full[sb], (e >> 1) & 1, &s_abort, hdr, 0xa740u)) {
+      const WalkEntry we = s_walk[slot];
+      if (we.bt < 0) break;
+      const bool text = we.text != 0;
+      const int par = e & 1;
+      // per-row data of the tile, one row per thread of the first 128
+      if (mrow < 128) {
+        const TileRow R = tile_row(G, text, we.bt, mrow);
+        const size_t rix = (size_t)R.t * G.hq + R.h;
+        int own = -1, c_hi = -1;
+        if (!text && R.valid) {
+          own = a.cube_ids[R.t];
+          const TileRow Rl = tile_row(G, false, we.bt, 0);
+          c_hi = a.cube_ids[min(Rl.t + kTileRows, G.n_vis) - 1];
+        }
+        s_lse[par][mrow] = R.valid ? a.lse[rix] : 0.f;
+        s_dot[par][mrow] = R.valid ? a.dot[rix] : 0.f;
+        s_lim[par][0][mrow] = piece_limit(a, pA, text, we.bt, mrow, R, own, c_hi, dense);
+        s_lim[par][1][mrow] = piece_limit(a, pB, text, we.bt, mrow, R, own, c_hi, dense);
+      }
+      mbar_arrive(&meta_full[par]);
+      if (!mbar_wait_warp(&meta_full[par], (e >> 1) & 1, &s_abort, hdr, 0xa870u)) {
+        ok = false;
+        break;
+      }
+      // every row thread has read the slot once the metadata is in
+      mbar_arrive(&w_empty[slot]);
+      if (!mbar_wait_warp(s_full, e & 1, &s_abort, hdr, 0xa880u)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[64], dp[64];
+      float pv[64];
       {
+        uint32_t sr[64];
         uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
         uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        uint32_t(&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
-        uint32_t(&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
-        tmem_ld32(tmem_base + lane_base + sb * 64, s0);
-        tmem_ld32(tmem_base + lane_base + sb * 64 + 32, s1);
-        tmem_ld32(tmem_base + lane_base + 128 + sb * 64, p0);
-        tmem_ld32(tmem_base + lane_base + 128 + sb * 64 + 32, p1);
-      }
-      tmem_ld_wait();
-      uint32_t pp[32], pd[32];
+        tmem_ld32(tmem_base + lane_base + hc * 64, s0);
+        tmem_ld32(tmem_base + lane_base + hc * 64 + 32, s1);
+        tmem_ld_wait();
+        uint32_t pp[32];
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int u = 2 * q;
-        const float p0 = u < lim ? ex2(fmaf(__uint_as_float(sr[u]), scale, -lse2)) : 0.f;
-        const float p1 = u + 1 < lim ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, -lse2)) : 0.f;
-        pp[q] = pack_bf16x2(p0, p1);
-        pd[q] = pack_bf16x2(p0 * (__uint_as_float(dp[u]) - dot),
-                            p1 * (__uint_as_float(dp[u + 1]) - dot));
+        for (int q = 0; q < 32; ++q) {
+#pragma unroll
+          for (int z = 0; z < 2; ++z) {
+            const int r = hc * 64 + 2 * q + z;
+            pv[2 * q + z] = kl < s_lim[par][kp][r]
+                                ? ex2(fmaf(__uint_as_float(sr[2 * q + z]), scale, -s_lse[par][r]))
+                                : 0.f;
+          }
+          pp[q] = pack_bf16x2(pv[2 * q], pv[2 * q + 1]);
+        }
+        tmem_st32(tmem_base + lane_base + hc * 64, pp);
+        tmem_st_wait();
       }
-      // the gradient MMAs of the previous entry have finished reading sP / sdS
-      if (e > 0 && !mbar_wait_warp(ps_empty, (e - 1) & 1, &s_abort, hdr, 0xa750u)) {
+      tc_fence_before();
+      mbar_arrive(p_ready);
+      if (!mbar_wait_warp(dp_full, e & 1, &s_abort, hdr, 0xa885u)) {
         ok = false;
         break;
       }
+      tc_fence_after();
+      {
+        uint32_t dp[64];
+        uint32_t(&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
+        uint32_t(&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
+        tmem_ld32(tmem_base + lane_base + 128 + hc * 64, p0);
+        tmem_ld32(tmem_base + lane_base + 128 + hc * 64 + 32, p1);
+        tmem_ld_wait();
+        uint32_t pd[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t off = sw128_offset(row, c);
-        *reinterpret_cast<uint4*>(sP + off) =
-            make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
-        *reinterpret_cast<uint4*>(sdS + off) =
-            make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
+        for (int q = 0; q < 32; ++q) {
+          float dv[2];
+#pragma unroll
+          for (int z = 0; z < 2; ++z) {
+            const int r = hc * 64 + 2 * q + z;
+            dv[z] = kl < s_lim[par][kp][r]
+                        ? pv[2 * q + z] * (__uint_as_float(dp[2 * q + z]) - s_dot[par][r])
+                        : 0.f;
+          }
+          pd[q] = pack_bf16x2(dv[0], dv[1]);
+        }
+        tmem_st32(tmem_base + lane_base + 128 + hc * 64, pd);
+        tmem_st_wait();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(ps_full);
+      mbar_arrive(ds_ready);
     }
-    // epilogue: thread = head dimension d, 64 keys of dV^T and dK^T
+    // epilogue: thread = key, 64 of the 128 head dimensions of dV and dK
     long long t0 = clock64();
     bool fin = ok;
-    if (ok && n_entries > 0) {
+    if (ok && e > 0) {
       fin = false;
       while (!(fin = mbar_try_wait(done, 0)) && clock64() - t0 < kWaitCycles) {
       }
-      if (!fin) set_status(hdr, ADASPARK_DEV_TIMEOUT, 0xa760u);
+      if (!fin) set_status(hdr, ADASPARK_DEV_TIMEOUT, 0xa890u);
     }
     fin = __all_sync(0xffffffffu, fin);
     if (fin) {
       tc_fence_after();
-      const int d = row;
+      const Piece& pc = kp == 0 ? pA : pB;
+      const bool kvalid = kl < pc.nk;
+      const size_t o = ((size_t)(pc.k0 + kl) * G.hkv + kv) * 128 + hc * 64;
 #pragma unroll 1
       for (int c = 0; c < 64; c += 32) {
         uint32_t v[32], k[32];
-        tmem_ld32(tmem_base + lane_base + 256 + c, v);
-        tmem_ld32(tmem_base + lane_base + 320 + c, k);
+        tmem_ld32(tmem_base + lane_base + 256 + hc * 64 + c, v);
+        tmem_ld32(tmem_base + lane_base + 384 + hc * 64 + c, k);
         tmem_ld_wait();
+        if (kvalid) {
+          float4* dv4 = reinterpret_cast<float4*>(a.dV + o + c);
+          float4* dk4 = reinterpret_cast<float4*>(a.dK + o + c);
+          const float sk = a.inv_sqrt_d;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int key = c + x;
-          if (key < B.nk) {
-            const size_t o = ((size_t)(B.k0 + key) * G.hkv + B.kv) * 128 + d;
-            a.dV[o] = n_entries > 0 ? __uint_as_float(v[x]) : 0.f;
-            a.dK[o] = n_entries > 0 ? __uint_as_float(k[x]) * a.inv_sqrt_d : 0.f;
+          for (int x = 0; x < 8; ++x) {
+            dv4[x] = e > 0 ? make_float4(__uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
+                                         __uint_as_float(v[4 * x + 2]),
+                                         __uint_as_float(v[4 * x + 3]))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            dk4[x] = e > 0 ? make_float4(__uint_as_float(k[4 * x]) * sk,
+                                         __uint_as_float(k[4 * x + 1]) * sk,
+                                         __uint_as_float(k[4 * x + 2]) * sk,
+                                         __uint_as_float(k[4 * x + 3]) * sk)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
           }
         }
       }
@@ -943,7 +1055,10 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a, cudaStream_t s) {
                     a)))
       return e;
   }
-  const int units = 4 * G.n_cubes + (G.n_tokens - G.n_vis + 63) / 64;
+  // key pieces (64 keys) and their pairs
+  if ((e = launch("attn_bwd_pieces", piece_table_kernel, dim3(1), dim3(1024), 0, s, a)))
+    return e;
+  const int units = (4 * G.n_cubes + (G.n_tokens - G.n_vis + 63) / 64 + 1) / 2;
   if (units > 0) {
     auto k = attn_bwd_dkv_kernel;
     if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,

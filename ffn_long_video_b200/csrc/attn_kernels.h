@@ -65,6 +65,7 @@ struct AttnBwdArgs {
   int32_t* inv_start;                 // [hkv * C * inv_chunks + 1] exclusive prefix
   int32_t* inv_list;                  // tile indices, ascending per (kv, j)
   int inv_chunks;                     // chunks of kInvChunk visual tiles per KV head
+  void* pieces;                       // key pieces of up to 64 keys (cube, k0, nk), cube order
   AttnGeom G;
   int kv_major;
   float scale_log2;                   // log2(e) / sqrt(d)

@@ -101,6 +101,7 @@ struct AttnBwdLayout {
   size_t inv_count;  // int32 [hkv][C][chunks]
   size_t inv_start;  // int32 [hkv * C * chunks + 1]
   size_t inv_list;   // int32 [n_vtiles][C] (capacity; filled per (kv, j) segment)
+  size_t pieces;     // int4 [4 C + text pieces] key pieces (cube, k0, nk, -)
   int chunks;        // chunks of kInvChunk visual tiles per KV head
   size_t total;
 };
@@ -117,6 +118,7 @@ __host__ __device__ inline AttnBwdLayout make_attn_bwd_layout(const AttnGeom& G)
   L.inv_start = o; o += align_up((nkey + 1) * 4);
   L.inv_list = o; o += align_up((size_t)(G.n_vtiles > 0 ? G.n_vtiles : 1) *
                                 (G.n_cubes > 0 ? G.n_cubes : 1) * 4);
+  L.pieces = o; o += align_up(((size_t)4 * G.n_cubes + (G.n_tokens - G.n_vis + 63) / 64 + 1) * 16);
   L.total = o;
   return L;
 }
