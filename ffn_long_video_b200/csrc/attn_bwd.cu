@@ -121,15 +121,31 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
 }
 
 // ------------------------------------------------------------------ dQ kernel
-// Warps: 0 TMA producer (K and V blocks), 1 TMEM allocator + MMA issuer,
-// 2-5 one thread per row, 6 block-descriptor filler (as in the forward).
-// TMEM (512 columns): dQ 0-127, S buffers 128 + 64 b, dP buffers 256 + 64 b.
+// One CTA per 128-row tile (the forward's tiles, order and block walk). The
+// tile's 64-key blocks are taken two at a time (consecutive blocks of its own
+// walk, so no block is added): per pair S = Q [K_a; K_b]^T and dP = dO
+// [V_a; V_b]^T are N = 128 products into TMEM and dQ += dS [K_a; K_b] a K = 128
+// product with dS read from TMEM. Two passes over the walk: the first sums
+// D_r = sum_j P_rj dP_rj, the second forms dS and dQ.
+// Warps: 0 TMA producer, 1 TMEM allocator + MMA issuer, 2-9 row threads (two
+// warps per TMEM lane quadrant, one thread per (row, half of the pair's 128
+// keys)), 10 block-descriptor filler. TMEM (512 columns): dQ 0-127, S buffers
+// 128-255 and 384-511 (pair m in buffer m % 2, so the next pair's S runs
+// while the row threads work on this one), dP 256-383.
 namespace dq {
-constexpr int THREADS = 224;
-constexpr int KST = 3, VST = 2;
+constexpr int THREADS = 352;
+constexpr int ROW_THREADS = 256;
+constexpr int FILLER_WARP = 10;
+constexpr int KST = 2, VST = 1;           // stages of 128-key K and V pairs
+constexpr int KP_BYTES = 2 * 16384;       // 128 keys x 128 dims bf16
+constexpr uint32_t COL_DP = 256;
+__device__ __forceinline__ uint32_t col_s(int m) { return (m & 1) ? 384u : 128u; }
 constexpr size_t SMEM_BYTES =
-    1024 + 2 * Q_BYTES + (KST + VST) * KB_BYTES + RING * sizeof(Desc) + 2048;
+    1024 + 2 * Q_BYTES + (KST + VST) * KP_BYTES + RING * sizeof(Desc) + 2048;
 }  // namespace dq
+
+// Desc.pass bits: 0 = pass, 1 = pad (empty block that evens a pass), 2 = end.
+constexpr int kDescPad = 2, kDescEnd = 4;
 
 __global__ void __launch_bounds__(dq::THREADS, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap mapK,
@@ -140,23 +156,26 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sdO = sQ + Q_BYTES;
-  uint8_t* sK = sdO + Q_BYTES;              // [KST][KB_BYTES]
-  uint8_t* sV = sK + KST * KB_BYTES;        // [VST][KB_BYTES]
-  Desc* ring = reinterpret_cast<Desc*>(sV + VST * KB_BYTES);
+  uint8_t* sK = sdO + Q_BYTES;              // [KST][KP_BYTES]
+  uint8_t* sV = sK + KST * KP_BYTES;        // [VST][KP_BYTES]
+  Desc* ring = reinterpret_cast<Desc*>(sV + VST * KP_BYTES);
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + RING);
   uint64_t* k_full = bars;                  // [KST]
   uint64_t* k_empty = k_full + KST;
   uint64_t* v_full = k_empty + KST;         // [VST]
   uint64_t* v_empty = v_full + VST;
   uint64_t* s_full = v_empty + VST;         // [2]
-  uint64_t* p_full = s_full + 2;            // [2]
-  uint64_t* q_full = p_full + 2;
+  uint64_t* dp_full = s_full + 2;
+  uint64_t* ds_ready = dp_full + 1;         // row threads done with the pair
+  uint64_t* q_full = ds_ready + 1;
   uint64_t* drain = q_full + 1;
-  uint64_t* r_full = drain + 1;             // [RING]
+  uint64_t* xch = drain + 1;                // halves of D_r exchanged
+  uint64_t* r_full = xch + 1;               // [RING]
   uint64_t* r_empty = r_full + RING;        // [RING]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(r_empty + RING);
   __shared__ volatile int s_abort;
   __shared__ int s_own_hi, s_bad, s_dense;
+  __shared__ float s_dpart[2][128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const AttnGeom& G = a.G;
@@ -172,16 +191,17 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
-    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_ready, ROW_THREADS);
     for (int r = 0; r < RING; ++r) {
       mbar_init(&r_full[r], 1);
-      mbar_init(&r_empty[r], 128);
+      mbar_init(&r_empty[r], ROW_THREADS);
     }
-    mbar_init(q_full, 128);
+    mbar_init(q_full, ROW_THREADS);
     mbar_init(drain, 1);
+    mbar_init(xch, ROW_THREADS);
     fence_mbar_init();
     s_abort = 0;
     s_bad = status_bad(hdr) ? 1 : 0;
@@ -202,8 +222,10 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
   const uint32_t tmem_base = *tmem_holder;
   const bool bad = s_bad != 0;
 
-  if (warp == 6) {
+  if (warp == FILLER_WARP) {
     // ------------------------------------------------------------ descriptor filler
+    // Both passes over the tile's blocks; a pass with an odd number of blocks
+    // gets a pad block, so pairs never straddle passes; then an end marker.
     int n_entries = 0, n_chunks = 0;
     bool use_list = false;
     if (!bad) {
@@ -222,97 +244,113 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
     const uint4* tmask = reinterpret_cast<const uint4*>(a.tile_mask) + (size_t)T.bt * G.n_cubes;
     int base = 0;
     bool ok = true;
-    for (int pass = 0; pass < 2; ++pass)
-    for (int e0 = 0; e0 < n_total && ok; e0 += 32) {
-      const int e = e0 + lane;
-      int j = -1, ks = 0, ke = 0;
-      uint4 m = make_uint4(~0u, ~0u, ~0u, ~0u);
-      if (e < n_entries) {
-        j = use_list ? (int)list[e] : e;
-        ks = a.cube_offsets[j];
-        ke = a.cube_offsets[j + 1];
-        if (use_list) m = tmask[j];
-      } else if (e < n_total) {
-        ks = G.n_vis + (e - n_entries) * 64;
-        ke = min(ks + 64, T.t_hi + 1);
-      }
-      const int nb = (ke - ks + 63) / 64;
-      int incl = nb;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
-      int idx = base + incl - nb;
-      for (int b = 0; b < nb; ++b, ++idx) {
-        const int slot = idx % RING;
-        if (!mbar_wait(&r_empty[slot], ((idx / RING) & 1) ^ 1, &s_abort, hdr, 0xa200u)) {
-          ok = false;
-          break;
+    auto put = [&](int idx, int k0, int nk, int j, int flags, uint4 m) -> bool {
+      const int slot = idx % RING;
+      if (!mbar_wait(&r_empty[slot], ((idx / RING) & 1) ^ 1, &s_abort, hdr, 0xa200u))
+        return false;
+      Desc& d = ring[slot];
+      d.k0 = k0;
+      d.nk = nk;
+      d.j = j;
+      d.pass = flags;
+      d.mask[0] = m.x;
+      d.mask[1] = m.y;
+      d.mask[2] = m.z;
+      d.mask[3] = m.w;
+      mbar_arrive(&r_full[slot]);
+      return true;
+    };
+    for (int pass = 0; pass < 2 && ok; ++pass) {
+      const int pass_begin = base;
+      for (int e0 = 0; e0 < n_total && ok; e0 += 32) {
+        const int e = e0 + lane;
+        int j = -1, ks = 0, ke = 0;
+        uint4 m = make_uint4(~0u, ~0u, ~0u, ~0u);
+        if (e < n_entries) {
+          j = use_list ? (int)list[e] : e;
+          ks = a.cube_offsets[j];
+          ke = a.cube_offsets[j + 1];
+          if (use_list) m = tmask[j];
+        } else if (e < n_total) {
+          ks = G.n_vis + (e - n_entries) * 64;
+          ke = min(ks + 64, T.t_hi + 1);
         }
-        Desc& d = ring[slot];
-        d.k0 = ks + 64 * b;
-        d.nk = min(64, ke - d.k0);
-        d.j = j;
-        d.pass = pass;
-        d.mask[0] = m.x;
-        d.mask[1] = m.y;
-        d.mask[2] = m.z;
-        d.mask[3] = m.w;
-        mbar_arrive(&r_full[slot]);
+        const int nb = (ke - ks + 63) / 64;
+        int incl = nb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        int idx = base + incl - nb;
+        for (int b = 0; b < nb && ok; ++b, ++idx)
+          ok = put(idx, ks + 64 * b, min(64, ke - ks - 64 * b), j, pass, m);
+        ok = __all_sync(0xffffffffu, ok);
+        base += total;
       }
-      ok = __all_sync(0xffffffffu, ok);
-      base += total;
+      if (ok && ((base - pass_begin) & 1)) {  // even the pass
+        if (lane == 0) ok = put(base, 0, 0, -1, pass | kDescPad, make_uint4(0, 0, 0, 0));
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        ++base;
+      }
     }
-    if (ok && lane == 0) {  // terminal descriptor
-      const int slot = base % RING;
-      if (mbar_wait(&r_empty[slot], ((base / RING) & 1) ^ 1, &s_abort, hdr, 0xa300u)) {
-        ring[slot].nk = 0;
-        mbar_arrive(&r_full[slot]);
-      }
+    if (ok && lane == 0) {  // end marker (both slots of a pair)
+      put(base, 0, 0, -1, kDescEnd, make_uint4(0, 0, 0, 0));
+      put(base + 1, 0, 0, -1, kDescEnd, make_uint4(0, 0, 0, 0));
     }
   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Pair m = blocks 2m and 2m + 1: K into keys 0-63 / 64-127 of a K stage,
+    // V likewise. A pad block loads the first block again (K enters the dQ
+    // product as a reduction operand, so its rows must hold finite values).
     if (lane == 0) {
-      int i = 0;
+      int m = 0;
       bool ok = true;
       while (ok) {
-        const int slot = i % RING;
-        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0xa400u)) {
+        const int sa = (2 * m) % RING, sb2 = (2 * m + 1) % RING;
+        if (!mbar_wait(&r_full[sa], ((2 * m) / RING) & 1, &s_abort, hdr, 0xa400u) ||
+            !mbar_wait(&r_full[sb2], ((2 * m + 1) / RING) & 1, &s_abort, hdr, 0xa401u)) {
           ok = false;
           break;
         }
-        const int k0 = ring[slot].k0, nk = ring[slot].nk;
-        if (nk == 0) break;
-        const int ks = i % KST, vs = i % VST;
-        if (!mbar_wait(&k_empty[ks], ((i / KST) & 1) ^ 1, &s_abort, hdr, 0xa410u)) {
+        const Desc da = ring[sa], db = ring[sb2];
+        if (da.pass & kDescEnd) break;
+        const int k0a = da.k0, k0b = db.nk > 0 ? db.k0 : da.k0;
+        const int ks = m % KST, vs = m % VST;
+        if (!mbar_wait(&k_empty[ks], ((m / KST) & 1) ^ 1, &s_abort, hdr, 0xa410u)) {
           ok = false;
           break;
         }
-        mbar_expect_tx(&k_full[ks], KB_BYTES);
-        tma_load_3d(&mapK, &k_full[ks], sK + ks * KB_BYTES, 0, T.kv, k0);
-        tma_load_3d(&mapK, &k_full[ks], sK + ks * KB_BYTES + 8192, 64, T.kv, k0);
-        if (!mbar_wait(&v_empty[vs], ((i / VST) & 1) ^ 1, &s_abort, hdr, 0xa420u)) {
+        uint8_t* kd = sK + ks * KP_BYTES;
+        mbar_expect_tx(&k_full[ks], KP_BYTES);
+        tma_load_3d(&mapK, &k_full[ks], kd, 0, T.kv, k0a);
+        tma_load_3d(&mapK, &k_full[ks], kd + 16384, 64, T.kv, k0a);
+        tma_load_3d(&mapK, &k_full[ks], kd + 8192, 0, T.kv, k0b);
+        tma_load_3d(&mapK, &k_full[ks], kd + 16384 + 8192, 64, T.kv, k0b);
+        if (!mbar_wait(&v_empty[vs], ((m / VST) & 1) ^ 1, &s_abort, hdr, 0xa420u)) {
           ok = false;
-          ++i;  // K of block i is in flight
+          ++m;  // K of pair m is in flight
           break;
         }
-        mbar_expect_tx(&v_full[vs], KB_BYTES);
-        tma_load_3d(&mapV, &v_full[vs], sV + vs * KB_BYTES, 0, T.kv, k0);
-        tma_load_3d(&mapV, &v_full[vs], sV + vs * KB_BYTES + 8192, 64, T.kv, k0);
-        ++i;
+        uint8_t* vd = sV + vs * KP_BYTES;
+        mbar_expect_tx(&v_full[vs], KP_BYTES);
+        tma_load_3d(&mapV, &v_full[vs], vd, 0, T.kv, k0a);
+        tma_load_3d(&mapV, &v_full[vs], vd + 16384, 64, T.kv, k0a);
+        tma_load_3d(&mapV, &v_full[vs], vd + 8192, 0, T.kv, k0b);
+        tma_load_3d(&mapV, &v_full[vs], vd + 16384 + 8192, 64, T.kv, k0b);
+        ++m;
       }
       if (!ok) {  // let copies already issued land before the CTA exits
         long long t0 = clock64();
         for (int k = 0; k < KST; ++k) {
-          const int jk = i - 1 - k;
+          const int jk = m - 1 - k;
           while (jk >= 0 && !mbar_try_wait(&k_full[jk % KST], (jk / KST) & 1) &&
                  clock64() - t0 < kWaitCycles) {
           }
         }
         for (int k = 0; k < VST; ++k) {
-          const int jv = i - 1 - k;
+          const int jv = m - 1 - k;
           while (jv >= 0 && !mbar_try_wait(&v_full[jv % VST], (jv / VST) & 1) &&
                  clock64() - t0 < kWaitCycles) {
           }
@@ -322,73 +360,79 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64);
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 128);
       constexpr uint32_t idesc_q = make_idesc_bf16(128, 128, true);
       const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sdO);
       bool ok = mbar_wait(q_full, 0, &s_abort, hdr, 0xa500u);
       tc_fence_after();
-      int i = 0, prev_pass = 0;
       bool dq_started = false;
-      // block blk: once its rows are done with S / dP, run dQ += dS K (second
-      // pass only) and free its K stage
-      auto finish = [&](int blk, int pass) -> bool {
-        const int pb = blk & 1;
-        if (!mbar_wait(&p_full[pb], (blk >> 1) & 1, &s_abort, hdr, 0xa510u)) return false;
+      int prev_flags = 0;
+      // pair m - 1's rows are done: its dQ product (second pass), then its K
+      // stage is free
+      auto finish = [&](int pm, int flags) -> bool {
+        if (!mbar_wait(ds_ready, pm & 1, &s_abort, hdr, 0xa510u)) return false;
         tc_fence_after();
-        const int ks = blk % KST;
-        if (pass == 1) {
-          const uint32_t k_addr = smem_u32(sK + ks * KB_BYTES);
-          const uint32_t ds_tmem = tmem_base + 128 + pb * 64;
+        const int ks = pm % KST;
+        if (flags & 1) {
+          const uint32_t k_addr = smem_u32(sK + ks * KP_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = make_sdesc_sw128(k_addr + kk * 2048, 8192, 1024);
-            umma_bf16_ts(tmem_base, ds_tmem + kk * 8, bd, idesc_q,
-                         (dq_started || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t bd = make_sdesc_sw128(k_addr + kk * 2048, 16384, 1024);
+            umma_bf16_ts(tmem_base, tmem_base + col_s(pm) + (kk >> 2) * 64 + (kk & 3) * 8, bd,
+                         idesc_q, (dq_started || kk > 0) ? 1u : 0u);
           }
           dq_started = true;
         }
         umma_commit(&k_empty[ks]);
         return true;
       };
-      while (ok) {
-        const int slot = i % RING;
-        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0xa520u)) {
+      int m = 0;
+      for (; ok; ++m) {
+        const int sa = (2 * m) % RING;
+        if (!mbar_wait(&r_full[sa], ((2 * m) / RING) & 1, &s_abort, hdr, 0xa520u)) {
           ok = false;
           break;
         }
-        if (ring[slot].nk == 0) break;
-        const int pass = ring[slot].pass;
-        const int ks = i % KST, vs = i % VST, sb = i & 1;
-        if (!mbar_wait(&k_full[ks], (i / KST) & 1, &s_abort, hdr, 0xa530u) ||
-            !mbar_wait(&v_full[vs], (i / VST) & 1, &s_abort, hdr, 0xa540u)) {
+        const int flags = ring[sa].pass;
+        if (flags & kDescEnd) break;
+        const int ks = m % KST, vs = m % VST;
+        if (!mbar_wait(&k_full[ks], (m / KST) & 1, &s_abort, hdr, 0xa530u) ||
+            !mbar_wait(&v_full[vs], (m / VST) & 1, &s_abort, hdr, 0xa540u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + ks * KB_BYTES);
-        const uint32_t v_addr = smem_u32(sV + vs * KB_BYTES);
+        const uint32_t k_addr = smem_u32(sK + ks * KP_BYTES);
+        const uint32_t v_addr = smem_u32(sV + vs * KP_BYTES);
+        // S of pair m into its buffer (the buffer's last reader, pair m - 2's
+        // dQ product, was issued before)
 #pragma unroll
         for (int dc = 0; dc < 2; ++dc)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t acc = (dc | kk) != 0 ? 1u : 0u;
-            umma_bf16(tmem_base + 128 + sb * 64,
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem_base + col_s(m),
                       make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024),
-                      make_sdesc_sw128(k_addr + dc * 8192 + kk * 32, 16, 1024), idesc_s, acc);
-            umma_bf16(tmem_base + 256 + sb * 64,
-                      make_sdesc_sw128(do_addr + dc * 16384 + kk * 32, 16, 1024),
-                      make_sdesc_sw128(v_addr + dc * 8192 + kk * 32, 16, 1024), idesc_s, acc);
-          }
-        umma_commit(&s_full[sb]);
-        umma_commit(&v_empty[vs]);
-        if (i > 0 && !finish(i - 1, prev_pass)) {
+                      make_sdesc_sw128(k_addr + dc * 16384 + kk * 32, 16, 1024), idesc_s,
+                      (dc | kk) != 0 ? 1u : 0u);
+        umma_commit(&s_full[m & 1]);
+        // dP has one buffer: pair m - 1's rows must be done with it first
+        if (m > 0 && !finish(m - 1, prev_flags)) {
           ok = false;
           break;
         }
-        prev_pass = pass;
-        ++i;
+#pragma unroll
+        for (int dc = 0; dc < 2; ++dc)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem_base + COL_DP,
+                      make_sdesc_sw128(do_addr + dc * 16384 + kk * 32, 16, 1024),
+                      make_sdesc_sw128(v_addr + dc * 16384 + kk * 32, 16, 1024), idesc_s,
+                      (dc | kk) != 0 ? 1u : 0u);
+        umma_commit(dp_full);
+        umma_commit(&v_empty[vs]);
+        prev_flags = flags;
       }
-      if (ok && i > 0) finish(i - 1, prev_pass);
+      if (ok && m > 0) finish(m - 1, prev_flags);
       umma_commit(drain);
       long long t0 = clock64();
       while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitCycles) {
@@ -398,6 +442,7 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
     // ------------------------------------------------------------ row threads
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
+    const int half = (warp - 2) >> 2;         // the pair's block: keys [64 half, +64)
     const TileRow R = tile_row(G, T.text, T.bt, row);
     const bool valid = R.valid;
     const int t = R.t, h = R.h;
@@ -408,7 +453,7 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
       const uint4* q4 = reinterpret_cast<const uint4*>(a.Q + rix * 128);
       const uint4* d4 = reinterpret_cast<const uint4*>(a.dO + rix * 128);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = half * 8; c < half * 8 + 8; ++c) {
         const uint32_t off = (c >> 3) * 16384 + sw128_offset(row, c & 7);
         *reinterpret_cast<uint4*>(sQ + off) = valid ? q4[c] : make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(sdO + off) = valid ? d4[c] : make_uint4(0, 0, 0, 0);
@@ -417,81 +462,111 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
       mbar_arrive(q_full);
     }
     const float lse2 = valid ? a.lse[rix] : 0.f;
-    float dot = 0.f;          // D_r, summed over the first pass
-    bool dot_stored = false;
+    float dot = 0.f;          // this half's part of D_r over the first pass
+    bool dot_done = false;
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
-    int i = 0;
+    int m = 0;
     bool ok = true;
     while (true) {
-      const int slot = i % RING;
-      if (!mbar_wait_warp(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0xa600u)) {
+      const int sa = (2 * m) % RING;
+      const int sme = (2 * m + half) % RING;  // this half's block
+      if (!mbar_wait_warp(&r_full[sa], ((2 * m) / RING) & 1, &s_abort, hdr, 0xa600u) ||
+          !mbar_wait_warp(&r_full[(2 * m + 1) % RING], ((2 * m + 1) / RING) & 1, &s_abort, hdr,
+                          0xa601u)) {
         ok = false;
         break;
       }
-      const Desc dsc = ring[slot];
-      if (dsc.nk == 0) break;
-      const int sb = i & 1;
-      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0xa610u)) {
+      const int flags = ring[sa].pass;
+      if (flags & kDescEnd) break;
+      const Desc dsc = ring[sme];
+      if (!mbar_wait_warp(&s_full[m & 1], (m >> 1) & 1, &s_abort, hdr, 0xa610u)) {
         ok = false;
         break;
       }
-      mbar_arrive(&r_empty[slot]);
+      // S of the pair landed: the producer and the MMA issuer are done with
+      // both descriptors
+      mbar_arrive(&r_empty[sa]);
+      mbar_arrive(&r_empty[(2 * m + 1) % RING]);
       tc_fence_after();
-      uint32_t sr[64], dp[64];
-      {
-        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        uint32_t(&p0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[0]);
-        uint32_t(&p1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&dp[32]);
-        tmem_ld32(tmem_base + lane_base + 128 + sb * 64, s0);
-        tmem_ld32(tmem_base + lane_base + 128 + sb * 64 + 32, s1);
-        tmem_ld32(tmem_base + lane_base + 256 + sb * 64, p0);
-        tmem_ld32(tmem_base + lane_base + 256 + sb * 64 + 32, p1);
-      }
-      tmem_ld_wait();
       bool row_on;
-      if (!valid) row_on = false;
+      if (!valid || dsc.nk <= 0) row_on = false;
       else if (T.text) row_on = true;
       else if (s_dense) row_on = dsc.j <= own;
       else row_on = ((dsc.mask[wq] >> lane) & 1u) != 0u;
       int lim = row_on ? dsc.nk : 0;
       if (row_on && (T.text || dsc.j == own)) lim = min(lim, t - dsc.k0 + 1);
-      if (dsc.pass == 0) {
+      if (lim < 0) lim = 0;
+      const bool pass1 = (flags & 1) != 0;
+      if (pass1 && !dot_done) {
+        // D_r = the two halves' sums, exchanged once through shared memory
+        s_dpart[half][row] = dot;
+        mbar_arrive(xch);
+        if (!mbar_wait_warp(xch, 0, &s_abort, hdr, 0xa630u)) {
+          ok = false;
+          break;
+        }
+        dot = s_dpart[0][row] + s_dpart[1][row];
+        if (valid && half == 0) a.dot[rix] = dot;
+        dot_done = true;
+      }
+      // P over this half's 64 keys, 32 at a time
+      float pv[64];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sr[32];
+        tmem_ld32(tmem_base + lane_base + col_s(m) + half * 64 + c * 32, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+          pv[c * 32 + u] =
+              c * 32 + u < lim ? ex2(fmaf(__uint_as_float(sr[u]), scale, -lse2)) : 0.f;
+      }
+      if (!mbar_wait_warp(dp_full, m & 1, &s_abort, hdr, 0xa615u)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (!pass1) {
         float ds[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) ds[k] = 0.f;
 #pragma unroll
-        for (int u = 0; u < 64; ++u) {
-          const float pu = u < lim ? ex2(fmaf(__uint_as_float(sr[u]), scale, -lse2)) : 0.f;
-          ds[u & 7] = fmaf(pu, __uint_as_float(dp[u]), ds[u & 7]);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(tmem_base + lane_base + COL_DP + half * 64 + c * 32, dp);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u)
+            ds[u & 7] = fmaf(pv[c * 32 + u], __uint_as_float(dp[u]), ds[u & 7]);
         }
         dot += ((ds[0] + ds[1]) + (ds[2] + ds[3])) + ((ds[4] + ds[5]) + (ds[6] + ds[7]));
       } else {
-        if (!dot_stored) {
-          if (valid) a.dot[rix] = dot;
-          dot_stored = true;
-        }
-        uint32_t pk[32];
+        // dS over keys 32c..32c+31 of this half goes to columns 16c..16c+15 of
+        // the half's S region, whose scores were read above
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const int u = 2 * q;
-          const float p0 = u < lim ? ex2(fmaf(__uint_as_float(sr[u]), scale, -lse2)) : 0.f;
-          const float p1 =
-              u + 1 < lim ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, -lse2)) : 0.f;
-          pk[q] = pack_bf16x2(p0 * (__uint_as_float(dp[u]) - dot),
-                              p1 * (__uint_as_float(dp[u + 1]) - dot));
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(tmem_base + lane_base + COL_DP + half * 64 + c * 32, dp);
+          tmem_ld_wait();
+          uint32_t pk[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int u = 2 * q;
+            pk[q] = pack_bf16x2(pv[c * 32 + u] * (__uint_as_float(dp[u]) - dot),
+                                pv[c * 32 + u + 1] * (__uint_as_float(dp[u + 1]) - dot));
+          }
+          tmem_st16(tmem_base + lane_base + col_s(m) + half * 64 + c * 16, pk);
         }
-        tmem_st32(tmem_base + lane_base + 128 + sb * 64, pk);
         tmem_st_wait();
       }
       tc_fence_before();
-      mbar_arrive(&p_full[sb]);
-      ++i;
+      mbar_arrive(ds_ready);
+      ++m;
     }
-    if (ok && !dot_stored && valid) a.dot[rix] = dot;
+    if (ok && !dot_done && valid && half == 0) a.dot[rix] = 0.f;  // no blocks at all
     long long t0 = clock64();
     bool done = ok;
-    if (ok && i > 0) {
+    if (ok && m > 0) {
       done = false;
       while (!(done = mbar_try_wait(drain, 0)) && clock64() - t0 < kWaitCycles) {
       }
@@ -502,19 +577,19 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
       tc_fence_after();
       float* dst = a.dQ + rix * 128;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = half * 64; c < half * 64 + 64; c += 32) {
         uint32_t o[32];
         tmem_ld32(tmem_base + lane_base + c, o);
         tmem_ld_wait();
         if (valid) {
           float4* d4 = reinterpret_cast<float4*>(dst + c);
-          const float s = a.inv_sqrt_d;
+          const float sc = a.inv_sqrt_d;
 #pragma unroll
           for (int x = 0; x < 8; ++x)
-            d4[x] = i > 0 ? make_float4(__uint_as_float(o[4 * x]) * s,
-                                        __uint_as_float(o[4 * x + 1]) * s,
-                                        __uint_as_float(o[4 * x + 2]) * s,
-                                        __uint_as_float(o[4 * x + 3]) * s)
+            d4[x] = m > 0 ? make_float4(__uint_as_float(o[4 * x]) * sc,
+                                        __uint_as_float(o[4 * x + 1]) * sc,
+                                        __uint_as_float(o[4 * x + 2]) * sc,
+                                        __uint_as_float(o[4 * x + 3]) * sc)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
