@@ -524,12 +524,17 @@ def attention_backward_given_sets(Q, K, V, dO, cube_offsets, n_vis, sel, with_ma
     return dQ, dK, dV
 
 
-def swiglu_ffn_backward(x, W_gate, W_up, W_down, df):
+def swiglu_ffn_backward(x, W_gate, W_up, W_down, df, with_magnitudes=False):
     """Gradients of f = swiglu_ffn(x) for the upstream gradient df [n, D]:
     with g = x W_gate^T, u = x W_up^T, silu(g) = g sigma(g), h = silu(g) u,
     dh = df W_down; du = dh silu(g); dg = dh u sigma(g) (1 + g (1 - sigma(g)));
     dx = dg W_gate + du W_up; dW_gate = dg^T x; dW_up = du^T x; dW_down = df^T h.
-    Returns float64 (dx, dW_gate, dW_up, dW_down)."""
+    Returns float64 (dx, dW_gate, dW_up, dW_down).  With ``with_magnitudes``
+    also, per gradient, the scale in which one relative rounding of the
+    intermediates df, dg, du and h (each rounded once, the error in df carried
+    through dh into dg and du) enters each element: a comparison that rounds
+    those intermediates to a format with unit roundoff r stays within about
+    r times this scale."""
     X, Wg, Wu, Wd, dF = _f64(x), _f64(W_gate), _f64(W_up), _f64(W_down), _f64(df)
     gate = X @ Wg.T
     up = X @ Wu.T
@@ -538,13 +543,23 @@ def swiglu_ffn_backward(x, W_gate, W_up, W_down, df):
     h = silu * up
     dh = dF @ Wd
     du = dh * silu
-    dg = dh * up * sig * (1.0 + gate * (1.0 - sig))
+    dsilu_u = up * sig * (1.0 + gate * (1.0 - sig))
+    dg = dh * dsilu_u
     dx = dg @ Wg + du @ Wu
-    return dx, dg.T @ X, du.T @ X, dF.T @ h
+    grads = (dx, dg.T @ X, du.T @ X, dF.T @ h)
+    if not with_magnitudes:
+        return grads
+    m_dh = np.abs(dF) @ np.abs(Wd)                  # df's rounding inside dh
+    m_dg = np.abs(dsilu_u) * m_dh + np.abs(dg)      # ... carried into dg, plus dg's own
+    m_du = np.abs(silu) * m_dh + np.abs(du)
+    aX = np.abs(X)
+    mags = (m_dg @ np.abs(Wg) + m_du @ np.abs(Wu), m_dg.T @ aX, m_du.T @ aX,
+            2.0 * (np.abs(dF).T @ np.abs(h)))         # df and h both rounded
+    return grads, mags
 
 
 def ffn_backward_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active, dy,
-                            cubes=None, text=True):
+                            cubes=None, text=True, with_magnitudes=False):
     """Gradients of ``ffn_given_sets`` (all cubes and the text rows) for the
     upstream gradient dy [N, D], the active set held fixed.
 
@@ -557,7 +572,9 @@ def ffn_backward_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active
     (dx [N, D], dW_gate [F, D], dW_up [F, D], dW_down [D, F]).  ``cubes`` /
     ``text`` restrict the rows to those cubes and (or not) the text tokens: dx
     is exact on them (NaN elsewhere) and the weight gradients hold only their
-    rows' contributions."""
+    rows' contributions.  ``with_magnitudes`` adds the rounding scales of
+    ``swiglu_ffn_backward`` (zero on the skipped rows' dx, whose gradient is
+    dy itself)."""
     N, D = x.shape
     off = np.asarray(cube_offsets)
     C = len(off) - 1
@@ -579,7 +596,13 @@ def ffn_backward_given_sets(x, W_gate, W_up, W_down, cube_offsets, n_vis, active
             df[a:b][act] += dY[a:b][~act].sum(axis=0) / int(act.sum())
     df[n_vis:] = dY[n_vis:]
     rows = np.nonzero(active & keep)[0]
-    dxr, dWg, dWu, dWd = swiglu_ffn_backward(X[rows], W_gate, W_up, W_down, df[rows])
+    res = swiglu_ffn_backward(X[rows], W_gate, W_up, W_down, df[rows],
+                              with_magnitudes=with_magnitudes)
+    dxr, dWg, dWu, dWd = res[0] if with_magnitudes else res
     dx = np.where(keep[:, None], dY, np.nan)
     dx[rows] += dxr
-    return dx, dWg, dWu, dWd
+    if not with_magnitudes:
+        return dx, dWg, dWu, dWd
+    mdx = np.zeros_like(dY)
+    mdx[rows] = res[1][0]
+    return (dx, dWg, dWu, dWd), (mdx, res[1][1], res[1][2], res[1][3])

@@ -186,12 +186,14 @@ def check_ffn(case, p=None, cubes=None, text=True, report=None, importance="l2")
 GRAD_TOL = (2e-2, 5e-3)
 
 
-# For sums that round one operand to bf16 (dS or P in the attention gradients)
-# a rigorous per-element bound also holds: RNE to 8 significant bits moves a
-# value by at most 2^-9 of itself, so |err| <= 2^-9 * sum |a| |b| over the
-# element's terms; 2^-8 leaves room for the fp32 accumulation and the ex2
-# approximation. It matters where the terms nearly cancel (each row's dS sums
-# to zero), which makes the gradient small next to its terms.
+# For sums that round an operand to bf16 (dS or P in the attention gradients;
+# df, dg, du, h in the FFN ones) a rigorous per-element bound also holds: RNE
+# to 8 significant bits moves a value by at most 2^-9 of itself, so |err| <=
+# 2^-9 times the oracle's rounding scale (sum |a| |b| over the element's terms,
+# with an upstream rounding carried through, e.g. df's into dg); 2^-8 leaves
+# room for the fp32 accumulation and the ex2 approximation. It matters where
+# the terms nearly cancel (each row's dS sums to zero; the rows of one cube are
+# near-duplicates), which makes the gradient small next to its terms.
 ROUND_BOUND = 2.0 ** -8
 
 
@@ -228,11 +230,12 @@ def run_ffn_backward(case, p=None):
 def check_ffn_backward(case, p=None, report=None):
     cfg, t = case["cfg"], case["t"]
     grads, act, dy = run_ffn_backward(case, p)
-    want = oracle.ffn_backward_given_sets(t["x"].cpu(), t["W_gate"].cpu(), t["W_up"].cpu(),
-                                          t["W_down"].cpu(), case["off_np"], cfg.n_vis, act,
-                                          dy.cpu())
-    for g, w, nm in zip(grads, want, ("dx", "dW_gate", "dW_up", "dW_down")):
-        check_grad(g.cpu().numpy(), w, nm, report)
+    want, mags = oracle.ffn_backward_given_sets(t["x"].cpu(), t["W_gate"].cpu(),
+                                                t["W_up"].cpu(), t["W_down"].cpu(),
+                                                case["off_np"], cfg.n_vis, act, dy.cpu(),
+                                                with_magnitudes=True)
+    for g, w, m, nm in zip(grads, want, mags, ("dx", "dW_gate", "dW_up", "dW_down")):
+        check_grad(g.cpu().numpy(), w, nm, report, magnitude=m)
     # a skipped token's gradient is its upstream gradient, bit for bit
     skipped = ~act
     skipped[cfg.n_vis:] = False

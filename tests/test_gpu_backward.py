@@ -97,3 +97,26 @@ def test_backward_full_size_3b_18k(case_18k):
     parity.check_grad(dx.cpu().numpy()[rows], want[rows], "dx", rep)
     assert all(torch.isfinite(x).all() for x in (dx, dWg, dWu, dWd))
     print(cfg.name, rep)
+
+
+EDGE = {
+    # no text tokens at all
+    "no-text": workloads.small_config(name="notext", grid=(4, 8, 8), cube=(4, 4, 2), n_text=0,
+                                      D=256, hq=4, hkv=2, F=256, seed=61),
+    # one query head per KV head (g = 1), odd number of 64-key pieces
+    "g1-odd": workloads.small_config(name="g1", grid=(4, 8, 8), cube=(4, 4, 4), n_text=9,
+                                     D=256, hq=2, hkv=2, F=256, seed=62,
+                                     cube_sizes=(64, 64, 64, 63, 1)),
+    # a single cube plus a short text tail
+    "one-cube": workloads.small_config(name="onecube", grid=(4, 4, 4), cube=(4, 4, 4),
+                                       n_text=5, D=256, hq=4, hkv=1, F=256, seed=63),
+}
+
+
+@pytest.mark.parametrize("name", list(EDGE))
+def test_backward_edge_layouts(name):
+    case = parity.make_case(EDGE[name])
+    rep = {}
+    parity.check_attn_backward(case, p=0.6, report=rep)
+    parity.check_ffn_backward(case, p=0.6, report=rep)
+    print(name, rep)

@@ -580,6 +580,23 @@ def test_backward_row_restrictions_agree_with_full():
     assert np.isnan(pdx[np.r_[0:4, 8:12, 16:N]]).all()
 
 
+def test_ffn_backward_magnitudes_bound_the_gradients():
+    """The rounding scales dominate the gradients they belong to (each is a sum
+    of absolute values over the same terms, plus non-negative extras), and the
+    dW_down scale is exactly twice |df|^T |h|."""
+    off, n_vis, x, Wg, Wu, Wd, active, dy = _tiny_ffn_case(29)
+    grads, mags = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd, off, n_vis, active, dy,
+                                                 with_magnitudes=True)
+    plain = oracle.ffn_backward_given_sets(x, Wg, Wu, Wd, off, n_vis, active, dy)
+    for g, p_, m in zip(grads, plain, mags):
+        assert np.array_equal(g, p_)
+    rows = active.copy()
+    rows[n_vis:] = True
+    assert (np.abs(grads[0] - dy)[rows] <= mags[0][rows] + 1e-12).all()
+    for g, m in zip(grads[1:], mags[1:]):
+        assert (np.abs(g) <= m + 1e-12).all()
+
+
 def _tiny_ffn_case(seed):
     rng = np.random.default_rng(seed)
     D, F = 3, 4
