@@ -20,12 +20,13 @@
 //   ffn_bwd_skip      per cube: G_c and dx of the skipped rows (HBM)
 //   ffn_bwd_df        df in compacted row order, bf16, plus its transpose (HBM)
 //   bwd_transpose     x_a^T, W_down^T, [W_gate^T | W_up^T] in bf16 (HBM)
-//   ffn_bwd_gemm<0>   per 128 x 128 tile of (rows, F): gate|up = x_a [W_gate;
+//   ffn_bwd_gemm<0>   per 128 x 64 tile of (rows, F): gate|up = x_a [W_gate;
 //                     W_up]^T and dh = df (W_down^T)^T share K = D, so one
-//                     k-loop feeds two MMAs (N = 256 and N = 128) into 384 TMEM
-//                     columns; the epilogue forms dg, du, h and stores [dg du]
-//                     row-major plus [dg du]^T and h^T (the K-major operands of
-//                     the weight-gradient GEMMs)
+//                     k-loop feeds two MMAs (N = 128 and N = 64) into 192 TMEM
+//                     columns, two such sets so the epilogue of one tile
+//                     overlaps the products of the next; the epilogue forms
+//                     dg, du, h and stores [dg du] row-major plus [dg du]^T and
+//                     h^T (the K-major operands of the weight-gradient GEMMs)
 //   ffn_bwd_gemm<1>   dx[idx] = dy[idx] + [dg du] [W_gate^T | W_up^T]^T (K = 2F)
 //   ffn_bwd_gemm<2>   weight gradients, K = active rows (a device count):
 //                     [dW_gate; dW_up] = [dg du]^T (x_a^T)^T, dW_down = df^T (h^T)^T
@@ -195,13 +196,13 @@ constexpr int TILE16K = BM * BK * 2;  // one 128-row x 64-column bf16 tile
 
 template <int MODE>
 struct Cfg {
-  // mode 0: A = x_a and df tiles; B = 128 W_gate + 128 W_up + 128 W_down^T rows
-  static constexpr int STAGES = MODE == 0 ? 2 : 4;
+  // mode 0: A = x_a and df tiles; B = 64 W_gate + 64 W_up + 64 W_down^T rows
+  static constexpr int STAGES = MODE == 0 ? 3 : 4;
   static constexpr int A_BYTES = MODE == 0 ? 2 * TILE16K : TILE16K;
-  static constexpr int B_BYTES = MODE == 0 ? 3 * TILE16K : 2 * TILE16K;
+  static constexpr int B_BYTES = MODE == 0 ? 3 * (TILE16K / 2) : 2 * TILE16K;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int BN = MODE == 0 ? 128 : 256;  // output columns per tile
-  static constexpr int NACC = MODE == 0 ? 1 : 2;    // accumulator sets in TMEM
+  static constexpr int BN = MODE == 0 ? 64 : 256;   // output columns per tile
+  static constexpr int NACC = 2;                    // accumulator sets in TMEM
   static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
 };
 
@@ -318,9 +319,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           tma_load_2d(&mA0, &full[s], sa, kb * BK, mt * BM);
           if (MODE == 0) {
             tma_load_2d(&mA1, &full[s], sa + TILE16K, kb * BK, mt * BM);
-            tma_load_2d(&mB0, &full[s], sb, kb * BK, nt * 128);
-            tma_load_2d(&mB1, &full[s], sb + TILE16K, kb * BK, nt * 128);
-            tma_load_2d(&mB2, &full[s], sb + 2 * TILE16K, kb * BK, nt * 128);
+            tma_load_2d(&mB0, &full[s], sb, kb * BK, nt * 64);
+            tma_load_2d(&mB1, &full[s], sb + TILE16K / 2, kb * BK, nt * 64);
+            tma_load_2d(&mB2, &full[s], sb + TILE16K, kb * BK, nt * 64);
           } else {
             tma_load_2d(&mB0, &full[s], sb, kb * BK, nt * 256);
           }
@@ -342,6 +343,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc256 = make_idesc_bf16(BM, 256);
       constexpr uint32_t idesc128 = make_idesc_bf16(BM, 128);
+      constexpr uint32_t idesc64 = make_idesc_bf16(BM, 64);
       int it = 0, tc = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tc) {
@@ -364,11 +366,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t acc = (kb | k) != 0 ? 1u : 0u;
             const uint64_t ad = make_sdesc_sw128(a_addr + k * 32, 16, 1024);
             const uint64_t bd = make_sdesc_sw128(b_addr + k * 32, 16, 1024);
-            umma_bf16(d0, ad, bd, idesc256, acc);
             if (MODE == 0) {
+              // gate|up (64 + 64 B rows) into columns 0-127 of the set, dh
+              // (64 W_down^T rows) into 128-191
+              umma_bf16(d0, ad, bd, idesc128, acc);
               const uint64_t ad1 = make_sdesc_sw128(a_addr + TILE16K + k * 32, 16, 1024);
-              const uint64_t bd2 = make_sdesc_sw128(b_addr + 2 * TILE16K + k * 32, 16, 1024);
-              umma_bf16(tmem_base + 256, ad1, bd2, idesc128, acc);
+              const uint64_t bd2 = make_sdesc_sw128(b_addr + TILE16K + k * 32, 16, 1024);
+              umma_bf16(d0 + 128, ad1, bd2, idesc64, acc);
+            } else {
+              umma_bf16(d0, ad, bd, idesc256, acc);
             }
           }
           umma_commit(&empty[s]);
@@ -400,13 +406,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (MODE == 0) {
         const bool padrow = i < m_pad;
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
+        for (int c = 0; c < 64; c += 32) {
           uint32_t g[32], u[32], dh[32];
           tmem_ld32(tb + c, g);
-          tmem_ld32(tb + 128 + c, u);
-          tmem_ld32(tb + 256 + c, dh);
+          tmem_ld32(tb + 64 + c, u);
+          tmem_ld32(tb + 128 + c, dh);
           tmem_ld_wait();
-          const int n0 = nt * 128 + c;
+          const int n0 = nt * 64 + c;
           float dg[32], du[32], hh[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -563,8 +569,8 @@ cudaError_t launch_ffn_backward_tc(const FfnBwdArgs& a, cudaStream_t s) {
   CUtensorMap mXa, mDf, mWg, mWu, mWdT, mDgu, mWguT, mDguT, mXaT, mDfT, mHT;
   const uint64_t mp = a.mp;
   if (!map2d(&mXa, a.xa, D, N, D, 128) || !map2d(&mDf, a.df, D, N, D, 128) ||
-      !map2d(&mWg, a.W_gate, D, F, D, 128) || !map2d(&mWu, a.W_up, D, F, D, 128) ||
-      !map2d(&mWdT, a.wdT, D, F, D, 128) || !map2d(&mDgu, a.dgu, 2 * F, N, 2 * F, 128) ||
+      !map2d(&mWg, a.W_gate, D, F, D, 64) || !map2d(&mWu, a.W_up, D, F, D, 64) ||
+      !map2d(&mWdT, a.wdT, D, F, D, 64) || !map2d(&mDgu, a.dgu, 2 * F, N, 2 * F, 128) ||
       !map2d(&mWguT, a.wguT, 2 * F, D, 2 * F, 256) ||
       !map2d(&mDguT, a.dguT, mp, 2 * F, mp, 128) || !map2d(&mXaT, a.xaT, mp, D, mp, 256) ||
       !map2d(&mDfT, a.dfT, mp, D, mp, 128) || !map2d(&mHT, a.hT, mp, F, mp, 256))
@@ -577,7 +583,7 @@ cudaError_t launch_ffn_backward_tc(const FfnBwdArgs& a, cudaStream_t s) {
   P.hdr = a.hdr;
   // dg, du, h
   P.k_blocks = D / 64;
-  P.n_tiles = F / 128;
+  P.n_tiles = F / 64;
   P.n_cols = F;
   P.dgu = a.dgu;
   P.dguT = a.dguT;
