@@ -40,7 +40,6 @@ namespace abwd {
 
 constexpr int RING = 64;
 constexpr int Q_BYTES = 128 * 256;   // 128 rows x 128 dims bf16 (two 64-dim halves)
-constexpr int KB_BYTES = 2 * 8192;   // one 64-key block of K or V (two 64-dim halves)
 
 struct Desc {
   int k0, nk, j, pass;  // pass: 0 sums D_r, 1 forms dS and dQ

@@ -56,7 +56,7 @@ bool layer_sizes_ok(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d
   if (d != 128 || hq < 1 || hkv < 1) return false;
   // GEMM shapes: K multiple of 64, output columns multiple of 32
   if (D % 64 != 0 || (hq * d) % 64 != 0) return false;
-  LayerLayout L;
+  LayerLayout L{};
   return layer_layout(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, &L);
 }
 
@@ -106,9 +106,8 @@ size_t adaspark_layer_workspace(int n_tokens, int n_vis, int n_cubes, int hq, in
                                 int D, int F, int dtype) {
   if (dtype != ADASPARK_BF16 || !layer_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F))
     return 0;
-  LayerLayout L;
-  layer_layout(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, &L);
-  return L.total;
+  LayerLayout L{};
+  return layer_layout(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, &L) ? L.total : 0;
 }
 
 int adaspark_layer_buffers(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d, int D,
@@ -116,8 +115,8 @@ int adaspark_layer_buffers(int n_tokens, int n_vis, int n_cubes, int hq, int hkv
   if (!offsets || dtype != ADASPARK_BF16 ||
       !layer_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F))
     return ADASPARK_EINVAL;
-  LayerLayout L;
-  layer_layout(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, &L);
+  LayerLayout L{};
+  if (!layer_layout(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, &L)) return ADASPARK_EINVAL;
   offsets[0] = L.q;
   offsets[1] = L.k;
   offsets[2] = L.v;
@@ -141,8 +140,8 @@ int adaspark_layer(const void* x, const void* W_q, const void* W_k, const void* 
   if (dtype != ADASPARK_BF16 || !layer_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F))
     return ADASPARK_EINVAL;
   if (!(p_attn > 0.f && p_attn <= 1.f) || !(p_ffn > 0.f && p_ffn <= 1.f)) return ADASPARK_EINVAL;
-  LayerLayout L;
-  layer_layout(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, &L);
+  LayerLayout L{};
+  if (!layer_layout(n_tokens, n_vis, n_cubes, hq, hkv, d, D, F, &L)) return ADASPARK_EINVAL;
   if (workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & (kLayerAlign - 1)))
     return ADASPARK_EINVAL;
   for (const void* ptr : {x, W_q, W_k, W_v, W_o, W_gate, W_up, W_down,
