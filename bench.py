@@ -190,8 +190,10 @@ def kernel_work(name, cfg, attn_stats, ffn_stats):
     # backward (selection straight-through); pairs = executed (tile, key block) pairs
     pairs = attn_stats["key_blocks"]
     if name == "attn_bwd_dq_tc":
-        # two passes of S = Q K^T and dP = dO V^T, then dQ += dS K
-        return 10.0 * 128 * 64 * cfg.d * pairs, "flop", "tensor"
+        # after a training-mode forward (the way bench.py runs it): S = Q K^T,
+        # dP = dO V^T and dQ += dS K once per block (an inference-mode forward
+        # would add a first pass of S and dP: 10 instead of 6)
+        return 6.0 * 128 * 64 * cfg.d * pairs, "flop", "tensor"
     if name == "attn_bwd_dkv_tc":
         # S, dP, dV^T += dO^T P, dK^T += Q^T dS
         return 8.0 * 128 * 64 * cfg.d * pairs, "flop", "tensor"
@@ -436,9 +438,9 @@ def run_ours(args, rank, world, device):
     # ---------------- backward (fine-tuning step), the forward's sets held fixed
     backward = None
     if not args.no_backward:
-        step()  # the sets of the timed workload (p = cfg.p) back in the workspaces
-        backward = measure_backward(args, cfg, lay, aws, fws, attn_stats, ffn_stats, world,
-                                    device, ms_step)
+        step()  # the sets of the timed workload (p = cfg.p) back in the FFN workspace
+        backward = measure_backward(args, cfg, lay, fws, attn_stats, ffn_stats, world, device,
+                                    ms_step)
 
     dense = workloads.dense_flops(cfg)
     sparsity = {
@@ -459,17 +461,41 @@ def run_ours(args, rank, world, device):
     }
 
 
-def measure_backward(args, cfg, lay, aws, fws, attn_stats, ffn_stats, world, device,
-                     forward_ms):
+def measure_backward(args, cfg, lay, fws, attn_stats, ffn_stats, world, device, forward_ms):
     """One backward step = adaspark_cube_attn_backward + adaspark_token_ffn_backward
     on the sets the forward left in its workspaces, for seeded upstream
-    gradients (dO bf16, dy fp32) resident in HBM; device-timed like the forward."""
+    gradients (dO bf16, dy fp32) resident in HBM; device-timed like the forward.
+    The attention forward of a training step is adaspark_cube_attn_train (same
+    sets; it keeps the fp32 output the backward takes D_r from); its time is
+    reported beside the inference call's."""
     import torch
     import ffn_long_video_b200 as fb
     import workloads
     N, n_vis = cfg.n_tokens, cfg.n_vis
     up = workloads.make_upstream(cfg)
     dO, dy = up["dO"].to(device), up["dy"].to(device)
+    out_t = torch.empty_like(lay["Q"])
+    aws = torch.empty(fb.cube_attn_train_workspace_bytes(N, n_vis, cfg.n_cubes, cfg.hq, cfg.hkv,
+                                                         cfg.d), dtype=torch.uint8,
+                      device=device)
+
+    def attn_train():
+        fb.cube_attn(lay["Q"], lay["K"], lay["V"], lay["cube_ids"], lay["cube_offsets"], n_vis,
+                     cfg.p, out=out_t, workspace=aws, train=True)
+
+    for _ in range(2):
+        attn_train()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    for _ in range(3):
+        attn_train()
+    f1.record()
+    torch.cuda.synchronize()
+    attn_train_ms = max_over_ranks(f0.elapsed_time(f1), world, device) / 3
+    code, det = fb.read_device_status(aws)
+    if code != fb.OK:
+        raise RuntimeError(f"training forward device status {code} detail {det:#x}")
     bufs = {"a": {}, "f": {}}
 
     def bwd():
@@ -505,9 +531,11 @@ def measure_backward(args, cfg, lay, aws, fws, attn_stats, ffn_stats, world, dev
     dname, (dn, dms) = max(ktimes.items(), key=lambda kv: kv[1][1])
     return {
         "what": "attention + FFN backward of the timed layer, cube and token sets of its "
-                "forward held fixed (straight-through selection); gradients fp32",
+                "forward held fixed (straight-through selection), attention forward in "
+                "training mode; gradients fp32",
         "ms_per_step": round(ms, 3), "value": world * N / (ms / 1e3), "unit": "tokens/s",
         "steps": steps, "forward_plus_backward_ms": round(forward_ms + ms, 3),
+        "attention_train_forward_ms": round(attn_train_ms, 3),
         "gpu_launches": launches,
         "roofline": roofline_of(dname, dn, dms, cfg, attn_stats, ffn_stats,
                                 load_traffic(dname, cfg.name)),

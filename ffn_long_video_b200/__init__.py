@@ -5,7 +5,8 @@ kernels.  Torch tensors supply device memory and the current CUDA stream.  The
 binding fails loudly when the library is missing; there is no fallback.
 
 Entry points (same names as include/adaspark.h, without the prefix):
-``cube_count``, ``cube_partition``, ``cube_attn``, ``cube_attn_topk``, ``cube_attn_backward``,
+``cube_count``, ``cube_partition``, ``cube_attn`` (and ``_train``), ``cube_attn_topk``,
+``cube_attn_backward``,
 ``attn_export_sets``,
 ``attn_read_stats``, ``token_ffn``, ``token_ffn_backward``, ``ffn_export_active``,
 ``ffn_read_stats``,
@@ -75,6 +76,9 @@ def lib():
                                                                                    vp]),
             "adaspark_cube_attn_topk": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 7 + [vp, vp, sz,
                                                                                     vp]),
+            "adaspark_cube_attn_train_workspace": (sz, [i32] * 7),
+            "adaspark_cube_attn_train": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 6 + [f32, vp, vp,
+                                                                                   sz, vp]),
             "adaspark_cube_attn_backward_workspace": (sz, [i32] * 7),
             "adaspark_cube_attn_backward": (i32, [vp] * 4 + [i32, vp, vp] + [i32] * 6 +
                                             [vp] * 5 + [sz, vp]),
@@ -176,8 +180,11 @@ def cube_attn_workspace_bytes(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype) -> in
     return int(lib().adaspark_cube_attn_workspace(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype))
 
 
-def cube_attn(Q, K, V, cube_ids, cube_offsets, n_vis, p, out=None, workspace=None, stream=None):
-    """AdaS-Attn on device tensors; returns (out, workspace)."""
+def cube_attn(Q, K, V, cube_ids, cube_offsets, n_vis, p, out=None, workspace=None, stream=None,
+              train=False):
+    """AdaS-Attn on device tensors; returns (out, workspace). ``train`` runs
+    adaspark_cube_attn_train (the workspace then also keeps the fp32 output
+    that makes the backward pass a single walk over the keys)."""
     import torch
     for t, nm in ((Q, "Q"), (K, "K"), (V, "V"), (cube_ids, "cube_ids"),
                   (cube_offsets, "cube_offsets")):
@@ -189,16 +196,22 @@ def cube_attn(Q, K, V, cube_ids, cube_offsets, n_vis, p, out=None, workspace=Non
     if out is None:
         out = torch.empty_like(Q)
     if workspace is None:
-        nb = cube_attn_workspace_bytes(N, n_vis, C, hq, hkv, d, dt)
+        nb = (cube_attn_train_workspace_bytes if train else cube_attn_workspace_bytes)(
+            N, n_vis, C, hq, hkv, d, dt)
         if nb == 0:
-            raise AdasparkError(EINVAL, "adaspark_cube_attn_workspace")
+            raise AdasparkError(EUNSUPPORTED if train and dt == FP32 else EINVAL,
+                                "adaspark_cube_attn_workspace")
         workspace = torch.empty(nb, dtype=torch.uint8, device=Q.device)
-    _check(lib().adaspark_cube_attn(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(cube_ids),
-                                    _ptr(cube_offsets), C, n_vis, N, hq, hkv, d, float(p),
-                                    _ptr(out), _ptr(workspace), workspace.numel(),
-                                    _stream(stream)),
-           "adaspark_cube_attn")
+    fn = lib().adaspark_cube_attn_train if train else lib().adaspark_cube_attn
+    _check(fn(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(cube_ids), _ptr(cube_offsets), C, n_vis, N, hq,
+              hkv, d, float(p), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "adaspark_cube_attn_train" if train else "adaspark_cube_attn")
     return out, workspace
+
+
+def cube_attn_train_workspace_bytes(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype=BF16) -> int:
+    return int(lib().adaspark_cube_attn_train_workspace(n_tokens, n_vis, n_cubes, hq, hkv, d,
+                                                         dtype))
 
 
 def cube_attn_topk(Q, K, V, cube_ids, cube_offsets, n_vis, k, out=None, workspace=None,

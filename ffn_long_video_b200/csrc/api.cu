@@ -58,16 +58,24 @@ size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq
 }  // extern "C"
 
 // AdaS-Attn with Top-p (topk == 0) or Top-K (topk > 0, p unused) selection.
+// fp32 O of a training-mode call, after the inference layout
+static size_t attn_train_bytes(const AttnGeom& G) {
+  return (size_t)G.n_tokens * G.hq * G.d * sizeof(float);
+}
+
 static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype,
                           const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
                           int n_vis, int n_tokens, int hq, int hkv, int d, float p, int topk,
-                          void* out, void* workspace, size_t workspace_bytes, void* stream) {
+                          void* out, void* workspace, size_t workspace_bytes, void* stream,
+                          bool train = false) {
   if (!Q || !K || !V || !cube_ids || !cube_offsets || !out || !workspace) return ADASPARK_EINVAL;
   if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return ADASPARK_EINVAL;
   if (topk < 0 || (topk == 0 && !p_valid(p))) return ADASPARK_EINVAL;
+  if (train && dtype != ADASPARK_BF16) return ADASPARK_EUNSUPPORTED;
   const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
   const AttnLayout L = make_attn_layout(G);
-  if (workspace_bytes < L.total || !aligned(workspace, kAlign)) return ADASPARK_EINVAL;
+  const size_t need = L.total + (train ? attn_train_bytes(G) : 0);
+  if (workspace_bytes < need || !aligned(workspace, kAlign)) return ADASPARK_EINVAL;
   const size_t es = dtype == ADASPARK_BF16 ? 2 : 4;
   if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) || es == 0)
     return ADASPARK_EINVAL;
@@ -80,6 +88,9 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   const int dense = topk == 0 && p >= 1.0f;
   if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
   if (dense && cudaMemsetAsync(&hdr->pad[0], kModeDense, 1, s) != cudaSuccess)
+    return ADASPARK_ECUDA;
+  if (train &&
+      cudaMemsetAsync(reinterpret_cast<uint8_t*>(&hdr->pad[0]) + 1, 1, 1, s) != cudaSuccess)
     return ADASPARK_ECUDA;
   rc = cuda_rc(launch_validate(cube_ids, cube_offsets, nullptr, n_cubes, n_vis, n_tokens, hdr, s));
   if (rc) return rc;
@@ -122,6 +133,7 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   aa.dense = dense;
   aa.scale_log2 = sa.zscale;
   aa.lse = reinterpret_cast<float*>(ws + L.lse);
+  aa.o32 = train ? reinterpret_cast<float*>(ws + L.total) : nullptr;
   // When the layer's K and V outgrow what L2 holds alongside the other
   // traffic, visual tiles run one KV head after another, so that the blocks in
   // use belong to one head; otherwise all heads of a token range run together
@@ -140,6 +152,22 @@ int adaspark_cube_attn(const void* Q, const void* K, const void* V, int dtype,
                        void* workspace, size_t workspace_bytes, void* stream) {
   return cube_attn_impl(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq, hkv,
                         d, p, 0, out, workspace, workspace_bytes, stream);
+}
+
+size_t adaspark_cube_attn_train_workspace(int n_tokens, int n_vis, int n_cubes, int hq,
+                                          int hkv, int d, int dtype) {
+  if (dtype != ADASPARK_BF16 || !attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype))
+    return 0;
+  const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
+  return make_attn_layout(G).total + attn_train_bytes(G);
+}
+
+int adaspark_cube_attn_train(const void* Q, const void* K, const void* V, int dtype,
+                             const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                             int n_vis, int n_tokens, int hq, int hkv, int d, float p, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  return cube_attn_impl(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq, hkv,
+                        d, p, 0, out, workspace, workspace_bytes, stream, true);
 }
 
 int adaspark_cube_attn_topk(const void* Q, const void* K, const void* V, int dtype,
@@ -315,6 +343,8 @@ int adaspark_cube_attn_backward(const void* Q, const void* K, const void* V, con
   a.tile_list = reinterpret_cast<const uint16_t*>(fws + FL.tile_list);
   a.tile_mask = reinterpret_cast<const uint32_t*>(fws + FL.tile_mask);
   a.lse = reinterpret_cast<const float*>(fws + FL.lse);
+  // read only when the forward ran in training mode (then its workspace holds it)
+  a.o32 = reinterpret_cast<const float*>(fws + FL.total);
   a.hdr = reinterpret_cast<WsHeader*>(ws + L.header);
   a.dot = reinterpret_cast<float*>(ws + L.dot);
   a.inv_count = reinterpret_cast<int32_t*>(ws + L.inv_count);

@@ -57,6 +57,25 @@ __global__ void __launch_bounds__(32) check_kernel(WsHeader* hdr, const WsHeader
   if (threadIdx.x == 0 && fhdr->status != 0u) set_status(hdr, fhdr->status, 0xa100u);
 }
 
+// D_r = dO_r . O_r from the fp32 O of a training-mode forward (one warp per
+// row); nothing to do otherwise (the dQ kernel then sums D_r in a first pass).
+__global__ void __launch_bounds__(256) dot_kernel(AttnBwdArgs a) {
+  if (status_bad(a.hdr) || !fwd_was_train(a.fhdr)) return;
+  const int rows = a.G.n_tokens * a.G.hq;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const uint2 g = reinterpret_cast<const uint2*>(a.dO + (size_t)r * 128)[lane];
+  const float4 o = reinterpret_cast<const float4*>(a.o32 + (size_t)r * 128)[lane];
+  const __nv_bfloat162* gb = reinterpret_cast<const __nv_bfloat162*>(&g);
+  const float2 g0 = __bfloat1622float2(gb[0]), g1 = __bfloat1622float2(gb[1]);
+  float s = g0.x * o.x;
+  s = fmaf(g0.y, o.y, s);
+  s = fmaf(g1.x, o.z, s);
+  s = fmaf(g1.y, o.w, s);
+  s = warp_sum(s);
+  if (lane == 0) a.dot[r] = s;
+}
+
 // Per (KV head, cube j): the visual tiles of the KV head with any row admitting
 // cube j, in ascending tile order. The tiles of a KV head are cut into chunks
 // of kInvChunk; thread (kv, j, chunk) counts (fill = 0) or writes (fill = 1)
@@ -173,7 +192,7 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
   uint64_t* r_empty = r_full + RING;        // [RING]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(r_empty + RING);
   __shared__ volatile int s_abort;
-  __shared__ int s_own_hi, s_bad, s_dense;
+  __shared__ int s_own_hi, s_bad, s_dense, s_train;
   __shared__ float s_dpart[2][128];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -206,6 +225,7 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
     s_bad = status_bad(hdr) ? 1 : 0;
     s_own_hi = (!T.text && !s_bad) ? a.cube_ids[T.t_hi] : -1;
     s_dense = fwd_was_dense(a.fhdr) ? 1 : 0;
+    s_train = fwd_was_train(a.fhdr) ? 1 : 0;
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&mapK);
@@ -259,7 +279,8 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
       mbar_arrive(&r_full[slot]);
       return true;
     };
-    for (int pass = 0; pass < 2 && ok; ++pass) {
+    // a training-mode forward left D_r already: the second pass alone
+    for (int pass = s_train ? 1 : 0; pass < 2 && ok; ++pass) {
       const int pass_begin = base;
       for (int e0 = 0; e0 < n_total && ok; e0 += 32) {
         const int e = e0 + lane;
@@ -461,8 +482,11 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
       mbar_arrive(q_full);
     }
     const float lse2 = valid ? a.lse[rix] : 0.f;
-    float dot = 0.f;          // this half's part of D_r over the first pass
-    bool dot_done = false;
+    // this half's part of D_r over the first pass, or D_r from the training
+    // forward's fp32 O
+    const bool have_dot = s_train != 0;
+    float dot = have_dot && valid ? a.dot[rix] : 0.f;
+    bool dot_done = have_dot;
     const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     int m = 0;
     bool ok = true;
@@ -563,6 +587,7 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
       ++m;
     }
     if (ok && !dot_done && valid && half == 0) a.dot[rix] = 0.f;  // no blocks at all
+
     long long t0 = clock64();
     bool done = ok;
     if (ok && m > 0) {
@@ -1096,6 +1121,11 @@ cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a, cudaStream_t s) {
   cudaError_t e;
   if ((e = launch("attn_bwd_check", check_kernel, dim3(1), dim3(32), 0, s, a.hdr, a.fhdr)))
     return e;
+  {
+    const int rows = G.n_tokens * G.hq;
+    if ((e = launch("attn_bwd_dot", dot_kernel, dim3((rows + 7) / 8), dim3(256), 0, s, a)))
+      return e;
+  }
   if (G.n_cubes > 0) {
     const int nc = a.inv_chunks;
     const dim3 g((G.n_cubes + 127) / 128, G.hkv * nc);

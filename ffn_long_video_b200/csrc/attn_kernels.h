@@ -39,6 +39,7 @@ struct AttnArgs {
   float scale_log2;                   // log2(e) / sqrt(d)
   int kv_major;                       // visual tiles ordered one KV head after another
   float* lse;                         // [N][hq] m + log2(l) per row (bf16 path), for the backward
+  float* o32;                         // [N][hq][d] fp32 O with P split hi + lo (training), or null
 };
 
 // Backward of AdaS-Attn (sets of a forward call held fixed).
@@ -65,6 +66,7 @@ struct AttnBwdArgs {
   int32_t* inv_start;                 // [hkv * C * inv_chunks + 1] exclusive prefix
   int32_t* inv_list;                  // tile indices, ascending per (kv, j)
   int inv_chunks;                     // chunks of kInvChunk visual tiles per KV head
+  const float* o32;                   // forward's fp32 O when it ran in training mode
   void* pieces;                       // key pieces of up to 64 keys (cube, k0, nk), cube order
   AttnGeom G;
   int kv_major;
@@ -75,6 +77,11 @@ struct AttnBwdArgs {
 // first byte of its header's pad[0], set by the forward's host code.
 __device__ __forceinline__ bool fwd_was_dense(const WsHeader* fhdr) {
   return reinterpret_cast<const volatile uint8_t*>(&fhdr->pad[0])[0] == 1u;
+}
+// The forward call ran in training mode (adaspark_cube_attn_train): its
+// workspace holds O in fp32 after the inference layout (second byte of pad[0]).
+__device__ __forceinline__ bool fwd_was_train(const WsHeader* fhdr) {
+  return reinterpret_cast<const volatile uint8_t*>(&fhdr->pad[0])[1] == 1u;
 }
 cudaError_t launch_attn_backward_tc(const AttnBwdArgs& a, cudaStream_t s);
 

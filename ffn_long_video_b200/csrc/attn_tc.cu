@@ -75,6 +75,11 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
 }
 
 
+// TRAIN: for a backward pass to follow, P goes to the PV product as a bf16
+// pair hi + lo (lo = P - hi, in the second half of the S buffer, whose
+// scores were read before), so O is exact to about 2^-17 of each term, and O is
+// also written in fp32 to a.o32; the backward takes D_r = dO_r . O_r from it.
+template <bool TRAIN>
 __global__ void __launch_bounds__(THREADS, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    AttnArgs a) {
@@ -286,6 +291,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = make_sdesc_sw128(v_addr + kk * 2048, 8192, 1024);
           umma_bf16_ts(tmem_base, p_tmem + kk * 8, bd, idesc_o, (blk > 0 || kk > 0) ? 1u : 0u);
+          if (TRAIN) umma_bf16_ts(tmem_base, p_tmem + 32 + kk * 8, bd, idesc_o, 1u);
         }
         umma_commit(&pv_done[pb]);
         umma_commit(&v_empty[s]);
@@ -452,6 +458,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           const float p0 = ex2(x0), p1 = ex2(x1);
           add2(ls[2 * (q & 3)], ls[2 * (q & 3) + 1], p0, p1);
           pk[q] = pack_bf16x2(p0, p1);
+          if (TRAIN) sr[2 * q] = __float_as_uint(p0), sr[2 * q + 1] = __float_as_uint(p1);
         }
       } else {
 #pragma unroll
@@ -462,9 +469,22 @@ __global__ void __launch_bounds__(THREADS, 2)
               (u + 1 < lim) ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, neg_m)) : 0.f;
           ls[q & 7] += p0 + p1;
           pk[q] = pack_bf16x2(p0, p1);
+          if (TRAIN) sr[u] = __float_as_uint(p0), sr[u + 1] = __float_as_uint(p1);
         }
       }
       tmem_st32(tmem_base + lane_base + 128 + sb * 64, pk);
+      if (TRAIN) {
+        // lo parts: P - bf16(P), pairs in the S buffer's columns 32-63
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const __nv_bfloat162 hv = *reinterpret_cast<const __nv_bfloat162*>(&pk[q]);
+          const float2 hf = __bfloat1622float2(hv);
+          pk[q] = pack_bf16x2(__uint_as_float(sr[2 * q]) - hf.x,
+                              __uint_as_float(sr[2 * q + 1]) - hf.y);
+        }
+        tmem_st_wait();
+        tmem_st32(tmem_base + lane_base + 128 + sb * 64 + 32, pk);
+      }
       tmem_st_wait();
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       tc_fence_before();
@@ -495,6 +515,15 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
           for (int x = 0; x < 4; ++x)
             d4[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+          if (TRAIN) {
+            float4* o4 = reinterpret_cast<float4*>(a.o32 + ((size_t)t * G.hq + h) * 128 + c);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              o4[x] = make_float4(__uint_as_float(o[4 * x]) * inv,
+                                  __uint_as_float(o[4 * x + 1]) * inv,
+                                  __uint_as_float(o[4 * x + 2]) * inv,
+                                  __uint_as_float(o[4 * x + 3]) * inv);
+          }
         }
       }
     }
@@ -524,7 +553,7 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   if (!encode_tmap_bf16(&mK, a.K, 3, dims, strides, box) ||
       !encode_tmap_bf16(&mV, a.V, 3, dims, strides, box))
     return cudaErrorInvalidValue;
-  auto k = fa::attn_tc_kernel;
+  auto k = a.o32 ? fa::attn_tc_kernel<true> : fa::attn_tc_kernel<false>;
   cudaError_t e =
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fa::SMEM_BYTES);
   if (e != cudaSuccess) return e;

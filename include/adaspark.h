@@ -152,6 +152,24 @@ int adaspark_cube_attn_topk(const void *Q, const void *K, const void *V, int dty
                             int n_vis, int n_tokens, int hq, int hkv, int d, int k, void *out,
                             void *workspace, size_t workspace_bytes, void *stream);
 
+/* Device workspace bytes needed by adaspark_cube_attn_train (0 when the sizes
+ * are invalid or dtype is not ADASPARK_BF16): adaspark_cube_attn_workspace
+ * plus an fp32 copy of the output. */
+size_t adaspark_cube_attn_train_workspace(int n_tokens, int n_vis, int n_cubes, int hq,
+                                          int hkv, int d, int dtype);
+
+/* adaspark_cube_attn for a step whose backward pass follows: the same sets and
+ * output, and P goes to the PV product as a bf16 pair (hi + lo) so that the
+ * workspace also keeps O in fp32 exact to about 2^-17 of each term; with it,
+ * adaspark_cube_attn_backward takes D_r = dO_r . O_r directly instead of
+ * summing it in an extra pass over the keys. Arguments as adaspark_cube_attn,
+ * with workspace >= adaspark_cube_attn_train_workspace(...) bytes. Only
+ * ADASPARK_BF16 (ADASPARK_FP32 returns ADASPARK_EUNSUPPORTED). */
+int adaspark_cube_attn_train(const void *Q, const void *K, const void *V, int dtype,
+                             const int32_t *cube_ids, const int32_t *cube_offsets, int n_cubes,
+                             int n_vis, int n_tokens, int hq, int hkv, int d, float p, void *out,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
 /* Device workspace bytes needed by adaspark_cube_attn_backward (0 when the
  * sizes are invalid or dtype is not ADASPARK_BF16). */
 size_t adaspark_cube_attn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int hq,
@@ -172,7 +190,8 @@ size_t adaspark_cube_attn_backward_workspace(int n_tokens, int n_vis, int n_cube
  *   Q, K, V, cube_ids, cube_offsets, sizes: exactly those of the forward call;
  *   dO [n_tokens, hq, d]: device bf16, the gradient of the forward's output;
  *   fwd_workspace: the forward call's workspace, untouched since (the backward
- *       reads its sets, mode and per-row log-sum-exp; it does not modify it);
+ *       reads its sets, mode and per-row log-sum-exp, and after
+ *       adaspark_cube_attn_train its fp32 output; it does not modify it);
  *   dQ [n_tokens, hq, d], dK / dV [n_tokens, hkv, d]: device float32, written
  *       in full (not accumulated into);
  *   workspace: device, >= adaspark_cube_attn_backward_workspace(...) bytes,

@@ -68,12 +68,14 @@ def excess_over_bf16(got, want):
     return float((np.abs(got - want) - ulp_bf16(want)).max()) if got.size else 0.0
 
 
-def run_attn(case, p=None, k=None):
-    """Run AdaS-Attn (Top-p, or Top-K when k is given) and export its sets."""
+def run_attn(case, p=None, k=None, train=False):
+    """Run AdaS-Attn (Top-p, or Top-K when k is given; the training-mode call
+    when ``train``) and export its sets."""
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
     if k is None:
-        out, ws = fb.cube_attn(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis, p)
+        out, ws = fb.cube_attn(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis, p,
+                               train=train)
     else:
         out, ws = fb.cube_attn_topk(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis,
                                     k)
@@ -85,12 +87,12 @@ def run_attn(case, p=None, k=None):
     return out, sel, ws
 
 
-def check_attn(case, p=None, tokens=None, report=None, k=None):
+def check_attn(case, p=None, tokens=None, report=None, k=None, train=False):
     """Selection parity + output parity of AdaS-Attn on ``tokens`` (default all);
-    Top-K selection when ``k`` is given."""
+    Top-K selection when ``k`` is given; the training-mode call when ``train``."""
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
-    out, gsel, ws = run_attn(case, p, k)
+    out, gsel, ws = run_attn(case, p, k, train)
     Qc, Kc, Vc = (t[k].cpu() for k in ("Q", "K", "V"))
     off = case["off_np"]
     if tokens is None:
@@ -244,12 +246,12 @@ def check_ffn_backward(case, p=None, report=None):
     return grads, act
 
 
-def run_attn_backward(case, p=None, k=None):
-    """Forward AdaS-Attn (Top-p, or Top-K when k is given), then its backward for
-    the case's seeded dO; returns the library's gradients, the forward's sets
-    [N, hq, C] (text rows False) and dO."""
+def run_attn_backward(case, p=None, k=None, train=False):
+    """Forward AdaS-Attn (Top-p, or Top-K when k is given; training mode when
+    ``train``), then its backward for the case's seeded dO; returns the
+    library's gradients, the forward's sets [N, hq, C] (text rows False) and dO."""
     cfg, t = case["cfg"], case["t"]
-    out, sel, fws = run_attn(case, p, k)
+    out, sel, fws = run_attn(case, p, k, train)
     dO = workloads.make_upstream(cfg)["dO"].to(t["Q"].device)
     dQ, dK, dV, bws = fb.cube_attn_backward(t["Q"], t["K"], t["V"], dO, case["ids"],
                                             case["off"], cfg.n_vis, fws)
@@ -261,9 +263,9 @@ def run_attn_backward(case, p=None, k=None):
     return (dQ, dK, dV), sets, dO, (out, fws)
 
 
-def check_attn_backward(case, p=None, k=None, report=None):
+def check_attn_backward(case, p=None, k=None, report=None, train=False):
     cfg, t = case["cfg"], case["t"]
-    grads, sets, dO, _ = run_attn_backward(case, p, k)
+    grads, sets, dO, _ = run_attn_backward(case, p, k, train)
     *want, mags = oracle.attention_backward_given_sets(
         t["Q"].cpu(), t["K"].cpu(), t["V"].cpu(), dO.cpu(), case["off_np"], cfg.n_vis, sets,
         with_magnitudes=True)

@@ -42,6 +42,21 @@ def test_attn_backward(bcase, p):
     print(bcase["cfg"].name, "attn", p, rep)
 
 
+@pytest.mark.parametrize("p", [0.7, 1.0])
+def test_attn_train_forward_and_backward(bcase, p):
+    """The training-mode forward: same sets, output within the forward bar; its
+    backward (D_r from the fp32 output, one walk over the keys) within the
+    gradient bar, and within rounding of the inference forward's backward."""
+    rep = {}
+    parity.check_attn(bcase, p=p, report=rep, train=True)
+    g_train, _ = parity.check_attn_backward(bcase, p=p, report=rep, train=True)
+    g_inf, _, _, _ = parity.run_attn_backward(bcase, p=p)
+    for a, b, nm in zip(g_train, g_inf, ("dQ", "dK", "dV")):
+        d = (a - b).double()
+        assert (d.norm() / b.double().norm()).item() < 5e-3, nm
+    print(bcase["cfg"].name, "attn train", p, rep)
+
+
 def test_attn_backward_topk_and_determinism(bcase):
     rep = {}
     g1, _ = parity.check_attn_backward(bcase, k=3, report=rep)
