@@ -13,23 +13,26 @@
 //
 // Two tcgen05 kernels, no atomics:
 //   attn_bwd_dq   one CTA per 128-row tile (the forward's tiles, order and
-//                 block walk), two passes over the row's key blocks with
-//                 S = Q K^T and dP = dO V^T per 64-key block in TMEM: the first
-//                 sums D_r = sum_j P_rj dP_rj in fp32 (stored for attn_bwd_dkv),
-//                 the second writes dS (bf16) back over S and runs
-//                 dQ += dS K with dS read from TMEM (K as an N-major operand).
-//                 D from the same fp32 P and dP makes each row's dS sum to zero
-//                 up to fp32 rounding; D = dO . O from the bf16 output would
-//                 leave a bias of about one bf16 ulp of O, which the near-
-//                 cancelling sum behind dQ turns into errors near 4% of its RMS.
-//   attn_bwd_dkv  one CTA per (KV head, 64-key block): walks the query tiles
-//                 that admit the block (inverted selection lists, then the
-//                 text tiles), S and dP as above, P and dS staged in shared
-//                 memory, then dV^T += dO^T P and dK^T += Q^T dS with M = 128
-//                 over the head dimension (both operands MN-major), so the
-//                 block's key and value gradients stay in TMEM until the end.
-// Small kernels before them: the inverted lists (per KV head and cube, the
-// visual tiles with any row admitting the cube, ascending).
+//                 block walk), the walk's 64-key blocks two at a time:
+//                 S = Q [K_a; K_b]^T and dP = dO [V_a; V_b]^T (N = 128) into
+//                 TMEM, dS (bf16) written back over S, dQ += dS [K_a; K_b]
+//                 (K = 128) with dS read from TMEM. D_r must agree with the
+//                 recomputed fp32 P: after a training-mode forward it is
+//                 dO . O from that call's fp32 output (dot_kernel); otherwise a
+//                 first walk sums D_r = sum_j P_rj dP_rj (stored for
+//                 attn_bwd_dkv). D = dO . O from the bf16 output would leave a
+//                 bias of about one bf16 ulp of O, which the near-cancelling
+//                 sum behind dQ turns into errors near 4% of its RMS.
+//   attn_bwd_dkv  transposed: one CTA per (KV head, pair of 64-key pieces),
+//                 walking the query tiles that admit either piece (the union of
+//                 the two cubes' inverted lists, then the text tiles):
+//                 S^T = K Q^T and dP^T = V dO^T with M = 128 keys, one thread
+//                 per key forming P^T and dS^T in TMEM, dV += P^T dO and
+//                 dK += dS^T Q with P^T / dS^T read from TMEM, so the pair's key
+//                 and value gradients stay in TMEM until the end.
+// Small kernels before them: D_r (training-mode forward only), the inverted
+// lists (per KV head and cube, the visual tiles with any row admitting the
+// cube, ascending) and the table of key pieces.
 #include <algorithm>
 
 #include "attn_kernels.h"
