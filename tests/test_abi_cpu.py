@@ -86,3 +86,57 @@ def test_calls_reject_bad_arguments_before_the_device():
     for code in (-1, 3):
         assert L.adaspark_token_ffn_ex(*fargs, 0.7, code, dummy, dummy, fws, None) == fb.EINVAL
     assert fb.status_string(fb.EDEVICE) == "device-side check failed"
+
+
+def test_backward_layer_and_train_calls_reject_bad_arguments_before_the_device():
+    L = fb.lib()
+    d = ctypes.c_void_p(256)
+    # workspace queries: bf16 only for the backward and the training forward
+    assert fb.cube_attn_backward_workspace_bytes(65792, 65536, 1024, 28, 4, 128) > 0
+    assert fb.cube_attn_backward_workspace_bytes(544, 512, 16, 4, 1, 64, fb.FP32) == 0
+    assert fb.token_ffn_backward_workspace_bytes(65792, 65536, 1024, 3584, 18944) > 0
+    assert fb.token_ffn_backward_workspace_bytes(544, 512, 16, 256, 512, fb.FP32) == 0
+    inf = fb.cube_attn_workspace_bytes(65792, 65536, 1024, 28, 4, 128, fb.BF16)
+    assert fb.cube_attn_train_workspace_bytes(65792, 65536, 1024, 28, 4, 128) == \
+        inf + 65792 * 28 * 128 * 4
+    # attention backward: fp32 unsupported, bad sizes / pointers / workspace rejected
+    ab = fb.cube_attn_backward_workspace_bytes(544, 512, 16, 4, 1, 128)
+    aargs = [d] * 4
+    geo = [d, d, 16, 512, 544, 4, 1, 128]
+    assert L.adaspark_cube_attn_backward(*aargs, fb.FP32, *geo, d, d, d, d, d, ab, None) == \
+        fb.EUNSUPPORTED
+    assert L.adaspark_cube_attn_backward(*aargs, fb.BF16, *geo, d, d, d, d, d, ab - 1, None) == \
+        fb.EINVAL
+    assert L.adaspark_cube_attn_backward(*aargs, fb.BF16, *geo, None, d, d, d, d, ab, None) == \
+        fb.EINVAL
+    assert L.adaspark_cube_attn_backward(*aargs, fb.BF16, d, d, 16, 512, 544, 5, 2, 128, d, d, d,
+                                         d, d, ab, None) == fb.EINVAL                 # hq % hkv
+    # training forward: fp32 unsupported, too small a workspace rejected
+    tw = fb.cube_attn_train_workspace_bytes(544, 512, 16, 4, 1, 128)
+    targs = [d, d, d, fb.BF16, d, d, 16, 512, 544, 4, 1, 128, 0.7, d, d]
+    assert L.adaspark_cube_attn_train(*targs, tw - 1, None) == fb.EINVAL
+    targs[3] = fb.FP32
+    assert L.adaspark_cube_attn_train(*targs, tw, None) == fb.EUNSUPPORTED
+    # FFN backward
+    fb_ws = fb.token_ffn_backward_workspace_bytes(544, 512, 16, 256, 512)
+    fargs = [d, d, d]
+    fgeo = [d, 16, 512, 544, 256, 512]
+    assert L.adaspark_token_ffn_backward(*fargs, fb.FP32, *fgeo, d, d, d, d, d, d, d, fb_ws,
+                                         None) == fb.EUNSUPPORTED
+    assert L.adaspark_token_ffn_backward(*fargs, fb.BF16, *fgeo, d, d, d, d, d, d, d, fb_ws - 8,
+                                         None) == fb.EINVAL
+    assert L.adaspark_token_ffn_backward(*fargs, fb.BF16, *fgeo, None, d, d, d, d, d, d, fb_ws,
+                                         None) == fb.EINVAL
+    assert L.adaspark_token_ffn_backward(*fargs, fb.BF16, d, 16, 512, 544, 250, 512, d, d, d, d, d,
+                                         d, d, fb_ws, None) == fb.EINVAL                # D % 64
+    # layer: fp32 unsupported, bad p rejected; RMSNorm: bad sizes rejected
+    lw = fb.layer_workspace_bytes(544, 512, 16, 4, 1, 128, 256, 512)
+    assert lw > 0
+    largs = [d] * 8
+    lgeo = [d, d, d, 16, 512, 544, 4, 1, 128, 256, 512]
+    assert L.adaspark_layer(*largs, fb.FP32, *lgeo, 0.7, 0.7, d, d, lw, None) == fb.EUNSUPPORTED
+    for pa, pf in ((0.0, 0.7), (0.7, 1.5)):
+        assert L.adaspark_layer(*largs, fb.BF16, *lgeo, pa, pf, d, d, lw, None) == fb.EINVAL
+    assert L.adaspark_layer(*largs, fb.BF16, *lgeo, 0.7, 0.7, d, d, lw - 1, None) == fb.EINVAL
+    assert L.adaspark_rmsnorm(d, fb.BF16, None, d, 4, 0, 1e-6, None) == fb.EINVAL
+    assert L.adaspark_rmsnorm(d, 7, None, d, 4, 64, 1e-6, None) == fb.EINVAL
