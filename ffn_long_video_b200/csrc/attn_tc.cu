@@ -367,24 +367,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       const Desc dsc = ring[slot];
       if (dsc.nk == 0) break;
-      const int sb = i & 1;
-      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0x7600u)) {
-        ok = false;
-        break;
-      }
-      // S_i has landed, so the producer and the MMA issuer have both consumed
-      // descriptor i: only now may the filler reuse its slot.
-      mbar_arrive(&r_empty[slot]);
-      tc_fence_after();
-      uint32_t sr[64];
-      {
-        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        tmem_ld32(tmem_base + lane_base + 128 + sb * 64, s0);
-        tmem_ld32(tmem_base + lane_base + 128 + sb * 64 + 32, s1);
-      }
-      tmem_ld_wait();
-
       // admitted keys [0, lim) of this row in the block
       bool row_on;
       if (!valid) row_on = false;
@@ -394,6 +376,39 @@ __global__ void __launch_bounds__(THREADS, 2)
       int lim = row_on ? dsc.nk : 0;
       if (row_on && (T.text || dsc.j == own)) lim = min(lim, t - dsc.k0 + 1);
       if (lim <= 0) row_on = false;
+      const int sb = i & 1;
+      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0x7600u)) {
+        ok = false;
+        break;
+      }
+      // S_i has landed, so the producer and the MMA issuer have both consumed
+      // descriptor i: only now may the filler reuse its slot.
+      mbar_arrive(&r_empty[slot]);
+      tc_fence_after();
+      if (!__any_sync(0xffffffffu, row_on)) {
+        // No row of this warp takes a key of the block (the tile's list holds
+        // the cube for other rows): P = 0 for its 32 rows, the value the
+        // general path gives them, without reading S.
+        uint32_t zero[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) zero[q] = 0u;
+        tmem_st32(tmem_base + lane_base + 128 + sb * 64, zero);
+        if (TRAIN) tmem_st32(tmem_base + lane_base + 128 + sb * 64 + 32, zero);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[sb]);
+        ++i;
+        continue;
+      }
+      uint32_t sr[64];
+      {
+        uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        tmem_ld32(tmem_base + lane_base + 128 + sb * 64, s0);
+        tmem_ld32(tmem_base + lane_base + 128 + sb * 64 + 32, s1);
+      }
+      tmem_ld_wait();
+
       // Blocks where every row of the warp takes all 64 keys or none need no
       // per-key mask: a row that takes none gets an offset of -inf, so its
       // probabilities come out as exact zeros.
