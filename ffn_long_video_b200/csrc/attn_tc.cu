@@ -63,6 +63,12 @@ __device__ __forceinline__ void fma2_bcast(float a0, float a1, float s, float c,
       : "=f"(o0), "=f"(o1)
       : "f"(a0), "f"(a1), "f"(s), "f"(c));
 }
+// max(a, b, c) in one instruction (three-input form of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 // (s0, s1) += (a0, a1)
 __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
   asm("{\n\t.reg .b64 ps, pa;\n\t"
@@ -415,13 +421,19 @@ __global__ void __launch_bounds__(THREADS, 2)
       const bool partial = __any_sync(0xffffffffu, row_on && lim < 64);
       float mraw = -INFINITY;
       if (!partial) {
+        // eight chains over columns 0-55, then the last eight columns
+        auto f = [&](int u) { return __uint_as_float(sr[u]); };
         float mx[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(f(k), f(k + 8), f(k + 16));
 #pragma unroll
-        for (int u = 8; u < 64; ++u) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(sr[u]));
-        const float m8 = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], f(k + 24), f(k + 32));
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], f(k + 40), f(k + 48));
+        const float t0 = fmax3(mx[0], mx[1], f(56)), t1 = fmax3(mx[2], mx[3], f(57));
+        const float t2 = fmax3(mx[4], mx[5], f(58)), t3 = fmax3(mx[6], mx[7], f(59));
+        const float t4 = fmax3(f(60), f(61), f(62));
+        const float m8 = fmax3(fmax3(t0, t1, t2), fmax3(t3, t4, f(63)), -INFINITY);
         mraw = row_on ? m8 : -INFINITY;
       } else {
         float mx[8];
