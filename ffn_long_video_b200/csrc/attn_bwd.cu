@@ -535,6 +535,28 @@ __global__ void __launch_bounds__(dq::THREADS, 1)
         if (valid && half == 0) a.dot[rix] = dot;
         dot_done = true;
       }
+      if (!__any_sync(0xffffffffu, lim > 0)) {
+        // No row of this warp takes a key of its block: P = 0, so its dS is
+        // zero (and its part of D_r in the first pass adds nothing); dS = 0
+        // goes over the scores without reading S or dP. The dP barrier is
+        // still waited on, which keeps its phase count.
+        if (!mbar_wait_warp(dp_full, m & 1, &s_abort, hdr, 0xa616u)) {
+          ok = false;
+          break;
+        }
+        if (pass1) {
+          uint32_t zero[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) zero[q] = 0u;
+          tmem_st16(tmem_base + lane_base + col_s(m) + half * 64, zero);
+          tmem_st16(tmem_base + lane_base + col_s(m) + half * 64 + 16, zero);
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(ds_ready);
+        ++m;
+        continue;
+      }
       // P over this half's 64 keys, 32 at a time
       float pv[64];
 #pragma unroll
@@ -752,6 +774,7 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
   __shared__ WalkEntry s_walk[RINGE];
   __shared__ float s_lse[2][128], s_dot[2][128];
   __shared__ int s_lim[2][2][128];          // [entry parity][piece][row]
+  __shared__ int s_on[2][2][4];             // [entry parity][piece][row quarter]: any row on
   __shared__ volatile int s_abort;
 
   const AttnGeom& G = a.G;
@@ -996,8 +1019,16 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
         }
         s_lse[par][mrow] = R.valid ? a.lse[rix] : 0.f;
         s_dot[par][mrow] = R.valid ? a.dot[rix] : 0.f;
-        s_lim[par][0][mrow] = piece_limit(a, pA, text, we.bt, mrow, R, own, c_hi, dense);
-        s_lim[par][1][mrow] = piece_limit(a, pB, text, we.bt, mrow, R, own, c_hi, dense);
+        const int limA = piece_limit(a, pA, text, we.bt, mrow, R, own, c_hi, dense);
+        const int limB = piece_limit(a, pB, text, we.bt, mrow, R, own, c_hi, dense);
+        s_lim[par][0][mrow] = limA;
+        s_lim[par][1][mrow] = limB;
+        const unsigned onA = __ballot_sync(0xffffffffu, limA > 0);
+        const unsigned onB = __ballot_sync(0xffffffffu, limB > 0);
+        if (lane == 0) {
+          s_on[par][0][mrow >> 5] = onA != 0u;
+          s_on[par][1][mrow >> 5] = onB != 0u;
+        }
       }
       mbar_arrive(&meta_full[par]);
       if (!mbar_wait_warp(&meta_full[par], (e >> 1) & 1, &s_abort, hdr, 0xa870u)) {
@@ -1011,6 +1042,28 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
         break;
       }
       tc_fence_after();
+      if (!(s_on[par][kp][2 * hc] | s_on[par][kp][2 * hc + 1])) {
+        // No row of this half takes a key of this warp's piece: P^T = 0 and
+        // dS^T = 0 go over S^T and dP^T without reading them; both barriers
+        // keep their order.
+        uint32_t zero[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) zero[q] = 0u;
+        tmem_st32(tmem_base + lane_base + hc * 64, zero);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_ready);
+        if (!mbar_wait_warp(dp_full, e & 1, &s_abort, hdr, 0xa886u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st32(tmem_base + lane_base + 128 + hc * 64, zero);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(ds_ready);
+        continue;
+      }
       float pv[64];
       {
         uint32_t sr[64];
