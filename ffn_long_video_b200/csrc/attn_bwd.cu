@@ -772,9 +772,12 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
   uint64_t* w_empty = w_full + RINGE;       // [RINGE]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(w_empty + RINGE);
   __shared__ WalkEntry s_walk[RINGE];
-  __shared__ float s_lse[2][128], s_dot[2][128];
+  // per row and piece: the row's log2-sum-exp, or +inf where the row takes no
+  // key of the piece (its P then comes out as an exact zero)
+  __shared__ float s_lse[2][2][128], s_dot[2][128];
   __shared__ int s_lim[2][2][128];          // [entry parity][piece][row]
   __shared__ int s_on[2][2][4];             // [entry parity][piece][row quarter]: any row on
+  __shared__ int s_part[2][2][4];           // ... any row taking only some keys of the piece
   __shared__ volatile int s_abort;
 
   const AttnGeom& G = a.G;
@@ -1017,17 +1020,23 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
           const TileRow Rl = tile_row(G, false, we.bt, 0);
           c_hi = a.cube_ids[min(Rl.t + kTileRows, G.n_vis) - 1];
         }
-        s_lse[par][mrow] = R.valid ? a.lse[rix] : 0.f;
+        const float lse = R.valid ? a.lse[rix] : 0.f;
         s_dot[par][mrow] = R.valid ? a.dot[rix] : 0.f;
         const int limA = piece_limit(a, pA, text, we.bt, mrow, R, own, c_hi, dense);
         const int limB = piece_limit(a, pB, text, we.bt, mrow, R, own, c_hi, dense);
         s_lim[par][0][mrow] = limA;
         s_lim[par][1][mrow] = limB;
+        s_lse[par][0][mrow] = limA > 0 ? lse : INFINITY;
+        s_lse[par][1][mrow] = limB > 0 ? lse : INFINITY;
         const unsigned onA = __ballot_sync(0xffffffffu, limA > 0);
         const unsigned onB = __ballot_sync(0xffffffffu, limB > 0);
+        const unsigned ptA = __ballot_sync(0xffffffffu, limA > 0 && limA < 64);
+        const unsigned ptB = __ballot_sync(0xffffffffu, limB > 0 && limB < 64);
         if (lane == 0) {
           s_on[par][0][mrow >> 5] = onA != 0u;
           s_on[par][1][mrow >> 5] = onB != 0u;
+          s_part[par][0][mrow >> 5] = ptA != 0u;
+          s_part[par][1][mrow >> 5] = ptB != 0u;
         }
       }
       mbar_arrive(&meta_full[par]);
@@ -1064,6 +1073,9 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
         mbar_arrive(ds_ready);
         continue;
       }
+      // Every row of the half takes all 64 keys of the piece or none: no
+      // per-key limit (rows taking none have lse = +inf, so P = 0).
+      const bool full = !(s_part[par][kp][2 * hc] | s_part[par][kp][2 * hc + 1]);
       float pv[64];
       {
         uint32_t sr[64];
@@ -1073,16 +1085,29 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
         tmem_ld32(tmem_base + lane_base + hc * 64 + 32, s1);
         tmem_ld_wait();
         uint32_t pp[32];
+        if (full) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+          for (int q = 0; q < 32; ++q) {
 #pragma unroll
-          for (int z = 0; z < 2; ++z) {
-            const int r = hc * 64 + 2 * q + z;
-            pv[2 * q + z] = kl < s_lim[par][kp][r]
-                                ? ex2(fmaf(__uint_as_float(sr[2 * q + z]), scale, -s_lse[par][r]))
-                                : 0.f;
+            for (int z = 0; z < 2; ++z) {
+              const int r = hc * 64 + 2 * q + z;
+              pv[2 * q + z] = ex2(fmaf(__uint_as_float(sr[2 * q + z]), scale, -s_lse[par][kp][r]));
+            }
+            pp[q] = pack_bf16x2(pv[2 * q], pv[2 * q + 1]);
           }
-          pp[q] = pack_bf16x2(pv[2 * q], pv[2 * q + 1]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const int r = hc * 64 + 2 * q + z;
+              pv[2 * q + z] =
+                  kl < s_lim[par][kp][r]
+                      ? ex2(fmaf(__uint_as_float(sr[2 * q + z]), scale, -s_lse[par][kp][r]))
+                      : 0.f;
+            }
+            pp[q] = pack_bf16x2(pv[2 * q], pv[2 * q + 1]);
+          }
         }
         tmem_st32(tmem_base + lane_base + hc * 64, pp);
         tmem_st_wait();
@@ -1102,17 +1127,30 @@ __global__ void __launch_bounds__(dkv::THREADS, 1)
         tmem_ld32(tmem_base + lane_base + 128 + hc * 64 + 32, p1);
         tmem_ld_wait();
         uint32_t pd[32];
+        if (full) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          float dv[2];
+          for (int q = 0; q < 32; ++q) {
+            float dv[2];
 #pragma unroll
-          for (int z = 0; z < 2; ++z) {
-            const int r = hc * 64 + 2 * q + z;
-            dv[z] = kl < s_lim[par][kp][r]
-                        ? pv[2 * q + z] * (__uint_as_float(dp[2 * q + z]) - s_dot[par][r])
-                        : 0.f;
+            for (int z = 0; z < 2; ++z) {
+              const int r = hc * 64 + 2 * q + z;
+              dv[z] = pv[2 * q + z] * (__uint_as_float(dp[2 * q + z]) - s_dot[par][r]);
+            }
+            pd[q] = pack_bf16x2(dv[0], dv[1]);
           }
-          pd[q] = pack_bf16x2(dv[0], dv[1]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) {
+            float dv[2];
+#pragma unroll
+            for (int z = 0; z < 2; ++z) {
+              const int r = hc * 64 + 2 * q + z;
+              dv[z] = kl < s_lim[par][kp][r]
+                          ? pv[2 * q + z] * (__uint_as_float(dp[2 * q + z]) - s_dot[par][r])
+                          : 0.f;
+            }
+            pd[q] = pack_bf16x2(dv[0], dv[1]);
+          }
         }
         tmem_st32(tmem_base + lane_base + 128 + hc * 64, pd);
         tmem_st_wait();
