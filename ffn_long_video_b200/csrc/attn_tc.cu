@@ -371,16 +371,20 @@ __global__ void __launch_bounds__(THREADS, 2)
         ok = false;
         break;
       }
-      const Desc dsc = ring[slot];
-      if (dsc.nk == 0) break;
+      // the descriptor's fields straight from shared memory (a local copy
+      // indexed by the warp's quadrant would live in local memory)
+      const int d_nk = ring[slot].nk;
+      if (d_nk == 0) break;
+      const int d_k0 = ring[slot].k0, d_j = ring[slot].j;
+      const uint32_t d_mask = ring[slot].mask[wq];
       // admitted keys [0, lim) of this row in the block
       bool row_on;
       if (!valid) row_on = false;
       else if (T.text) row_on = true;
-      else if (a.dense) row_on = dsc.j <= own;
-      else row_on = ((dsc.mask[wq] >> lane) & 1u) != 0u;
-      int lim = row_on ? dsc.nk : 0;
-      if (row_on && (T.text || dsc.j == own)) lim = min(lim, t - dsc.k0 + 1);
+      else if (a.dense) row_on = d_j <= own;
+      else row_on = ((d_mask >> lane) & 1u) != 0u;
+      int lim = row_on ? d_nk : 0;
+      if (row_on && (T.text || d_j == own)) lim = min(lim, t - d_k0 + 1);
       if (lim <= 0) row_on = false;
       const int sb = i & 1;
       if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0x7600u)) {
