@@ -1,0 +1,124 @@
+"""Host-side arithmetic of bench.py (no GPU): the algorithmic work per launch,
+the roofline entry built from it, the check that ties recorded DRAM counters
+to the kernel source they were taken on, and the clock-sample filter."""
+import hashlib
+import os
+
+import pytest
+
+import bench
+import workloads
+
+CFG = workloads.CONFIGS[3]   # the 64K-token 7B-shaped layer
+ATTN = {"key_blocks": 1000, "candidate_pairs": 5000}
+FFN = {"active_visual": 300, "text_tokens": 20, "skipped_visual": 40}
+
+
+def test_kernel_work_counts():
+    d, D, F = CFG.d, CFG.D, CFG.F
+    M = 320
+    # attention: Q K^T and P V, 2 flops per multiply-add, 128 rows x 64 keys x d per block
+    assert bench.kernel_work("attn_tc", CFG, ATTN, FFN) == (2 * 2 * 128 * 64 * d * 1000, "flop",
+                                                             "tensor")
+    assert bench.kernel_work("ffn_gemm1_tc", CFG, ATTN, FFN)[0] == 2 * 2 * M * D * F
+    assert bench.kernel_work("ffn_gemm2_tc", CFG, ATTN, FFN)[0] == 2 * M * D * F
+    # three bf16 parts of the cube means, two passes, 2 d flops per (row, cube) pair
+    assert bench.kernel_work("select_tc", CFG, ATTN, FFN)[0] == 3 * 2 * 2 * d * 5000
+    # backward: S, dP, dQ (three products) and S, dP, dV, dK (four) per block
+    assert bench.kernel_work("attn_bwd_dq_tc", CFG, ATTN, FFN)[0] == 3 * 2 * 128 * 64 * d * 1000
+    assert bench.kernel_work("attn_bwd_dkv_tc", CFG, ATTN, FFN)[0] == 4 * 2 * 128 * 64 * d * 1000
+    # recompute gate and up plus dh = df W_down: three D x F products per row
+    assert bench.kernel_work("ffn_bwd_gemm_hdg_tc", CFG, ATTN, FFN)[0] == 3 * 2 * M * D * F
+    # HBM kernels: bytes moved
+    assert bench.kernel_work("ffn_compensate", CFG, ATTN, FFN) == (40 * D * (2 + 4), "byte", "hbm")
+    assert bench.kernel_work("ffn_select", CFG, ATTN, FFN)[0] == CFG.n_vis * D * 2
+    assert bench.kernel_work("no_such_kernel", CFG, ATTN, FFN) == (None, None, None)
+
+
+def test_roofline_fraction(monkeypatch):
+    peaks = {"hbm_gbs": 5000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1000.0}
+    monkeypatch.setattr(bench, "load_peaks", lambda: (dict(peaks), "measured"))
+    attn = {"key_blocks": 5_000_000, "candidate_pairs": 0}   # about the 64K layer's
+    work = bench.kernel_work("attn_tc", CFG, attn, FFN)[0]
+    # two launches of 25 ms each
+    r = bench.roofline_of("attn_tc", 2, 50.0, CFG, attn, FFN, traffic=123)
+    achieved = work / 25e-3 / 1e12
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(achieved, rel=1e-3)
+    assert r["peak"] == 1000.0                       # the sustained figure
+    assert r["frac"] == pytest.approx(achieved / 1000.0, rel=1e-3)
+    assert r["traffic"] == 123 and r["ms_per_launch"] == 25.0
+    h = bench.roofline_of("ffn_select", 1, 2.0, CFG, ATTN, FFN, traffic=None)
+    gbs = CFG.n_vis * CFG.D * 2 / 2e-3 / 1e9
+    assert h["bound"] == "hbm" and h["achieved"] == pytest.approx(gbs, rel=1e-3)
+    assert h["frac"] == pytest.approx(gbs / 5000.0, rel=1e-3)
+    assert bench.roofline_of("no_such_kernel", 1, 1.0, CFG, ATTN, FFN, None) is None
+
+
+def test_kernel_table_shares():
+    t = bench.kernel_table({"attn_tc": (2, 30.0), "ffn_select": (1, 10.0)}, CFG, ATTN, FFN)
+    assert list(t) == ["attn_tc", "ffn_select"]      # largest share first
+    assert t["attn_tc"]["share"] == 0.75 and t["ffn_select"]["share"] == 0.25
+    assert t["attn_tc"]["ms_per_launch"] == 15.0
+    assert "tflops" in t["attn_tc"] and "gbs" in t["ffn_select"]
+
+
+def _write_profile(root, kernel, workload, nbytes, sha):
+    os.makedirs(os.path.join(root, "profiles"), exist_ok=True)
+    with open(os.path.join(root, "profiles", f"{kernel}_{workload}.md"), "w") as f:
+        f.write(f"# summary\n\n- traffic-bytes-per-launch: `{nbytes}`\n- source-sha256: `{sha}`\n")
+
+
+def test_traffic_tied_to_kernel_source(tmp_path, monkeypatch):
+    root = str(tmp_path)
+    csrc = os.path.join(root, "ffn_long_video_b200", "csrc")
+    os.makedirs(csrc)
+    src = b"// kernel source\n"
+    with open(os.path.join(csrc, "attn_tc.cu"), "wb") as f:
+        f.write(src)
+    monkeypatch.setattr(bench, "ROOT", root)
+    assert bench.load_traffic("attn_tc", "w") is None                     # no summary
+    _write_profile(root, "attn_tc", "w", 4096, hashlib.sha256(src).hexdigest())
+    assert bench.load_traffic("attn_tc", "w") == 4096                     # same source
+    with open(os.path.join(csrc, "attn_tc.cu"), "ab") as f:
+        f.write(b"// edited\n")
+    assert bench.load_traffic("attn_tc", "w") is None                     # source changed
+    _write_profile(root, "no_such_kernel", "w", 1, "0" * 64)
+    assert bench.load_traffic("no_such_kernel", "w") is None              # unknown kernel
+
+
+class _FakeProc:
+    stdout = iter(())
+
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+    def kill(self):
+        pass
+
+
+def test_clock_samples_inside_the_region():
+    s = bench.ClockSampler(0)
+    s.proc = _FakeProc()
+    s.t0, s.t1 = 100.0, 110.0
+
+    def line(mhz, cap="Not Active", thermal="Not Active"):
+        return f"0, {mhz}, 1965, 900.0, 0x4, Not Active, {thermal}, Not Active, {cap}"
+    s.lines = [(99.0, line(500, thermal="Active")),      # before the region: dropped
+               (101.0, line(1700, cap="Active")),
+               (105.0, line(1800)),
+               (110.05, line(1900)),                      # within one period after the end
+               (111.0, line(600, thermal="Active")),      # after it: dropped
+               (106.0, "garbled")]
+    r = s.stop()
+    assert r["samples"] == 3
+    assert r["sm_mhz"] == 1800.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_sampler_without_nvidia_smi():
+    s = bench.ClockSampler(0)
+    assert s.stop()["reasons"] == ["nvidia-smi unavailable"]
