@@ -26,7 +26,8 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device. The host-side
 // symbol is only a stand-in: the address is looked up once per device, with
-// that device current, and cached.
+// that device current, and cached for the life of the process (a
+// cudaDeviceReset would invalidate it; the header says so).
 int scratch_on_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ADASPARK_ECUDA;
@@ -51,8 +52,14 @@ extern "C" int adaspark_cube_attn_noalloc(const void* Q, const void* K, const vo
       adaspark_cube_attn_workspace(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype);
   if (need == 0) return ADASPARK_EINVAL;                       // invalid sizes
   if (need > (size_t)ADASPARK_NOALLOC_SCRATCH_BYTES) return ADASPARK_EINVAL;  // too large
+  // the device check comes first, so that a device without this library's
+  // device code reports ADASPARK_EUNSUPPORTED rather than a failed lookup
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ADASPARK_ECUDA;
+  int rc = adaspark_device_check(dev);
+  if (rc != ADASPARK_OK) return rc;
   void* scratch = nullptr;
-  const int rc = scratch_on_current_device(&scratch);
+  rc = scratch_on_current_device(&scratch);
   if (rc != ADASPARK_OK) return rc;
   // adaspark_cube_attn clears the parts of the workspace that must start at
   // zero (status word and counters) at the start of every call.

@@ -57,9 +57,12 @@ typedef enum { ADASPARK_BF16 = 0, ADASPARK_FP32 = 1 } adaspark_dtype;
 /* Bits of the device status word (adaspark_read_device_status detail). */
 #define ADASPARK_DEV_BAD_LAYOUT   0x1u  /* cube_ids / cube_offsets / text_mask inconsistent */
 #define ADASPARK_DEV_TIMEOUT      0x2u  /* a bounded wait inside a kernel expired          */
-#define ADASPARK_DEV_RANGE        0x4u  /* a row's largest cube score is out of range:     */
-                                        /* |q.kbar| * log2(e) / sqrt(d) must stay below    */
-                                        /* 2^18; such a row keeps only its own cube        */
+#define ADASPARK_DEV_RANGE        0x4u  /* a value left the range the kernels represent   */
+                                        /* exactly: AdaS-Attn: a row's largest cube score  */
+                                        /* |q.kbar| * log2(e) / sqrt(d) reached 2^20 (the  */
+                                        /* row then keeps only its own cube); AdaS-FFN: a  */
+                                        /* SwiGLU activation or a W_down weight beyond the */
+                                        /* fp16 range +-65504 (see adaspark_token_ffn)     */
 
 /* Human-readable name of a return code. Never NULL. */
 const char *adaspark_status_string(int status);
@@ -246,7 +249,12 @@ int adaspark_attn_read_stats(const void *workspace, adaspark_attn_stats *stats, 
  *     contents: calls whose kernels may overlap on the GPU (different streams
  *     without ordering between them) race and give wrong results; serialize
  *     them. adaspark_attn_export_sets / adaspark_attn_read_stats cannot read
- *     this array (use adaspark_cube_attn for those). */
+ *     this array (use adaspark_cube_attn for those).
+ *   - The cached address belongs to the device context it was looked up in:
+ *     after cudaDeviceReset() on a device, this entry point must not be called
+ *     on that device again in the same process.
+ *   - A device that is not sm_100 gives ADASPARK_EUNSUPPORTED before any
+ *     lookup. */
 #define ADASPARK_NOALLOC_SCRATCH_BYTES (32u << 20)
 int adaspark_cube_attn_noalloc(const void *Q, const void *K, const void *V, int dtype,
                                const int32_t *cube_ids, const int32_t *cube_offsets,
@@ -283,6 +291,13 @@ size_t adaspark_token_ffn_workspace(int n_tokens, int n_vis, int n_cubes, int D,
  *   p in (0, 1]; D % 64 == 0 and F % 128 == 0 for BF16 (D, F multiples of 4 for FP32);
  *   y [n_tokens, D]: device float32 (the residual stream is kept in fp32);
  *   workspace: device, >= adaspark_token_ffn_workspace(...) bytes, 256-byte aligned.
+ * Precision (BF16): the products accumulate in fp32; the SwiGLU activations
+ * feed the down projection as fp16 (3 more mantissa bits than bf16) and W_down
+ * is converted to fp16 for it (exact for |w| >= 2^-14, absolute error below
+ * 2^-25 under that). An activation whose magnitude exceeds 65504 (stored
+ * saturated) or a W_down weight beyond +-65504 sets ADASPARK_DEV_RANGE in the
+ * status word (detail code 0x65 and 0x66 respectively): the output then
+ * differs from the exact FFN and must not be used.
  * Errors as for adaspark_cube_attn. */
 int adaspark_token_ffn(const void *x, const void *W_gate, const void *W_up, const void *W_down,
                        int dtype, const int32_t *cube_ids, const int32_t *cube_offsets,

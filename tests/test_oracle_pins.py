@@ -658,3 +658,105 @@ def test_ffn_backward_dense_equals_autograd_and_skipped_rows():
     _, _, _, dWd_c0 = oracle.ffn_backward_given_sets(x[:6], Wg, Wu, Wd, off[:2], 6, active[:6],
                                                      dy[:6])
     assert np.abs(dWd_c0 - df0.T @ h).max() < 1e-12
+
+
+# ---------------------------------------------------------------- rounding scales, from above
+# The rounding scales returned with ``with_magnitudes`` widen the GPU gradient
+# bound, so an inflated scale would loosen the comparison. Above, they are
+# pinned from below (they dominate the gradients). Here they are pinned from
+# above: in cases where every term of a gradient element has one sign the
+# scale must equal the gradient's magnitude (attention) or exactly twice it
+# (FFN, where two roundings enter each term), so a scale inflated by any factor
+# fails; and each attention scale is compared with its sum of absolute terms
+# written out one term at a time.
+
+def test_attention_magnitudes_equal_gradients_for_single_terms():
+    """Query row 1 of cube 0 admits keys 0 and 1; with K_1 = 0 its dQ has the
+    single term dS_10 K_0 / sqrt(d), so mQ = |dQ| there. The last key of the
+    last cube (no text, one query head per KV head) is admitted by its own row
+    only, so mK = |dK| there. With dO > 0 every P^T dO term is positive, so
+    mV = dV everywhere."""
+    rng = np.random.default_rng(31)
+    off = np.array([0, 2, 4, 7])
+    n_vis, hq, hkv, d = 7, 2, 2, 5
+    Q, K, V = _qkv(rng, n_vis, hq, hkv, d)
+    K[1] = 0.0                 # row 1 sees keys {0, 1}: only key 0 contributes to dQ
+    K[4] = 0.0                 # row 5 (cube 2, second token) sees {4, 5} + selections
+    sel = np.zeros((n_vis, hq, 3), dtype=bool)
+    dO = rng.standard_normal((n_vis, hq, d))
+    dQ, dK, dV, (mQ, mK, mV) = oracle.attention_backward_given_sets(
+        Q, K, V, dO, off, n_vis, sel, with_magnitudes=True)
+    for t in (1, 5):
+        assert np.abs(dQ[t]).min() > 1e-6                 # the case is not degenerate
+        np.testing.assert_allclose(mQ[t], np.abs(dQ[t]), rtol=1e-12, atol=0)
+    np.testing.assert_allclose(mK[n_vis - 1], np.abs(dK[n_vis - 1]), rtol=1e-12, atol=0)
+    assert np.abs(dK[n_vis - 1]).min() > 1e-6
+    _, _, dVp, (_, _, mVp) = oracle.attention_backward_given_sets(
+        Q, K, V, np.abs(dO) + 0.1, off, n_vis, sel, with_magnitudes=True)
+    np.testing.assert_allclose(mVp, dVp, rtol=1e-12, atol=0)
+
+
+def test_attention_magnitudes_term_by_term():
+    """mQ, mK and mV equal their sums of absolute terms, taken one (row, key)
+    term at a time; the row's probabilities are read from the pinned forward
+    (one-hot values make the output the probability vector itself)."""
+    rng = np.random.default_rng(32)
+    off = np.array([0, 3, 5, 8])
+    n_vis, n_text, hq, hkv, d = 8, 2, 4, 2, 3
+    N = n_vis + n_text
+    g = hq // hkv
+    Q, K, V = _qkv(rng, N, hq, hkv, d)
+    sel = rng.random((N, hq, 3)) < 0.5
+    dO = rng.standard_normal((N, hq, d))
+    *_, (mQ, mK, mV) = oracle.attention_backward_given_sets(Q, K, V, dO, off, n_vis, sel,
+                                                            with_magnitudes=True)
+    # P[t, h, u] from the forward with one-hot values (head dim N for V)
+    onehot = np.zeros((N, hkv, N))
+    for u in range(N):
+        onehot[u, :, u] = 1.0
+    Qp = np.zeros((N, hq, N))
+    Kp = np.zeros((N, hkv, N))
+    Qp[:, :, :d] = Q * math.sqrt(N / d)     # same logits at head dim N
+    Kp[:, :, :d] = K
+    P = oracle.attention_given_sets(Qp, Kp, onehot, off, n_vis, sel)
+    wQ, wK, wV = np.zeros_like(Q), np.zeros_like(K), np.zeros_like(V)
+    for t in range(N):
+        for h in range(hq):
+            kv = h // g
+            dP = [float(dO[t, h] @ V[u, kv]) for u in range(N)]
+            D = sum(P[t, h, u] * dP[u] for u in range(N))
+            for u in range(N):
+                if P[t, h, u] == 0.0:
+                    continue
+                dS = P[t, h, u] * (dP[u] - D)
+                for c in range(d):
+                    wQ[t, h, c] += abs(dS) * abs(K[u, kv, c]) / math.sqrt(d)
+                    wK[u, kv, c] += abs(dS) * abs(Q[t, h, c]) / math.sqrt(d)
+                    wV[u, kv, c] += P[t, h, u] * abs(dO[t, h, c])
+    for m, w in ((mQ, wQ), (mK, wK), (mV, wV)):
+        np.testing.assert_allclose(m, w, rtol=1e-9, atol=1e-12)
+
+
+def test_ffn_magnitudes_twice_the_gradients_when_terms_are_positive():
+    """With x, the three weights and dy all positive, every term of every
+    gradient is positive, and each rounding scale counts each term twice (df and
+    dg / du / h each rounded once): the scales equal exactly twice the
+    gradients (dx without its dy part)."""
+    rng = np.random.default_rng(33)
+    D, F = 5, 7
+    off = np.array([0, 3, 4, 8])
+    n_vis, n_text = 8, 2
+    N = n_vis + n_text
+    x = rng.random((N, D)) + 0.1
+    Wg, Wu, Wd = (rng.random(s) * 0.5 + 0.05 for s in ((F, D), (F, D), (D, F)))
+    active = np.array([True, False, True, True, True, False, True, False, True, True])
+    dy = rng.random((N, D)) + 0.1
+    (dx, dWg, dWu, dWd), (mdx, mWg, mWu, mWd) = oracle.ffn_backward_given_sets(
+        x, Wg, Wu, Wd, off, n_vis, active, dy, with_magnitudes=True)
+    rows = active.copy()
+    rows[n_vis:] = True
+    np.testing.assert_allclose(mdx[rows], 2.0 * (dx - dy)[rows], rtol=1e-12, atol=0)
+    assert not mdx[~rows].any()
+    for m, gr in ((mWg, dWg), (mWu, dWu), (mWd, dWd)):
+        assert gr.min() > 0.0
+        np.testing.assert_allclose(m, 2.0 * gr, rtol=1e-12, atol=0)
