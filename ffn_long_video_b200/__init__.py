@@ -104,6 +104,7 @@ def lib():
             "adaspark_timer_read": (i32, [ctypes.POINTER(_KernelTime), i32, ctypes.POINTER(i32)]),
             "adaspark_launch_count": (ctypes.c_uint64, []),
             "adaspark_device_check": (i32, [i32]),
+            "adaspark_debug_wait_expiry": (i32, [i32, ctypes.c_longlong]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -478,6 +479,14 @@ def timer_read(max_entries: int = 64) -> dict:
     _check(lib().adaspark_timer_read(buf, max_entries, ctypes.byref(n)), "adaspark_timer_read")
     return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms))
             for i in range(n.value)}
+
+
+def debug_wait_expiry(on: bool, wait_cycles: int = 2_000_000):
+    """Test hook of the bounded waits (adaspark_debug_wait_expiry): while on,
+    bf16 AdaS-Attn launches withhold their first key block and give up after
+    wait_cycles SM cycles, reporting ADASPARK_DEV_TIMEOUT."""
+    _check(lib().adaspark_debug_wait_expiry(1 if on else 0, int(wait_cycles)),
+           "adaspark_debug_wait_expiry")
 
 
 def launch_count() -> int:

@@ -44,6 +44,11 @@ bool ffn_sizes_ok(int n_tokens, int n_vis, int n_cubes, int D, int F, int dtype)
 
 int cuda_rc(cudaError_t e) { return e == cudaSuccess ? ADASPARK_OK : ADASPARK_ECUDA; }
 
+// Test hook of the bounded waits (adaspark_debug_wait_expiry): the wait limit
+// of the bf16 attention kernel and whether its first descriptor is withheld.
+long long g_attn_wait_limit = kWaitCycles;
+int g_attn_withhold_first = 0;
+
 }  // namespace
 
 extern "C" {
@@ -134,6 +139,8 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   aa.scale_log2 = sa.zscale;
   aa.lse = reinterpret_cast<float*>(ws + L.lse);
   aa.o32 = train ? reinterpret_cast<float*>(ws + L.total) : nullptr;
+  aa.wait_limit = g_attn_wait_limit;
+  aa.withhold_first = g_attn_withhold_first;
   // When the layer's K and V outgrow what L2 holds alongside the other
   // traffic, visual tiles run one KV head after another, so that the blocks in
   // use belong to one head; otherwise all heads of a token range run together
@@ -448,6 +455,18 @@ int adaspark_ffn_read_stats(const void* workspace, adaspark_ffn_stats* stats, vo
   const WsHeader* hdr = static_cast<const WsHeader*>(workspace);
   static_assert(sizeof(adaspark_ffn_stats) == sizeof(hdr->stats), "stats size");
   return cuda_rc(cudaMemcpy(stats, hdr->stats, sizeof(adaspark_ffn_stats), cudaMemcpyDeviceToHost));
+}
+
+int adaspark_debug_wait_expiry(int on, long long wait_cycles) {
+  if (!on) {
+    g_attn_wait_limit = kWaitCycles;
+    g_attn_withhold_first = 0;
+    return ADASPARK_OK;
+  }
+  if (wait_cycles < 100000 || wait_cycles > kWaitCycles) return ADASPARK_EINVAL;
+  g_attn_wait_limit = wait_cycles;
+  g_attn_withhold_first = 1;
+  return ADASPARK_OK;
 }
 
 int adaspark_read_device_status(const void* workspace, uint32_t* detail, void* stream) {

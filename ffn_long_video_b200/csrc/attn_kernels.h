@@ -40,6 +40,8 @@ struct AttnArgs {
   int kv_major;                       // visual tiles ordered one KV head after another
   float* lse;                         // [N][hq] m + log2(l) per row (bf16 path), for the backward
   float* o32;                         // [N][hq][d] fp32 O with P split hi + lo (training), or null
+  long long wait_limit;               // SM cycles before a wait gives up (bf16 kernel)
+  int withhold_first;                 // test hook: the first descriptor is never announced
 };
 
 // Backward of AdaS-Attn (sets of a forward call held fixed).

@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   const AttnGeom& G = a.G;
   WsHeader* hdr = a.hdr;
   const TileInfo T = decode_tile(G, a.kv_major != 0);
+  const long long WL = a.wait_limit;  // cycles before any wait of this kernel gives up
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -197,7 +198,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       int idx = base + incl - nb;
       for (int b = 0; b < nb; ++b, ++idx) {
         const int slot = idx % RING;
-        if (!mbar_wait(&r_empty[slot], ((idx / RING) & 1) ^ 1, &s_abort, hdr, 0x7a00u)) {
+        if (!mbar_wait(&r_empty[slot], ((idx / RING) & 1) ^ 1, &s_abort, hdr, 0x7a00u, WL)) {
           ok = false;
           break;
         }
@@ -209,16 +210,19 @@ __global__ void __launch_bounds__(THREADS, 2)
         d.mask[1] = m.y;
         d.mask[2] = m.z;
         d.mask[3] = m.w;
-        mbar_arrive(&r_full[slot]);
+        // (test hook: with withhold_first the first descriptor is never
+        // announced, so every wait for it runs out and the kernel reports
+        // ADASPARK_DEV_TIMEOUT)
+        if (!(a.withhold_first && idx == 0)) mbar_arrive(&r_full[slot]);
       }
       ok = __all_sync(0xffffffffu, ok);
       base += total;
     }
     if (ok && lane == 0) {  // terminal descriptor
       const int slot = base % RING;
-      if (mbar_wait(&r_empty[slot], ((base / RING) & 1) ^ 1, &s_abort, hdr, 0x7b00u)) {
+      if (mbar_wait(&r_empty[slot], ((base / RING) & 1) ^ 1, &s_abort, hdr, 0x7b00u, WL)) {
         ring[slot].nk = 0;
-        mbar_arrive(&r_full[slot]);
+        if (!(a.withhold_first && base == 0)) mbar_arrive(&r_full[slot]);
       }
     }
   } else if (warp == 0) {
@@ -232,7 +236,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       bool ok = true;
       auto load_v = [&](int blk, int k0) -> bool {
         const int s = blk % STAGES;
-        if (!mbar_wait(&v_empty[s], ((blk / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7110u)) return false;
+        if (!mbar_wait(&v_empty[s], ((blk / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7110u, WL)) return false;
         mbar_expect_tx(&v_full[s], K_BYTES);
         tma_load_3d(&mapV, &v_full[s], sV + s * K_BYTES, 0, T.kv, k0);
         tma_load_3d(&mapV, &v_full[s], sV + s * K_BYTES + 8192, 64, T.kv, k0);
@@ -241,14 +245,14 @@ __global__ void __launch_bounds__(THREADS, 2)
       };
       while (ok) {
         const int slot = i % RING;
-        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7000u)) {
+        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7000u, WL)) {
           ok = false;
           break;
         }
         const int k0 = ring[slot].k0, nk = ring[slot].nk;
         if (nk == 0) break;
         const int s = i % STAGES;
-        if (!mbar_wait(&k_empty[s], ((i / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7100u)) {
+        if (!mbar_wait(&k_empty[s], ((i / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7100u, WL)) {
           ok = false;
           break;
         }
@@ -268,10 +272,10 @@ __global__ void __launch_bounds__(THREADS, 2)
           long long t0 = clock64();
           const int jk = i - 1 - k, jv = nv - 1 - k;
           while (jk >= 0 && !mbar_try_wait(&k_full[jk % STAGES], (jk / STAGES) & 1) &&
-                 clock64() - t0 < kWaitCycles) {
+                 clock64() - t0 < WL) {
           }
           while (jv >= 0 && !mbar_try_wait(&v_full[jv % STAGES], (jv / STAGES) & 1) &&
-                 clock64() - t0 < kWaitCycles) {
+                 clock64() - t0 < WL) {
           }
         }
       }
@@ -282,14 +286,14 @@ __global__ void __launch_bounds__(THREADS, 2)
       constexpr uint32_t idesc_s = make_idesc_bf16(128, 64);
       constexpr uint32_t idesc_o = make_idesc_bf16(128, 128, true);
       const uint32_t q_addr = smem_u32(sQ);
-      bool ok = mbar_wait(q_full, 0, &s_abort, hdr, 0x7200u);
+      bool ok = mbar_wait(q_full, 0, &s_abort, hdr, 0x7200u, WL);
       tc_fence_after();
       int i = 0;
       auto issue_pv = [&](int blk) -> bool {
         const int pb = blk & 1;
-        if (!mbar_wait(&p_full[pb], (blk >> 1) & 1, &s_abort, hdr, 0x7300u)) return false;
+        if (!mbar_wait(&p_full[pb], (blk >> 1) & 1, &s_abort, hdr, 0x7300u, WL)) return false;
         const int s = blk % STAGES;
-        if (!mbar_wait(&v_full[s], (blk / STAGES) & 1, &s_abort, hdr, 0x7310u)) return false;
+        if (!mbar_wait(&v_full[s], (blk / STAGES) & 1, &s_abort, hdr, 0x7310u, WL)) return false;
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sKV + STAGES * K_BYTES + s * K_BYTES);
         const uint32_t p_tmem = tmem_base + 128 + pb * 64;
@@ -305,14 +309,14 @@ __global__ void __launch_bounds__(THREADS, 2)
       };
       while (ok) {
         const int slot = i % RING;
-        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7d00u)) {
+        if (!mbar_wait(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7d00u, WL)) {
           ok = false;
           break;
         }
         if (ring[slot].nk == 0) break;
         const int s = i % STAGES;
         const int sb = i & 1;
-        if (!mbar_wait(&k_full[s], (i / STAGES) & 1, &s_abort, hdr, 0x7400u)) {
+        if (!mbar_wait(&k_full[s], (i / STAGES) & 1, &s_abort, hdr, 0x7400u, WL)) {
           ok = false;
           break;
         }
@@ -338,7 +342,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (ok && i > 0) issue_pv(i - 1);
       umma_commit(drain);
       long long t0 = clock64();
-      while (!mbar_try_wait(drain, 0) && clock64() - t0 < kWaitCycles) {
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < WL) {
       }
     }
   } else {
@@ -367,7 +371,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     bool ok = true;
     while (true) {
       const int slot = i % RING;
-      if (!mbar_wait_warp(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7e00u)) {
+      if (!mbar_wait_warp(&r_full[slot], (i / RING) & 1, &s_abort, hdr, 0x7e00u, WL)) {
         ok = false;
         break;
       }
@@ -387,7 +391,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (row_on && (T.text || d_j == own)) lim = min(lim, t - d_k0 + 1);
       if (lim <= 0) row_on = false;
       const int sb = i & 1;
-      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0x7600u)) {
+      if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0x7600u, WL)) {
         ok = false;
         break;
       }
@@ -456,7 +460,7 @@ __global__ void __launch_bounds__(THREADS, 2)
                                                                          : ex2(m_used - m_new);
         if (i > 0) {
           if (!mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr,
-                              0x7700u)) {
+                              0x7700u, WL)) {
             ok = false;
             break;
           }
@@ -524,7 +528,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     // final: O / l once the last PV has landed
     if (ok && i > 0 &&
-        mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr, 0x7900u)) {
+        mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr, 0x7900u, WL)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       // the row's softmax is 2^(s * scale - lse): kept for the backward pass

@@ -119,19 +119,21 @@ __device__ __forceinline__ bool mbar_try_wait_parked(uint64_t* bar, uint32_t par
   return ok != 0;
 }
 
-// A wait that gives up after ~2^31 SM cycles (about a second): on expiry it
-// records ADASPARK_DEV_TIMEOUT, raises the CTA-wide abort flag and returns
-// false so the caller can leave its loop. It also returns false at once when
-// another thread of the CTA has raised the abort flag.
+// A wait that gives up after `limit` SM cycles (by default ~2^31, about a
+// second): on expiry it records ADASPARK_DEV_TIMEOUT, raises the CTA-wide
+// abort flag and returns false so the caller can leave its loop. It also
+// returns false at once when another thread of the CTA has raised the abort
+// flag.
 constexpr long long kWaitCycles = 2000000000LL;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          WsHeader* hdr, uint32_t where) {
+                                          WsHeader* hdr, uint32_t where,
+                                          long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long start = clock64();
   while (true) {
     if (mbar_try_wait_parked(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - start > kWaitCycles) {
+    if (clock64() - start > limit) {
       *abort_flag = 1;
       set_status(hdr, ADASPARK_DEV_TIMEOUT, where);
       return false;
@@ -143,8 +145,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // saw the phase complete (so warp-collective tcgen05 ops after it never diverge).
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
                                                volatile int* abort_flag, WsHeader* hdr,
-                                               uint32_t where) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, hdr, where);
+                                               uint32_t where, long long limit = kWaitCycles) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, hdr, where, limit);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(wq * 32) << 16) + b * BN;
       if (MODE == 0) {
         __half* H = reinterpret_cast<__half*>(P.f.h);
+        float hmax = 0.f;  // largest |h| of this row's slice, before the fp16 store
 #pragma unroll 1
         for (int c = 0; c < 128; c += 32) {
           uint32_t g[32], u[32];
@@ -243,6 +244,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               const float h0 = silu(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
               const float h1 =
                   silu(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              hmax = fmaxf(hmax, fmaxf(fabsf(h0), fabsf(h1)));
               pk[i] = pack_f16x2_sat(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(H + (size_t)m * P.f.F + n0);
@@ -251,6 +253,9 @@ __global__ void __launch_bounds__(THREADS, 1)
               dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
           }
         }
+        // an activation beyond the fp16 range was stored saturated: the down
+        // projection would then differ from the exact FFN
+        if (hmax > 65504.f) set_status(hdr, ADASPARK_DEV_RANGE, 0x6500u);
       } else if (MODE == 2) {
 #pragma unroll 1
         for (int c = 0; c < BN; c += 32) {
@@ -370,11 +375,13 @@ static bool map_rows(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
   return encode_tmap_16(m, base, 2, dims, strides, box, fp16);
 }
 
-// W_down bf16 -> fp16 (exact for |w| >= 2^-14; smaller magnitudes keep an
-// absolute error below 2^-25). 8 elements per thread.
+// W_down bf16 -> fp16 (exact for 2^-14 <= |w| <= 65504; smaller magnitudes
+// keep an absolute error below 2^-25; a weight beyond +-65504 would become
+// infinite and sets ADASPARK_DEV_RANGE). 8 elements per thread.
 __global__ void wdown_to_fp16_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst,
                                      size_t n8, WsHeader* hdr) {
   if (status_bad(hdr)) return;
+  float wmax = 0.f;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
        i += (size_t)gridDim.x * blockDim.x) {
     const uint4 v = reinterpret_cast<const uint4*>(src)[i];
@@ -384,11 +391,13 @@ __global__ void wdown_to_fp16_kernel(const __nv_bfloat16* __restrict__ src, __ha
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float2 f = __bfloat1622float2(b[k]);
+      wmax = fmaxf(wmax, fmaxf(fabsf(f.x), fabsf(f.y)));
       const __half2 hv = __floats2half2_rn(f.x, f.y);
       op[k] = *reinterpret_cast<const uint32_t*>(&hv);
     }
     reinterpret_cast<uint4*>(dst)[i] = o;
   }
+  if (wmax > 65504.f) set_status(hdr, ADASPARK_DEV_RANGE, 0x6600u);
 }
 
 cudaError_t launch_wdown_to_fp16(const FfnArgs& a, cudaStream_t s) {

@@ -296,7 +296,7 @@ size_t adaspark_token_ffn_workspace(int n_tokens, int n_vis, int n_cubes, int D,
  * is converted to fp16 for it (exact for |w| >= 2^-14, absolute error below
  * 2^-25 under that). An activation whose magnitude exceeds 65504 (stored
  * saturated) or a W_down weight beyond +-65504 sets ADASPARK_DEV_RANGE in the
- * status word (detail code 0x65 and 0x66 respectively): the output then
+ * status word (internal codes 0x65xx and 0x66xx of the detail): the output then
  * differs from the exact FFN and must not be used.
  * Errors as for adaspark_cube_attn. */
 int adaspark_token_ffn(const void *x, const void *W_gate, const void *W_up, const void *W_down,
@@ -433,6 +433,20 @@ int adaspark_rmsnorm(const void *x, int x_dtype, const void *weight, void *out, 
  * ADASPARK_DEV_* bits in bits 0-7 and an internal code of the first failing
  * check in bits 8-23. The word is cleared by the next call on the workspace. */
 int adaspark_read_device_status(const void *workspace, uint32_t *detail, void *stream);
+
+/* Test hook for the bounded waits inside the kernels (not for production use;
+ * the AdaSpark pages have no counterpart). Every wait on another warp or on the
+ * tensor core is bounded; when a bound runs out the kernel records
+ * ADASPARK_DEV_TIMEOUT, lets its issued copies and products finish, frees its
+ * tensor memory and returns, and the device stays usable. With on != 0, every
+ * later bf16 adaspark_cube_attn / _topk / _train launch of this process runs
+ * its attention kernel with waits bounded by wait_cycles SM cycles (1e5 ..
+ * 2e9) and withholds the announcement of each tile's first key block, so those
+ * waits run out: the call then reports ADASPARK_EDEVICE with
+ * ADASPARK_DEV_TIMEOUT. on == 0 restores the normal bound (about 2e9 cycles)
+ * and behaviour. Process-wide, not thread-safe; ADASPARK_EINVAL for a bound
+ * outside the range. */
+int adaspark_debug_wait_expiry(int on, long long wait_cycles);
 
 /* Per-kernel timing with CUDA events recorded on the launching stream around
  * each launch of this library. Off by default; process-wide; not thread-safe. */

@@ -96,3 +96,68 @@ def test_score_range_is_flagged_and_device_stays_usable():
     Q, K, V, ids, off = _small_inputs(scale=1.0)
     code, detail = _attn_status(Q, K, V, ids, off, 256)
     assert code == fb.OK, (code, detail)
+
+
+# AdaS-FFN feeds the down projection in fp16: values beyond its range must be
+# reported, not silently saturated or turned into infinities.
+_FFN_RANGE_CFG = workloads.small_config(name="ffn-range", grid=(4, 8, 8), cube=(4, 4, 4),
+                                        n_text=16, D=256, hq=4, hkv=1, F=512, seed=61)
+
+
+def _ffn_status(case, **weights):
+    t = dict(case["t"], **weights)
+    cfg = case["cfg"]
+    y, ws = fb.token_ffn(t["x"], t["W_gate"], t["W_up"], t["W_down"], case["ids"], case["off"],
+                         case["text"], cfg.n_vis, cfg.p)
+    torch.cuda.synchronize()
+    return fb.read_device_status(ws)
+
+
+def test_ffn_activation_beyond_fp16_is_flagged_and_device_stays_usable():
+    """Gate and up weights scaled 1000x make silu(g) * u reach ~1e5 > 65504: the
+    fp16 store would saturate, so RANGE is reported (code 0x65xx); the same
+    layer with its own weights then runs clean."""
+    case = parity.make_case(_FFN_RANGE_CFG)
+    t = case["t"]
+    code, detail = _ffn_status(case, W_gate=(t["W_gate"].float() * 1000).to(torch.bfloat16),
+                               W_up=(t["W_up"].float() * 1000).to(torch.bfloat16))
+    assert code == fb.EDEVICE and (detail & fb.DEV_RANGE), (code, hex(detail))
+    assert (detail >> 8) & 0xff00 == 0x6500, hex(detail)
+    code, detail = _ffn_status(case)
+    assert code == fb.OK, (code, hex(detail))
+
+
+def test_ffn_wdown_beyond_fp16_is_flagged():
+    """One W_down weight of 70144 (a bf16 value above the fp16 maximum 65504)
+    would become infinite in the fp16 copy: RANGE is reported (code 0x66xx)."""
+    case = parity.make_case(_FFN_RANGE_CFG)
+    wd = case["t"]["W_down"].clone()
+    wd[3, 7] = 70000.0
+    assert float(wd[3, 7]) > 65504.0
+    code, detail = _ffn_status(case, W_down=wd)
+    assert code == fb.EDEVICE and (detail & fb.DEV_RANGE), (code, hex(detail))
+    assert (detail >> 8) & 0xff00 == 0x6600, hex(detail)
+
+
+def test_bounded_wait_expiry_reports_timeout_and_device_stays_usable():
+    """Every wait inside the attention kernel is bounded. The test hook makes
+    each tile withhold the announcement of its first key block and bounds the
+    waits by 2e6 SM cycles (about a millisecond): the producer, the MMA issuer
+    and the softmax warps wait for a descriptor that never comes, give up,
+    report ADASPARK_DEV_TIMEOUT (a location code 0x7xxx of this kernel), free
+    their tensor memory and return. A normal call afterwards on the same device
+    succeeds and matches the oracle."""
+    cfg = workloads.small_config(name="wait-expiry", grid=(4, 8, 8), cube=(4, 4, 4), n_text=16,
+                                 D=256, hq=4, hkv=1, F=256, seed=62)
+    case = parity.make_case(cfg)
+    t = case["t"]
+    fb.debug_wait_expiry(True, 2_000_000)
+    try:
+        _, ws = fb.cube_attn(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis, cfg.p)
+        torch.cuda.synchronize()
+        code, detail = fb.read_device_status(ws)
+    finally:
+        fb.debug_wait_expiry(False)
+    assert code == fb.EDEVICE and (detail & fb.DEV_TIMEOUT), (code, hex(detail))
+    assert (detail >> 8) & 0xf000 == 0x7000, hex(detail)
+    parity.check_attn(case)
