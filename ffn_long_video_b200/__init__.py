@@ -40,12 +40,14 @@ class _AttnStats(ctypes.Structure):
     _fields_ = [("visual_rows", ctypes.c_uint64), ("candidate_pairs", ctypes.c_uint64),
                 ("selected_pairs", ctypes.c_uint64), ("overflow_rows", ctypes.c_uint64),
                 ("tiles", ctypes.c_uint64), ("key_blocks", ctypes.c_uint64),
-                ("key_block_keys", ctypes.c_uint64), ("reserved", ctypes.c_uint64 * 9)]
+                ("key_block_keys", ctypes.c_uint64), ("near_margin_rows", ctypes.c_uint64),
+                ("reserved", ctypes.c_uint64 * 8)]
 
 
 class _FfnStats(ctypes.Structure):
     _fields_ = [("active_visual", ctypes.c_uint64), ("skipped_visual", ctypes.c_uint64),
-                ("text_tokens", ctypes.c_uint64), ("reserved", ctypes.c_uint64 * 13)]
+                ("text_tokens", ctypes.c_uint64), ("near_margin_cubes", ctypes.c_uint64),
+                ("reserved", ctypes.c_uint64 * 12)]
 
 
 class _KernelTime(ctypes.Structure):
@@ -76,6 +78,8 @@ def lib():
                                                                                    vp]),
             "adaspark_cube_attn_topk": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 7 + [vp, vp, sz,
                                                                                     vp]),
+            "adaspark_cube_attn_uniform": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 7 +
+                                           [vp, vp, sz, vp]),
             "adaspark_cube_attn_train_workspace": (sz, [i32] * 7),
             "adaspark_cube_attn_train": (i32, [vp, vp, vp, i32, vp, vp] + [i32] * 6 + [f32, vp, vp,
                                                                                    sz, vp]),
@@ -242,6 +246,33 @@ def cube_attn_topk(Q, K, V, cube_ids, cube_offsets, n_vis, k, out=None, workspac
     return out, workspace
 
 
+def cube_attn_uniform(Q, K, V, cube_ids, cube_offsets, n_vis, k, out=None, workspace=None,
+                      stream=None):
+    """AdaS-Attn with Uniform Sampling (k evenly spaced preceding cubes);
+    returns (out, workspace)."""
+    import torch
+    for t, nm in ((Q, "Q"), (K, "K"), (V, "V"), (cube_ids, "cube_ids"),
+                  (cube_offsets, "cube_offsets")):
+        _need(t, nm)
+    N, hq, d = Q.shape
+    hkv = K.shape[1]
+    C = cube_offsets.numel() - 1
+    dt = _dtype_code(Q)
+    if out is None:
+        out = torch.empty_like(Q)
+    if workspace is None:
+        nb = cube_attn_workspace_bytes(N, n_vis, C, hq, hkv, d, dt)
+        if nb == 0:
+            raise AdasparkError(EINVAL, "adaspark_cube_attn_workspace")
+        workspace = torch.empty(nb, dtype=torch.uint8, device=Q.device)
+    _check(lib().adaspark_cube_attn_uniform(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(cube_ids),
+                                            _ptr(cube_offsets), C, n_vis, N, hq, hkv, d, int(k),
+                                            _ptr(out), _ptr(workspace), workspace.numel(),
+                                            _stream(stream)),
+           "adaspark_cube_attn_uniform")
+    return out, workspace
+
+
 def attn_export_sets(workspace, cube_ids, n_cubes, n_vis, n_tokens, hq, hkv, d, dtype,
                      stream=None):
     """Selected sets of the last cube_attn call as a bool tensor [n_vis, hq, C] (host)."""
@@ -256,6 +287,21 @@ def attn_export_sets(workspace, cube_ids, n_cubes, n_vis, n_tokens, hq, hkv, d, 
     unpacked = np.unpackbits(b.view(np.uint8).reshape(n_vis, hq, W * 4), axis=-1,
                              bitorder="little")
     return unpacked[:, :, :n_cubes].astype(bool)
+
+
+def attn_export_bits(workspace, cube_ids, n_cubes, n_vis, n_tokens, hq, hkv, d, dtype,
+                     stream=None):
+    """Selected sets of the last cube_attn call as packed bits on the device:
+    int32 [n_vis, hq, ceil(C/32)], bit j of row (t, h) set when cube j is in
+    its set (the own cube is not marked)."""
+    import torch
+    W = (n_cubes + 31) // 32
+    bits = torch.zeros(max(n_vis, 1) * hq * W, dtype=torch.int32, device=workspace.device)
+    _check(lib().adaspark_attn_export_sets(_ptr(workspace), _ptr(cube_ids), n_cubes, n_vis,
+                                           n_tokens, hq, hkv, d, dtype, _ptr(bits),
+                                           _stream(stream)),
+           "adaspark_attn_export_sets")
+    return bits[: n_vis * hq * W].view(n_vis, hq, W)
 
 
 def attn_read_stats(workspace, stream=None) -> dict:

@@ -72,7 +72,7 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
                           const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
                           int n_vis, int n_tokens, int hq, int hkv, int d, float p, int topk,
                           void* out, void* workspace, size_t workspace_bytes, void* stream,
-                          bool train = false) {
+                          bool train = false, bool uniform = false) {
   if (!Q || !K || !V || !cube_ids || !cube_offsets || !out || !workspace) return ADASPARK_EINVAL;
   if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return ADASPARK_EINVAL;
   if (topk < 0 || (topk == 0 && !p_valid(p))) return ADASPARK_EINVAL;
@@ -115,7 +115,10 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   sa.zscale = (float)(1.4426950408889634 / std::sqrt((double)d));
   sa.topk = topk;
 
-  if (!dense && n_vis > 0 && G.n_vtiles > 0) {
+  if (uniform && n_vis > 0 && G.n_vtiles > 0) {
+    rc = cuda_rc(launch_select_uniform(sa, s));
+    if (rc) return rc;
+  } else if (!dense && n_vis > 0 && G.n_vtiles > 0) {
     rc = cuda_rc(launch_cube_mean(K, dtype, cube_offsets, const_cast<float*>(sa.kbar),
                                   const_cast<__nv_bfloat16*>(sa.kbar_split), G, hdr, s));
     if (rc) return rc;
@@ -184,6 +187,15 @@ int adaspark_cube_attn_topk(const void* Q, const void* K, const void* V, int dty
   if (k < 1) return ADASPARK_EINVAL;
   return cube_attn_impl(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq, hkv,
                         d, 0.5f, k, out, workspace, workspace_bytes, stream);
+}
+
+int adaspark_cube_attn_uniform(const void* Q, const void* K, const void* V, int dtype,
+                               const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                               int n_vis, int n_tokens, int hq, int hkv, int d, int k, void* out,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (k < 1) return ADASPARK_EINVAL;
+  return cube_attn_impl(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq, hkv,
+                        d, 0.5f, k, out, workspace, workspace_bytes, stream, false, true);
 }
 
 int adaspark_attn_export_sets(const void* workspace, const int32_t* cube_ids, int n_cubes,

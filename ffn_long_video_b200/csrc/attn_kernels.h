@@ -94,6 +94,7 @@ cudaError_t launch_cube_mean(const void* K, int dtype, const int32_t* off, float
                              cudaStream_t s);
 cudaError_t launch_select_simt(const SelectArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_select_tc(const SelectArgs& a, cudaStream_t s);
+cudaError_t launch_select_uniform(const SelectArgs& a, cudaStream_t s);
 cudaError_t launch_export_sets(const int32_t* tile_count, const uint16_t* tile_list,
                                const uint32_t* tile_mask, const int32_t* cube_ids,
                                const AttnGeom& G, int dense, uint32_t* bits, cudaStream_t s);

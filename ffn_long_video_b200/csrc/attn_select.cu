@@ -179,11 +179,13 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
   const unsigned v_cand = __reduce_add_sync(0xffffffffu, (unsigned)ncand);
   const unsigned v_sel = __reduce_add_sync(0xffffffffu, (unsigned)nsel);
   const unsigned v_ext = __reduce_add_sync(0xffffffffu, (unsigned)extra);
+  const unsigned v_near = __reduce_add_sync(0xffffffffu, (valid && s.near) ? 1u : 0u);
   if (lane == 0) {
     atomicAdd((unsigned long long*)&a.hdr->stats[0], (unsigned long long)v_rows);
     atomicAdd((unsigned long long*)&a.hdr->stats[1], (unsigned long long)v_cand);
     atomicAdd((unsigned long long*)&a.hdr->stats[2], (unsigned long long)v_sel);
     atomicAdd((unsigned long long*)&a.hdr->stats[3], (unsigned long long)v_ext);
+    if (v_near) atomicAdd((unsigned long long*)&a.hdr->stats[7], (unsigned long long)v_near);
   }
   __threadfence_block();
   __syncthreads();
@@ -262,6 +264,60 @@ cudaError_t launch_select_simt(const SelectArgs& a, int dtype, cudaStream_t s) {
     return launch_select_simt_t<float, 128>(a, s);
   }
   return launch_select_simt_t<__nv_bfloat16, 128>(a, s);
+}
+
+// ---------------------------------------------------------------------------
+// Uniform Sampling (the content-independent strategy of the AdaSpark paper's
+// selection-strategy ablation, read as k of the i preceding cubes at even
+// spacing from the first, floor(m i / k), or all of them when i <= k): the
+// tile masks and lists of the attention written directly, without scores.
+// One CTA of 128 threads (one per row) per visual tile.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool uniform_member(int i, int k, int j) {
+  if (j >= i) return false;
+  if (i <= k) return true;
+  // the smallest m with m i / k >= j is ceil(j k / i); j is taken when it maps back to j
+  const long long m = ((long long)j * k + i - 1) / i;
+  return m < k && (m * i) / k == j;
+}
+
+__global__ void __launch_bounds__(128) select_uniform_kernel(SelectArgs a) {
+  __shared__ int s_hi, s_wcnt[4];
+  const AttnGeom& G = a.G;
+  const int vt = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (status_bad(a.hdr)) return;
+  const TileRow R = tile_row(G, false, vt, tid);
+  const int own = R.valid ? a.cube_ids[R.t] : -1;
+  if (tid == 0) s_hi = -1;
+  __syncthreads();
+  if (R.valid) atomicMax(&s_hi, own);
+  __syncthreads();
+  const int c_hi = s_hi;
+  if (c_hi < 0) return;
+  uint32_t* tmask = a.tile_mask + (size_t)vt * G.n_cubes * 4;
+  for (int j = 0; j <= c_hi; ++j) {
+    const bool in = R.valid && (j == own || uniform_member(own, a.topk, j));
+    const unsigned w = __ballot_sync(0xffffffffu, in);
+    if (lane == 0) tmask[(size_t)j * 4 + warp] = w;
+  }
+  const int cand = own > 0 ? own : 0;
+  const unsigned v_rows = __reduce_add_sync(0xffffffffu, (R.valid && own > 0) ? 1u : 0u);
+  const unsigned v_cand = __reduce_add_sync(0xffffffffu, (unsigned)cand);
+  const unsigned v_sel = __reduce_add_sync(0xffffffffu, (unsigned)min(cand, a.topk));
+  if (lane == 0) {
+    atomicAdd((unsigned long long*)&a.hdr->stats[0], (unsigned long long)v_rows);
+    atomicAdd((unsigned long long*)&a.hdr->stats[1], (unsigned long long)v_cand);
+    atomicAdd((unsigned long long*)&a.hdr->stats[2], (unsigned long long)v_sel);
+  }
+  __threadfence_block();
+  __syncthreads();
+  compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes, a.tile_count + vt, c_hi, s_wcnt,
+                    tid);
+}
+
+cudaError_t launch_select_uniform(const SelectArgs& a, cudaStream_t s) {
+  if (a.G.n_vtiles == 0) return cudaSuccess;
+  return launch("select_uniform", select_uniform_kernel, dim3(a.G.n_vtiles), dim3(128), 0, s, a);
 }
 
 cudaError_t launch_export_sets(const int32_t* tile_count, const uint16_t* tile_list,

@@ -101,19 +101,29 @@ __global__ void __launch_bounds__(256) ffn_select_kernel(FfnArgs a) {
     float total = 0.f;
     for (int u = 0; u < n; ++u) total += s_w[u];
     int k = n;
+    bool near = false;
     if (total > 0.f) {
       const float target = a.p * total;
       float cum = 0.f;
       for (int i = 0; i < n; ++i) {
-        cum += s_w[(int)(0xFFFFFFFFu - (unsigned)(keys[i] & 0xFFFFFFFFull))];
+        const float wi = s_w[(int)(0xFFFFFFFFu - (unsigned)(keys[i] & 0xFFFFFFFFull))];
+        cum += wi;
         if (cum >= target) {
           k = i + 1;
+          // within 1e-5 of flipping: C_k - p, p - C_(k-1) (k > 1), w_(k) - w_(k+1)
+          float m = cum - target;
+          if (i > 0) m = fminf(m, wi - (cum - target));
+          if (i + 1 < n)
+            m = fminf(m, wi - s_w[(int)(0xFFFFFFFFu - (unsigned)(keys[i + 1] & 0xFFFFFFFFull))]);
+          near = m < 1e-5f * total;
           break;
         }
       }
+      if (k == n && cum < target) near = true;  // rounding left the target unmet
     }
     s_k = k;
     a.cube_count[j] = k;
+    if (near) atomicAdd((unsigned long long*)&a.hdr->stats[3], 1ull);
   }
   __syncthreads();
   if (tid < n) {

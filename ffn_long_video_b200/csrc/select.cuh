@@ -133,6 +133,30 @@ static __device__ __noinline__ void offer_full(float* lz_col, int* lj_col, bool 
   }
 }
 
+// Whether a Top-p cut that closed at sorted list entry i lies within thr of
+// flipping, in the margin terms of the parity protocol, from the fp32 masses
+// (units of 2^ref): C_k* - p (= over, the mass taken beyond the need),
+// p - C_(k*-1) (only when k* > 1) and P_(k*) - P_(k*+1). The next score is the
+// next list entry when there is one; when the list held the whole cut bin and
+// the next score lies in a lower bin, its mass is bounded by the bin's lower
+// edge; when the list was full the next score is unknown and the row counts as
+// near.
+static __device__ __noinline__ bool near_cut(const float* lz_col, int i, int n, float over,
+                                             float zs, float ref, float thr, bool kstar_gt1,
+                                             int kcut_lo) {
+  const float mi = fast_exp2(fmaf(lz_col[i * kRows], zs, -ref));
+  float m = over;
+  if (kstar_gt1) m = fminf(m, mi - over);
+  if (i + 1 < n) {
+    m = fminf(m, mi - fast_exp2(fmaf(lz_col[(i + 1) * kRows], zs, -ref)));
+  } else if (n == kL) {
+    return true;
+  } else if (kcut_lo != INT_MIN) {
+    m = fminf(m, mi - __int_as_float(kcut_lo << 20));
+  }
+  return m < thr;
+}
+
 struct RowSel {
   float* hist_col;   // &hist[0][row]
   float* lz_col;     // list scores, in the histogram's place
@@ -151,6 +175,9 @@ struct RowSel {
   bool bounded;      // only keys after (bz, bj) are offered (extra passes)
   bool range_err;    // a score outside +-kZLimit log2 units
   bool count_mode;   // Top-K: bins count scores instead of summing masses
+  bool any_above;    // some score lies above the cut bin (then k* > 1)
+  bool near;         // the closed cut lies within 1e-5 of a flip (Top-p only)
+  float Z;           // total mass of the row (units of 2^ref), from finish1
   float bz;
   int bj;
 
@@ -173,6 +200,9 @@ struct RowSel {
     bounded = false;
     range_err = false;
     count_mode = count;
+    any_above = false;
+    near = false;
+    Z = 0.f;
     bz = 0.f;
     bj = 0;
 #pragma unroll 8
@@ -246,6 +276,8 @@ struct RowSel {
       cum += m;
     }
     need = target - cum;
+    this->Z = Z;
+    any_above = cum > 0.f;
     open = true;
     lsorted = false;   // the emission pass appends the cut bin in column order
     kcut = kc;
@@ -310,11 +342,15 @@ struct RowSel {
       cum += count_mode ? 1.f : mass(lz_col[i * kRows]);
       if (cum >= need) {
         open = false;
+        if (!count_mode)
+          near = near_cut(lz_col, i, n, cum - need, zs, ref, 1e-5f * Z,
+                          any_above || bounded || i > 0, kcut_lo);
         return i + 1;
       }
     }
     if (n < kL) {  // the whole cut bin was offered: rounding left need unmet
       open = false;
+      near = !count_mode;
       return n;
     }
     need -= cum;

@@ -329,11 +329,13 @@ __global__ void __launch_bounds__(THREADS, 2)
         const unsigned v_cand = __reduce_add_sync(0xffffffffu, (unsigned)ncand);
         const unsigned v_sel = __reduce_add_sync(0xffffffffu, (unsigned)nsel);
         const unsigned v_ext = __reduce_add_sync(0xffffffffu, (unsigned)extra);
+        const unsigned v_near = __reduce_add_sync(0xffffffffu, (valid && s.near) ? 1u : 0u);
         if (lane == 0) {
           atomicAdd((unsigned long long*)&hdr->stats[0], (unsigned long long)v_rows);
           atomicAdd((unsigned long long*)&hdr->stats[1], (unsigned long long)v_cand);
           atomicAdd((unsigned long long*)&hdr->stats[2], (unsigned long long)v_sel);
           atomicAdd((unsigned long long*)&hdr->stats[3], (unsigned long long)v_ext);
+          if (v_near) atomicAdd((unsigned long long*)&hdr->stats[7], (unsigned long long)v_near);
         }
       }
       __threadfence_block();

@@ -107,7 +107,11 @@ typedef struct {
   uint64_t tiles;            /* 128-row attention tiles executed (visual + text)    */
   uint64_t key_blocks;       /* executed (tile, key block) pairs                    */
   uint64_t key_block_keys;   /* keys covered by those blocks (for executed FLOPs)   */
-  uint64_t reserved[9];
+  uint64_t near_margin_rows; /* Top-p rows whose cut lies within 1e-5 of flipping:  */
+                             /* min(C_k* - p, p - C_k*-1, P_(k*) - P_(k*+1)) < 1e-5, */
+                             /* from the fp32 masses (a row whose next score is     */
+                             /* not known counts as near); 0 for Top-K             */
+  uint64_t reserved[8];
 } adaspark_attn_stats;
 
 /* Device workspace bytes needed by adaspark_cube_attn for these sizes
@@ -154,6 +158,22 @@ int adaspark_cube_attn_topk(const void *Q, const void *K, const void *V, int dty
                             const int32_t *cube_ids, const int32_t *cube_offsets, int n_cubes,
                             int n_vis, int n_tokens, int hq, int hkv, int d, int k, void *out,
                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* AdaS-Attn with Uniform Sampling in place of Top-p: the other strategy of the
+ * AdaSpark paper's selection-strategy ablation that does not look at the
+ * content (row "Uniform Sampling"; the pages name it without defining it).
+ * Read here as: a query of cube i takes k of its i preceding cubes at even
+ * spacing from the first, cubes floor(m * i / k) for m = 0..k-1, and every
+ * preceding cube when i <= k; every query head of every token of cube i has
+ * the same set, and the own cube is attended causally as always. No cube mean
+ * keys or scores are computed. Arguments, layout, workspace and outputs as for
+ * adaspark_cube_attn with k (>= 1) in place of p; adaspark_attn_export_sets
+ * reads its sets. Errors: as adaspark_cube_attn, and ADASPARK_EINVAL for
+ * k < 1. */
+int adaspark_cube_attn_uniform(const void *Q, const void *K, const void *V, int dtype,
+                               const int32_t *cube_ids, const int32_t *cube_offsets, int n_cubes,
+                               int n_vis, int n_tokens, int hq, int hkv, int d, int k, void *out,
+                               void *workspace, size_t workspace_bytes, void *stream);
 
 /* Device workspace bytes needed by adaspark_cube_attn_train (0 when the sizes
  * are invalid or dtype is not ADASPARK_BF16): adaspark_cube_attn_workspace
@@ -269,7 +289,10 @@ typedef struct {
   uint64_t active_visual;   /* visual tokens that went through the FFN      */
   uint64_t skipped_visual;  /* visual tokens updated by mean compensation   */
   uint64_t text_tokens;     /* text tokens (always dense)                   */
-  uint64_t reserved[13];
+  uint64_t near_margin_cubes; /* cubes whose Top-p cut lies within 1e-5 of   */
+                              /* flipping (the margin of adaspark_attn_stats, */
+                              /* on the importance shares, fp32)              */
+  uint64_t reserved[12];
 } adaspark_ffn_stats;
 
 /* Device workspace bytes needed by adaspark_token_ffn (0 when invalid). */

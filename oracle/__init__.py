@@ -13,6 +13,9 @@ Parity status per function (what pins it is in ``tests/test_oracle_pins.py``):
 * ``cube_mean_keys``        pinned (invariants: zero residual sum, constant cubes)
 * ``top_p``                 pinned (exhaustive subset enumeration, closed forms)
 * ``top_k``                 pinned (exhaustive k-subset enumeration, closed forms)
+* ``uniform_cubes``, ``select_cubes_uniform``
+                            pinned (hand values, even-spacing and count
+                            invariants, equal sets across heads and tokens)
 * ``select_cubes``          pinned (uniform closed form, 2-cube sigmoid cut, GQA map)
 * ``attention_given_sets``  pinned (torch SDPA in float64 with a mask; first token)
 * ``ffn_select``            pinned (closed forms on scaled tokens, brute force)
@@ -38,6 +41,8 @@ from .adaspark_ref import (  # noqa: F401
     top_k,
     top_k_margin,
     select_cubes,
+    select_cubes_uniform,
+    uniform_cubes,
     token_importance,
     linear,
     rmsnorm,

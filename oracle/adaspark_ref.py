@@ -215,8 +215,37 @@ def top_k_margin(P, k):
     return out.reshape(P.shape[:-1])
 
 
+def uniform_cubes(i, k):
+    """Uniform Sampling, the content-independent strategy of the AdaSpark
+    paper's selection-strategy ablation (the pages name it without defining
+    it; reading: k of the i preceding cubes at even spacing from the first,
+    j_m = floor(m * i / k) for m = 0..k-1, every preceding cube when i <= k).
+    Returns the ascending cube indices."""
+    if int(k) != k or k < 1:
+        raise ValueError("k must be a positive integer")
+    if i <= k:
+        return np.arange(i)
+    return (np.arange(k) * i) // k
+
+
+def select_cubes_uniform(cube_offsets, n_vis, hq, k, tokens=None):
+    """AdaS-Attn sets under Uniform Sampling (``uniform_cubes``): every query
+    head of every token of cube i gets the same set. Returns a boolean array
+    sel[len(tokens), hq, C] like ``select_cubes`` (own cube not marked)."""
+    off = np.asarray(cube_offsets)
+    C = len(off) - 1
+    if tokens is None:
+        tokens = np.arange(n_vis)
+    tokens = np.asarray(tokens)
+    cube_of = np.searchsorted(off, tokens, side="right") - 1
+    sel = np.zeros((len(tokens), hq, C), dtype=bool)
+    for r, i in enumerate(cube_of):
+        sel[r, :, uniform_cubes(int(i), k)] = True
+    return sel
+
+
 def select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=None, with_margin=False,
-                 k=None):
+                 k=None, kbar=None):
     """AdaS-Attn cube selection (key design 2, formula P_i and S_i).
 
     For visual token t in cube i and query head h: P = softmax over the
@@ -226,7 +255,9 @@ def select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=None, with_margin
     sel[len(tokens), hq, C] (sel[r, h, j] is True when cube j is selected; the
     own cube is not marked here, it is always attended causally) and, when
     asked, the cut margins [len(tokens), hq] (+inf where nothing can flip).
-    ``tokens`` defaults to every visual token.
+    ``tokens`` defaults to every visual token.  ``kbar`` may pass the cube mean
+    keys of ``cube_mean_keys(K, cube_offsets)`` when the caller has them (they
+    belong to the layer, not to the selected rows).
     """
     if k is None:
         _check_p(p)
@@ -234,7 +265,8 @@ def select_cubes(Q, K, cube_offsets, n_vis, hq, hkv, p, tokens=None, with_margin
     C = len(off) - 1
     d = Q.shape[-1]
     g = hq // hkv
-    kbar = cube_mean_keys(K, off)
+    if kbar is None:
+        kbar = cube_mean_keys(K, off)
     if tokens is None:
         tokens = np.arange(n_vis)
     tokens = np.asarray(tokens)

@@ -103,12 +103,16 @@ def excess_over_bf16(got, want):
     return float((np.abs(got - want) - allow).max())
 
 
-def run_attn(case, p=None, k=None, train=False):
-    """Run AdaS-Attn (Top-p, or Top-K when k is given; the training-mode call
-    when ``train``) and export its sets."""
+def run_attn(case, p=None, k=None, train=False, uniform=None):
+    """Run AdaS-Attn (Top-p, or Top-K when k is given, or Uniform Sampling of
+    ``uniform`` cubes; the training-mode call when ``train``) and export its
+    sets."""
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
-    if k is None:
+    if uniform is not None:
+        out, ws = fb.cube_attn_uniform(t["Q"], t["K"], t["V"], case["ids"], case["off"],
+                                       cfg.n_vis, uniform)
+    elif k is None:
         out, ws = fb.cube_attn(t["Q"], t["K"], t["V"], case["ids"], case["off"], cfg.n_vis, p,
                                train=train)
     else:
@@ -122,20 +126,26 @@ def run_attn(case, p=None, k=None, train=False):
     return out, sel, ws
 
 
-def check_attn(case, p=None, tokens=None, report=None, k=None, train=False):
+def check_attn(case, p=None, tokens=None, report=None, k=None, train=False, uniform=None):
     """Selection parity + output parity of AdaS-Attn on ``tokens`` (default all);
-    Top-K selection when ``k`` is given; the training-mode call when ``train``."""
+    Top-K selection when ``k`` is given, Uniform Sampling of ``uniform`` cubes
+    (integer sets, compared exactly) when that is given; the training-mode call
+    when ``train``."""
     cfg, t = case["cfg"], case["t"]
     p = cfg.p if p is None else p
-    out, gsel, ws = run_attn(case, p, k, train)
+    out, gsel, ws = run_attn(case, p, k, train, uniform)
     Qc, Kc, Vc = (t[k].cpu() for k in ("Q", "K", "V"))
     off = case["off_np"]
     if tokens is None:
         tokens = np.arange(cfg.n_tokens)
     tokens = np.asarray(tokens)
     vis = tokens[tokens < cfg.n_vis]
-    osel, margin = oracle.select_cubes(Qc, Kc, off, cfg.n_vis, cfg.hq, cfg.hkv, p, tokens=vis,
-                                       with_margin=True, k=k)
+    if uniform is not None:
+        osel = oracle.select_cubes_uniform(off, cfg.n_vis, cfg.hq, uniform, tokens=vis)
+        margin = np.full(osel.shape[:2], np.inf)
+    else:
+        osel, margin = oracle.select_cubes(Qc, Kc, off, cfg.n_vis, cfg.hq, cfg.hkv, p,
+                                           tokens=vis, with_margin=True, k=k)
     g = gsel[vis]
     diff_rows = (osel != g).any(axis=2)
     near = margin < MARGIN
@@ -153,7 +163,8 @@ def check_attn(case, p=None, tokens=None, report=None, k=None, train=False):
             c = int(np.searchsorted(off, tok, side="right") - 1)
             P = oracle.softmax(oracle.cube_scores(Qf[tok, h], kbar[:c, h // g_of], cfg.d))
             assert near_cut_ok(P, g[r, h, :c], p, k), (tok, int(h))
-    _record("attn", cfg, p, k, g.shape[0] * g.shape[1], near.sum(), n_near_mismatch)
+    if uniform is None:
+        _record("attn", cfg, p, k, g.shape[0] * g.shape[1], near.sum(), n_near_mismatch)
     # outputs against the oracle on the library's own sets
     sel_full = np.zeros((len(tokens), cfg.hq, cfg.n_cubes), dtype=bool)
     is_vis = tokens < cfg.n_vis

@@ -122,3 +122,47 @@ def test_clock_samples_inside_the_region():
 def test_clock_sampler_without_nvidia_smi():
     s = bench.ClockSampler(0)
     assert s.stop()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_popcount32_matches_python():
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(5)
+    v = rng.integers(-2**31, 2**31, size=1000, dtype=np.int64).astype(np.int32)
+    got = bench.popcount32(torch.from_numpy(v)).numpy()
+    want = [bin(int(x) & 0xFFFFFFFF).count("1") for x in v]
+    assert list(got) == want
+
+
+def test_useful_pairs_count_every_admitted_key():
+    """Selected cubes' keys + own-cube causal prefixes + text causal prefixes,
+    over all heads, counted against a brute-force walk of a tiny layer."""
+    cfg = workloads.small_config(name="pairs", grid=(2, 4, 4), cube=(2, 2, 2), n_text=5, D=64,
+                                 hq=3, hkv=1, F=128)
+    sizes, off = cfg.sizes, cfg.offsets
+    selected_pairs = 17           # any count: each selected cube brings n_c keys
+    brute = selected_pairs * int(sizes[0])
+    for h in range(cfg.hq):
+        for t in range(cfg.n_tokens):
+            if t < cfg.n_vis:
+                c = int((off <= t).sum()) - 1
+                brute += t - int(off[c]) + 1
+            else:
+                brute += t + 1
+    assert bench.useful_attention_pairs(cfg, selected_pairs) == brute
+
+
+def test_oracle_sample_extrapolates_a_small_layer():
+    """The CPU baseline on a tiny layer: every term of the extrapolation is
+    there, the layer time is their sum and the value is tokens per second."""
+    lay = workloads.make_layer(workloads.CONFIGS[1])
+    r = bench.oracle_sample(workloads.CONFIGS[1], lay, budget_s=0.5)
+    assert r["value"] > 0 and r["cores"] >= 1
+    terms = r["extrapolation"].replace("setup", "").split("+")
+    total = 0.0
+    for term in terms:
+        parts = term.replace("s", "").split("x")
+        total += float(parts[0]) * float(parts[1]) if len(parts) == 2 else float(parts[0])
+    assert abs(total - r["layer_s_extrapolated"]) <= 0.05 + 0.01 * total
+    assert abs(r["value"] - workloads.CONFIGS[1].n_tokens / r["layer_s_extrapolated"]) \
+        <= 0.05 * r["value"]

@@ -1,8 +1,9 @@
 """Selection variants against the float64 oracle (needs a B200): Top-K cube
 selection (the fixed-size strategy of the paper's ablation of selection
 strategies; sets bit for bit except at near-ties, P_(k) - P_(k+1) below the
-1e-5 margin) and the AdaS-FFN importance alternatives (energy share, softmax of
-norms). Outputs are compared on the library's own sets within the stated
+1e-5 margin), Uniform Sampling (the content-independent strategy of the same
+ablation; sets exactly) and the AdaS-FFN importance alternatives (energy share,
+softmax of norms). Outputs are compared on the library's own sets within the stated
 tolerance."""
 import numpy as np
 import pytest
@@ -46,6 +47,26 @@ def test_topk_full_size_sampled():
     rep = {}
     parity.check_attn(c, k=16, tokens=_sample_tokens(cfg, 32, 5), report=rep)
     print(cfg.name, "top-16", rep)
+
+
+# ------------------------------------------------- Uniform Sampling
+@pytest.mark.parametrize("k", [1, 3, 8, 1000])
+def test_uniform_small(case, k):
+    """Uniform Sampling (k evenly spaced preceding cubes): sets equal to the
+    oracle's exactly (no scores, so no margin), outputs on those sets."""
+    rep = {}
+    parity.check_attn(case, uniform=k, report=rep)
+    print(case["cfg"].name, "uniform", k, rep)
+
+
+def test_uniform_full_size_sampled():
+    """The 7B-shaped 64K layer with 70 evenly spaced cubes (about the mean
+    Top-p set size at p = 0.7 there), sampled tokens (all heads)."""
+    cfg = workloads.CONFIGS[3]
+    c = parity.make_case(cfg)
+    rep = {}
+    parity.check_attn(c, uniform=70, tokens=_sample_tokens(cfg, 24, 6), report=rep)
+    print(cfg.name, "uniform-70", rep)
 
 
 # ------------------------------------------------- AdaS-FFN importance variants

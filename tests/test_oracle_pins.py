@@ -760,3 +760,50 @@ def test_ffn_magnitudes_twice_the_gradients_when_terms_are_positive():
     for m, gr in ((mWg, dWg), (mWu, dWu), (mWd, dWd)):
         assert gr.min() > 0.0
         np.testing.assert_allclose(m, 2.0 * gr, rtol=1e-12, atol=0)
+
+
+def test_select_cubes_with_given_means_is_the_same_selection():
+    """Passing the layer's cube means (computed once per layer) changes nothing."""
+    rng = np.random.default_rng(34)
+    off = np.array([0, 4, 8, 12, 16, 20])
+    Q, K, _ = _qkv(rng, 24, 4, 2, 8)
+    a, ma = oracle.select_cubes(Q, K, off, 20, 4, 2, 0.6, with_margin=True)
+    b, mb = oracle.select_cubes(Q, K, off, 20, 4, 2, 0.6, with_margin=True,
+                                kbar=oracle.cube_mean_keys(K, off))
+    assert np.array_equal(a, b) and np.array_equal(ma, mb)
+
+
+# ---------------------------------------------------------------- Uniform Sampling
+def test_uniform_cubes_hand_values():
+    """k of the i preceding cubes at even spacing from the first (floor(m i / k)),
+    all of them when i <= k, none for the first cube."""
+    assert oracle.uniform_cubes(10, 3).tolist() == [0, 3, 6]
+    assert oracle.uniform_cubes(7, 7).tolist() == list(range(7))
+    assert oracle.uniform_cubes(3, 5).tolist() == [0, 1, 2]
+    assert oracle.uniform_cubes(0, 4).tolist() == []
+    assert oracle.uniform_cubes(1000, 4).tolist() == [0, 250, 500, 750]
+    with pytest.raises(ValueError):
+        oracle.uniform_cubes(5, 0)
+
+
+@pytest.mark.parametrize("i,k", [(i, k) for i in range(1, 40) for k in (1, 2, 3, 5, 8, 13)])
+def test_uniform_cubes_even_spacing(i, k):
+    """min(i, k) distinct ascending preceding cubes, starting at cube 0, whose gaps
+    (including the one up to cube i) are floor(i/k) or ceil(i/k)."""
+    j = oracle.uniform_cubes(i, k)
+    assert len(j) == min(i, k) and len(set(j.tolist())) == len(j)
+    assert (np.diff(j) > 0).all() and j[0] == 0 and j[-1] < i
+    if i > k:
+        gaps = np.diff(np.append(j, i))
+        assert gaps.min() >= i // k and gaps.max() <= -(-i // k)
+
+
+def test_select_cubes_uniform_shares_the_set_across_heads_and_tokens():
+    off = np.array([0, 3, 5, 9, 12, 16])
+    sel = oracle.select_cubes_uniform(off, 16, 4, 2)
+    for t in range(16):
+        c = int(np.searchsorted(off, t, side="right") - 1)
+        want = np.zeros(5, bool)
+        want[oracle.uniform_cubes(c, 2)] = True
+        for h in range(4):
+            assert np.array_equal(sel[t, h], want)
