@@ -143,11 +143,16 @@ __global__ void __launch_bounds__(128) select_simt_kernel(SelectArgs a) {
           for (int e = 0; e < D; ++e) acc = fmaf(q[e], kr[e], acc);
           if (pass == 0) s.pass1(acc);
           else if (pass == 1) selb = s.pass2(acc, j, true);
-          else s.pass_more(acc, j);
+          else selb = s.pass_more(acc, j);
         }
         if (pass == 1) {
           const unsigned w = __ballot_sync(0xffffffffu, selb || own == j);
           if (lane == 0) tmask[(size_t)j * 4 + warp] = w;
+          nsel += selb;
+        } else if (pass >= 2) {
+          // fine bins above a row's fine cut, selected outright
+          const unsigned w = __ballot_sync(0xffffffffu, selb);
+          if (w != 0u && lane == 0) atomicOr(&tmask[(size_t)j * 4 + warp], w);
           nsel += selb;
         }
       }

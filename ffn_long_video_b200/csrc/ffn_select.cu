@@ -1,6 +1,8 @@
 // AdaS-FFN token selection, compaction and mean compensation (key design 3 of
 // the AdaSpark note: rank tokens of a cube by L2 norm, Top-p through the FFN,
 // skipped tokens y_k = x_k + m_bar_i). HBM-bound SIMT kernels.
+#include <algorithm>
+
 #include "ffn_kernels.h"
 
 namespace adaspark {
@@ -222,35 +224,38 @@ __global__ void __launch_bounds__(256) ffn_compact_kernel(FfnArgs a) {
 }
 
 // Skipped visual rows: y_k = x_k + sums_c / |M_c| (mean of FFN over the cube's
-// active tokens). One block per 4 rows.
+// active tokens). Each warp walks the tokens with a grid-wide stride and takes
+// the skipped ones, so every resident warp has rows to move (a warp per token
+// would leave most warps without work: most tokens are active).
 template <typename T>
 __global__ void __launch_bounds__(256) ffn_compensate_kernel(FfnArgs a) {
   if (status_bad(a.hdr)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + warp;
-  if (t >= a.n_vis) return;
-  if (a.active[t]) return;
-  const int c = a.cube_ids[t];
-  const float inv = 1.f / (float)a.cube_count[c];
-  const T* xr = reinterpret_cast<const T*>(a.x) + (size_t)t * a.D;
-  const float* sr = a.sums + (size_t)c * a.D;
-  float* yr = a.y + (size_t)t * a.D;
-  // one 16-byte load of x per lane and step (8 bf16 or 4 fp32 features), the
-  // matching sums and stores; two steps in flight
+  const int n_warps = gridDim.x * 8;
   constexpr int kN = Vec8<T>::kN;
-#pragma unroll 2
-  for (int e = lane * kN; e < a.D; e += 32 * kN) {
-    float xv[8];
-    Vec8<T>::load(xr + e, xv);
+  for (int t = blockIdx.x * 8 + warp; t < a.n_vis; t += n_warps) {
+    if (a.active[t]) continue;
+    const int c = a.cube_ids[t];
+    const float inv = 1.f / (float)a.cube_count[c];
+    const T* xr = reinterpret_cast<const T*>(a.x) + (size_t)t * a.D;
+    const float* sr = a.sums + (size_t)c * a.D;
+    float* yr = a.y + (size_t)t * a.D;
+    // one 16-byte load of x per lane and step (8 bf16 or 4 fp32 features),
+    // the matching sums and stores; four steps in flight
+#pragma unroll 4
+    for (int e = lane * kN; e < a.D; e += 32 * kN) {
+      float xv[8];
+      Vec8<T>::load(xr + e, xv);
 #pragma unroll
-    for (int h = 0; h < kN; h += 4) {
-      const float4 sv = *reinterpret_cast<const float4*>(sr + e + h);
-      float4 o;
-      o.x = xv[h] + sv.x * inv;
-      o.y = xv[h + 1] + sv.y * inv;
-      o.z = xv[h + 2] + sv.z * inv;
-      o.w = xv[h + 3] + sv.w * inv;
-      *reinterpret_cast<float4*>(yr + e + h) = o;
+      for (int h = 0; h < kN; h += 4) {
+        const float4 sv = *reinterpret_cast<const float4*>(sr + e + h);
+        float4 o;
+        o.x = xv[h] + sv.x * inv;
+        o.y = xv[h + 1] + sv.y * inv;
+        o.z = xv[h + 2] + sv.z * inv;
+        o.w = xv[h + 3] + sv.w * inv;
+        *reinterpret_cast<float4*>(yr + e + h) = o;
+      }
     }
   }
 }
@@ -280,7 +285,10 @@ cudaError_t launch_ffn_compact(const FfnArgs& a, int dtype, cudaStream_t s) {
 
 cudaError_t launch_ffn_compensate(const FfnArgs& a, int dtype, cudaStream_t s) {
   if (a.n_vis == 0 || a.dense) return cudaSuccess;
-  const int blocks = (a.n_vis + 7) / 8;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int blocks = std::min((a.n_vis + 7) / 8, sms * 8);
   if (dtype == ADASPARK_BF16)
     return launch("ffn_compensate", ffn_compensate_kernel<__nv_bfloat16>, dim3(blocks), dim3(256),
                   0, s, a);

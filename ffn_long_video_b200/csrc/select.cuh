@@ -14,11 +14,19 @@
 //          cut bin are appended to a per-row list of kL entries. Sorted into
 //          the (s desc, index asc) order and walked until the cumulative mass
 //          reaches p * Z, the list ends the cut. A cut bin larger than the
-//          list is collected again in the next pass, keeping its kL best.
-//  more    if the cut lies beyond the kL best scores of the cut bin, those kL
-//          are selected, the required mass is reduced by theirs, and another
-//          pass collects the next kL below the last one; repeated until the cut
-//          is found (bounded by the size of the cut bin).
+//          list turns the row's storage into a finer histogram of the cut bin
+//          (64 bins of 1/512 octave; for the window's lowest bin, the next 8
+//          octaves below it in 1/8-octave bins), filled for the rest of the
+//          pass from the list's entries and the bin's remaining scores.
+//  pass 3  (rows with a finer histogram) the fine cut bin is found the same
+//          way; scores of fine bins above it are selected outright, and the
+//          scores of the fine cut bin are listed, sorted and walked as above.
+//  more    if the cut lies beyond the kL best scores of the (fine) cut bin,
+//          those kL are selected, the required mass is reduced by theirs, and
+//          another pass collects the next kL below the last one; repeated
+//          until the cut is found (bounded by the size of that bin). With the
+//          finer histogram this is rare: a crowded cut bin costs one pass more
+//          instead of one pass per kL of its scores.
 // This reproduces "smallest prefix of the (P desc, index asc) order whose
 // cumulative mass reaches p" up to fp32 rounding of the masses, for any score
 // distribution (ties included), without memory beyond the per-row list.
@@ -139,11 +147,11 @@ static __device__ __noinline__ void offer_full(float* lz_col, int* lj_col, bool 
 // p - C_(k*-1) (only when k* > 1) and P_(k*) - P_(k*+1). The next score is the
 // next list entry when there is one; when the list held the whole cut bin and
 // the next score lies in a lower bin, its mass is bounded by the bin's lower
-// edge; when the list was full the next score is unknown and the row counts as
-// near.
+// edge `edge` (negative when nothing lies below the bin); when the list was
+// full the next score is unknown and the row counts as near.
 static __device__ __noinline__ bool near_cut(const float* lz_col, int i, int n, float over,
                                              float zs, float ref, float thr, bool kstar_gt1,
-                                             int kcut_lo) {
+                                             float edge) {
   const float mi = fast_exp2(fmaf(lz_col[i * kRows], zs, -ref));
   float m = over;
   if (kstar_gt1) m = fminf(m, mi - over);
@@ -151,10 +159,29 @@ static __device__ __noinline__ bool near_cut(const float* lz_col, int i, int n, 
     m = fminf(m, mi - fast_exp2(fmaf(lz_col[(i + 1) * kRows], zs, -ref)));
   } else if (n == kL) {
     return true;
-  } else if (kcut_lo != INT_MIN) {
-    m = fminf(m, mi - __int_as_float(kcut_lo << 20));
+  } else if (edge >= 0.f) {
+    m = fminf(m, mi - edge);
   }
   return m < thr;
+}
+
+// Fine bin of a mass u inside a crowded cut bin: (bits(u) >> sh) - base,
+// clamped to [0, kB - 1] (bin 0 also takes everything below).
+__device__ __forceinline__ int fine_bin(float u, int sh, int base) {
+  return min(max((int)(__float_as_uint(u) >> sh) - base, 0), kB - 1);
+}
+
+// The emission pass found the cut bin larger than the list: the row's column
+// (list scores in rows [0, kL), indices above) becomes a histogram of kB fine
+// bins of the cut bin, filled with the listed scores and the one that did not
+// fit (u_new). Count mode adds one per score instead of its mass.
+static __device__ __noinline__ void start_fine(float* col, float zs, float ref, int sh, int base,
+                                               bool count, float u_new) {
+  float u[kL];
+  for (int i = 0; i < kL; ++i) u[i] = fast_exp2(fmaf(col[i * kRows], zs, -ref));
+  for (int b = 0; b < kB; ++b) col[b * kRows] = 0.f;
+  for (int i = 0; i < kL; ++i) col[fine_bin(u[i], sh, base) * kRows] += count ? 1.f : u[i];
+  col[fine_bin(u_new, sh, base) * kRows] += count ? 1.f : u_new;
 }
 
 struct RowSel {
@@ -170,13 +197,18 @@ struct RowSel {
   float need;        // mass still to take from the cut bin (units of 2^ref)
   int ln;            // list entries
   bool lsorted;      // list in (score desc, index asc) order
-  bool ovf;          // the emission pass met more cut-bin scores than the list holds
   bool open;         // cut not found yet
   bool bounded;      // only keys after (bz, bj) are offered (extra passes)
   bool range_err;    // a score outside +-kZLimit log2 units
   bool count_mode;   // Top-K: bins count scores instead of summing masses
   bool any_above;    // some score lies above the cut bin (then k* > 1)
   bool near;         // the closed cut lies within 1e-5 of a flip (Top-p only)
+  bool sub;          // emission pass: the cut bin overflowed the list; its
+                     // scores go to the fine histogram instead
+  bool fine;         // the cut lies in fine bin fcut of the cut bin
+  bool femit;        // first pass after the fine cut: emit its upper fine bins
+  int fsh, fbase;    // fine bin of a mass: fine_bin(u, fsh, fbase)
+  int fcut;
   float Z;           // total mass of the row (units of 2^ref), from finish1
   float bz;
   int bj;
@@ -195,13 +227,18 @@ struct RowSel {
     need = 0.f;
     ln = 0;
     lsorted = true;
-    ovf = false;
     open = false;
     bounded = false;
     range_err = false;
     count_mode = count;
     any_above = false;
     near = false;
+    sub = false;
+    fine = false;
+    femit = false;
+    fsh = 20;
+    fbase = 0;
+    fcut = 0;
     Z = 0.f;
     bz = 0.f;
     bj = 0;
@@ -284,20 +321,32 @@ struct RowSel {
     kcut_lo = kc == klo ? INT_MIN : kc;   // the lowest bin holds everything below it
   }
 
-  // Emission pass, one score, without branches: true when the score lies
-  // above the cut bin (selected outright); a cut-bin score is appended to the
-  // list. The list has one spare slot, so the append writes unconditionally;
-  // a cut-bin score that finds the list full sets ovf, and the row then
-  // collects its cut bin again, in order, in an extra pass.
+  // Emission pass, one score: true when the score lies above the cut bin
+  // (selected outright); a cut-bin score is appended to the list. The list
+  // has one spare slot, so the append writes unconditionally. A cut-bin score
+  // that finds the list full turns the column into the fine histogram of the
+  // cut bin (start_fine), which takes the bin's scores from then on.
   __device__ __forceinline__ bool pass2(float score, int j, bool valid) {
-    const int k = mass_key(mass(score));
+    const float u = mass(score);
+    const int k = mass_key(u);
     const bool above = valid && k > kcut;
     const bool inb = valid && k >= kcut_lo && k <= kcut;
-    lz_col[ln * kRows] = score;
-    lj_col[ln * kRows] = j;
-    const bool room = ln < kL;
-    ovf = ovf || (inb && !room);
-    ln += (inb && room) ? 1 : 0;
+    if (!sub) {
+      lz_col[ln * kRows] = score;
+      lj_col[ln * kRows] = j;
+      const bool room = ln < kL;
+      ln += (inb && room) ? 1 : 0;
+      if (inb && !room) {
+        // fine bins: 1/512 octave inside a regular cut bin; for the window's
+        // lowest bin (which holds everything below), the 8 octaves below it
+        sub = true;
+        fsh = kcut_lo == INT_MIN ? 20 : 14;
+        fbase = kcut_lo == INT_MIN ? klo - (kB - 1) : kcut << 6;
+        start_fine(hist_col, zs, ref, fsh, fbase, count_mode, u);
+      }
+    } else if (inb) {
+      hist_col[fine_bin(u, fsh, fbase) * kRows] += count_mode ? 1.f : u;
+    }
     return above;
   }
 
@@ -314,24 +363,49 @@ struct RowSel {
     }
   }
 
-  // Extra pass for a row whose cut is still open.
-  __device__ __forceinline__ void pass_more(float score, int j) {
-    if (!open) return;
-    const int k = mass_key(mass(score));
-    if (k >= kcut_lo && k <= kcut) offer(score, j);
+  // Extra pass for a row whose cut is still open: offers the scores of the
+  // (fine) cut bin to the list. In the first pass after a fine cut, true for
+  // a score of a fine bin above it (selected outright).
+  __device__ __forceinline__ bool pass_more(float score, int j) {
+    if (!open) return false;
+    const float u = mass(score);
+    const int k = mass_key(u);
+    if (k < kcut_lo || k > kcut) return false;
+    if (fine) {
+      const int f = fine_bin(u, fsh, fbase);
+      if (f > fcut) return femit;
+      if (f < fcut) return false;
+    }
+    offer(score, j);
+    return false;
   }
 
   // After a pass over the cut bin: how many leading list entries are selected.
   // Closes the cut when reached (or when the bin is exhausted); otherwise all
-  // kL entries are taken and the next pass starts after the last of them. A
-  // list that overflowed during the emission pass is dropped unused: the next
-  // pass collects the best kL of the cut bin in order.
+  // kL entries are taken and the next pass starts after the last of them.
+  // After an emission pass that filled the fine histogram, finds the fine cut
+  // bin instead (walking the fine bins from the top, like finish1) and leaves
+  // the row open: the next pass emits the fine bins above it and lists it.
   __device__ __forceinline__ int settle() {
     if (!open) return 0;
-    if (ovf) {
-      ovf = false;
+    femit = false;
+    if (sub) {
+      float cum = 0.f;
+      int b = kB - 1;
+      for (; b > 0; --b) {
+        const float m = hist_col[b * kRows];
+        if (cum + m >= need) break;
+        cum += m;
+      }
+      need -= cum;
+      any_above = any_above || cum > 0.f;
+      fcut = b;
+      sub = false;
+      fine = true;
+      femit = true;
       ln = 0;
       lsorted = true;
+      bounded = false;
       return 0;
     }
     const int n = ln;
@@ -344,7 +418,7 @@ struct RowSel {
         open = false;
         if (!count_mode)
           near = near_cut(lz_col, i, n, cum - need, zs, ref, 1e-5f * Z,
-                          any_above || bounded || i > 0, kcut_lo);
+                          any_above || bounded || i > 0, lower_edge());
         return i + 1;
       }
     }
@@ -358,6 +432,13 @@ struct RowSel {
     bz = lz_col[(kL - 1) * kRows];
     bj = lj_col[(kL - 1) * kRows];
     return n;
+  }
+
+  // Lower mass edge of the bin the list collects (the cut bin, or its fine
+  // cut bin); negative when that bin also holds everything below it.
+  __device__ __forceinline__ float lower_edge() const {
+    if (fine) return (fsh == 20 && fcut == 0) ? -1.f : __int_as_float((fbase + fcut) << fsh);
+    return kcut_lo == INT_MIN ? -1.f : __int_as_float(kcut_lo << 20);
   }
 
   __device__ __forceinline__ int list_j(int i) const { return lj_col[i * kRows]; }

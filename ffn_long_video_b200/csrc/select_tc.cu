@@ -265,13 +265,24 @@ __global__ void __launch_bounds__(THREADS, 2)
                 if (s.pass2(__uint_as_float(acc[c]), j0 + q * 8 + c, q * 8 + c < nv)) gb |= 1u << c;
               bits |= gb << (q * 8);
             } else if (s.open) {
+              uint32_t gb = 0u;
 #pragma unroll
               for (int c = 0; c < 8; ++c)
-                if (q * 8 + c < nv) s.pass_more(__uint_as_float(acc[c]), j0 + q * 8 + c);
+                if (q * 8 + c < nv && s.pass_more(__uint_as_float(acc[c]), j0 + q * 8 + c))
+                  gb |= 1u << c;
+              bits |= gb << (q * 8);
             }
           }
           tc_fence_before();
           mbar_arrive(&s_empty[sb]);
+          if (pass >= 2 && __any_sync(0xffffffffu, bits != 0u)) {
+            // fine bins above a row's fine cut: selected outright in the first
+            // pass after the fine cut was found
+            nsel += __popc(bits);
+            const uint32_t word = sel::warp_transpose32(bits, lane);
+            const int jl = j0 + lane;
+            if (word != 0u && jl < c_hi) atomicOr(&tmask[(size_t)jl * 4 + wq], word);
+          }
           if (pass == 1) {
             nsel += __popc(bits);
             // lane L now takes the mask word of column j0 + L (bit r = row r)
