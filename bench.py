@@ -434,6 +434,8 @@ def run_ours(args, rank, world, device):
     cfg = resolve_config(args)
     if fb.device_check(torch.cuda.current_device()) != fb.OK:
         raise RuntimeError("not an sm_100 device")
+    if args.only:
+        return run_only(args, cfg, device)
     if cfg.n_layers > 1:
         return run_stack(args, cfg, world, device)
     dt = fb.BF16 if cfg.dtype == "bf16" else fb.FP32
@@ -535,6 +537,52 @@ def run_ours(args, rank, world, device):
                            "kernels": kernel_table(dense_kt, cfg, attn_stats, ffn_stats)},
         "sparsity": sparsity, "backward": backward, "cfg": cfg, "lay": lay,
     }
+
+
+def run_only(args, cfg, device):
+    """Profiling mode: one of the two calls alone, with only its own inputs,
+    output and workspace on the device (about 1.3 GB for AdaS-Attn at 64K), so
+    that a profiler capture of one launch moves little memory. Prints the
+    call's time; not a bench line."""
+    import torch
+    import ffn_long_video_b200 as fb
+    import workloads
+    dt = fb.BF16 if cfg.dtype == "bf16" else fb.FP32
+    lay = workloads.make_layer(cfg, project_on=device)
+    ids = np.concatenate([np.repeat(np.arange(cfg.n_cubes, dtype=np.int32), cfg.sizes),
+                          np.full(cfg.n_text, -1, np.int32)])
+    t_ids = torch.from_numpy(ids).to(device)
+    t_off = torch.from_numpy(cfg.offsets).to(device)
+    if args.only == "attn":
+        Q, K, V = (lay[k].to(device) for k in ("Q", "K", "V"))
+        del lay
+        torch.cuda.empty_cache()
+        out = torch.empty_like(Q)
+        ws = torch.empty(fb.cube_attn_workspace_bytes(cfg.n_tokens, cfg.n_vis, cfg.n_cubes, cfg.hq,
+                                                      cfg.hkv, cfg.d, dt), dtype=torch.uint8,
+                         device=device)
+        step = lambda: fb.cube_attn(Q, K, V, t_ids, t_off, cfg.n_vis, cfg.p, out=out,
+                                    workspace=ws)
+    else:
+        x, Wg, Wu, Wd = (lay[k].to(device) for k in ("x", "W_gate", "W_up", "W_down"))
+        del lay
+        torch.cuda.empty_cache()
+        text = torch.from_numpy((ids == -1).astype(np.uint8)).to(device)
+        y = torch.empty((cfg.n_tokens, cfg.D), dtype=torch.float32, device=device)
+        ws = torch.empty(fb.token_ffn_workspace_bytes(cfg.n_tokens, cfg.n_vis, cfg.n_cubes, cfg.D,
+                                                      cfg.F, dt), dtype=torch.uint8, device=device)
+        step = lambda: fb.token_ffn(x, Wg, Wu, Wd, t_ids, t_off, text, cfg.n_vis, cfg.p, y=y,
+                                    workspace=ws)
+    for _ in range(args.warmup):
+        step()
+    ms, kt = timed_steps(step, args.steps, torch.cuda.current_stream(), ktimer=True)
+    code, det = fb.read_device_status(ws)
+    if code != fb.OK:
+        raise RuntimeError(f"device status {code} detail {det:#x}")
+    print(json.dumps({"only": args.only, "workload": cfg.name, "ms_per_call": ms / args.steps,
+                      "kernels": {k: round(v[1] / v[0], 4) for k, v in kt.items()},
+                      "device_bytes": torch.cuda.memory_reserved()}))
+    raise SystemExit(0)
 
 
 def measure_e2e(args, cfg, lay, out, y, aws, fws, world, device):
@@ -956,6 +1004,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward-pass measurement")
+    ap.add_argument("--only", choices=["attn", "ffn"], default=None,
+                    help="profiling mode: run one call alone (small device footprint)")
     args = ap.parse_args()
 
     import torch

@@ -171,6 +171,29 @@ __device__ __forceinline__ int fine_bin(float u, int sh, int base) {
   return min(max((int)(__float_as_uint(u) >> sh) - base, 0), kB - 1);
 }
 
+// The emission pass of a group of scores found the cut bin larger than the
+// list: the list holds kL of the bin's scores and the group's in-bin scores
+// after its first `skip` ones did not fit. The row's column becomes the fine
+// histogram of the cut bin, filled with all of them (count mode adds one per
+// score instead of its mass).
+static __device__ __noinline__ void group_to_fine(float* col, float zs, float ref, int sh, int base,
+                                                  bool count, const float* grp, uint32_t inb,
+                                                  int skip) {
+  float u[kL];
+  for (int i = 0; i < kL; ++i) u[i] = fast_exp2(fmaf(col[i * kRows], zs, -ref));
+  for (int b = 0; b < kB; ++b) col[b * kRows] = 0.f;
+  for (int i = 0; i < kL; ++i) col[fine_bin(u[i], sh, base) * kRows] += count ? 1.f : u[i];
+  for (int c = 0; c < 8; ++c) {
+    if (!((inb >> c) & 1u)) continue;
+    if (skip > 0) {
+      --skip;
+      continue;
+    }
+    const float v = fast_exp2(fmaf(grp[c], zs, -ref));
+    col[fine_bin(v, sh, base) * kRows] += count ? 1.f : v;
+  }
+}
+
 // The emission pass found the cut bin larger than the list: the row's column
 // (list scores in rows [0, kL), indices above) becomes a histogram of kB fine
 // bins of the cut bin, filled with the listed scores and the one that did not
@@ -346,6 +369,55 @@ struct RowSel {
       }
     } else if (inb) {
       hist_col[fine_bin(u, fsh, fbase) * kRows] += count_mode ? 1.f : u;
+    }
+    return above;
+  }
+
+  // Emission pass over 8 consecutive scores (columns j0 .. j0 + 7, the first
+  // nv of them candidates): the same decisions as pass2 score by score, with
+  // the masses and keys of the group computed first (independent, so their
+  // latencies overlap) and nothing more done for a group without a cut-bin
+  // score, the common case. Returns the outright selections as bits.
+  __device__ __forceinline__ uint32_t emit8(const uint32_t (&acc)[8], int j0, int nv) {
+    int k[8];
+    float u[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      u[c] = mass(__uint_as_float(acc[c]));
+      k[c] = mass_key(u[c]);
+    }
+    uint32_t above = 0u, inb = 0u;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const bool v = c < nv;
+      above |= (v && k[c] > kcut) ? (1u << c) : 0u;
+      inb |= (v && k[c] >= kcut_lo && k[c] <= kcut) ? (1u << c) : 0u;
+    }
+    if (inb == 0u) return above;
+    if (!sub) {
+      const int ln0 = ln;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        lz_col[ln * kRows] = __uint_as_float(acc[c]);
+        lj_col[ln * kRows] = j0 + c;
+        ln += (((inb >> c) & 1u) && ln < kL) ? 1 : 0;
+      }
+      if (__popc(inb) > kL - ln0) {
+        // the cut bin overflows the list: fine bins, 1/512 octave inside a
+        // regular cut bin; for the window's lowest bin (which holds everything
+        // below), the 8 octaves below it
+        float grp[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) grp[c] = __uint_as_float(acc[c]);
+        sub = true;
+        fsh = kcut_lo == INT_MIN ? 20 : 14;
+        fbase = kcut_lo == INT_MIN ? klo - (kB - 1) : kcut << 6;
+        group_to_fine(hist_col, zs, ref, fsh, fbase, count_mode, grp, inb, kL - ln0);
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if ((inb >> c) & 1u) hist_col[fine_bin(u[c], fsh, fbase) * kRows] += count_mode ? 1.f : u[c];
     }
     return above;
   }

@@ -259,11 +259,7 @@ __global__ void __launch_bounds__(THREADS, 2)
             tmem_ld8(tcol + q * 8, acc);
             tmem_ld_wait();
             if (pass == 1) {
-              uint32_t gb = 0u;
-#pragma unroll
-              for (int c = 0; c < 8; ++c)
-                if (s.pass2(__uint_as_float(acc[c]), j0 + q * 8 + c, q * 8 + c < nv)) gb |= 1u << c;
-              bits |= gb << (q * 8);
+              bits |= s.emit8(acc, j0 + q * 8, nv - q * 8) << (q * 8);
             } else if (s.open) {
               uint32_t gb = 0u;
 #pragma unroll

@@ -79,6 +79,13 @@ def test_calls_reject_bad_arguments_before_the_device():
     for k in (0, -3):
         assert L.adaspark_cube_attn_topk(*args, k, dummy, dummy, ws_bytes, None) == fb.EINVAL
     assert L.adaspark_cube_attn_topk(*args, 4, dummy, dummy, ws_bytes - 1, None) == fb.EINVAL
+    for k in (0, -3):
+        assert L.adaspark_cube_attn_uniform(*args, k, dummy, dummy, ws_bytes, None) == fb.EINVAL
+    assert L.adaspark_cube_attn_uniform(*args, 4, dummy, dummy, ws_bytes - 1, None) == fb.EINVAL
+    # the wait-expiry test hook takes bounds of 1e5 .. 2e9 cycles; off is always accepted
+    for cycles in (0, 99_999, 2_000_000_001):
+        assert L.adaspark_debug_wait_expiry(1, cycles) == fb.EINVAL
+    assert L.adaspark_debug_wait_expiry(0, 0) == fb.OK
     fws = fb.token_ffn_workspace_bytes(544, 512, 16, 256, 512, fb.FP32)
     fargs = [dummy] * 4 + [fb.FP32, dummy, dummy, dummy, 16, 512, 544, 256, 512]
     assert L.adaspark_token_ffn(*fargs, 2.0, dummy, dummy, fws, None) == fb.EINVAL
