@@ -542,8 +542,9 @@ def run_ours(args, rank, world, device):
 def run_only(args, cfg, device):
     """Profiling mode: one of the two calls alone, with only its own inputs,
     output and workspace on the device (about 1.3 GB for AdaS-Attn at 64K), so
-    that a profiler capture of one launch moves little memory. Prints the
-    call's time; not a bench line."""
+    that a profiler capture of one launch moves little memory; or ("step") the
+    step's two calls with nothing else, for a list of its launches. Prints the
+    time per step; not a bench line."""
     import torch
     import ffn_long_video_b200 as fb
     import workloads
@@ -553,7 +554,23 @@ def run_only(args, cfg, device):
                           np.full(cfg.n_text, -1, np.int32)])
     t_ids = torch.from_numpy(ids).to(device)
     t_off = torch.from_numpy(cfg.offsets).to(device)
-    if args.only == "attn":
+    if args.only == "step":
+        lay = {k: v.to(device) for k, v in lay.items()}
+        text = torch.from_numpy((ids == -1).astype(np.uint8)).to(device)
+        out = torch.empty_like(lay["Q"])
+        y = torch.empty((cfg.n_tokens, cfg.D), dtype=torch.float32, device=device)
+        aws = torch.empty(fb.cube_attn_workspace_bytes(cfg.n_tokens, cfg.n_vis, cfg.n_cubes,
+                                                       cfg.hq, cfg.hkv, cfg.d, dt),
+                          dtype=torch.uint8, device=device)
+        ws = torch.empty(fb.token_ffn_workspace_bytes(cfg.n_tokens, cfg.n_vis, cfg.n_cubes, cfg.D,
+                                                      cfg.F, dt), dtype=torch.uint8, device=device)
+
+        def step():
+            fb.cube_attn(lay["Q"], lay["K"], lay["V"], t_ids, t_off, cfg.n_vis, cfg.p, out=out,
+                         workspace=aws)
+            fb.token_ffn(lay["x"], lay["W_gate"], lay["W_up"], lay["W_down"], t_ids, t_off, text,
+                         cfg.n_vis, cfg.p, y=y, workspace=ws)
+    elif args.only == "attn":
         Q, K, V = (lay[k].to(device) for k in ("Q", "K", "V"))
         del lay
         torch.cuda.empty_cache()
@@ -1004,8 +1021,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward-pass measurement")
-    ap.add_argument("--only", choices=["attn", "ffn"], default=None,
-                    help="profiling mode: run one call alone (small device footprint)")
+    ap.add_argument("--only", choices=["attn", "ffn", "step"], default=None,
+                    help="profiling mode: one call alone (small device footprint), or the "
+                         "step's two calls without the extra measurements")
     args = ap.parse_args()
 
     import torch
