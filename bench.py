@@ -217,42 +217,53 @@ def kernel_work(name, cfg, attn_stats, ffn_stats):
     return None, None, None
 
 
-def kernel_table(ktimes, cfg, attn_stats, ffn_stats):
-    """Per kernel: ms per launch, share of the summed kernel time, and the
-    achieved TFLOP/s or GB/s where its algorithmic work is known."""
+def kernel_table(ktimes, calls, cfg, attn_stats, ffn_stats):
+    """Per kernel: ms per library call (a call may launch a kernel several
+    times, e.g. the attention once per KV head), launches per call, share of
+    the summed kernel time, and the achieved TFLOP/s or GB/s where its
+    algorithmic work per call is known. `ktimes` covers `calls` calls."""
     total = sum(v[1] for v in ktimes.values()) or 1.0
     kernels = {}
     for k, (n, ms) in sorted(ktimes.items(), key=lambda kv: -kv[1][1]):
         w, u, b = kernel_work(k, cfg, attn_stats, ffn_stats)
-        e = {"ms_per_launch": round(ms / n, 4), "share": round(ms / total, 4)}
+        e = {"ms_per_call": round(ms / calls, 4), "launches_per_call": round(n / calls, 2),
+             "share": round(ms / total, 4)}
         if w is not None:
             if b == "tensor":
-                e["tflops"] = round(w / (ms / n / 1e3) / 1e12, 1)
+                e["tflops"] = round(w / (ms / calls / 1e3) / 1e12, 1)
             else:
-                e["gbs"] = round(w / (ms / n / 1e3) / 1e9, 1)
+                e["gbs"] = round(w / (ms / calls / 1e3) / 1e9, 1)
         kernels[k] = e
     return kernels
 
 
-def roofline_of(name, n, ms, cfg, attn_stats, ffn_stats, traffic):
-    """Roofline entry of one kernel from its timer totals (n launches, ms)."""
+def roofline_of(name, calls, ms, cfg, attn_stats, ffn_stats, traffic, launches=None):
+    """Roofline entry of one kernel from its timer total `ms` over `calls`
+    library calls (its algorithmic work is counted per call). `traffic` is the
+    DRAM bytes of one launch; with several launches per call it is scaled to
+    the call only when they are equal pieces of it (not known here), so it is
+    reported per launch with the launch count beside it."""
     work, unit, bound = kernel_work(name, cfg, attn_stats, ffn_stats)
     if work is None:
         return None
     peaks, peak_src = load_peaks()
-    per_launch_ms = ms / n
+    per_launch_ms = ms / calls
     if bound == "tensor":
         achieved = work / (per_launch_ms / 1e3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         return {"kernel": name, "bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a step)",
-                "traffic": traffic, "ms_per_launch": round(per_launch_ms, 4)}
+                "traffic": traffic if (launches or calls) == calls else None,
+                "ms_per_call": round(per_launch_ms, 4),
+                "launches_per_call": round((launches or calls) / calls, 2)}
     achieved = work / (per_launch_ms / 1e3) / 1e9
     peak = peaks["hbm_gbs"]
     return {"kernel": name, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
             "unit": "GB/s", "frac": round(achieved / peak, 4), "peak_source": f"{peak_src} hbm_gbs",
-            "traffic": traffic, "ms_per_launch": round(per_launch_ms, 4)}
+            "traffic": traffic if (launches or calls) == calls else None,
+            "ms_per_call": round(per_launch_ms, 4),
+            "launches_per_call": round((launches or calls) / calls, 2)}
 
 
 def max_over_ranks(v, world, device="cpu"):
@@ -313,7 +324,7 @@ def useful_attention_pairs(cfg, selected_pairs):
     return selected_pairs * n_c + cfg.hq * (own + text)
 
 
-def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, dense_ktimes):
+def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, calls, dense_ktimes):
     """What the timed call selected and computed (read from the library after
     the timed region): cubes per row and keep ratio per cube as histograms,
     useful against executed attention FLOPs, the near-margin counters."""
@@ -382,8 +393,8 @@ def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, dense_k
     sel = [ktimes[k] for k in ("select_tc", "select_simt", "cube_mean_keys", "validate")
            if k in ktimes]
     if attn:
-        a_ms = attn[1] / attn[0]
-        s_ms = sum(v[1] / v[0] for v in sel)
+        a_ms = attn[1] / calls                      # per call (one launch per KV head or one)
+        s_ms = sum(v[1] / calls for v in sel)
         out["attention_ms"] = round(a_ms, 4)
         out["selection_ms"] = round(s_ms, 4)
         out["useful_tflops"] = round(useful / (a_ms / 1e3) / 1e12, 1)
@@ -394,7 +405,7 @@ def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, dense_k
                                   "peak_source": f"{src} bf16_tflops_sustained"}
         dattn = dense_ktimes.get("attn_tc") or dense_ktimes.get("attn_simt")
         if dattn:
-            d_ms = dattn[1] / dattn[0]
+            d_ms = dattn[1]                          # one call
             out["dense_attention_ms"] = round(d_ms, 4)
             out["sparse_attention_with_selection_over_dense"] = round((a_ms + s_ms) / d_ms, 4)
     return out
@@ -502,8 +513,9 @@ def run_ours(args, rank, world, device):
 
     # ---------------- roofline of the dominant kernel
     dname, (dn, dms) = max(ktimes.items(), key=lambda kv: kv[1][1])
-    roof = roofline_of(dname, dn, dms, cfg, attn_stats, ffn_stats, load_traffic(dname, cfg.name))
-    kernels = kernel_table(ktimes, cfg, attn_stats, ffn_stats)
+    roof = roofline_of(dname, args.steps, dms, cfg, attn_stats, ffn_stats,
+                       load_traffic(dname, cfg.name), launches=dn)
+    kernels = kernel_table(ktimes, args.steps, cfg, attn_stats, ffn_stats)
 
     # ---------------- e2e through the C ABI with host buffers
     e2e = measure_e2e(args, cfg, lay, out, y, aws, fws, world, device)
@@ -518,7 +530,8 @@ def run_ours(args, rank, world, device):
     # ---------------- the timed workload's sets back in the workspaces
     step()
     torch.cuda.synchronize()
-    sparsity = realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, dense_kt)
+    sparsity = realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, args.steps,
+                                 dense_kt)
 
     # ---------------- backward (fine-tuning step), the forward's sets held fixed
     backward = None
@@ -534,7 +547,7 @@ def run_ours(args, rank, world, device):
                            "value": world * N / (dense_ms / 1e3),
                            "dense_tflop": round((dense["attn"] + dense["ffn"]) / 1e12, 2),
                            "sparse_over_dense": round(ms_step / dense_ms, 4),
-                           "kernels": kernel_table(dense_kt, cfg, attn_stats, ffn_stats)},
+                           "kernels": kernel_table(dense_kt, 1, cfg, attn_stats, ffn_stats)},
         "sparsity": sparsity, "backward": backward, "cfg": cfg, "lay": lay,
     }
 
@@ -804,7 +817,9 @@ def run_stack(args, cfg, world, device):
     att0, ffn0 = stats[0]
     dname, (dn, dms) = max(ktimes.items(), key=lambda kv: kv[1][1])
     # kernel work of layer 0's counters (the layers differ a little)
-    roof = roofline_of(dname, dn, dms, cfg, att0, ffn0, load_traffic(dname, cfg.name))
+    calls = args.steps * cfg.n_layers
+    roof = roofline_of(dname, calls, dms, cfg, att0, ffn0, load_traffic(dname, cfg.name),
+                       launches=dn)
     per_layer = []
     for att, ffn in stats:
         useful = 4.0 * cfg.d * useful_attention_pairs(cfg, att["selected_pairs"])
@@ -821,7 +836,7 @@ def run_stack(args, cfg, world, device):
     return {
         "value": value, "ms_per_step": ms_step, "launches": launches // args.steps,
         "clocks": clk, "roofline": roof,
-        "kernels": kernel_table(ktimes, cfg, att0, ffn0), "e2e": None,
+        "kernels": kernel_table(ktimes, calls, cfg, att0, ffn0), "e2e": None,
         "e2e_note": "not measured for the stack (every step would copy four layers' inputs)",
         "stack": {"layers": cfg.n_layers, "core_ms_per_layer": round(ms_step / cfg.n_layers, 3),
                   "with_projections_ms_per_step": round(full_ms, 3),
@@ -908,9 +923,9 @@ def measure_backward(args, cfg, lay, fws, attn_stats, ffn_stats, world, device, 
         "steps": steps, "forward_plus_backward_ms": round(forward_ms + ms, 3),
         "attention_train_forward_ms": round(attn_train_ms, 3),
         "gpu_launches": launches,
-        "roofline": roofline_of(dname, dn, dms, cfg, attn_stats, ffn_stats,
-                                load_traffic(dname, cfg.name)),
-        "kernels": kernel_table(ktimes, cfg, attn_stats, ffn_stats),
+        "roofline": roofline_of(dname, steps, dms, cfg, attn_stats, ffn_stats,
+                                load_traffic(dname, cfg.name), launches=dn),
+        "kernels": kernel_table(ktimes, steps, cfg, attn_stats, ffn_stats),
     }
 
 

@@ -284,6 +284,7 @@ int adaspark_token_ffn_ex(const void* x, const void* W_gate, const void* W_up,
   a.h = ws + L.h;
   a.sums = reinterpret_cast<float*>(ws + L.sums);
   a.wd16 = ws + L.wd16;
+  a.skip = reinterpret_cast<int32_t*>(ws + L.skip);
   a.hdr = reinterpret_cast<WsHeader*>(ws + L.header);
   a.n_tokens = n_tokens;
   a.n_vis = n_vis;

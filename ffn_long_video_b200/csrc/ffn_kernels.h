@@ -25,6 +25,7 @@ struct FfnArgs {
   void* h;              // [N][F]
   float* sums;          // [C][D]
   void* wd16;           // [D][F] fp16 copy of W_down (bf16 path)
+  int32_t* skip;        // [n_vis] skipped visual rows, cube by cube
   WsHeader* hdr;
   int n_tokens, n_vis, n_cubes, D, F;
   float p;

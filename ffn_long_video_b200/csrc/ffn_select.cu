@@ -1,8 +1,6 @@
 // AdaS-FFN token selection, compaction and mean compensation (key design 3 of
 // the AdaSpark note: rank tokens of a cube by L2 norm, Top-p through the FFN,
 // skipped tokens y_k = x_k + m_bar_i). HBM-bound SIMT kernels.
-#include <algorithm>
-
 #include "ffn_kernels.h"
 
 namespace adaspark {
@@ -187,9 +185,14 @@ __global__ void __launch_bounds__(256) ffn_compact_kernel(FfnArgs a) {
     const int base = a.cube_offsets[j];
     const int n = a.cube_offsets[j + 1] - base;
     if (tid == 0) {
-      int c = 0;
-      for (int u = 0; u < n; ++u)
+      // skipped rows go to their own list: before cube j lie base tokens, of
+      // which cube_start[j] are active
+      int32_t* skip = a.skip + (base - a.cube_start[j]);
+      int c = 0, k = 0;
+      for (int u = 0; u < n; ++u) {
         if (a.active[base + u]) s_rows[c++] = base + u;
+        else skip[k++] = base + u;
+      }
       s_cnt = c;
     }
     __syncthreads();
@@ -224,38 +227,37 @@ __global__ void __launch_bounds__(256) ffn_compact_kernel(FfnArgs a) {
 }
 
 // Skipped visual rows: y_k = x_k + sums_c / |M_c| (mean of FFN over the cube's
-// active tokens). Each warp walks the tokens with a grid-wide stride and takes
-// the skipped ones, so every resident warp has rows to move (a warp per token
-// would leave most warps without work: most tokens are active).
+// active tokens). One warp per skipped row, taken from the compaction's list
+// of skipped rows (so the warps of the first blocks all have a row, and the
+// blocks past the list's end exit at once).
 template <typename T>
 __global__ void __launch_bounds__(256) ffn_compensate_kernel(FfnArgs a) {
   if (status_bad(a.hdr)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n_warps = gridDim.x * 8;
+  const int i = blockIdx.x * 8 + warp;
+  if (i >= a.n_vis - a.cube_start[a.n_cubes]) return;
+  const int t = a.skip[i];
+  const int c = a.cube_ids[t];
+  const float inv = 1.f / (float)a.cube_count[c];
+  const T* xr = reinterpret_cast<const T*>(a.x) + (size_t)t * a.D;
+  const float* sr = a.sums + (size_t)c * a.D;
+  float* yr = a.y + (size_t)t * a.D;
+  // one 16-byte load of x per lane and step (8 bf16 or 4 fp32 features), the
+  // matching sums and stores; four steps in flight
   constexpr int kN = Vec8<T>::kN;
-  for (int t = blockIdx.x * 8 + warp; t < a.n_vis; t += n_warps) {
-    if (a.active[t]) continue;
-    const int c = a.cube_ids[t];
-    const float inv = 1.f / (float)a.cube_count[c];
-    const T* xr = reinterpret_cast<const T*>(a.x) + (size_t)t * a.D;
-    const float* sr = a.sums + (size_t)c * a.D;
-    float* yr = a.y + (size_t)t * a.D;
-    // one 16-byte load of x per lane and step (8 bf16 or 4 fp32 features),
-    // the matching sums and stores; four steps in flight
 #pragma unroll 4
-    for (int e = lane * kN; e < a.D; e += 32 * kN) {
-      float xv[8];
-      Vec8<T>::load(xr + e, xv);
+  for (int e = lane * kN; e < a.D; e += 32 * kN) {
+    float xv[8];
+    Vec8<T>::load(xr + e, xv);
 #pragma unroll
-      for (int h = 0; h < kN; h += 4) {
-        const float4 sv = *reinterpret_cast<const float4*>(sr + e + h);
-        float4 o;
-        o.x = xv[h] + sv.x * inv;
-        o.y = xv[h + 1] + sv.y * inv;
-        o.z = xv[h + 2] + sv.z * inv;
-        o.w = xv[h + 3] + sv.w * inv;
-        *reinterpret_cast<float4*>(yr + e + h) = o;
-      }
+    for (int h = 0; h < kN; h += 4) {
+      const float4 sv = *reinterpret_cast<const float4*>(sr + e + h);
+      float4 o;
+      o.x = xv[h] + sv.x * inv;
+      o.y = xv[h + 1] + sv.y * inv;
+      o.z = xv[h + 2] + sv.z * inv;
+      o.w = xv[h + 3] + sv.w * inv;
+      *reinterpret_cast<float4*>(yr + e + h) = o;
     }
   }
 }
@@ -285,10 +287,7 @@ cudaError_t launch_ffn_compact(const FfnArgs& a, int dtype, cudaStream_t s) {
 
 cudaError_t launch_ffn_compensate(const FfnArgs& a, int dtype, cudaStream_t s) {
   if (a.n_vis == 0 || a.dense) return cudaSuccess;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int blocks = std::min((a.n_vis + 7) / 8, sms * 8);
+  const int blocks = (a.n_vis + 7) / 8;
   if (dtype == ADASPARK_BF16)
     return launch("ffn_compensate", ffn_compensate_kernel<__nv_bfloat16>, dim3(blocks), dim3(256),
                   0, s, a);

@@ -136,6 +136,7 @@ struct FfnLayout {
   size_t h;           // dtype [n_tokens][F] SwiGLU activations
   size_t sums;        // float [C][D] per-cube sums of FFN over active rows
   size_t wd16;        // fp16 [D][F] copy of W_down (bf16 path)
+  size_t skip;        // int32 [n_vis] skipped visual rows, cube by cube
   size_t total;
 };
 
@@ -154,6 +155,7 @@ __host__ __device__ inline FfnLayout make_ffn_layout(int n_tokens, int n_vis, in
   L.h = o; o += align_up((size_t)n_tokens * F * esize, 1024);
   L.sums = o; o += align_up((size_t)(n_cubes > 0 ? n_cubes : 1) * D * 4);
   L.wd16 = o; o += align_up(esize == 2 ? (size_t)D * F * 2 : 0, 1024);
+  L.skip = o; o += align_up((size_t)(n_vis > 0 ? n_vis : 1) * 4);
   L.total = o;
   return L;
 }

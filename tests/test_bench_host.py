@@ -40,14 +40,20 @@ def test_roofline_fraction(monkeypatch):
     monkeypatch.setattr(bench, "load_peaks", lambda: (dict(peaks), "measured"))
     attn = {"key_blocks": 5_000_000, "candidate_pairs": 0}   # about the 64K layer's
     work = bench.kernel_work("attn_tc", CFG, attn, FFN)[0]
-    # two launches of 25 ms each
-    r = bench.roofline_of("attn_tc", 2, 50.0, CFG, attn, FFN, traffic=123)
+    # two calls of 25 ms each, one launch per call
+    r = bench.roofline_of("attn_tc", 2, 50.0, CFG, attn, FFN, traffic=123, launches=2)
     achieved = work / 25e-3 / 1e12
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(achieved, rel=1e-3)
     assert r["peak"] == 1000.0                       # the sustained figure
     assert r["frac"] == pytest.approx(achieved / 1000.0, rel=1e-3)
-    assert r["traffic"] == 123 and r["ms_per_launch"] == 25.0
+    assert r["traffic"] == 123 and r["ms_per_call"] == 25.0
+    # the same calls as five launches each (one per KV head and the text
+    # tiles): the work and time per call are unchanged; one launch's DRAM
+    # counters no longer describe a call
+    r5 = bench.roofline_of("attn_tc", 2, 50.0, CFG, attn, FFN, traffic=123, launches=10)
+    assert r5["achieved"] == r["achieved"] and r5["traffic"] is None
+    assert r5["launches_per_call"] == 5.0
     h = bench.roofline_of("ffn_select", 1, 2.0, CFG, ATTN, FFN, traffic=None)
     gbs = CFG.n_vis * CFG.D * 2 / 2e-3 / 1e9
     assert h["bound"] == "hbm" and h["achieved"] == pytest.approx(gbs, rel=1e-3)
@@ -56,10 +62,11 @@ def test_roofline_fraction(monkeypatch):
 
 
 def test_kernel_table_shares():
-    t = bench.kernel_table({"attn_tc": (2, 30.0), "ffn_select": (1, 10.0)}, CFG, ATTN, FFN)
+    # one call; the attention launched twice in it
+    t = bench.kernel_table({"attn_tc": (2, 30.0), "ffn_select": (1, 10.0)}, 1, CFG, ATTN, FFN)
     assert list(t) == ["attn_tc", "ffn_select"]      # largest share first
     assert t["attn_tc"]["share"] == 0.75 and t["ffn_select"]["share"] == 0.25
-    assert t["attn_tc"]["ms_per_launch"] == 15.0
+    assert t["attn_tc"]["ms_per_call"] == 30.0 and t["attn_tc"]["launches_per_call"] == 2.0
     assert "tflops" in t["attn_tc"] and "gbs" in t["ffn_select"]
 
 
