@@ -25,8 +25,7 @@ bool attn_sizes_ok(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d,
   if (n_vis == 0 && n_cubes != 0) return false;
   if ((long long)n_cubes > n_vis) return false;
   if (hq < 1 || hkv < 1 || hq % hkv != 0 || hkv * d > 1024) return false;
-  if (dtype == ADASPARK_BF16) return d == 128;
-  if (dtype == ADASPARK_FP32) return d == 64 || d == 128;
+  if (dtype == ADASPARK_BF16 || dtype == ADASPARK_FP32) return d == 64 || d == 128;
   return false;
 }
 
@@ -317,7 +316,9 @@ int adaspark_token_ffn_ex(const void* x, const void* W_gate, const void* W_up,
 
 size_t adaspark_cube_attn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int hq,
                                              int hkv, int d, int dtype) {
-  if (dtype != ADASPARK_BF16 || !attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype))
+  // the backward kernels are built for head_dim 128
+  if (dtype != ADASPARK_BF16 || d != 128 ||
+      !attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype))
     return 0;
   return make_attn_bwd_layout(make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d)).total;
 }
@@ -334,6 +335,7 @@ int adaspark_cube_attn_backward(const void* Q, const void* K, const void* V, con
   if (dtype == ADASPARK_FP32) return ADASPARK_EUNSUPPORTED;
   if (dtype != ADASPARK_BF16 || !attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype))
     return ADASPARK_EINVAL;
+  if (d != 128) return ADASPARK_EUNSUPPORTED;   // the backward kernels are built for 128
   const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
   const AttnBwdLayout L = make_attn_bwd_layout(G);
   if (workspace_bytes < L.total || !aligned(workspace, kAlign) || !aligned(fwd_workspace, kAlign))

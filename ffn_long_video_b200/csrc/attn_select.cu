@@ -44,41 +44,57 @@ __global__ void validate_layout_kernel(const int32_t* __restrict__ cube_ids,
 // kbar[kv][j][:] = mean of K over cube j (fp64 accumulation, fp32 result) and
 // its split kbar = hi + mid + lo into bf16 parts (products with bf16 queries are
 // exact, so three tensor-core passes reproduce the fp32 dot product).
-// One block per cube, one thread per (kv, dim) element.
-// ---------------------------------------------------------------------------
+// One block per cube; each thread sums one 16-byte vector of a token's row
+// (8 bf16 or 4 fp32 elements of one KV head) over the cube's tokens.
 template <typename T>
 __global__ void cube_mean_kernel(const T* __restrict__ K, const int32_t* __restrict__ off,
                                  float* __restrict__ kbar, __nv_bfloat16* __restrict__ split,
                                  int n_cubes, int hkv, int d, WsHeader* hdr) {
+  constexpr int V = 16 / sizeof(T);
   if (status_bad(hdr)) return;
   const int j = blockIdx.x;
-  const int e = threadIdx.x;  // kv * d + dim
   const int row = hkv * d;
+  const int e = threadIdx.x * V;  // first (kv * d + dim) element of this thread
   if (e >= row) return;
   const int a = off[j], b = off[j + 1];
-  // four independent partial sums keep several loads in flight (bf16 sums of
-  // a cube are exact in fp64, so the order does not change the result)
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
-  int t = a;
-  for (; t + 4 <= b; t += 4) {
+  // two interleaved partial sums keep two loads in flight (bf16 sums of a
+  // cube are exact in fp64 for any realistic spread of magnitudes; the order
+  // is fixed, so the result is deterministic in any case)
+  double acc0[V], acc1[V];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u] += (double)to_f32(K[(size_t)(t + u) * row + e]);
+  for (int i = 0; i < V; ++i) acc0[i] = acc1[i] = 0.0;
+  auto add = [&](double (&acc)[V], int t) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(K + (size_t)t * row + e);
+    const T* v = reinterpret_cast<const T*>(&raw);
+#pragma unroll
+    for (int i = 0; i < V; ++i) acc[i] += (double)to_f32(v[i]);
+  };
+  int t = a;
+  for (; t + 2 <= b; t += 2) {
+    add(acc0, t);
+    add(acc1, t + 1);
   }
-  for (; t < b; ++t) acc[0] += (double)to_f32(K[(size_t)t * row + e]);
-  const double sum = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  const float mean = (float)(sum / (double)(b - a));
+  if (t < b) add(acc0, t);
   const int kv = e / d, dim = e - kv * d;
   const size_t o = ((size_t)kv * n_cubes + j) * d + dim;
-  kbar[o] = mean;
-  const __nv_bfloat16 hi = __float2bfloat16_rn(mean);
-  const float r1 = mean - __bfloat162float(hi);
-  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-  const float r2 = r1 - __bfloat162float(mid);
-  const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
   const size_t plane = (size_t)hkv * n_cubes * d;
-  split[o] = hi;
-  split[plane + o] = mid;
-  split[2 * plane + o] = lo;
+  float mean[V];
+  __nv_bfloat16 hi[V], mid[V], lo[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    mean[i] = (float)((acc0[i] + acc1[i]) / (double)(b - a));
+    hi[i] = __float2bfloat16_rn(mean[i]);
+    const float r1 = mean[i] - __bfloat162float(hi[i]);
+    mid[i] = __float2bfloat16_rn(r1);
+    lo[i] = __float2bfloat16_rn(r1 - __bfloat162float(mid[i]));
+  }
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    kbar[o + i] = mean[i];
+    split[o + i] = hi[i];
+    split[plane + o + i] = mid[i];
+    split[2 * plane + o + i] = lo[i];
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -248,10 +264,10 @@ cudaError_t launch_cube_mean(const void* K, int dtype, const int32_t* off, float
   const int threads = G.hkv * G.d;
   if (dtype == ADASPARK_BF16)
     return launch("cube_mean_keys", cube_mean_kernel<__nv_bfloat16>, dim3(G.n_cubes),
-                  dim3(threads), 0, s, (const __nv_bfloat16*)K, off, kbar, split, G.n_cubes,
+                  dim3(threads / 8), 0, s, (const __nv_bfloat16*)K, off, kbar, split, G.n_cubes,
                   G.hkv, G.d, hdr);
-  return launch("cube_mean_keys", cube_mean_kernel<float>, dim3(G.n_cubes), dim3(threads), 0, s,
-                (const float*)K, off, kbar, split, G.n_cubes, G.hkv, G.d, hdr);
+  return launch("cube_mean_keys", cube_mean_kernel<float>, dim3(G.n_cubes), dim3(threads / 4),
+                0, s, (const float*)K, off, kbar, split, G.n_cubes, G.hkv, G.d, hdr);
 }
 
 template <typename T, int D>

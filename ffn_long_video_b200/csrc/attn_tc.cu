@@ -35,14 +35,23 @@ namespace fa {
 constexpr int STAGES = 2;
 constexpr int THREADS = 224;
 constexpr int RING = 64;
-constexpr int Q_BYTES = 128 * 256;        // 128 rows x 128 dims bf16 (two 64-dim halves)
-constexpr int KV_BYTES = 4 * 8192;        // K (2 halves) + V (2 halves), 64 keys each
-constexpr int K_BYTES = 2 * 8192;         // one K (or V) block: two 64-dim halves
+// Head dimension D (64 or 128) in 64-dim halves: the query tile is 128 rows x
+// D dims bf16, a K (or V) block 64 keys x D dims, each stored as 64-dim halves
+// of 8 KB (per 64 rows) in the 128-byte swizzled layout.
+template <int D> struct Dim {
+  static constexpr int HALVES = D / 64;
+  static constexpr int Q_BYTES = 128 * 2 * D;
+  static constexpr int K_BYTES = HALVES * 8192;   // one K (or V) block
+  static constexpr int KV_BYTES = 2 * K_BYTES;
+};
 struct Desc {
   int k0, nk, j, pad;
   uint32_t mask[4];
 };
-constexpr size_t SMEM_BYTES = 1024 + Q_BYTES + STAGES * KV_BYTES + RING * sizeof(Desc) + 2048;
+template <int D>
+constexpr size_t smem_bytes() {
+  return 1024 + Dim<D>::Q_BYTES + STAGES * Dim<D>::KV_BYTES + RING * sizeof(Desc) + 2048;
+}
 constexpr float kRescale = 8.0f;          // log2 headroom before O is rescaled
 
 __device__ __forceinline__ float ex2(float x) {
@@ -85,10 +94,12 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
 // pair hi + lo (lo = P - hi, in the second half of the S buffer, whose
 // scores were read before), so O is exact to about 2^-17 of each term, and O is
 // also written in fp32 to a.o32; the backward takes D_r = dO_r . O_r from it.
-template <bool TRAIN>
+template <bool TRAIN, int D>
 __global__ void __launch_bounds__(THREADS, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    AttnArgs a) {
+  constexpr int Q_BYTES = Dim<D>::Q_BYTES, K_BYTES = Dim<D>::K_BYTES, KV_BYTES = Dim<D>::KV_BYTES;
+  constexpr int HALVES = Dim<D>::HALVES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -238,8 +249,9 @@ __global__ void __launch_bounds__(THREADS, 2)
         const int s = blk % STAGES;
         if (!mbar_wait(&v_empty[s], ((blk / STAGES) & 1) ^ 1, &s_abort, hdr, 0x7110u, WL)) return false;
         mbar_expect_tx(&v_full[s], K_BYTES);
-        tma_load_3d(&mapV, &v_full[s], sV + s * K_BYTES, 0, T.kv, k0);
-        tma_load_3d(&mapV, &v_full[s], sV + s * K_BYTES + 8192, 64, T.kv, k0);
+#pragma unroll
+        for (int hf = 0; hf < HALVES; ++hf)
+          tma_load_3d(&mapV, &v_full[s], sV + s * K_BYTES + hf * 8192, hf * 64, T.kv, k0);
         nv = blk + 1;
         return true;
       };
@@ -257,8 +269,9 @@ __global__ void __launch_bounds__(THREADS, 2)
           break;
         }
         mbar_expect_tx(&k_full[s], K_BYTES);
-        tma_load_3d(&mapK, &k_full[s], sK + s * K_BYTES, 0, T.kv, k0);
-        tma_load_3d(&mapK, &k_full[s], sK + s * K_BYTES + 8192, 64, T.kv, k0);
+#pragma unroll
+        for (int hf = 0; hf < HALVES; ++hf)
+          tma_load_3d(&mapK, &k_full[s], sK + s * K_BYTES + hf * 8192, hf * 64, T.kv, k0);
         if (i > 0 && !load_v(i - 1, prev_k0)) {
           ok = false;
           break;
@@ -284,7 +297,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = make_idesc_bf16(128, 64);
-      constexpr uint32_t idesc_o = make_idesc_bf16(128, 128, true);
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, D, true);
       const uint32_t q_addr = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, &s_abort, hdr, 0x7200u, WL);
       tc_fence_after();
@@ -324,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, 2)
         const uint32_t k_addr = smem_u32(sKV + s * K_BYTES);
         const uint32_t d_s = tmem_base + 128 + sb * 64;
 #pragma unroll
-        for (int dc = 0; dc < 2; ++dc)
+        for (int dc = 0; dc < HALVES; ++dc)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024);
@@ -356,9 +369,9 @@ __global__ void __launch_bounds__(THREADS, 2)
     const float scale = a.scale_log2;
     {
       const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
-      const uint4* src = reinterpret_cast<const uint4*>(Qg + ((size_t)t * G.hq + h) * 128);
+      const uint4* src = reinterpret_cast<const uint4*>(Qg + ((size_t)t * G.hq + h) * D);
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
+      for (int c = 0; c < D / 8; ++c) {
         const uint4 v = valid ? src[c] : make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(sQ + (c >> 3) * 16384 + sw128_offset(row, c & 7)) = v;
       }
@@ -466,7 +479,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           }
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < 128; c += 32) {
+          for (int c = 0; c < D; c += 32) {
             uint32_t o[32];
             tmem_ld32(tmem_base + lane_base + c, o);
             tmem_ld_wait();
@@ -534,9 +547,9 @@ __global__ void __launch_bounds__(THREADS, 2)
       // the row's softmax is 2^(s * scale - lse): kept for the backward pass
       if (valid && a.lse) a.lse[(size_t)t * G.hq + h] = m_used + __log2f(l);
       __nv_bfloat16* dst =
-          reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * 128;
+          reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * D;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
         tmem_ld32(tmem_base + lane_base + c, o);
         tmem_ld_wait();
@@ -551,7 +564,7 @@ __global__ void __launch_bounds__(THREADS, 2)
           for (int x = 0; x < 4; ++x)
             d4[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
           if (TRAIN) {
-            float4* o4 = reinterpret_cast<float4*>(a.o32 + ((size_t)t * G.hq + h) * 128 + c);
+            float4* o4 = reinterpret_cast<float4*>(a.o32 + ((size_t)t * G.hq + h) * D + c);
 #pragma unroll
             for (int x = 0; x < 8; ++x)
               o4[x] = make_float4(__uint_as_float(o[4 * x]) * inv,
@@ -588,11 +601,12 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   if (!encode_tmap_bf16(&mK, a.K, 3, dims, strides, box) ||
       !encode_tmap_bf16(&mV, a.V, 3, dims, strides, box))
     return cudaErrorInvalidValue;
-  auto k = a.o32 ? fa::attn_tc_kernel<true> : fa::attn_tc_kernel<false>;
-  cudaError_t e =
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fa::SMEM_BYTES);
+  auto k = G.d == 64 ? (a.o32 ? fa::attn_tc_kernel<true, 64> : fa::attn_tc_kernel<false, 64>)
+                     : (a.o32 ? fa::attn_tc_kernel<true, 128> : fa::attn_tc_kernel<false, 128>);
+  const size_t smem = G.d == 64 ? fa::smem_bytes<64>() : fa::smem_bytes<128>();
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch("attn_tc", k, dim3(blocks), dim3(fa::THREADS), fa::SMEM_BYTES, s, mK, mV, a);
+  return launch("attn_tc", k, dim3(blocks), dim3(fa::THREADS), smem, s, mK, mV, a);
 }
 
 }  // namespace adaspark

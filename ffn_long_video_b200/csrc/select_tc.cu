@@ -33,13 +33,19 @@ constexpr int STAGES = 3;
 constexpr int SBUF = 4;                         // TMEM score buffers
 constexpr int THREADS = 192;
 constexpr int BOX_BYTES = NC * 128;             // 32 cubes x 64 dims bf16
-constexpr int CHUNK_BYTES = 6 * BOX_BYTES;      // 3 parts x 2 halves
-constexpr size_t SMEM_BYTES = 1024 + STAGES * CHUNK_BYTES + sizeof(sel::Smem) + 256;
+// kbar chunk of head dimension D: 3 parts x D / 64 halves of BOX_BYTES
+template <int D> constexpr int chunk_bytes() { return 3 * (D / 64) * BOX_BYTES; }
+template <int D> constexpr size_t smem_bytes() {
+  return 1024 + STAGES * chunk_bytes<D>() + sizeof(sel::Smem) + 256;
+}
 constexpr int TMEM_COLS = 256;                  // S buffers 0..127, Q tile 128..191
 constexpr int Q_COL = 128;
 
+template <int D>
 __global__ void __launch_bounds__(THREADS, 2)
     select_tc_kernel(const __grid_constant__ CUtensorMap mapKb, SelectArgs a) {
+  constexpr int HALVES = D / 64;                // 64-dim halves of a query / kbar row
+  constexpr int CHUNK_BYTES = chunk_bytes<D>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -119,9 +125,9 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
           for (int part = 0; part < 3; ++part)
 #pragma unroll
-            for (int dc = 0; dc < 2; ++dc)
-              tma_load_3d(&mapKb, &k_full[s], st + (part * 2 + dc) * BOX_BYTES, dc * 64, c * NC,
-                          part * G.hkv + kv);
+            for (int dc = 0; dc < HALVES; ++dc)
+              tma_load_3d(&mapKb, &k_full[s], st + (part * HALVES + dc) * BOX_BYTES, dc * 64,
+                          c * NC, part * G.hkv + kv);
         }
       }
       if (!ok) {
@@ -161,11 +167,11 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
           for (int part = 0; part < 3; ++part)
 #pragma unroll
-            for (int dc = 0; dc < 2; ++dc)
+            for (int dc = 0; dc < HALVES; ++dc)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t bd =
-                    make_sdesc_sw128(k_addr + (part * 2 + dc) * BOX_BYTES + kk * 32, 16, 1024);
+                const uint64_t bd = make_sdesc_sw128(
+                    k_addr + (part * HALVES + dc) * BOX_BYTES + kk * 32, 16, 1024);
                 umma_bf16_ts(d, q_tmem + dc * 32 + kk * 8, bd, idesc,
                              (part | dc | kk) != 0 ? 1u : 0u);
               }
@@ -187,12 +193,12 @@ __global__ void __launch_bounds__(THREADS, 2)
     const int t = R.t, h = R.h;
     const int own = valid ? a.cube_ids[t] : -1;
     {
-      // query row -> 64 TMEM columns of this row's lane (two bf16 per column)
+      // query row -> D / 2 TMEM columns of this row's lane (two bf16 per column)
       const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
-      const uint4* src = reinterpret_cast<const uint4*>(Qg + ((size_t)t * G.hq + h) * 128);
+      const uint4* src = reinterpret_cast<const uint4*>(Qg + ((size_t)t * G.hq + h) * D);
       const uint32_t qlane = tmem_base + ((uint32_t)(wq * 32) << 16) + Q_COL;
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < HALVES; ++half) {
         uint32_t r[32];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -370,11 +376,11 @@ cudaError_t launch_select_tc(const SelectArgs& a, cudaStream_t s) {
   const uint64_t strides[2] = {(uint64_t)G.d * 2, (uint64_t)G.n_cubes * G.d * 2};
   const uint32_t box[3] = {64, (uint32_t)seltc::NC, 1};
   if (!encode_tmap_bf16(&m, a.kbar_split, 3, dims, strides, box)) return cudaErrorInvalidValue;
-  auto k = seltc::select_tc_kernel;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)seltc::SMEM_BYTES);
+  auto k = G.d == 64 ? seltc::select_tc_kernel<64> : seltc::select_tc_kernel<128>;
+  const size_t smem = G.d == 64 ? seltc::smem_bytes<64>() : seltc::smem_bytes<128>();
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch("select_tc", k, dim3(G.n_vtiles), dim3(seltc::THREADS), seltc::SMEM_BYTES, s, m, a);
+  return launch("select_tc", k, dim3(G.n_vtiles), dim3(seltc::THREADS), smem, s, m, a);
 }
 
 }  // namespace adaspark

@@ -132,7 +132,7 @@ size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq
  * A text token attends densely and causally to every earlier token.
  *
  *   Q [n_tokens, hq, d], K/V [n_tokens, hkv, d]: device, row-major, element type
- *       `dtype` (BF16 for d = 128, FP32 for d = 64 or 128);
+ *       `dtype` (BF16 or FP32), d = 64 or 128;
  *   cube_ids [n_tokens], cube_offsets [n_cubes + 1]: device int32 (layout above);
  *   n_vis = cube_offsets[n_cubes] (checked on the device);
  *   p in (0, 1]; hq % hkv == 0; every cube holds 1..256 tokens;
@@ -194,7 +194,7 @@ int adaspark_cube_attn_train(const void *Q, const void *K, const void *V, int dt
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /* Device workspace bytes needed by adaspark_cube_attn_backward (0 when the
- * sizes are invalid or dtype is not ADASPARK_BF16). */
+ * sizes are invalid, dtype is not ADASPARK_BF16 or d is not 128). */
 size_t adaspark_cube_attn_backward_workspace(int n_tokens, int n_vis, int n_cubes, int hq,
                                              int hkv, int d, int dtype);
 
@@ -223,9 +223,10 @@ size_t adaspark_cube_attn_backward_workspace(int n_tokens, int n_vis, int n_cube
  * dS are rounded to bf16 as operands; the softmax is recomputed in fp32, and
  * D_r is summed from the same fp32 P and dP rather than taken from the bf16
  * output, so each row's dS sums to zero up to fp32 rounding).
- * Deterministic: no atomics. Only ADASPARK_BF16 (ADASPARK_FP32 returns
- * ADASPARK_EUNSUPPORTED); a forward call that reported a device error makes
- * this call report ADASPARK_EDEVICE. Other errors as for adaspark_cube_attn. */
+ * Deterministic: no atomics. Only ADASPARK_BF16 with d = 128 (ADASPARK_FP32
+ * and d = 64 return ADASPARK_EUNSUPPORTED); a forward call that reported a
+ * device error makes this call report ADASPARK_EDEVICE. Other errors as for
+ * adaspark_cube_attn. */
 int adaspark_cube_attn_backward(const void *Q, const void *K, const void *V, const void *dO,
                                 int dtype, const int32_t *cube_ids,
                                 const int32_t *cube_offsets, int n_cubes, int n_vis,

@@ -60,7 +60,10 @@ def test_workspace_queries():
     assert fb.cube_attn_workspace_bytes(65792, 65536, 1024, 28, 4, 128, fb.BF16) > 0
     assert fb.cube_attn_workspace_bytes(544, 512, 16, 4, 1, 64, fb.FP32) > 0
     assert fb.cube_attn_workspace_bytes(544, 512, 16, 5, 2, 64, fb.FP32) == 0   # hq % hkv
-    assert fb.cube_attn_workspace_bytes(544, 512, 16, 4, 1, 64, fb.BF16) == 0   # bf16 needs d=128
+    assert fb.cube_attn_workspace_bytes(544, 512, 16, 4, 1, 64, fb.BF16) > 0    # bf16, d = 64
+    assert fb.cube_attn_workspace_bytes(544, 512, 16, 4, 1, 96, fb.BF16) == 0   # d in {64, 128}
+    # the backward is built for d = 128 only
+    assert fb.cube_attn_backward_workspace_bytes(544, 512, 16, 4, 1, 64) == 0
     assert fb.cube_attn_workspace_bytes(544, 600, 16, 4, 1, 64, fb.FP32) == 0   # n_vis > n_tokens
     assert fb.token_ffn_workspace_bytes(65792, 65536, 1024, 3584, 18944, fb.BF16) > 0
     assert fb.token_ffn_workspace_bytes(544, 512, 16, 250, 512, fb.FP32) == 0
@@ -98,6 +101,10 @@ def test_calls_reject_bad_arguments_before_the_device():
 def test_backward_layer_and_train_calls_reject_bad_arguments_before_the_device():
     L = fb.lib()
     d = ctypes.c_void_p(256)
+    # the attention backward is built for head_dim 128: bf16 with d = 64 is
+    # refused before any device work
+    assert L.adaspark_cube_attn_backward(d, d, d, d, fb.BF16, d, d, 16, 512, 544, 4, 1, 64, d, d,
+                                         d, d, d, 1 << 30, None) == fb.EUNSUPPORTED
     # workspace queries: bf16 only for the backward and the training forward
     assert fb.cube_attn_backward_workspace_bytes(65792, 65536, 1024, 28, 4, 128) > 0
     assert fb.cube_attn_backward_workspace_bytes(544, 512, 16, 4, 1, 64, fb.FP32) == 0

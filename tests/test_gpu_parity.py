@@ -29,6 +29,9 @@ SMALL = {
                                           n_text=9, D=128, hq=4, hkv=1, d=64, F=256,
                                           dtype="fp32", seed=8,
                                           cube_sizes=(1, 63, 32, 32, 40, 24, 60, 1, 1, 2)),
+    # bf16 with head_dim 64 (one 64-dim half per query and key row)
+    "d64-bf16": workloads.small_config(name="d64", grid=(8, 16, 16), cube=(4, 4, 4), n_text=40,
+                                       D=256, hq=8, hkv=2, d=64, F=256, seed=15),
 }
 
 
@@ -159,7 +162,7 @@ def test_262k_four_layer_stack_sampled():
 
 
 # ------------------------------------------------------------------ cut-bin stress
-@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("fp32", 64)])
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("fp32", 64)])
 def test_attn_uniform_means_closed_form(dtype, d):
     """Every key identical -> every cube mean identical -> P uniform over the c
     preceding cubes: exact ties, the cut bin holds all of them, and the Top-p
@@ -235,3 +238,13 @@ def test_attn_crowded_cut_bins():
         st = fb.attn_read_stats(ws)
         print("crowded", p, rep, "rows needing extra passes", st["overflow_rows"])
         assert st["overflow_rows"] > 0
+
+
+def test_attn_d64_training_mode_and_variants():
+    """bf16 with head_dim 64 through the training-mode forward (P as a bf16
+    pair, fp32 O kept), Top-K and Uniform Sampling, against the oracle."""
+    case = parity.make_case(SMALL["d64-bf16"])
+    for kw in ({"train": True}, {"k": 3}, {"uniform": 4}):
+        rep = {}
+        parity.check_attn(case, report=rep, **kw)
+        print("d64", kw, rep)
