@@ -44,37 +44,54 @@ __global__ void validate_layout_kernel(const int32_t* __restrict__ cube_ids,
 // kbar[kv][j][:] = mean of K over cube j (fp64 accumulation, fp32 result) and
 // its split kbar = hi + mid + lo into bf16 parts (products with bf16 queries are
 // exact, so three tensor-core passes reproduce the fp32 dot product).
-// One block per cube; each thread sums one 16-byte vector of a token's row
-// (8 bf16 or 4 fp32 elements of one KV head) over the cube's tokens.
+// One block per cube: thread (x, y) sums one 16-byte vector of a token's row
+// (8 bf16 or 4 fp32 elements of one KV head) over the cube's tokens y, y + S,
+// y + 2S, ... (S = blockDim.y token slices; eight loads in flight per thread),
+// and the S partial sums meet in shared memory.
+constexpr int kMeanThreads = 256;
 template <typename T>
-__global__ void cube_mean_kernel(const T* __restrict__ K, const int32_t* __restrict__ off,
-                                 float* __restrict__ kbar, __nv_bfloat16* __restrict__ split,
-                                 int n_cubes, int hkv, int d, WsHeader* hdr) {
+__global__ void __launch_bounds__(kMeanThreads)
+    cube_mean_kernel(const T* __restrict__ K, const int32_t* __restrict__ off,
+                     float* __restrict__ kbar, __nv_bfloat16* __restrict__ split, int n_cubes,
+                     int hkv, int d, WsHeader* hdr) {
   constexpr int V = 16 / sizeof(T);
+  __shared__ double part[kMeanThreads * V];
   if (status_bad(hdr)) return;
   const int j = blockIdx.x;
-  const int row = hkv * d;
-  const int e = threadIdx.x * V;  // first (kv * d + dim) element of this thread
-  if (e >= row) return;
+  const int row = hkv * d;               // blockDim.x * V == row (the launcher's shape)
+  const int x = threadIdx.x, y = threadIdx.y, S = blockDim.y;
+  const int e = x * V;                   // first (kv * d + dim) element of this thread
   const int a = off[j], b = off[j + 1];
-  // two interleaved partial sums keep two loads in flight (bf16 sums of a
-  // cube are exact in fp64 for any realistic spread of magnitudes; the order
-  // is fixed, so the result is deterministic in any case)
-  double acc0[V], acc1[V];
+  // bf16 sums of a cube are exact in fp64 for any realistic spread of
+  // magnitudes; the order is fixed, so the result is deterministic in any case
+  constexpr int U = 8;
+  double acc0[V];
 #pragma unroll
-  for (int i = 0; i < V; ++i) acc0[i] = acc1[i] = 0.0;
-  auto add = [&](double (&acc)[V], int t) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(K + (size_t)t * row + e);
-    const T* v = reinterpret_cast<const T*>(&raw);
+  for (int i = 0; i < V; ++i) acc0[i] = 0.0;
+  for (int t = a + y; t < b; t += U * S) {
+    uint4 raw[U];
 #pragma unroll
-    for (int i = 0; i < V; ++i) acc[i] += (double)to_f32(v[i]);
-  };
-  int t = a;
-  for (; t + 2 <= b; t += 2) {
-    add(acc0, t);
-    add(acc1, t + 1);
+    for (int u = 0; u < U; ++u) {
+      const int tt = t + u * S;
+      raw[u] = tt < b ? __ldg(reinterpret_cast<const uint4*>(K + (size_t)tt * row + e))
+                      : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const T* v = reinterpret_cast<const T*>(&raw[u]);
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc0[i] += (double)to_f32(v[i]);
+    }
   }
-  if (t < b) add(acc0, t);
+  if (S > 1) {
+#pragma unroll
+    for (int i = 0; i < V; ++i) part[(y * blockDim.x + x) * V + i] = acc0[i];
+    __syncthreads();
+    if (y != 0) return;
+    for (int z = 1; z < S; ++z)
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc0[i] += part[(z * blockDim.x + x) * V + i];
+  }
   const int kv = e / d, dim = e - kv * d;
   const size_t o = ((size_t)kv * n_cubes + j) * d + dim;
   const size_t plane = (size_t)hkv * n_cubes * d;
@@ -82,7 +99,7 @@ __global__ void cube_mean_kernel(const T* __restrict__ K, const int32_t* __restr
   __nv_bfloat16 hi[V], mid[V], lo[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) {
-    mean[i] = (float)((acc0[i] + acc1[i]) / (double)(b - a));
+    mean[i] = (float)(acc0[i] / (double)(b - a));
     hi[i] = __float2bfloat16_rn(mean[i]);
     const float r1 = mean[i] - __bfloat162float(hi[i]);
     mid[i] = __float2bfloat16_rn(r1);
@@ -261,13 +278,16 @@ cudaError_t launch_validate(const int32_t* cube_ids, const int32_t* off, const u
 cudaError_t launch_cube_mean(const void* K, int dtype, const int32_t* off, float* kbar,
                              __nv_bfloat16* split, const AttnGeom& G, WsHeader* hdr,
                              cudaStream_t s) {
-  const int threads = G.hkv * G.d;
+  // hkv * d <= 1024 (attn_sizes_ok): at most 128 (bf16) or 256 (fp32) vector
+  // threads per token row, and up to 8 token slices within 256 threads
+  const int rx = G.hkv * G.d / (dtype == ADASPARK_BF16 ? 8 : 4);
+  const int sy = std::max(1, std::min(8, kMeanThreads / rx));
   if (dtype == ADASPARK_BF16)
     return launch("cube_mean_keys", cube_mean_kernel<__nv_bfloat16>, dim3(G.n_cubes),
-                  dim3(threads / 8), 0, s, (const __nv_bfloat16*)K, off, kbar, split, G.n_cubes,
+                  dim3(rx, sy), 0, s, (const __nv_bfloat16*)K, off, kbar, split, G.n_cubes,
                   G.hkv, G.d, hdr);
-  return launch("cube_mean_keys", cube_mean_kernel<float>, dim3(G.n_cubes), dim3(threads / 4),
-                0, s, (const float*)K, off, kbar, split, G.n_cubes, G.hkv, G.d, hdr);
+  return launch("cube_mean_keys", cube_mean_kernel<float>, dim3(G.n_cubes), dim3(rx, sy), 0, s,
+                (const float*)K, off, kbar, split, G.n_cubes, G.hkv, G.d, hdr);
 }
 
 template <typename T, int D>

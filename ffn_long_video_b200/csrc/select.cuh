@@ -61,6 +61,13 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// max(a, b, c) in one instruction (three-input form of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // (s1, j1) comes before (s2, j2) in the (score desc, index asc) order.
 __device__ __forceinline__ bool before(float s1, int j1, float s2, int j2) {
   return s1 > s2 || (s1 == s2 && j1 < j2);
@@ -308,6 +315,28 @@ struct RowSel {
   __device__ __forceinline__ void add_score(float u, bool valid) {
     const int k = max(mass_key(valid ? u : 0.f), klo);
     hist_col[(k & (kB - 1)) * kRows] += valid ? (count_mode ? 1.f : u) : 0.f;
+  }
+
+  // Histogram update of four scores of a full chunk (keys within the window,
+  // which raise() has made reach the chunk's maximum). The four bins are read
+  // before any is written; a score whose bin equals an earlier one's adds to
+  // that score's new value, and the stores go out in order, so every bin ends
+  // with exactly the sums of one update after another.
+  __device__ __forceinline__ void add_quad(float u0, float u1, float u2, float u3) {
+    const int k0 = max(mass_key(u0), klo) & (kB - 1), k1 = max(mass_key(u1), klo) & (kB - 1);
+    const int k2 = max(mass_key(u2), klo) & (kB - 1), k3 = max(mass_key(u3), klo) & (kB - 1);
+    const float w0 = count_mode ? 1.f : u0, w1 = count_mode ? 1.f : u1;
+    const float w2 = count_mode ? 1.f : u2, w3 = count_mode ? 1.f : u3;
+    const float h0 = hist_col[k0 * kRows], h1 = hist_col[k1 * kRows];
+    const float h2 = hist_col[k2 * kRows], h3 = hist_col[k3 * kRows];
+    const float v0 = h0 + w0;
+    const float v1 = (k1 == k0 ? v0 : h1) + w1;
+    const float v2 = (k2 == k1 ? v1 : k2 == k0 ? v0 : h2) + w2;
+    const float v3 = (k3 == k2 ? v2 : k3 == k1 ? v1 : k3 == k0 ? v0 : h3) + w3;
+    hist_col[k0 * kRows] = v0;
+    hist_col[k1 * kRows] = v1;
+    hist_col[k2 * kRows] = v2;
+    hist_col[k3 * kRows] = v3;
   }
 
   // One score of the histogram pass (raises the window when needed).

@@ -242,7 +242,22 @@ __global__ void __launch_bounds__(THREADS, 2)
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&s_empty[sb]);
-            if (nv > 0) {
+            if (nv >= NC) {
+              // a full chunk: no candidate tests; the maximum as a tree
+              auto f = [&](int u) { return __uint_as_float(acc[u]); };
+              float mx[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) mx[k] = sel::fmax3(f(k), f(k + 8), f(k + 16));
+#pragma unroll
+              for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], f(k + 24));
+              s.raise(sel::fmax3(sel::fmax3(mx[0], mx[1], mx[2]), sel::fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7])));
+              if (!s.range_err) {
+#pragma unroll
+                for (int c = 0; c < NC; c += 4)
+                  s.add_quad(s.mass(f(c)), s.mass(f(c + 1)), s.mass(f(c + 2)), s.mass(f(c + 3)));
+              }
+            } else if (nv > 0) {
               // the chunk maximum first: the window moves at most once per chunk
               float m = -INFINITY;
 #pragma unroll
