@@ -53,7 +53,7 @@ bool layer_layout(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d, 
 }
 
 bool layer_sizes_ok(int n_tokens, int n_vis, int n_cubes, int hq, int hkv, int d, int D, int F) {
-  if (d != 128 || hq < 1 || hkv < 1) return false;
+  if ((d != 64 && d != 128) || hq < 1 || hkv < 1) return false;
   // GEMM shapes: K multiple of 64, output columns multiple of 32
   if (D % 64 != 0 || (hq * d) % 64 != 0) return false;
   LayerLayout L{};

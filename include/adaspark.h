@@ -426,7 +426,7 @@ size_t adaspark_layer_workspace(int n_tokens, int n_vis, int n_cubes, int hq, in
  *   layout arguments and p as for the two calls; y [n_tokens, D] fp32;
  *   workspace: device, >= adaspark_layer_workspace(...) bytes, 256-byte aligned;
  *   it also holds Q, K, V, a and h (see adaspark_layer_buffers).
- * Requires d = 128 and D a multiple of 64. ADASPARK_EUNSUPPORTED for FP32,
+ * Requires d = 64 or 128 and D a multiple of 64. ADASPARK_EUNSUPPORTED for FP32,
  * ADASPARK_EINVAL for bad arguments; device-detected problems of any stage are
  * reported by adaspark_read_device_status on the layer workspace. */
 int adaspark_layer(const void *x, const void *W_q, const void *W_k, const void *W_v,

@@ -18,6 +18,9 @@ LAYERS = {
     # a ragged row count (not a multiple of the 128-row GEMM tile) and 3 KV heads
     "ragged": workloads.small_config(name="layer-ragged", grid=(4, 8, 8), cube=(4, 4, 4),
                                      n_text=23, D=384, hq=6, hkv=3, F=640, seed=42),
+    # head_dim 64
+    "d64": workloads.small_config(name="layer-d64", grid=(4, 8, 8), cube=(4, 4, 4),
+                                  n_text=40, D=256, hq=8, hkv=2, d=64, F=512, seed=43),
 }
 
 

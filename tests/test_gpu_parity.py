@@ -32,6 +32,9 @@ SMALL = {
     # bf16 with head_dim 64 (one 64-dim half per query and key row)
     "d64-bf16": workloads.small_config(name="d64", grid=(8, 16, 16), cube=(4, 4, 4), n_text=40,
                                        D=256, hq=8, hkv=2, d=64, F=256, seed=15),
+    "ragged-d64": workloads.small_config(name="ragged-d64", grid=(4, 8, 8), cube=(4, 4, 2),
+                                         n_text=21, D=192, hq=6, hkv=3, d=64, F=384, seed=16,
+                                         cube_sizes=(3, 61, 32, 7, 57, 33, 1, 31, 2, 29)),
 }
 
 
