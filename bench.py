@@ -311,6 +311,46 @@ def _hist(values, n_bins, top):
             for b, c in enumerate(counts) if c]
 
 
+def rows_per_block(bits, n_cubes, thresholds=(1, 2, 4, 8, 16, 32, 64)):
+    """How the union walk spends its blocks. The attention runs one 128-row
+    tile per (128 consecutive visual tokens, query head) and walks every cube
+    that any of its rows selected; for each such (tile, cube) block, r = how
+    many of the 128 rows selected the cube and w = how many of the tile's four
+    32-row warps hold one of them (a warp with none skips its softmax work).
+    `bits` is the exported set tensor int32 [n_vis, hq, ceil(C/32)] (own cube
+    not marked). Returns the histogram of r, and for each R in `thresholds`
+    the fractions of blocks, of selected (row, cube) pairs and of active
+    warp-blocks that lie in blocks with r <= R."""
+    torch = torch_mod()
+    n_vis, hq, W = bits.shape
+    T = -(-n_vis // 128)
+    shifts = torch.arange(32, device=bits.device, dtype=torch.int32)
+    hist = torch.zeros(129, dtype=torch.int64, device=bits.device)
+    pairs_r = torch.zeros(129, dtype=torch.float64, device=bits.device)
+    warps_r = torch.zeros(129, dtype=torch.float64, device=bits.device)
+    for h in range(hq):
+        b = bits[:, h, :]
+        if T * 128 != n_vis:
+            b = torch.cat([b, b.new_zeros(T * 128 - n_vis, W)])
+        u = ((b.unsqueeze(-1) >> shifts) & 1).to(torch.uint8).reshape(T * 128, W * 32)[:, :n_cubes]
+        r = u.reshape(T, 128, n_cubes).sum(1, dtype=torch.int64).flatten()
+        w = u.reshape(T, 4, 32, n_cubes).amax(2).sum(1, dtype=torch.int64).flatten()
+        hist += torch.bincount(r, minlength=129)
+        pairs_r += torch.bincount(r, weights=r.double(), minlength=129)
+        warps_r += torch.bincount(r, weights=w.double(), minlength=129)
+    h_, p_, w_ = hist.cpu().numpy(), pairs_r.cpu().numpy(), warps_r.cpu().numpy()
+    blocks, pairs, warps = h_[1:].sum(), p_[1:].sum(), w_[1:].sum()
+    return {
+        "blocks": int(blocks), "pairs": int(round(pairs)), "active_warp_blocks": int(round(warps)),
+        "mean_rows": round(float(pairs / max(blocks, 1)), 2),
+        "r_le": {str(R): {"blocks": round(float(h_[1:R + 1].sum() / max(blocks, 1)), 4),
+                          "pairs": round(float(p_[1:R + 1].sum() / max(pairs, 1)), 4),
+                          "active_warp_blocks": round(float(w_[1:R + 1].sum() / max(warps, 1)), 4)}
+                 for R in thresholds},
+        "histogram_r_1_to_128": [int(v) for v in h_[1:]],
+    }
+
+
 def useful_attention_pairs(cfg, selected_pairs):
     """(row, key) pairs the method itself computes in AdaS-Attn: the keys of
     every selected cube, the own cube's causal prefix of every visual row and
@@ -339,6 +379,7 @@ def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, calls, 
     for t0 in range(0, cfg.n_vis, 8192):
         per_row.append(popcount32(bits[t0:t0 + 8192]).sum(dim=-1).reshape(-1))
     per_row = torch.cat(per_row)
+    per_block = rows_per_block(bits, C)
     del bits
     own = torch.repeat_interleave(torch.arange(C, device=per_row.device),
                                   torch.as_tensor(cfg.sizes, device=per_row.device))
@@ -377,6 +418,11 @@ def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, calls, 
         "executed_over_useful": round(executed / max(useful, 1.0), 3),
         "useful_over_dense": round(useful / dense_attn, 4),
         "executed_key_blocks": attn_stats["key_blocks"],
+        "rows_per_executed_block": dict(
+            per_block, what="selected cubes of 128-row tiles (own cubes, which every tile "
+                            "walks causally, not counted): r = rows of the tile that chose the "
+                            "cube; fractions of blocks, pairs and active 32-row warp-blocks in "
+                            "blocks with r <= R"),
         "overflow_rows": attn_stats["overflow_rows"],
         "near_margin": {
             "attn_rows": attn_stats["near_margin_rows"],

@@ -173,3 +173,49 @@ def test_oracle_sample_extrapolates_a_small_layer():
     assert abs(total - r["layer_s_extrapolated"]) <= 0.05 + 0.01 * total
     assert abs(r["value"] - workloads.CONFIGS[1].n_tokens / r["layer_s_extrapolated"]) \
         <= 0.05 * r["value"]
+
+
+def test_rows_per_block_brute_force():
+    """Per (128-row tile, cube) block: rows that chose the cube and active warps,
+    against a plain loop over a random set tensor with a ragged last tile."""
+    import numpy as np
+    import torch
+    rng = np.random.default_rng(5)
+    n_vis, hq, C = 300, 2, 40
+    sel = rng.random((n_vis, hq, C)) < 0.07
+    W = (C + 31) // 32
+    words = np.zeros((n_vis, hq, W), dtype=np.int64)
+    for j in range(C):
+        words[:, :, j // 32] |= sel[:, :, j].astype(np.int64) << (j % 32)
+    bits = torch.from_numpy(words.astype(np.uint32).view(np.int32))
+    got = bench.rows_per_block(bits, C, thresholds=(1, 3))
+    hist = np.zeros(129, dtype=np.int64)
+    pairs_le = {1: 0, 3: 0}
+    warps_le = {1: 0, 3: 0}
+    blocks_le = {1: 0, 3: 0}
+    tot_pairs = tot_warps = 0
+    for h in range(hq):
+        for t0 in range(0, n_vis, 128):
+            rows = sel[t0:t0 + 128, h, :]
+            for j in range(C):
+                r = int(rows[:, j].sum())
+                if r == 0:
+                    continue
+                w = sum(int(rows[q:q + 32, j].any()) for q in range(0, rows.shape[0], 32))
+                hist[r] += 1
+                tot_pairs += r
+                tot_warps += w
+                for R in (1, 3):
+                    if r <= R:
+                        blocks_le[R] += 1
+                        pairs_le[R] += r
+                        warps_le[R] += w
+    blocks = hist[1:].sum()
+    assert got["blocks"] == blocks and got["pairs"] == tot_pairs
+    assert got["active_warp_blocks"] == tot_warps
+    assert got["histogram_r_1_to_128"] == hist[1:].tolist()
+    for R in (1, 3):
+        e = got["r_le"][str(R)]
+        assert e["blocks"] == round(blocks_le[R] / blocks, 4)
+        assert e["pairs"] == round(pairs_le[R] / tot_pairs, 4)
+        assert e["active_warp_blocks"] == round(warps_le[R] / tot_warps, 4)
