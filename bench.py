@@ -179,6 +179,9 @@ def kernel_work(name, cfg, attn_stats, ffn_stats):
         return 4.0 * M * cfg.D * cfg.F, "flop", "tensor"
     if name.startswith("ffn_gemm2"):
         return 2.0 * M * cfg.D * cfg.F, "flop", "tensor"
+    if name == "attn_tc_gather":
+        # the split walk's gathered tiles: QK^T + PV per (gathered tile, 64-key block)
+        return 4.0 * 128 * 64 * cfg.d * attn_stats.get("gathered_blocks", 0), "flop", "tensor"
     if name.startswith("attn_tc"):
         # QK^T + PV per executed (128-row tile, 64-key block)
         return 4.0 * 128 * 64 * cfg.d * attn_stats["key_blocks"], "flop", "tensor"
@@ -398,7 +401,9 @@ def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, calls, 
     keep_hist = torch.bincount(per_cube, minlength=n_c + 1).cpu().tolist()
     useful_pairs = useful_attention_pairs(cfg, attn_stats["selected_pairs"])
     useful = 4.0 * cfg.d * useful_pairs
-    executed = 4.0 * 128 * 64 * cfg.d * attn_stats["key_blocks"]
+    # the tiles' own blocks and the split walk's gathered blocks
+    executed = 4.0 * 128 * 64 * cfg.d * (attn_stats["key_blocks"] +
+                                         attn_stats.get("gathered_blocks", 0))
     dense_attn = workloads_mod().dense_flops(cfg)["attn"]
     out = {
         "what": "read from the library after the timed region (exported sets, active flags, "
@@ -418,6 +423,11 @@ def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, calls, 
         "executed_over_useful": round(executed / max(useful, 1.0), 3),
         "useful_over_dense": round(useful / dense_attn, 4),
         "executed_key_blocks": attn_stats["key_blocks"],
+        "split_walk": {"pairs_in_gathered_tiles": attn_stats.get("split_pairs", 0),
+                       "gathered_blocks": attn_stats.get("gathered_blocks", 0),
+                       "what": "selected (row, cube) pairs of cubes that few of a tile's rows "
+                               "chose, run in gathered 128-row tiles and merged into their rows "
+                               "(adaspark_set_split_rows)"},
         "rows_per_executed_block": dict(
             per_block, what="selected cubes of 128-row tiles (own cubes, which every tile "
                             "walks causally, not counted): r = rows of the tile that chose the "
@@ -436,10 +446,12 @@ def realised_sparsity(cfg, lay, aws, fws, attn_stats, ffn_stats, ktimes, calls, 
     peaks, src = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     attn = ktimes.get("attn_tc") or ktimes.get("attn_simt")
-    sel = [ktimes[k] for k in ("select_tc", "select_simt", "cube_mean_keys", "validate")
-           if k in ktimes]
+    gath = ktimes.get("attn_tc_gather")
+    sel = [ktimes[k] for k in ("select_tc", "select_simt", "cube_mean_keys", "validate",
+                               "split_prefix", "split_scatter") if k in ktimes]
     if attn:
-        a_ms = attn[1] / calls                      # per call (one launch per KV head or one)
+        # per call: the tiles' walk plus the split walk's gathered tiles
+        a_ms = attn[1] / calls + (gath[1] / calls if gath else 0.0)
         s_ms = sum(v[1] / calls for v in sel)
         out["attention_ms"] = round(a_ms, 4)
         out["selection_ms"] = round(s_ms, 4)
@@ -869,7 +881,7 @@ def run_stack(args, cfg, world, device):
     per_layer = []
     for att, ffn in stats:
         useful = 4.0 * cfg.d * useful_attention_pairs(cfg, att["selected_pairs"])
-        executed = 4.0 * 128 * 64 * cfg.d * att["key_blocks"]
+        executed = 4.0 * 128 * 64 * cfg.d * (att["key_blocks"] + att.get("gathered_blocks", 0))
         per_layer.append({
             "mean_cubes_per_row": round(att["selected_pairs"] / max(1, att["visual_rows"]), 2),
             "selected_fraction": round(att["selected_pairs"] / max(1, att["candidate_pairs"]), 4),
@@ -928,6 +940,10 @@ def measure_backward(args, cfg, lay, fws, attn_stats, ffn_stats, world, device, 
     code, det = fb.read_device_status(aws)
     if code != fb.OK:
         raise RuntimeError(f"training forward device status {code} detail {det:#x}")
+    # the training-mode forward walks each tile's whole list (no split walk):
+    # its counters give the blocks the backward executes
+    attn_stats = dict(attn_stats, **{k: v for k, v in fb.attn_read_stats(aws).items()
+                                     if k in ("key_blocks", "tiles")})
     bufs = {"a": {}, "f": {}}
 
     def bwd():

@@ -41,7 +41,8 @@ class _AttnStats(ctypes.Structure):
                 ("selected_pairs", ctypes.c_uint64), ("overflow_rows", ctypes.c_uint64),
                 ("tiles", ctypes.c_uint64), ("key_blocks", ctypes.c_uint64),
                 ("key_block_keys", ctypes.c_uint64), ("near_margin_rows", ctypes.c_uint64),
-                ("reserved", ctypes.c_uint64 * 8)]
+                ("split_pairs", ctypes.c_uint64), ("gathered_blocks", ctypes.c_uint64),
+                ("reserved", ctypes.c_uint64 * 6)]
 
 
 class _FfnStats(ctypes.Structure):
@@ -109,6 +110,7 @@ def lib():
             "adaspark_launch_count": (ctypes.c_uint64, []),
             "adaspark_device_check": (i32, [i32]),
             "adaspark_debug_wait_expiry": (i32, [i32, ctypes.c_longlong]),
+            "adaspark_set_split_rows": (i32, [i32]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -533,6 +535,15 @@ def debug_wait_expiry(on: bool, wait_cycles: int = 2_000_000):
     wait_cycles SM cycles, reporting ADASPARK_DEV_TIMEOUT."""
     _check(lib().adaspark_debug_wait_expiry(1 if on else 0, int(wait_cycles)),
            "adaspark_debug_wait_expiry")
+
+
+def set_split_rows(rows: int):
+    """adaspark_set_split_rows: a tile's selected cube that at most `rows` of its
+    rows chose runs in a gathered tile (0: the single walk)."""
+    _check(lib().adaspark_set_split_rows(int(rows)), "adaspark_set_split_rows")
+
+
+SPLIT_ROWS_DEFAULT = 8
 
 
 def launch_count() -> int:

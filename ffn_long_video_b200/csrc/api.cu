@@ -5,6 +5,15 @@
 #include "attn_kernels.h"
 #include "ffn_kernels.h"
 
+namespace adaspark {
+int cube_attn_single_walk(const void* Q, const void* K, const void* V, int dtype,
+                          const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                          int n_vis, int n_tokens, int hq, int hkv, int d, float p, void* out,
+                          void* workspace, size_t workspace_bytes, void* stream);
+size_t cube_attn_single_walk_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv,
+                                       int d, int dtype);
+}  // namespace adaspark
+
 using namespace adaspark;
 
 namespace {
@@ -47,6 +56,9 @@ int cuda_rc(cudaError_t e) { return e == cudaSuccess ? ADASPARK_OK : ADASPARK_EC
 // of the bf16 attention kernel and whether its first descriptor is withheld.
 long long g_attn_wait_limit = kWaitCycles;
 int g_attn_withhold_first = 0;
+// Split walk of the bf16 forward (adaspark_set_split_rows): a tile's selected
+// cube that at most this many of its rows chose runs in a gathered tile.
+int g_split_rows = kSplitRowsDefault;
 
 }  // namespace
 
@@ -56,7 +68,8 @@ size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq
                                     int dtype) {
   if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return 0;
   const AttnGeom G = make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d);
-  return make_attn_layout(G).total;
+  // the bf16 path's split walk keeps its records after the common layout
+  return make_attn_layout(G).total + (dtype == ADASPARK_BF16 ? make_split_layout(G).total : 0);
 }
 
 }  // extern "C"
@@ -71,7 +84,7 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
                           const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
                           int n_vis, int n_tokens, int hq, int hkv, int d, float p, int topk,
                           void* out, void* workspace, size_t workspace_bytes, void* stream,
-                          bool train = false, bool uniform = false) {
+                          bool train = false, bool uniform = false, bool allow_split = true) {
   if (!Q || !K || !V || !cube_ids || !cube_offsets || !out || !workspace) return ADASPARK_EINVAL;
   if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return ADASPARK_EINVAL;
   if (topk < 0 || (topk == 0 && !p_valid(p))) return ADASPARK_EINVAL;
@@ -93,6 +106,36 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return ADASPARK_ECUDA;
   if (dense && cudaMemsetAsync(&hdr->pad[0], kModeDense, 1, s) != cudaSuccess)
     return ADASPARK_ECUDA;
+  // Split walk: bf16 Top-p / Top-K inference calls whose workspace holds the
+  // split region (as adaspark_cube_attn_workspace sizes it).
+  const SplitLayout SL = make_split_layout(G);
+  const bool split = allow_split && g_split_rows > 0 && dtype == ADASPARK_BF16 && !train &&
+                     !dense && !uniform && n_vis > 0 && G.n_vtiles > 0 &&
+                     workspace_bytes >= L.total + SL.total;
+  SplitArgs sp{};
+  if (split) {
+    uint8_t* r = ws + L.total;
+    sp.rows = g_split_rows;
+    sp.cap = SL.cap;
+    sp.max_mtiles = SL.max_mtiles;
+    sp.walk_count = reinterpret_cast<int32_t*>(r + SL.walk_count);
+    sp.walk_list = reinterpret_cast<uint16_t*>(r + SL.walk_list);
+    sp.row_off = reinterpret_cast<int32_t*>(r + SL.row_off);
+    sp.row_cnt = reinterpret_cast<int32_t*>(r + SL.row_cnt);
+    sp.rec_row = reinterpret_cast<int32_t*>(r + SL.rec_row);
+    sp.rec_cube = reinterpret_cast<int32_t*>(r + SL.rec_cube);
+    sp.rec_gpos = reinterpret_cast<int32_t*>(r + SL.rec_gpos);
+    sp.grp_cnt = reinterpret_cast<int32_t*>(r + SL.grp_cnt);
+    sp.grp_base = reinterpret_cast<int32_t*>(r + SL.grp_base);
+    sp.grp_tile = reinterpret_cast<int32_t*>(r + SL.grp_tile);
+    sp.grec = reinterpret_cast<int32_t*>(r + SL.grec);
+    sp.mtile = reinterpret_cast<int32_t*>(r + SL.mtile);
+    sp.part_o = reinterpret_cast<__nv_bfloat16*>(r + SL.part_o);
+    sp.part_lse = reinterpret_cast<float*>(r + SL.part_lse);
+    if (cudaMemsetAsync(sp.grp_cnt, 0, (size_t)G.hkv * n_cubes * sizeof(int32_t), s) !=
+        cudaSuccess)
+      return ADASPARK_ECUDA;
+  }
   if (train &&
       cudaMemsetAsync(reinterpret_cast<uint8_t*>(&hdr->pad[0]) + 1, 1, 1, s) != cudaSuccess)
     return ADASPARK_ECUDA;
@@ -113,6 +156,7 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   sa.p = p;
   sa.zscale = (float)(1.4426950408889634 / std::sqrt((double)d));
   sa.topk = topk;
+  sa.sp = sp;
 
   if (uniform && n_vis > 0 && G.n_vtiles > 0) {
     rc = cuda_rc(launch_select_uniform(sa, s));
@@ -123,6 +167,10 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
     if (rc) return rc;
     rc = cuda_rc(dtype == ADASPARK_BF16 ? launch_select_tc(sa, s) : launch_select_simt(sa, dtype, s));
     if (rc) return rc;
+    if (split) {
+      rc = cuda_rc(launch_split_build(sp, G, hdr, s));
+      if (rc) return rc;
+    }
   }
 
   AttnArgs aa;
@@ -143,14 +191,37 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
   aa.o32 = train ? reinterpret_cast<float*>(ws + L.total) : nullptr;
   aa.wait_limit = g_attn_wait_limit;
   aa.withhold_first = g_attn_withhold_first;
+  aa.sp = sp;
   // When the layer's K and V outgrow what L2 holds alongside the other
   // traffic, visual tiles run one KV head after another, so that the blocks in
   // use belong to one head; otherwise all heads of a token range run together
   // (fewer CTAs then read the same lines at once).
   const double kv_bytes = 2.0 * n_tokens * hkv * d * (dtype == ADASPARK_BF16 ? 2 : 4);
   aa.kv_major = kv_bytes > 64.0 * 1024 * 1024 ? 1 : 0;
-  if (dtype == ADASPARK_BF16) return cuda_rc(launch_attn_tc(aa, s));
+  if (dtype == ADASPARK_BF16) {
+    if (split) {  // the gathered tiles first: the tiles' epilogues merge their results
+      rc = cuda_rc(launch_attn_tc_gather(aa, s));
+      if (rc) return rc;
+    }
+    return cuda_rc(launch_attn_tc(aa, s));
+  }
   return cuda_rc(launch_attn_simt(aa, dtype, s));
+}
+
+// adaspark_cube_attn on the common layout alone (no split walk): the entry
+// point with the library-held scratch array.
+int adaspark::cube_attn_single_walk(const void* Q, const void* K, const void* V, int dtype,
+                          const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                          int n_vis, int n_tokens, int hq, int hkv, int d, float p, void* out,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  return cube_attn_impl(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq, hkv,
+                        d, p, 0, out, workspace, workspace_bytes, stream, false, false, false);
+}
+
+size_t adaspark::cube_attn_single_walk_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv,
+                                       int d, int dtype) {
+  if (!attn_sizes_ok(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype)) return 0;
+  return make_attn_layout(make_attn_geom(n_tokens, n_vis, n_cubes, hq, hkv, d)).total;
 }
 
 extern "C" {
@@ -470,6 +541,12 @@ int adaspark_ffn_read_stats(const void* workspace, adaspark_ffn_stats* stats, vo
   const WsHeader* hdr = static_cast<const WsHeader*>(workspace);
   static_assert(sizeof(adaspark_ffn_stats) == sizeof(hdr->stats), "stats size");
   return cuda_rc(cudaMemcpy(stats, hdr->stats, sizeof(adaspark_ffn_stats), cudaMemcpyDeviceToHost));
+}
+
+int adaspark_set_split_rows(int rows) {
+  if (rows < 0 || rows > kTileRows) return ADASPARK_EINVAL;
+  g_split_rows = rows;
+  return ADASPARK_OK;
 }
 
 int adaspark_debug_wait_expiry(int on, long long wait_cycles) {

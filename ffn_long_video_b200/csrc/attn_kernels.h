@@ -7,6 +7,28 @@
 
 namespace adaspark {
 
+// Device pointers of the split walk (SplitLayout), shared by the selection,
+// the regrouping kernels and the attention; rows == 0: no split.
+struct SplitArgs {
+  int rows;                           // a cube chosen by at most this many rows leaves the walk
+  int cap;                            // record capacity
+  int max_mtiles;
+  int32_t* walk_count;
+  uint16_t* walk_list;
+  int32_t* row_off;
+  int32_t* row_cnt;
+  int32_t* rec_row;
+  int32_t* rec_cube;
+  int32_t* rec_gpos;
+  int32_t* grp_cnt;
+  int32_t* grp_base;
+  int32_t* grp_tile;
+  int32_t* grec;
+  int32_t* mtile;
+  __nv_bfloat16* part_o;
+  float* part_lse;
+};
+
 struct SelectArgs {
   const void* Q;
   const int32_t* cube_ids;
@@ -21,6 +43,7 @@ struct SelectArgs {
   float p;
   float zscale;                       // log2(e) / sqrt(d)
   int topk;                           // > 0: Top-K with this k instead of Top-p
+  SplitArgs sp;
 };
 
 struct AttnArgs {
@@ -42,6 +65,7 @@ struct AttnArgs {
   float* o32;                         // [N][hq][d] fp32 O with P split hi + lo (training), or null
   long long wait_limit;               // SM cycles before a wait gives up (bf16 kernel)
   int withhold_first;                 // test hook: the first descriptor is never announced
+  SplitArgs sp;                       // split walk (sp.rows == 0: none)
 };
 
 // Backward of AdaS-Attn (sets of a forward call held fixed).
@@ -100,5 +124,11 @@ cudaError_t launch_export_sets(const int32_t* tile_count, const uint16_t* tile_l
                                const AttnGeom& G, int dense, uint32_t* bits, cudaStream_t s);
 cudaError_t launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t s);
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
+// Split walk: group the records by (KV head, cube) and number the gathered
+// tiles (after the selection), then run the gathered tiles (before the tiles'
+// own walk, whose epilogue merges their partial results).
+cudaError_t launch_split_build(const SplitArgs& sp, const AttnGeom& G, WsHeader* hdr,
+                               cudaStream_t s);
+cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t s);
 
 }  // namespace adaspark

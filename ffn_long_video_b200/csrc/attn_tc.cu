@@ -94,7 +94,11 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
 // pair hi + lo (lo = P - hi, in the second half of the S buffer, whose
 // scores were read before), so O is exact to about 2^-17 of each term, and O is
 // also written in fp32 to a.o32; the backward takes D_r = dO_r . O_r from it.
-template <bool TRAIN, int D>
+// GATHER: a gathered tile of the split walk (see SplitLayout): its rows are
+// records (row, cube) of one (KV head, cube) group, taken from many tiles; it
+// walks that cube's keys alone and writes each record's normalised output and
+// log2-sum-exp, which the row's own tile merges at the end of its walk.
+template <bool TRAIN, int D, bool GATHER>
 __global__ void __launch_bounds__(THREADS, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    AttnArgs a) {
@@ -125,9 +129,36 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const AttnGeom& G = a.G;
   WsHeader* hdr = a.hdr;
-  const TileInfo T = decode_tile(G, a.kv_major != 0);
+  TileInfo T;
+  int g_cube = 0, g_first = 0, g_count = 0;   // gathered tile: cube, first record slot, rows
+  if (GATHER) {
+    // the launch covers the largest possible number of gathered tiles; the
+    // regrouping counted the ones that exist
+    const int m_tile = blockIdx.x;
+    if (m_tile >= (int)*reinterpret_cast<const volatile uint32_t*>(&hdr->sched[1])) return;
+    const int grp = a.sp.mtile[m_tile];
+    T.text = false;
+    T.kv = grp / G.n_cubes;
+    T.bt = 0;
+    T.t_hi = 0;
+    g_cube = grp - T.kv * G.n_cubes;
+    g_first = a.sp.grp_base[grp] + (m_tile - a.sp.grp_tile[grp]) * kTileRows;
+    g_count = min(kTileRows, a.sp.grp_base[grp + 1] - g_first);
+  } else {
+    T = decode_tile(G, a.kv_major != 0);
+  }
+  // the tile walks only part of its list, the rest in gathered tiles
+  const bool split = !GATHER && !TRAIN && a.sp.rows > 0 && !T.text && !a.dense;
   const long long WL = a.wait_limit;  // cycles before any wait of this kernel gives up
 
+  if (warp == 2) {
+    // the descriptor ring's barriers, one slot per lane and round
+    for (int r = lane; r < RING; r += 32) {
+      mbar_init(&r_full[r], 1);
+      mbar_init(&r_empty[r], 128);
+    }
+    fence_mbar_init();
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&k_full[s], 1);
@@ -140,16 +171,12 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_init(&p_full[b], 128);
       mbar_init(&pv_done[b], 1);
     }
-    for (int r = 0; r < RING; ++r) {
-      mbar_init(&r_full[r], 1);
-      mbar_init(&r_empty[r], 128);
-    }
     mbar_init(q_full, 128);
     mbar_init(drain, 1);
     fence_mbar_init();
     s_abort = 0;
     s_bad = status_bad(hdr) ? 1 : 0;
-    s_own_hi = (!T.text && !s_bad) ? a.cube_ids[T.t_hi] : -1;
+    s_own_hi = (!GATHER && !T.text && !s_bad) ? a.cube_ids[T.t_hi] : -1;
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&mapK);
@@ -173,15 +200,17 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (T.text) {
         n_entries = G.n_cubes;
         n_chunks = (T.t_hi - G.n_vis) / 64 + 1;
+      } else if (GATHER) {
+        n_entries = 1;
       } else if (a.dense) {
         n_entries = s_own_hi + 1;
       } else {
-        n_entries = a.tile_count[T.bt];
+        n_entries = split ? a.sp.walk_count[T.bt] : a.tile_count[T.bt];
         use_list = true;
       }
     }
     const int n_total = n_entries + n_chunks;
-    const uint16_t* list = a.tile_list + (size_t)T.bt * G.n_cubes;
+    const uint16_t* list = (split ? a.sp.walk_list : a.tile_list) + (size_t)T.bt * G.n_cubes;
     const uint4* tmask = reinterpret_cast<const uint4*>(a.tile_mask) + (size_t)T.bt * G.n_cubes;
     int base = 0;
     bool ok = true;
@@ -190,10 +219,18 @@ __global__ void __launch_bounds__(THREADS, 2)
       int j = -1, ks = 0, ke = 0;
       uint4 m = make_uint4(~0u, ~0u, ~0u, ~0u);
       if (e < n_entries) {
-        j = use_list ? (int)list[e] : e;
+        j = GATHER ? g_cube : use_list ? (int)list[e] : e;
         ks = a.cube_offsets[j];
         ke = a.cube_offsets[j + 1];
-        if (use_list) m = tmask[j];
+        if (use_list) {
+          m = tmask[j];
+        } else if (GATHER) {  // the gathered tile's rows that exist
+          auto word = [&](int w) {
+            const int r = g_count - 32 * w;
+            return r >= 32 ? ~0u : r > 0 ? (1u << r) - 1u : 0u;
+          };
+          m = make_uint4(word(0), word(1), word(2), word(3));
+        }
       } else if (e < n_total) {
         ks = G.n_vis + (e - n_entries) * 64;
         ke = min(ks + 64, T.t_hi + 1);
@@ -362,10 +399,20 @@ __global__ void __launch_bounds__(THREADS, 2)
     // ------------------------------------------------------------ softmax rows
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    const TileRow R = tile_row(G, T.text, T.bt, row);
+    TileRow R;
+    int rec = 0;                                // GATHER: this row's record
+    if (GATHER) {
+      R.valid = row < g_count;
+      rec = R.valid ? a.sp.grec[g_first + row] : 0;
+      const int rid = R.valid ? a.sp.rec_row[rec] : 0;
+      R.t = rid / G.hq;
+      R.h = rid - R.t * G.hq;
+    } else {
+      R = tile_row(G, T.text, T.bt, row);
+    }
     const bool valid = R.valid;
     const int t = R.t, h = R.h;
-    const int own = (!T.text && valid) ? a.cube_ids[t] : -1;
+    const int own = (!GATHER && !T.text && valid) ? a.cube_ids[t] : -1;
     const float scale = a.scale_log2;
     {
       const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
@@ -544,10 +591,33 @@ __global__ void __launch_bounds__(THREADS, 2)
         mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr, 0x7900u, WL)) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const float lse_own = m_used + __log2f(l);
+      // Merge of the row's gathered partial results (split walk): with M the
+      // largest of the log2-sum-exps, the row's softmax over all its keys is
+      // the sum of the parts' normalised outputs weighted by 2^(lse - M) / S,
+      // S the sum of those powers; lse of the whole row = M + log2 S.
+      int mcnt = 0, moff = 0;
+      float w_own = 1.f, M = 0.f, inv_S = 1.f, lse_row = lse_own;
+      if (split && valid) {
+        const size_t rid = (size_t)t * G.hq + h;
+        mcnt = a.sp.row_cnt[rid];
+        moff = a.sp.row_off[rid];
+        if (mcnt > 0) {
+          M = lse_own;
+          for (int k = 0; k < mcnt; ++k) M = fmaxf(M, a.sp.part_lse[moff + k]);
+          float S = ex2(lse_own - M);
+          for (int k = 0; k < mcnt; ++k) S += ex2(a.sp.part_lse[moff + k] - M);
+          inv_S = 1.f / S;
+          w_own = ex2(lse_own - M) * inv_S;
+          lse_row = M + __log2f(S);
+        }
+      }
       // the row's softmax is 2^(s * scale - lse): kept for the backward pass
-      if (valid && a.lse) a.lse[(size_t)t * G.hq + h] = m_used + __log2f(l);
+      if (!GATHER && valid && a.lse) a.lse[(size_t)t * G.hq + h] = lse_row;
+      if (GATHER && valid) a.sp.part_lse[rec] = lse_own;
       __nv_bfloat16* dst =
-          reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * D;
+          GATHER ? a.sp.part_o + (size_t)rec * D
+                 : reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
@@ -555,10 +625,37 @@ __global__ void __launch_bounds__(THREADS, 2)
         tmem_ld_wait();
         if (valid) {
           uint32_t pk[16];
+          if (mcnt == 0) {
 #pragma unroll
-          for (int x = 0; x < 16; ++x)
-            pk[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv,
-                                __uint_as_float(o[2 * x + 1]) * inv);
+            for (int x = 0; x < 16; ++x)
+              pk[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv,
+                                  __uint_as_float(o[2 * x + 1]) * inv);
+          } else {
+            float f[32];
+            const float s_own = inv * w_own;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) f[x] = __uint_as_float(o[x]) * s_own;
+#pragma unroll 1
+            for (int k = 0; k < mcnt; ++k) {
+              const float wk = ex2(a.sp.part_lse[moff + k] - M) * inv_S;
+              const uint4* src =
+                  reinterpret_cast<const uint4*>(a.sp.part_o + (size_t)(moff + k) * D + c);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 v = src[q];
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int z = 0; z < 4; ++z) {
+                  const float2 pf = __bfloat1622float2(
+                      *reinterpret_cast<const __nv_bfloat162*>(&w4[z]));
+                  f[8 * q + 2 * z] = fmaf(wk, pf.x, f[8 * q + 2 * z]);
+                  f[8 * q + 2 * z + 1] = fmaf(wk, pf.y, f[8 * q + 2 * z + 1]);
+                }
+              }
+            }
+#pragma unroll
+            for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(f[2 * x], f[2 * x + 1]);
+          }
           uint4* d4 = reinterpret_cast<uint4*>(dst + c);
 #pragma unroll
           for (int x = 0; x < 4; ++x)
@@ -576,8 +673,13 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
     }
     if (warp == 2 && lane == 0 && !bad) {
-      atomicAdd((unsigned long long*)&hdr->stats[4], 1ull);
-      atomicAdd((unsigned long long*)&hdr->stats[5], (unsigned long long)i);
+      if (GATHER) {  // gathered tiles and their blocks are counted apart
+        atomicAdd((unsigned long long*)&hdr->stats[8], (unsigned long long)g_count);
+        atomicAdd((unsigned long long*)&hdr->stats[9], (unsigned long long)i);
+      } else {
+        atomicAdd((unsigned long long*)&hdr->stats[4], 1ull);
+        atomicAdd((unsigned long long*)&hdr->stats[5], (unsigned long long)i);
+      }
     }
   }
   tc_fence_before();
@@ -601,12 +703,35 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   if (!encode_tmap_bf16(&mK, a.K, 3, dims, strides, box) ||
       !encode_tmap_bf16(&mV, a.V, 3, dims, strides, box))
     return cudaErrorInvalidValue;
-  auto k = G.d == 64 ? (a.o32 ? fa::attn_tc_kernel<true, 64> : fa::attn_tc_kernel<false, 64>)
-                     : (a.o32 ? fa::attn_tc_kernel<true, 128> : fa::attn_tc_kernel<false, 128>);
+  auto k = G.d == 64
+               ? (a.o32 ? fa::attn_tc_kernel<true, 64, false> : fa::attn_tc_kernel<false, 64, false>)
+               : (a.o32 ? fa::attn_tc_kernel<true, 128, false>
+                        : fa::attn_tc_kernel<false, 128, false>);
   const size_t smem = G.d == 64 ? fa::smem_bytes<64>() : fa::smem_bytes<128>();
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch("attn_tc", k, dim3(blocks), dim3(fa::THREADS), smem, s, mK, mV, a);
+}
+
+// The gathered tiles of the split walk: a grid of the largest possible count
+// (SplitLayout::max_mtiles); tiles past the count the regrouping wrote exit at
+// once.
+cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t s) {
+  const AttnGeom& G = a.G;
+  if (a.sp.rows <= 0 || a.sp.max_mtiles <= 0 || G.n_vtiles == 0) return cudaSuccess;
+  CUtensorMap mK, mV;
+  const uint64_t dims[3] = {(uint64_t)G.d, (uint64_t)G.hkv, (uint64_t)G.n_tokens};
+  const uint64_t strides[2] = {(uint64_t)G.d * 2, (uint64_t)G.hkv * G.d * 2};
+  const uint32_t box[3] = {64, 1, 64};
+  if (!encode_tmap_bf16(&mK, a.K, 3, dims, strides, box) ||
+      !encode_tmap_bf16(&mV, a.V, 3, dims, strides, box))
+    return cudaErrorInvalidValue;
+  auto k = G.d == 64 ? fa::attn_tc_kernel<false, 64, true> : fa::attn_tc_kernel<false, 128, true>;
+  const size_t smem = G.d == 64 ? fa::smem_bytes<64>() : fa::smem_bytes<128>();
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch("attn_tc_gather", k, dim3(a.sp.max_mtiles), dim3(fa::THREADS), smem, s, mK, mV,
+                a);
 }
 
 }  // namespace adaspark

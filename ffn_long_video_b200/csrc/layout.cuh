@@ -94,6 +94,63 @@ __host__ __device__ inline AttnLayout make_attn_layout(const AttnGeom& G) {
   return L;
 }
 
+// Split walk of the bf16 forward (after the layout above; a training-mode call,
+// which never splits, keeps its fp32 O in the same place). A visual tile's
+// selected cubes that at most `split rows` of its 128 rows chose (and that are
+// no row's own cube) leave the tile's walk; their (row, cube) pairs, the
+// records, are regrouped by (KV head, cube) into gathered 128-row tiles whose
+// partial results the tile merges into its rows at the end.
+struct SplitLayout {
+  size_t walk_count;  // int32 [n_vtiles]       blocks the tile itself walks
+  size_t walk_list;   // uint16 [n_vtiles][C]   their cube ids, ascending
+  size_t row_off;     // int32 [n_vis * hq]     first record of a visual row
+  size_t row_cnt;     // int32 [n_vis * hq]     its number of records
+  size_t rec_row;     // int32 [cap]            record -> row (t * hq + h), -1 unused
+  size_t rec_cube;    // int32 [cap]            record -> cube
+  size_t rec_gpos;    // int32 [cap]            record -> place in its group
+  size_t grp_cnt;     // int32 [hkv * C]        records per (KV head, cube)
+  size_t grp_base;    // int32 [hkv * C + 1]    exclusive prefix of grp_cnt
+  size_t grp_tile;    // int32 [hkv * C + 1]    exclusive prefix of gathered tiles
+  size_t grec;        // int32 [cap]            records grouped by (KV head, cube)
+  size_t mtile;       // int32 [max_mtiles]     gathered tile -> group
+  size_t part_o;      // bf16 [cap][d]          a record's normalised partial output
+  size_t part_lse;    // float [cap]            and its log2-sum-exp
+  int cap;            // records
+  int max_mtiles;     // cap / 128 + hkv * C (the gathered launch's grid)
+  size_t total;
+};
+
+constexpr int kSplitRecordsPerRow = 6;  // record capacity per visual row
+constexpr int kSplitRowsDefault = 8;    // default of adaspark_set_split_rows
+
+__host__ __device__ inline SplitLayout make_split_layout(const AttnGeom& G) {
+  SplitLayout L;
+  const size_t rows = (size_t)G.n_vis * G.hq;
+  const size_t groups = (size_t)G.hkv * (G.n_cubes > 0 ? G.n_cubes : 1);
+  size_t cap = rows * kSplitRecordsPerRow;
+  if (cap > (size_t)0x3fffffff) cap = 0x3fffffff;
+  L.cap = (int)cap;
+  L.max_mtiles = (int)((cap + kTileRows - 1) / kTileRows + groups);
+  size_t o = 0;
+  L.walk_count = o; o += align_up((size_t)(G.n_vtiles > 0 ? G.n_vtiles : 1) * 4);
+  L.walk_list = o; o += align_up((size_t)(G.n_vtiles > 0 ? G.n_vtiles : 1) *
+                                 (G.n_cubes > 0 ? G.n_cubes : 1) * 2);
+  L.row_off = o; o += align_up((rows > 0 ? rows : 1) * 4);
+  L.row_cnt = o; o += align_up((rows > 0 ? rows : 1) * 4);
+  L.rec_row = o; o += align_up((cap > 0 ? cap : 1) * 4);
+  L.rec_cube = o; o += align_up((cap > 0 ? cap : 1) * 4);
+  L.rec_gpos = o; o += align_up((cap > 0 ? cap : 1) * 4);
+  L.grp_cnt = o; o += align_up(groups * 4);
+  L.grp_base = o; o += align_up((groups + 1) * 4);
+  L.grp_tile = o; o += align_up((groups + 1) * 4);
+  L.grec = o; o += align_up((cap > 0 ? cap : 1) * 4);
+  L.mtile = o; o += align_up((size_t)L.max_mtiles * 4);
+  L.part_o = o; o += align_up((cap > 0 ? cap : 1) * (size_t)G.d * 2);
+  L.part_lse = o; o += align_up((cap > 0 ? cap : 1) * 4);
+  L.total = o;
+  return L;
+}
+
 // Workspace of adaspark_cube_attn_backward.
 struct AttnBwdLayout {
   size_t header;

@@ -44,12 +44,22 @@ int scratch_on_current_device(void** out) {
 
 }  // namespace
 
+namespace adaspark {
+int cube_attn_single_walk(const void* Q, const void* K, const void* V, int dtype,
+                          const int32_t* cube_ids, const int32_t* cube_offsets, int n_cubes,
+                          int n_vis, int n_tokens, int hq, int hkv, int d, float p, void* out,
+                          void* workspace, size_t workspace_bytes, void* stream);
+size_t cube_attn_single_walk_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv,
+                                       int d, int dtype);
+}  // namespace adaspark
+
 extern "C" int adaspark_cube_attn_noalloc(const void* Q, const void* K, const void* V, int dtype,
                                           const int32_t* cube_ids, const int32_t* cube_offsets,
                                           int n_cubes, int n_vis, int n_tokens, int hq, int hkv,
                                           int d, float p, void* out, void* stream) {
+  // the common layout alone: this entry point always runs the single walk
   const size_t need =
-      adaspark_cube_attn_workspace(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype);
+      adaspark::cube_attn_single_walk_workspace(n_tokens, n_vis, n_cubes, hq, hkv, d, dtype);
   if (need == 0) return ADASPARK_EINVAL;                       // invalid sizes
   if (need > (size_t)ADASPARK_NOALLOC_SCRATCH_BYTES) return ADASPARK_EINVAL;  // too large
   // the device check comes first, so that a device without this library's
@@ -63,7 +73,7 @@ extern "C" int adaspark_cube_attn_noalloc(const void* Q, const void* K, const vo
   if (rc != ADASPARK_OK) return rc;
   // adaspark_cube_attn clears the parts of the workspace that must start at
   // zero (status word and counters) at the start of every call.
-  return adaspark_cube_attn(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis, n_tokens, hq,
-                            hkv, d, p, out, scratch, (size_t)ADASPARK_NOALLOC_SCRATCH_BYTES,
-                            stream);
+  return adaspark::cube_attn_single_walk(Q, K, V, dtype, cube_ids, cube_offsets, n_cubes, n_vis,
+                                         n_tokens, hq, hkv, d, p, out, scratch,
+                                         (size_t)ADASPARK_NOALLOC_SCRATCH_BYTES, stream);
 }

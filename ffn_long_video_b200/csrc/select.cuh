@@ -34,6 +34,7 @@
 
 #include <limits.h>
 
+#include "attn_kernels.h"
 #include "common.cuh"
 
 namespace adaspark {
@@ -572,8 +573,8 @@ __device__ __forceinline__ uint32_t warp_transpose32(uint32_t x, int lane) {
 // Shared tile epilogue: compact the cube columns with any row bit into the
 // tile's ascending list. 128 threads.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void compact_tile_list(const uint32_t* tmask, uint16_t* list,
-                                                  int32_t* count, int c_hi, int* s_wcnt, int tid) {
+__device__ __forceinline__ int compact_tile_list(const uint32_t* tmask, uint16_t* list,
+                                                 int32_t* count, int c_hi, int* s_wcnt, int tid) {
   const int warp = tid >> 5, lane = tid & 31;
   int total = 0;
   for (int base = 0; base <= c_hi; base += 128) {
@@ -594,6 +595,152 @@ __device__ __forceinline__ void compact_tile_list(const uint32_t* tmask, uint16_
     total += chunk_total;
   }
   if (tid == 0) *count = total;
+  return total;
+}
+
+// Split walk of a visual tile (see SplitLayout): the tile's list (n cubes,
+// ascending) is divided into the cubes the tile walks itself and the sparse
+// ones, chosen by at most sp.rows of its rows and below the tile's lowest own
+// cube c_lo (so no row of the tile has one as its own cube); at most kSparseMax
+// per tile (later candidates stay in the walk). Each row's selections among
+// the sparse cubes become records (row, cube), in ascending cube order, at
+// row_off[row]; space for the tile's records is taken from the counter
+// hdr->sched[0]; when it would pass the capacity the tile keeps its whole list
+// (its reserved records are marked unused). Each sparse cube takes a range of
+// its (KV head, cube) group at once (grp_cnt), and each record its place in
+// that range (rec_gpos, the row's rank among the cube's rows in the tile), so
+// the regrouping needs no atomics. 128 threads, thread tid = tile row; `stage`
+// is shared scratch of kSparseMax * 24 bytes (the per-row selection storage,
+// free by now).
+constexpr int kSparseMax = 1024;
+__device__ __forceinline__ void split_tile(const uint32_t* tmask, const uint16_t* list, int n,
+                                           const SplitArgs& sp, int vt, int C, int c_lo, int kv,
+                                           int rid, bool valid, uint8_t* stage, int* s_wcnt,
+                                           int* s_misc, WsHeader* hdr, int tid) {
+  const int warp = tid >> 5, lane = tid & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  uint4* s_mask = reinterpret_cast<uint4*>(stage);                       // [kSparseMax]
+  int* s_p0 = reinterpret_cast<int*>(stage + kSparseMax * 16);            // [kSparseMax]
+  uint16_t* s_j = reinterpret_cast<uint16_t*>(stage + kSparseMax * 20);   // [kSparseMax]
+  uint16_t* walk = sp.walk_list + (size_t)vt * C;
+  int n_walk = 0, n_sp = 0;
+  for (int base = 0; base < n; base += 128) {
+    const int e = base + tid;
+    int j = -1;
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    bool cand = false;
+    if (e < n) {
+      j = __ldcg(list + e);
+      w = __ldcg(reinterpret_cast<const uint4*>(tmask + (size_t)j * 4));
+      const int r = __popc(w.x) + __popc(w.y) + __popc(w.z) + __popc(w.w);
+      cand = j < c_lo && r <= sp.rows;
+    }
+    const unsigned bc = __ballot_sync(0xffffffffu, cand);
+    if (lane == 0) s_wcnt[warp] = __popc(bc);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int pc = n_sp;
+    for (int q = 0; q < warp; ++q) pc += s_wcnt[q];
+    const int tc = s_wcnt[0] + s_wcnt[1] + s_wcnt[2] + s_wcnt[3];
+    const int ps = pc + __popc(bc & lt);
+    const bool sp_e = cand && ps < kSparseMax;
+    const bool keep = e < n && !sp_e;
+    const unsigned bk = __ballot_sync(0xffffffffu, keep);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (lane == 0) s_wcnt[warp] = __popc(bk);
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    int pk = n_walk;
+    for (int q = 0; q < warp; ++q) pk += s_wcnt[q];
+    const int tk = s_wcnt[0] + s_wcnt[1] + s_wcnt[2] + s_wcnt[3];
+    if (keep) walk[pk + __popc(bk & lt)] = (uint16_t)j;
+    if (sp_e) {
+      s_mask[ps] = w;
+      s_j[ps] = (uint16_t)j;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    n_walk += tk;
+    n_sp = min(n_sp + tc, kSparseMax);
+  }
+  // this row's records: its bits among the sparse cubes, 32 cubes at a time
+  // (lane L reads its warp's word of cube k0 + L; the transpose gives each
+  // lane, a row, its bits over those 32 cubes)
+  const uint32_t* s_w = reinterpret_cast<const uint32_t*>(s_mask);
+  auto row_bits = [&](int k0) {
+    const uint32_t x = k0 + lane < n_sp ? s_w[(k0 + lane) * 4 + warp] : 0u;
+    return sel::warp_transpose32(x, lane);
+  };
+  int cnt = 0;
+  for (int k0 = 0; k0 < n_sp; k0 += 32) cnt += __popc(row_bits(k0));
+  if (!valid) cnt = 0;
+  int incl = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) s_wcnt[warp] = incl;
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  int excl = incl - cnt;
+  for (int q = 0; q < warp; ++q) excl += s_wcnt[q];
+  const int total = s_wcnt[0] + s_wcnt[1] + s_wcnt[2] + s_wcnt[3];
+  if (tid == 0) {
+    // once the counter has passed the capacity no tile takes space any more,
+    // so it stays far below 2^32 (at most the capacity plus the records of
+    // the tiles that raced past it)
+    unsigned b = 0;
+    bool fits = true;
+    if (total > 0) {
+      if (*reinterpret_cast<volatile unsigned*>(&hdr->sched[0]) >= (unsigned)sp.cap) {
+        b = (unsigned)sp.cap;
+        fits = false;
+      } else {
+        b = atomicAdd(&hdr->sched[0], (unsigned)total);
+        fits = (unsigned long long)b + (unsigned)total <= (unsigned long long)sp.cap;
+      }
+    }
+    s_misc[0] = (int)min(b, (unsigned)sp.cap);
+    s_misc[1] = fits ? 1 : 0;
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const int rbase = s_misc[0];
+  const bool fits = s_misc[1] != 0;
+  if (!fits) {
+    for (int e = tid; e < n; e += 128) walk[e] = __ldcg(list + e);
+    if (tid == 0) sp.walk_count[vt] = n;
+    // the records this tile reserved below the capacity are marked unused
+    const long long hi = min((long long)rbase + total, (long long)sp.cap);
+    for (long long i = (long long)rbase + tid; i < hi; i += 128) sp.rec_row[i] = -1;
+    if (valid) sp.row_cnt[rid] = 0;
+    return;
+  }
+  if (tid == 0) sp.walk_count[vt] = n_walk;
+  // each sparse cube's range in its group
+  for (int k = tid; k < n_sp; k += 128) {
+    const uint4 w = s_mask[k];
+    s_p0[k] = atomicAdd(&sp.grp_cnt[(size_t)kv * C + s_j[k]],
+                        __popc(w.x) + __popc(w.y) + __popc(w.z) + __popc(w.w));
+  }
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+  const int o = rbase + excl;
+  if (valid) {
+    sp.row_off[rid] = o;
+    sp.row_cnt[rid] = cnt;
+  }
+  int k2 = 0;
+  for (int k0 = 0; k0 < n_sp; k0 += 32) {   // warp-uniform: every lane transposes
+    uint32_t b = row_bits(k0);
+    if (!valid) b = 0u;
+    while (b) {
+      const int k = k0 + __ffs(b) - 1;
+      b &= b - 1u;
+      // rank of this row among the cube's rows in the tile
+      int rank = __popc(s_w[k * 4 + warp] & lt);
+      for (int q = 0; q < warp; ++q) rank += __popc(s_w[k * 4 + q]);
+      sp.rec_row[o + k2] = rid;
+      sp.rec_cube[o + k2] = s_j[k];
+      sp.rec_gpos[o + k2] = s_p0[k] + rank;
+      ++k2;
+    }
+  }
 }
 
 }  // namespace adaspark

@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(THREADS, 2)
   uint64_t* decide = drain + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(decide + 1);
   __shared__ volatile int s_abort;
-  __shared__ int s_hi, s_bad, s_wcnt[4];
+  __shared__ int s_hi, s_bad, s_wcnt[8], s_misc[2];
   __shared__ volatile int s_more[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -368,9 +368,20 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
       __threadfence_block();
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (!s_bad)
-        compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes, a.tile_count + vt, c_hi,
-                          s_wcnt, row);
+      if (!s_bad) {
+        const uint16_t* list = a.tile_list + (size_t)vt * G.n_cubes;
+        const int n = compact_tile_list(tmask, a.tile_list + (size_t)vt * G.n_cubes,
+                                        a.tile_count + vt, c_hi, s_wcnt, row);
+        if (a.sp.rows > 0) {
+          __threadfence_block();
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+          // the tile's lowest own cube: that of its first row
+          const int c_lo = a.cube_ids[tile_row(G, false, vt, 0).t];
+          static_assert(sizeof(sel::Smem) >= kSparseMax * 24, "split staging");
+          split_tile(tmask, list, n, a.sp, vt, G.n_cubes, c_lo, kv, t * G.hq + h, valid,
+                     reinterpret_cast<uint8_t*>(ss), s_wcnt, s_misc, hdr, row);
+        }
+      }
     }
   }
   tc_fence_before();

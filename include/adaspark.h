@@ -111,11 +111,16 @@ typedef struct {
                              /* min(C_k* - p, p - C_k*-1, P_(k*) - P_(k*+1)) < 1e-5, */
                              /* from the fp32 masses (a row whose next score is     */
                              /* not known counts as near); 0 for Top-K             */
-  uint64_t reserved[8];
+  uint64_t split_pairs;      /* (row, cube) pairs run in gathered tiles (split walk) */
+  uint64_t gathered_blocks;  /* (gathered tile, key block) pairs they executed       */
+  uint64_t reserved[6];
 } adaspark_attn_stats;
 
 /* Device workspace bytes needed by adaspark_cube_attn for these sizes
- * (0 when the sizes are invalid). */
+ * (0 when the sizes are invalid). For ADASPARK_BF16 this includes the region
+ * of the split walk (adaspark_set_split_rows); the common layout alone, the
+ * ADASPARK_FP32 figure for the same sizes, is also accepted and then runs the
+ * single walk. */
 size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv,
                                     int d, int dtype);
 
@@ -259,9 +264,10 @@ int adaspark_attn_read_stats(const void *workspace, adaspark_attn_stats *stats, 
  * adaspark_cube_attn, without the workspace: the kernels use a fixed array of
  * ADASPARK_NOALLOC_SCRATCH_BYTES that the library keeps in device memory on
  * every GPU where its device code is loaded, until the process exits.
- *   - Returns ADASPARK_EINVAL when the sizes are invalid or when
- *     adaspark_cube_attn_workspace() for them exceeds
- *     ADASPARK_NOALLOC_SCRATCH_BYTES (check that first).
+ *   - Runs the single walk (no split walk). Returns ADASPARK_EINVAL when the
+ *     sizes are invalid or when the single walk's workspace for them
+ *     (adaspark_cube_attn_workspace with dtype ADASPARK_FP32, the common
+ *     layout) exceeds ADASPARK_NOALLOC_SCRATCH_BYTES (check that first).
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current); make that first call before any stream
  *     capture.
@@ -471,6 +477,23 @@ int adaspark_read_device_status(const void *workspace, uint32_t *detail, void *s
  * and behaviour. Process-wide, not thread-safe; ADASPARK_EINVAL for a bound
  * outside the range. */
 int adaspark_debug_wait_expiry(int on, long long wait_cycles);
+
+/* Split walk of the bf16 forward (adaspark_cube_attn and adaspark_cube_attn_topk;
+ * not the training-mode call, Uniform Sampling, p = 1, or the allocation-free
+ * entry point). A visual attention tile (128 consecutive visual tokens of one
+ * query head) walks the key blocks of every cube any of its rows selected. A
+ * selected cube that at most `rows` of the tile's rows chose, and that is no
+ * row's own cube, leaves the tile's walk: its (row, cube) pairs are regrouped
+ * by (KV head, cube) into gathered 128-row tiles, run over that cube's keys
+ * alone, and each row merges their normalised partial outputs (bf16) by their
+ * log2-sum-exps at the end of its own walk. The sets and the softmax are
+ * those of the single walk; only the rounding of the merged parts differs.
+ * Needs the workspace adaspark_cube_attn_workspace returns for BF16 (a smaller
+ * workspace that still holds the common layout runs the single walk); a tile
+ * whose records would pass the workspace's record capacity (6 per visual row)
+ * keeps its whole walk. rows = 0 turns it off; default 8. Process-wide, not
+ * thread-safe; ADASPARK_EINVAL for rows outside [0, 128]. */
+int adaspark_set_split_rows(int rows);
 
 /* Per-kernel timing with CUDA events recorded on the launching stream around
  * each launch of this library. Off by default; process-wide; not thread-safe. */

@@ -110,9 +110,18 @@ def test_backward_layer_and_train_calls_reject_bad_arguments_before_the_device()
     assert fb.cube_attn_backward_workspace_bytes(544, 512, 16, 4, 1, 64, fb.FP32) == 0
     assert fb.token_ffn_backward_workspace_bytes(65792, 65536, 1024, 3584, 18944) > 0
     assert fb.token_ffn_backward_workspace_bytes(544, 512, 16, 256, 512, fb.FP32) == 0
+    # the common layout (the fp32 figure) plus the fp32 output of a training call;
+    # the bf16 inference figure adds the split walk's region instead
+    common = fb.cube_attn_workspace_bytes(65792, 65536, 1024, 28, 4, 128, fb.FP32)
     inf = fb.cube_attn_workspace_bytes(65792, 65536, 1024, 28, 4, 128, fb.BF16)
     assert fb.cube_attn_train_workspace_bytes(65792, 65536, 1024, 28, 4, 128) == \
-        inf + 65792 * 28 * 128 * 4
+        common + 65792 * 28 * 128 * 4
+    assert inf > common
+    # the split walk's threshold: 0 .. 128 rows
+    assert L.adaspark_set_split_rows(-1) == fb.EINVAL
+    assert L.adaspark_set_split_rows(129) == fb.EINVAL
+    assert L.adaspark_set_split_rows(0) == fb.OK
+    assert L.adaspark_set_split_rows(fb.SPLIT_ROWS_DEFAULT) == fb.OK
     # attention backward: fp32 unsupported, bad sizes / pointers / workspace rejected
     ab = fb.cube_attn_backward_workspace_bytes(544, 512, 16, 4, 1, 128)
     aargs = [d] * 4
