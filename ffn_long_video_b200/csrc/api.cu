@@ -129,7 +129,8 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
     sp.grp_base = reinterpret_cast<int32_t*>(r + SL.grp_base);
     sp.grp_tile = reinterpret_cast<int32_t*>(r + SL.grp_tile);
     sp.grec = reinterpret_cast<int32_t*>(r + SL.grec);
-    sp.mtile = reinterpret_cast<int32_t*>(r + SL.mtile);
+    sp.grow = reinterpret_cast<int32_t*>(r + SL.grow);
+    sp.mt_info = reinterpret_cast<int4*>(r + SL.mt_info);
     sp.part_o = reinterpret_cast<__nv_bfloat16*>(r + SL.part_o);
     sp.part_lse = reinterpret_cast<float*>(r + SL.part_lse);
     if (cudaMemsetAsync(sp.grp_cnt, 0, (size_t)G.hkv * n_cubes * sizeof(int32_t), s) !=
@@ -168,7 +169,7 @@ static int cube_attn_impl(const void* Q, const void* K, const void* V, int dtype
     rc = cuda_rc(dtype == ADASPARK_BF16 ? launch_select_tc(sa, s) : launch_select_simt(sa, dtype, s));
     if (rc) return rc;
     if (split) {
-      rc = cuda_rc(launch_split_build(sp, G, hdr, s));
+      rc = cuda_rc(launch_split_build(sp, G, cube_offsets, hdr, s));
       if (rc) return rc;
     }
   }

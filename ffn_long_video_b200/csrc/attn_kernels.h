@@ -24,7 +24,8 @@ struct SplitArgs {
   int32_t* grp_base;
   int32_t* grp_tile;
   int32_t* grec;
-  int32_t* mtile;
+  int32_t* grow;
+  int4* mt_info;
   __nv_bfloat16* part_o;
   float* part_lse;
 };
@@ -127,8 +128,8 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
 // Split walk: group the records by (KV head, cube) and number the gathered
 // tiles (after the selection), then run the gathered tiles (before the tiles'
 // own walk, whose epilogue merges their partial results).
-cudaError_t launch_split_build(const SplitArgs& sp, const AttnGeom& G, WsHeader* hdr,
-                               cudaStream_t s);
+cudaError_t launch_split_build(const SplitArgs& sp, const AttnGeom& G,
+                               const int32_t* cube_offsets, WsHeader* hdr, cudaStream_t s);
 cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t s);
 
 }  // namespace adaspark

@@ -69,16 +69,27 @@ __global__ void __launch_bounds__(1024) split_prefix_kernel(SplitArgs sp, int n_
   }
 }
 
-// Gathered tile -> group table, and the records placed group by group at the
-// places the selection gave them. Grid-stride over groups, then records.
+// Gathered tile table (first record slot, rows | KV head << 8, the cube's
+// first and end token) and the records placed group by group at the places the
+// selection gave them, with their rows beside them. Grid-stride over groups,
+// then records.
 __global__ void __launch_bounds__(256) split_scatter_kernel(SplitArgs sp, int n_groups, int C,
-                                                            int hq, int g_size, WsHeader* hdr) {
+                                                            int hq, int g_size,
+                                                            const int32_t* cube_offsets,
+                                                            WsHeader* hdr) {
   if (status_bad(hdr)) return;
   const int stride = gridDim.x * blockDim.x;
   const int first = blockIdx.x * blockDim.x + threadIdx.x;
   for (int g = first; g < n_groups; g += stride) {
     const int t0 = sp.grp_tile[g], t1 = min(sp.grp_tile[g + 1], sp.max_mtiles);
-    for (int m = t0; m < t1; ++m) sp.mtile[m] = g;
+    if (t0 >= t1) continue;
+    const int kv = g / C, cube = g - kv * C;
+    const int b0 = sp.grp_base[g], b1 = sp.grp_base[g + 1];
+    const int ks = cube_offsets[cube], ke = cube_offsets[cube + 1];
+    for (int m = t0; m < t1; ++m) {
+      const int f = b0 + (m - t0) * kTileRows;
+      sp.mt_info[m] = make_int4(f, min(kTileRows, b1 - f) | (kv << 8), ks, ke);
+    }
   }
   const int n_rec = (int)min((long long)hdr->sched[0], (long long)sp.cap);
   for (int i = first; i < n_rec; i += stride) {
@@ -86,21 +97,23 @@ __global__ void __launch_bounds__(256) split_scatter_kernel(SplitArgs sp, int n_
     if (rid < 0) continue;                      // reserved by a tile that did not split
     const int kv = (rid % hq) / g_size;
     const int g = kv * C + sp.rec_cube[i];
-    sp.grec[sp.grp_base[g] + sp.rec_gpos[i]] = i;
+    const int slot = sp.grp_base[g] + sp.rec_gpos[i];
+    sp.grec[slot] = i;
+    sp.grow[slot] = rid;
   }
 }
 
 }  // namespace split
 
-cudaError_t launch_split_build(const SplitArgs& sp, const AttnGeom& G, WsHeader* hdr,
-                               cudaStream_t s) {
+cudaError_t launch_split_build(const SplitArgs& sp, const AttnGeom& G,
+                               const int32_t* cube_offsets, WsHeader* hdr, cudaStream_t s) {
   const int n_groups = G.hkv * G.n_cubes;
   if (n_groups == 0) return cudaSuccess;
   cudaError_t e = launch("split_prefix", split::split_prefix_kernel, dim3(1), dim3(1024), 0, s,
                          sp, n_groups, hdr);
   if (e != cudaSuccess) return e;
   return launch("split_scatter", split::split_scatter_kernel, dim3(148 * 4), dim3(256), 0, s, sp,
-                n_groups, G.n_cubes, G.hq, G.g, hdr);
+                n_groups, G.n_cubes, G.hq, G.g, cube_offsets, hdr);
 }
 
 }  // namespace adaspark

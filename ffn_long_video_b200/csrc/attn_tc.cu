@@ -94,11 +94,7 @@ __device__ __forceinline__ void add2(float& s0, float& s1, float a0, float a1) {
 // pair hi + lo (lo = P - hi, in the second half of the S buffer, whose
 // scores were read before), so O is exact to about 2^-17 of each term, and O is
 // also written in fp32 to a.o32; the backward takes D_r = dO_r . O_r from it.
-// GATHER: a gathered tile of the split walk (see SplitLayout): its rows are
-// records (row, cube) of one (KV head, cube) group, taken from many tiles; it
-// walks that cube's keys alone and writes each record's normalised output and
-// log2-sum-exp, which the row's own tile merges at the end of its walk.
-template <bool TRAIN, int D, bool GATHER>
+template <bool TRAIN, int D>
 __global__ void __launch_bounds__(THREADS, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                    AttnArgs a) {
@@ -129,26 +125,9 @@ __global__ void __launch_bounds__(THREADS, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const AttnGeom& G = a.G;
   WsHeader* hdr = a.hdr;
-  TileInfo T;
-  int g_cube = 0, g_first = 0, g_count = 0;   // gathered tile: cube, first record slot, rows
-  if (GATHER) {
-    // the launch covers the largest possible number of gathered tiles; the
-    // regrouping counted the ones that exist
-    const int m_tile = blockIdx.x;
-    if (m_tile >= (int)*reinterpret_cast<const volatile uint32_t*>(&hdr->sched[1])) return;
-    const int grp = a.sp.mtile[m_tile];
-    T.text = false;
-    T.kv = grp / G.n_cubes;
-    T.bt = 0;
-    T.t_hi = 0;
-    g_cube = grp - T.kv * G.n_cubes;
-    g_first = a.sp.grp_base[grp] + (m_tile - a.sp.grp_tile[grp]) * kTileRows;
-    g_count = min(kTileRows, a.sp.grp_base[grp + 1] - g_first);
-  } else {
-    T = decode_tile(G, a.kv_major != 0);
-  }
+  const TileInfo T = decode_tile(G, a.kv_major != 0);
   // the tile walks only part of its list, the rest in gathered tiles
-  const bool split = !GATHER && !TRAIN && a.sp.rows > 0 && !T.text && !a.dense;
+  const bool split = !TRAIN && a.sp.rows > 0 && !T.text && !a.dense;
   const long long WL = a.wait_limit;  // cycles before any wait of this kernel gives up
 
   if (warp == 2) {
@@ -176,7 +155,7 @@ __global__ void __launch_bounds__(THREADS, 2)
     fence_mbar_init();
     s_abort = 0;
     s_bad = status_bad(hdr) ? 1 : 0;
-    s_own_hi = (!GATHER && !T.text && !s_bad) ? a.cube_ids[T.t_hi] : -1;
+    s_own_hi = (!T.text && !s_bad) ? a.cube_ids[T.t_hi] : -1;
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&mapK);
@@ -200,8 +179,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (T.text) {
         n_entries = G.n_cubes;
         n_chunks = (T.t_hi - G.n_vis) / 64 + 1;
-      } else if (GATHER) {
-        n_entries = 1;
       } else if (a.dense) {
         n_entries = s_own_hi + 1;
       } else {
@@ -219,18 +196,10 @@ __global__ void __launch_bounds__(THREADS, 2)
       int j = -1, ks = 0, ke = 0;
       uint4 m = make_uint4(~0u, ~0u, ~0u, ~0u);
       if (e < n_entries) {
-        j = GATHER ? g_cube : use_list ? (int)list[e] : e;
+        j = use_list ? (int)list[e] : e;
         ks = a.cube_offsets[j];
         ke = a.cube_offsets[j + 1];
-        if (use_list) {
-          m = tmask[j];
-        } else if (GATHER) {  // the gathered tile's rows that exist
-          auto word = [&](int w) {
-            const int r = g_count - 32 * w;
-            return r >= 32 ? ~0u : r > 0 ? (1u << r) - 1u : 0u;
-          };
-          m = make_uint4(word(0), word(1), word(2), word(3));
-        }
+        if (use_list) m = tmask[j];
       } else if (e < n_total) {
         ks = G.n_vis + (e - n_entries) * 64;
         ke = min(ks + 64, T.t_hi + 1);
@@ -399,20 +368,10 @@ __global__ void __launch_bounds__(THREADS, 2)
     // ------------------------------------------------------------ softmax rows
     const int wq = warp & 3;
     const int row = wq * 32 + lane;
-    TileRow R;
-    int rec = 0;                                // GATHER: this row's record
-    if (GATHER) {
-      R.valid = row < g_count;
-      rec = R.valid ? a.sp.grec[g_first + row] : 0;
-      const int rid = R.valid ? a.sp.rec_row[rec] : 0;
-      R.t = rid / G.hq;
-      R.h = rid - R.t * G.hq;
-    } else {
-      R = tile_row(G, T.text, T.bt, row);
-    }
+    const TileRow R = tile_row(G, T.text, T.bt, row);
     const bool valid = R.valid;
     const int t = R.t, h = R.h;
-    const int own = (!GATHER && !T.text && valid) ? a.cube_ids[t] : -1;
+    const int own = (!T.text && valid) ? a.cube_ids[t] : -1;
     const float scale = a.scale_log2;
     {
       const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
@@ -613,11 +572,8 @@ __global__ void __launch_bounds__(THREADS, 2)
         }
       }
       // the row's softmax is 2^(s * scale - lse): kept for the backward pass
-      if (!GATHER && valid && a.lse) a.lse[(size_t)t * G.hq + h] = lse_row;
-      if (GATHER && valid) a.sp.part_lse[rec] = lse_own;
-      __nv_bfloat16* dst =
-          GATHER ? a.sp.part_o + (size_t)rec * D
-                 : reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * D;
+      if (valid && a.lse) a.lse[(size_t)t * G.hq + h] = lse_row;
+      __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(a.out) + ((size_t)t * G.hq + h) * D;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
@@ -673,13 +629,451 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
     }
     if (warp == 2 && lane == 0 && !bad) {
-      if (GATHER) {  // gathered tiles and their blocks are counted apart
-        atomicAdd((unsigned long long*)&hdr->stats[8], (unsigned long long)g_count);
-        atomicAdd((unsigned long long*)&hdr->stats[9], (unsigned long long)i);
-      } else {
-        atomicAdd((unsigned long long*)&hdr->stats[4], 1ull);
-        atomicAdd((unsigned long long*)&hdr->stats[5], (unsigned long long)i);
+      atomicAdd((unsigned long long*)&hdr->stats[4], 1ull);
+      atomicAdd((unsigned long long*)&hdr->stats[5], (unsigned long long)i);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 256);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Gathered tiles of the split walk (see SplitLayout), persistent: CTA b takes
+// gathered tiles b, b + grid, b + 2 grid, ... A gathered tile holds up to 128
+// records (row, cube) of one (KV head, cube) group, query rows of many tiles
+// and heads; it walks that cube's keys alone (no causal part: the cube lies
+// below every row's own cube) and writes each record's normalised output
+// (bf16) and log2-sum-exp, which the row's own tile merges at the end of its
+// walk. The next tile's query rows are copied into the second Q buffer
+// (cp.async) while the current tile computes, and its first scores are
+// computed while the current tile's output is read, so one tile's chain of
+// latencies overlaps the next one's.
+//   warp 0     TMA producer: K and V blocks (one stage each)
+//   warp 1     TMEM allocator + tcgen05.mma issuer (S into two buffers, O)
+//   warps 2-5  one thread per row: Q copies, softmax, epilogue
+// ---------------------------------------------------------------------------
+constexpr int G_THREADS = 192;
+template <int D>
+constexpr size_t gather_smem_bytes() {
+  return 1024 + 2 * Dim<D>::Q_BYTES + 2 * Dim<D>::K_BYTES + 512;
+}
+
+struct GTile {
+  int kv, first, count, ks, ke;   // KV head, first record slot, rows, the cube's tokens
+};
+__device__ __forceinline__ GTile gather_tile(const AttnArgs& a, int m) {
+  const int4 v = a.sp.mt_info[m];
+  GTile g;
+  g.first = v.x;
+  g.count = v.y & 0xff;
+  g.kv = v.y >> 8;
+  g.ks = v.z;
+  g.ke = v.w;
+  return g;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(G_THREADS, 2)
+    attn_gather_kernel(const __grid_constant__ CUtensorMap mapK,
+                       const __grid_constant__ CUtensorMap mapV, AttnArgs a) {
+  constexpr int Q_BYTES = Dim<D>::Q_BYTES, K_BYTES = Dim<D>::K_BYTES;
+  constexpr int HALVES = Dim<D>::HALVES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;                       // [2][Q_BYTES]
+  uint8_t* sK = sQ + 2 * Q_BYTES;
+  uint8_t* sV = sK + K_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + K_BYTES);
+  uint64_t* k_full = bars;
+  uint64_t* k_empty = k_full + 1;
+  uint64_t* v_full = k_empty + 1;
+  uint64_t* v_empty = v_full + 1;
+  uint64_t* s_full = v_empty + 1;           // [2]
+  uint64_t* p_full = s_full + 2;            // [2]
+  uint64_t* pv_done = p_full + 2;           // [2]
+  uint64_t* q_full = pv_done + 2;           // [2]
+  uint64_t* o_free = q_full + 2;
+  uint64_t* drain = o_free + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const AttnGeom& G = a.G;
+  WsHeader* hdr = a.hdr;
+  const long long WL = a.wait_limit;
+  // the regrouping counted the gathered tiles; CTAs beyond them have none
+  const int total = (int)*reinterpret_cast<const volatile uint32_t*>(&hdr->sched[1]);
+  // (a bad status set before this launch left the count at 0)
+  if ((int)blockIdx.x >= total) return;
+  const int step = gridDim.x;
+
+  if (threadIdx.x == 0) {
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+      mbar_init(&q_full[b], 128);
+    }
+    mbar_init(o_free, 128);
+    mbar_init(drain, 1);
+    fence_mbar_init();
+    s_abort = 0;
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      // block i: K_i (stage free once S_{i-1} is done), then V_i (free once
+      // PV_{i-1} is done)
+      int i = 0, nv = 0;
+      bool ok = true;
+      GTile gn = gather_tile(a, blockIdx.x);
+      for (int m = blockIdx.x; ok && m < total; m += step) {
+        const GTile g = gn;
+        if (m + step < total) gn = gather_tile(a, m + step);   // in flight meanwhile
+        for (int k0 = g.ks; k0 < g.ke; k0 += 64) {
+          if (!mbar_wait(k_empty, (i & 1) ^ 1, &s_abort, hdr, 0x7a00u, WL)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(k_full, K_BYTES);
+#pragma unroll
+          for (int hf = 0; hf < HALVES; ++hf)
+            tma_load_3d(&mapK, k_full, sK + hf * 8192, hf * 64, g.kv, k0);
+          ++i;
+          if (!mbar_wait(v_empty, (nv & 1) ^ 1, &s_abort, hdr, 0x7a10u, WL)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(v_full, K_BYTES);
+#pragma unroll
+          for (int hf = 0; hf < HALVES; ++hf)
+            tma_load_3d(&mapV, v_full, sV + hf * 8192, hf * 64, g.kv, k0);
+          ++nv;
+        }
       }
+      if (!ok) {  // let copies already issued land before the CTA exits
+        long long t0 = clock64();
+        while (i > 0 && !mbar_try_wait(k_full, (i - 1) & 1) && clock64() - t0 < WL) {
+        }
+        while (nv > 0 && !mbar_try_wait(v_full, (nv - 1) & 1) && clock64() - t0 < WL) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = make_idesc_bf16(128, 64);
+      constexpr uint32_t idesc_o = make_idesc_bf16(128, D, true);
+      int i = 0, k = 0;
+      bool ok = true, prev_first = false;
+      int prev_tile = 0;
+      // PV of block blk: its P, its V, and (first block of a tile after the
+      // first) the previous tile's output read out of O
+      auto issue_pv = [&](int blk, bool first, int tile) -> bool {
+        const int pb = blk & 1;
+        if (!mbar_wait(&p_full[pb], (blk >> 1) & 1, &s_abort, hdr, 0x7b00u, WL)) return false;
+        if (!mbar_wait(v_full, blk & 1, &s_abort, hdr, 0x7b10u, WL)) return false;
+        if (first && tile > 0 &&
+            !mbar_wait(o_free, (tile - 1) & 1, &s_abort, hdr, 0x7b20u, WL))
+          return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sV);
+        const uint32_t p_tmem = tmem_base + 128 + pb * 64;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = make_sdesc_sw128(v_addr + kk * 2048, 8192, 1024);
+          umma_bf16_ts(tmem_base, p_tmem + kk * 8, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_done[pb]);
+        umma_commit(v_empty);
+        return true;
+      };
+      GTile gn = gather_tile(a, blockIdx.x);
+      for (int m = blockIdx.x; ok && m < total; m += step, ++k) {
+        const GTile g = gn;
+        if (m + step < total) gn = gather_tile(a, m + step);   // in flight meanwhile
+        // the previous tile's last PV first: its output does not wait for
+        // this tile's keys
+        if (i > 0 && !issue_pv(i - 1, prev_first, prev_tile)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&q_full[k & 1], (k >> 1) & 1, &s_abort, hdr, 0x7b30u, WL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQ + (k & 1) * Q_BYTES);
+        for (int k0 = g.ks; k0 < g.ke; k0 += 64, ++i) {
+          if (!mbar_wait(k_full, i & 1, &s_abort, hdr, 0x7b40u, WL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sK);
+          const uint32_t d_s = tmem_base + 128 + (i & 1) * 64;
+#pragma unroll
+          for (int dc = 0; dc < HALVES; ++dc)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = make_sdesc_sw128(q_addr + dc * 16384 + kk * 32, 16, 1024);
+              const uint64_t bd = make_sdesc_sw128(k_addr + dc * 8192 + kk * 32, 16, 1024);
+              umma_bf16(d_s, ad, bd, idesc_s, (dc | kk) != 0 ? 1u : 0u);
+            }
+          umma_commit(&s_full[i & 1]);
+          umma_commit(k_empty);
+          // within a tile, the previous block's PV after this block's S
+          if (k0 != g.ks && !issue_pv(i - 1, prev_first, prev_tile)) {
+            ok = false;
+            break;
+          }
+          prev_first = k0 == g.ks;
+          prev_tile = k;
+        }
+      }
+      if (ok && i > 0) issue_pv(i - 1, prev_first, prev_tile);
+      umma_commit(drain);
+      long long t0 = clock64();
+      while (!mbar_try_wait(drain, 0) && clock64() - t0 < WL) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ rows
+    const int wq = warp & 3;                // the TMEM lane quadrant this warp may access
+    const int row = wq * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+    const float scale = a.scale_log2;
+    // Row data arrive in stages, each a tile ahead of its use: the tile table
+    // entry three tiles ahead, the records and rows two ahead, the query copy
+    // one ahead.
+    auto row_rec = [&](const GTile& g, int& rec, int& rid) {
+      const bool v = row < g.count;
+      rec = v ? a.sp.grec[g.first + row] : 0;
+      rid = v ? a.sp.grow[g.first + row] : 0;
+    };
+    // the row's query into Q buffer qb, 16-byte copies (zeros for a row past
+    // the tile's count), completed before q_full is announced
+    auto copy_q = [&](int qb, bool valid, int rid) {
+      const __nv_bfloat16* Qg = reinterpret_cast<const __nv_bfloat16*>(a.Q);
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(Qg + (size_t)rid * D);
+      const uint32_t dst = smem_u32(sQ + qb * Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c)
+        cp_async16(dst + (c >> 3) * 16384 + sw128_offset(row, c & 7), src + c * 16,
+                   valid ? 16u : 0u);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const GTile g_none{0, 0, 0, 0, 0};
+    GTile g = gather_tile(a, blockIdx.x);
+    GTile g1 = blockIdx.x + step < total ? gather_tile(a, blockIdx.x + step) : g_none;
+    GTile g2 = blockIdx.x + 2 * step < total ? gather_tile(a, blockIdx.x + 2 * step) : g_none;
+    int rec, rid, rec1, rid1;
+    row_rec(g, rec, rid);
+    row_rec(g1, rec1, rid1);
+    bool valid = row < g.count;
+    copy_q(0, valid, rid);
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    mbar_arrive(&q_full[0]);
+    int i = 0, k = 0, pairs = 0;
+    bool ok = true;
+    for (int m = blockIdx.x; ok && m < total; m += step, ++k) {
+      const bool has_next = m + step < total;
+      // the next tile's queries, copied while this one computes
+      if (has_next) copy_q((k + 1) & 1, row < g1.count, rid1);
+      // records and rows two tiles ahead, the table entry three ahead
+      int rec2 = 0, rid2 = 0;
+      row_rec(g2, rec2, rid2);
+      const GTile g3 = m + 3 * step < total ? gather_tile(a, m + 3 * step) : g_none;
+      pairs += g.count;
+      float m_used = -INFINITY, l = 0.f;
+      for (int k0 = g.ks; k0 < g.ke; k0 += 64, ++i) {
+        const int sb = i & 1;
+        const bool row_on = valid;
+        const int lim = row_on ? min(64, g.ke - k0) : 0;
+        if (!mbar_wait_warp(&s_full[sb], (i >> 1) & 1, &s_abort, hdr, 0x7c00u, WL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (!__any_sync(0xffffffffu, row_on)) {
+          uint32_t zero[32];
+#pragma unroll
+          for (int q = 0; q < 32; ++q) zero[q] = 0u;
+          tmem_st32(tmem_base + lane_base + 128 + sb * 64, zero);
+        } else {
+          uint32_t sr[64];
+          {
+            uint32_t(&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+            uint32_t(&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+            tmem_ld32(tmem_base + lane_base + 128 + sb * 64, s0);
+            tmem_ld32(tmem_base + lane_base + 128 + sb * 64 + 32, s1);
+          }
+          tmem_ld_wait();
+          const bool partial = __any_sync(0xffffffffu, row_on && lim < 64);
+          float mraw = -INFINITY;
+          if (!partial) {
+            auto f = [&](int u) { return __uint_as_float(sr[u]); };
+            float mx[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) mx[q] = fmax3(f(q), f(q + 8), f(q + 16));
+#pragma unroll
+            for (int q = 0; q < 8; ++q) mx[q] = fmax3(mx[q], f(q + 24), f(q + 32));
+#pragma unroll
+            for (int q = 0; q < 8; ++q) mx[q] = fmax3(mx[q], f(q + 40), f(q + 48));
+            const float t0 = fmax3(mx[0], mx[1], f(56)), t1 = fmax3(mx[2], mx[3], f(57));
+            const float t2 = fmax3(mx[4], mx[5], f(58)), t3 = fmax3(mx[6], mx[7], f(59));
+            const float t4 = fmax3(f(60), f(61), f(62));
+            const float m8 = fmax3(fmax3(t0, t1, t2), fmax3(t3, t4, f(63)), -INFINITY);
+            mraw = row_on ? m8 : -INFINITY;
+          } else {
+            float mx[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) mx[q] = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < 64; ++u)
+              if (u < lim) mx[u & 7] = fmaxf(mx[u & 7], __uint_as_float(sr[u]));
+            mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          }
+          const float m_new = fmaxf(m_used, mraw * scale);
+          const bool want = m_new > m_used + kRescale;
+          if (__any_sync(0xffffffffu, want)) {
+            const float factor = (m_used == -INFINITY || m_new == -INFINITY) ? 1.f
+                                                                             : ex2(m_used - m_new);
+            if (k0 != g.ks) {  // O holds this tile's earlier blocks
+              if (!mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr,
+                                  0x7c10u, WL)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+#pragma unroll 1
+              for (int c = 0; c < D; c += 32) {
+                uint32_t o[32];
+                tmem_ld32(tmem_base + lane_base + c, o);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                  o[x] = __float_as_uint(__uint_as_float(o[x]) * factor);
+                tmem_st32(tmem_base + lane_base + c, o);
+              }
+            }
+            l *= factor;
+            if (m_new != -INFINITY) m_used = m_new;
+          }
+          const float neg_m = row_on ? -m_used : -INFINITY;
+          float ls[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) ls[q] = 0.f;
+          uint32_t pk[32];
+          if (!partial) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              float x0, x1;
+              fma2_bcast(__uint_as_float(sr[2 * q]), __uint_as_float(sr[2 * q + 1]), scale,
+                         neg_m, x0, x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              add2(ls[2 * (q & 3)], ls[2 * (q & 3) + 1], p0, p1);
+              pk[q] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const int u = 2 * q;
+              const float p0 = (u < lim) ? ex2(fmaf(__uint_as_float(sr[u]), scale, neg_m)) : 0.f;
+              const float p1 =
+                  (u + 1 < lim) ? ex2(fmaf(__uint_as_float(sr[u + 1]), scale, neg_m)) : 0.f;
+              ls[q & 7] += p0 + p1;
+              pk[q] = pack_bf16x2(p0, p1);
+            }
+          }
+          tmem_st32(tmem_base + lane_base + 128 + sb * 64, pk);
+          l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[sb]);
+        if (k0 == g.ks && has_next) {  // the next tile's queries are in
+          cp_async_wait_all();
+          fence_proxy_async_smem();
+          mbar_arrive(&q_full[(k + 1) & 1]);
+        }
+      }
+      if (!ok) break;
+      // the tile's output: O / l once its last PV has landed, then O is free
+      if (!mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr, 0x7c20u,
+                          WL)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      __nv_bfloat16* dst = a.sp.part_o + (size_t)rec * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tmem_base + lane_base + c, o);
+        tmem_ld_wait();
+        if (valid) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            pk[x] = pack_bf16x2(__uint_as_float(o[2 * x]) * inv,
+                                __uint_as_float(o[2 * x + 1]) * inv);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            d4[x] = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(o_free);
+      if (valid) a.sp.part_lse[rec] = m_used + __log2f(l);
+      g = g1;
+      rec = rec1;
+      valid = row < g.count;
+      g1 = g2;
+      rec1 = rec2;
+      rid1 = rid2;
+      g2 = g3;
+    }
+    cp_async_wait_all();   // no copy outlives the CTA
+    if (warp == 2 && lane == 0 && ok) {
+      atomicAdd((unsigned long long*)&hdr->stats[8], (unsigned long long)pairs);
+      atomicAdd((unsigned long long*)&hdr->stats[9], (unsigned long long)i);
     }
   }
   tc_fence_before();
@@ -703,22 +1097,27 @@ cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
   if (!encode_tmap_bf16(&mK, a.K, 3, dims, strides, box) ||
       !encode_tmap_bf16(&mV, a.V, 3, dims, strides, box))
     return cudaErrorInvalidValue;
-  auto k = G.d == 64
-               ? (a.o32 ? fa::attn_tc_kernel<true, 64, false> : fa::attn_tc_kernel<false, 64, false>)
-               : (a.o32 ? fa::attn_tc_kernel<true, 128, false>
-                        : fa::attn_tc_kernel<false, 128, false>);
+  auto k = G.d == 64 ? (a.o32 ? fa::attn_tc_kernel<true, 64> : fa::attn_tc_kernel<false, 64>)
+                     : (a.o32 ? fa::attn_tc_kernel<true, 128> : fa::attn_tc_kernel<false, 128>);
   const size_t smem = G.d == 64 ? fa::smem_bytes<64>() : fa::smem_bytes<128>();
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch("attn_tc", k, dim3(blocks), dim3(fa::THREADS), smem, s, mK, mV, a);
 }
 
-// The gathered tiles of the split walk: a grid of the largest possible count
-// (SplitLayout::max_mtiles); tiles past the count the regrouping wrote exit at
-// once.
+// The gathered tiles of the split walk: two persistent CTAs per SM (fewer when
+// fewer gathered tiles can exist); CTAs past the count the regrouping wrote
+// exit at once.
 cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t s) {
   const AttnGeom& G = a.G;
   if (a.sp.rows <= 0 || a.sp.max_mtiles <= 0 || G.n_vtiles == 0) return cudaSuccess;
+  static int n_sm = 0;
+  if (n_sm == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n_sm = 148;
+  }
   CUtensorMap mK, mV;
   const uint64_t dims[3] = {(uint64_t)G.d, (uint64_t)G.hkv, (uint64_t)G.n_tokens};
   const uint64_t strides[2] = {(uint64_t)G.d * 2, (uint64_t)G.hkv * G.d * 2};
@@ -726,12 +1125,12 @@ cudaError_t launch_attn_tc_gather(const AttnArgs& a, cudaStream_t s) {
   if (!encode_tmap_bf16(&mK, a.K, 3, dims, strides, box) ||
       !encode_tmap_bf16(&mV, a.V, 3, dims, strides, box))
     return cudaErrorInvalidValue;
-  auto k = G.d == 64 ? fa::attn_tc_kernel<false, 64, true> : fa::attn_tc_kernel<false, 128, true>;
-  const size_t smem = G.d == 64 ? fa::smem_bytes<64>() : fa::smem_bytes<128>();
+  auto k = G.d == 64 ? fa::attn_gather_kernel<64> : fa::attn_gather_kernel<128>;
+  const size_t smem = G.d == 64 ? fa::gather_smem_bytes<64>() : fa::gather_smem_bytes<128>();
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch("attn_tc_gather", k, dim3(a.sp.max_mtiles), dim3(fa::THREADS), smem, s, mK, mV,
-                a);
+  const int grid = std::min(a.sp.max_mtiles, 2 * n_sm);
+  return launch("attn_tc_gather", k, dim3(grid), dim3(fa::G_THREADS), smem, s, mK, mV, a);
 }
 
 }  // namespace adaspark

@@ -112,7 +112,9 @@ struct SplitLayout {
   size_t grp_base;    // int32 [hkv * C + 1]    exclusive prefix of grp_cnt
   size_t grp_tile;    // int32 [hkv * C + 1]    exclusive prefix of gathered tiles
   size_t grec;        // int32 [cap]            records grouped by (KV head, cube)
-  size_t mtile;       // int32 [max_mtiles]     gathered tile -> group
+  size_t grow;        // int32 [cap]            their rows, in the same order
+  size_t mt_info;     // int4 [max_mtiles]      gathered tile: first slot, rows | kv << 8, cube's
+                      //                        first and end token
   size_t part_o;      // bf16 [cap][d]          a record's normalised partial output
   size_t part_lse;    // float [cap]            and its log2-sum-exp
   int cap;            // records
@@ -144,7 +146,8 @@ __host__ __device__ inline SplitLayout make_split_layout(const AttnGeom& G) {
   L.grp_base = o; o += align_up((groups + 1) * 4);
   L.grp_tile = o; o += align_up((groups + 1) * 4);
   L.grec = o; o += align_up((cap > 0 ? cap : 1) * 4);
-  L.mtile = o; o += align_up((size_t)L.max_mtiles * 4);
+  L.grow = o; o += align_up((cap > 0 ? cap : 1) * 4);
+  L.mt_info = o; o += align_up((size_t)L.max_mtiles * 16);
   L.part_o = o; o += align_up((cap > 0 ? cap : 1) * (size_t)G.d * 2);
   L.part_lse = o; o += align_up((cap > 0 ? cap : 1) * 4);
   L.total = o;
