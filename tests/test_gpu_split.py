@@ -118,3 +118,40 @@ def test_split_walk_backward_after_inference_forward(case):
     for a, b, nm in zip(grads[0], grads[8], ("dQ", "dK", "dV")):
         scale = float(a.abs().max()) + 1e-12
         assert float((a - b).abs().max()) <= 2e-2 * scale, nm
+
+
+# gathered tiles over several 64-key pieces (128-token cubes, online softmax
+# across the pieces), ragged cubes (pieces shorter than 64 keys) and head_dim 64
+MORE = {
+    "cubes-8x8x2": workloads.small_config(name="split-8x8x2", grid=(8, 32, 32), cube=(8, 8, 2),
+                                          n_text=19, D=256, hq=8, hkv=2, F=256, seed=4242),
+    "ragged": workloads.small_config(name="split-ragged", grid=(8, 16, 16), cube=(4, 4, 2),
+                                     n_text=23, D=256, hq=6, hkv=3, F=256, seed=4343,
+                                     cube_sizes=(121, 81, 88, 115, 75, 100, 107, 29, 8, 39, 37,
+                                                 112, 117, 1, 64, 106, 17, 103, 16, 60, 105,
+                                                 39, 44, 36, 93, 33, 127, 57, 62, 56)),
+    "d64": workloads.small_config(name="split-d64", grid=(16, 16, 16), cube=(4, 4, 4), n_text=37,
+                                  D=256, hq=8, hkv=2, d=64, F=256, seed=4444),
+}
+
+
+@pytest.mark.parametrize("name", list(MORE))
+def test_split_walk_pieces_ragged_and_d64(name):
+    case = parity.make_case(MORE[name])
+    single, bits0, st0 = _run(case, 0)
+    for rows in (8, 128):
+        split, bits1, st1 = _run(case, rows)
+        assert torch.equal(bits0, bits1)
+        if rows == 128:
+            assert st1["split_pairs"] > 0, st1
+        d = (split.float() - single.float()).abs()
+        assert float((d - 4 * single.float().abs() * 2.0 ** -8).max()) <= 2e-3, (rows,
+                                                                                float(d.max()))
+        fb.set_split_rows(rows)
+        try:
+            rep = {}
+            parity.check_attn(case, report=rep)
+            print(name, "rows", rows, "split pairs", st1["split_pairs"], "gathered blocks",
+                  st1["gathered_blocks"], rep)
+        finally:
+            fb.set_split_rows(fb.SPLIT_ROWS_DEFAULT)
