@@ -122,7 +122,7 @@ typedef struct {
  * ADASPARK_FP32 figure for the same sizes, is also accepted and then runs the
  * single walk. The split walk's region holds up to 6 records per visual
  * (token, query head) row, each with a bf16 partial output of d elements:
- * about (12 d + 48) bytes per visual row, 3.6 GB for 65536 visual tokens, 28
+ * about (12 d + 152) bytes per visual row, 3.1 GB for 65536 visual tokens, 28
  * query heads and d = 128. */
 size_t adaspark_cube_attn_workspace(int n_tokens, int n_vis, int n_cubes, int hq, int hkv,
                                     int d, int dtype);
