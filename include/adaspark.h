@@ -263,8 +263,10 @@ int adaspark_attn_read_stats(const void *workspace, adaspark_attn_stats *stats, 
  * e.g. a plugin that its host framework gives only input and output buffers, a
  * serving loop that must not allocate (allocation may synchronize the device
  * or fragment a fixed budget), or a process whose device memory belongs to
- * another allocator. Same computation, arguments and errors as
- * adaspark_cube_attn, without the workspace: the kernels use a fixed array of
+ * another allocator. Same computation (as the single walk: the output of
+ * adaspark_cube_attn with adaspark_set_split_rows(0), bit for bit), arguments
+ * and errors as adaspark_cube_attn, without the workspace: the kernels use a
+ * fixed array of
  * ADASPARK_NOALLOC_SCRATCH_BYTES that the library keeps in device memory on
  * every GPU where its device code is loaded, until the process exits.
  *   - Runs the single walk (no split walk). Returns ADASPARK_EINVAL when the
