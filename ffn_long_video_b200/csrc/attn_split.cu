@@ -6,8 +6,8 @@
 // chose costs the tile a whole block for those rows. Such (row, cube) pairs,
 // the records the selection writes, are regrouped here by (KV head, cube):
 // every group becomes ceil(count / 128) gathered tiles of query rows from
-// many tiles, run by the attention kernel's gathered form over the cube's
-// keys alone; each record's partial result (normalised output and
+// many tiles, run by the gathered-tile kernel (attn_gather_kernel) over the
+// cube's keys alone; each record's partial result (normalised output and
 // log2-sum-exp) is merged into its row at the end of the row's own walk.
 #include "attn_kernels.h"
 
