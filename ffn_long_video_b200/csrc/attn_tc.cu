@@ -8,6 +8,10 @@
 // sequence of 64-key blocks: the cubes of its selection list (cubes where any
 // row has its bit set) cut into 64-key pieces, or every cube then the text keys
 // for a text tile. Rows that did not select a cube are masked inside the block.
+// With the split walk (attn_split.cu) a visual tile walks only the cubes that
+// more than a few of its rows chose (and its own cubes); each row then merges
+// the partial results of its other cubes, computed beforehand by the
+// gathered-tile kernel at the end of this file, with its own.
 //   warp 6     block-descriptor filler: reads the list, cube offsets and row
 //              masks from global memory 32 entries at a time and feeds a
 //              64-slot shared-memory ring, far ahead of the consumers
