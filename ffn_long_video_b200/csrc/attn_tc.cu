@@ -549,21 +549,6 @@ __global__ void __launch_bounds__(THREADS, 2)
       mbar_arrive(&p_full[sb]);
       ++i;
     }
-    // the row's records (split walk), their parts requested into L2 while
-    // the last PV runs
-    int mcnt = 0, moff = 0;
-    if (split && valid) {
-      const size_t rid = (size_t)t * G.hq + h;
-      mcnt = a.sp.row_cnt[rid];
-      moff = a.sp.row_off[rid];
-      for (int k = 0; k < mcnt; ++k) {
-        const char* po = reinterpret_cast<const char*>(a.sp.part_o + (size_t)(moff + k) * D);
-#pragma unroll
-        for (int b = 0; b < D * 2; b += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(po + b));
-      }
-      for (int k = 0; k < mcnt; k += 32)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.sp.part_lse + moff + k));
-    }
     // final: O / l once the last PV has landed
     if (ok && i > 0 &&
         mbar_wait_warp(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, &s_abort, hdr, 0x7900u, WL)) {
@@ -574,8 +559,12 @@ __global__ void __launch_bounds__(THREADS, 2)
       // largest of the log2-sum-exps, the row's softmax over all its keys is
       // the sum of the parts' normalised outputs weighted by 2^(lse - M) / S,
       // S the sum of those powers; lse of the whole row = M + log2 S.
+      int mcnt = 0, moff = 0;
       float w_own = 1.f, M = 0.f, inv_S = 1.f, lse_row = lse_own;
       if (split && valid) {
+        const size_t rid = (size_t)t * G.hq + h;
+        mcnt = a.sp.row_cnt[rid];
+        moff = a.sp.row_off[rid];
         if (mcnt > 0) {
           M = lse_own;
           for (int k = 0; k < mcnt; ++k) M = fmaxf(M, a.sp.part_lse[moff + k]);
@@ -728,6 +717,7 @@ __global__ void __launch_bounds__(G_THREADS, 2)
   __shared__ volatile int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const AttnGeom& G = a.G;
   WsHeader* hdr = a.hdr;
   const long long WL = a.wait_limit;
   // the regrouping counted the gathered tiles; CTAs beyond them have none
