@@ -11,7 +11,9 @@ that any row takes runs for all 128 rows. Measured here:
   heads, 32 x 4, 16 x 8), and 64-token single-head tiles, which would need
   M = 64 products;
 * one set per KV group from the group's mean query (the GQA-shared variant):
-  more selected pairs, and more executed blocks.
+  more selected pairs, and more executed blocks;
+* the split walk: the cubes that at most 8 of a tile's rows chose, moved to
+  gathered tiles, are many blocks but few pairs.
 The numbers printed are the figures quoted in the design notes."""
 import math
 
@@ -105,3 +107,44 @@ def test_group_shared_sets(study):
     # no fewer executed blocks than per-head sets
     assert pairs_shared > 1.8 * pairs
     assert t_shared > 0.95 * t128
+
+
+def test_split_walk_study(study):
+    """The split walk on the oracle's sets: a tile's cubes below its lowest own
+    cube that at most 8 of its 128 rows chose leave the tile's walk and run in
+    gathered 128-row tiles per (KV head, cube). Most of the blocks such cubes
+    cost move out, with only a small share of the selected pairs."""
+    sel, _ = study
+    T, hq, C = sel.shape
+    off = CFG.offsets
+    g = hq // CFG.hkv
+    base = off[SLICE[0]]
+    tiles = blocks = kept = moved_pairs = pairs = 0
+    warps_all = warps_moved = 0
+    groups = {}
+    for h in range(hq):
+        for s0 in range(0, T, 128):
+            rows = sel[s0:s0 + 128, h]                    # [128, C]
+            c_lo = int(np.searchsorted(off, base + s0, side="right") - 1)
+            r = rows.sum(axis=0)
+            w = np.array([rows[q:q + 32].any(axis=0) for q in range(0, rows.shape[0], 32)]).sum(0)
+            tiles += 1
+            for j in np.nonzero(r)[0]:
+                blocks += 1
+                pairs += int(r[j])
+                warps_all += int(w[j])
+                if j < c_lo and r[j] <= 8:
+                    moved_pairs += int(r[j])
+                    warps_moved += int(w[j])
+                    key = (h // g, int(j))
+                    groups[key] = groups.get(key, 0) + int(r[j])
+                else:
+                    kept += 1
+    gathered = sum(math.ceil(n / 128) for n in groups.values())
+    print(f"tiles {tiles}: blocks {blocks} -> kept {kept} + gathered {gathered}; "
+          f"pairs moved {moved_pairs / pairs:.3f}; warp-blocks moved "
+          f"{warps_moved / warps_all:.3f}")
+    # the moved blocks are many, their pairs few, and the gathered tiles pack them
+    assert kept + gathered < 0.8 * blocks
+    assert moved_pairs < 0.15 * pairs
+    assert warps_moved > 2.0 * moved_pairs / pairs * warps_all
